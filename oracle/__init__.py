@@ -1,0 +1,238 @@
+"""any4 oracle: plain fp64 CPU implementation of the any4 W4A16 path.
+
+TEST INFRASTRUCTURE.  Only tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline leg (and its ``--impl reference`` arm) may import this package.  The
+product path (learned_bit_lut_any4_b200) never imports it and shares no code
+with it.
+
+Every function follows "any4: Learned 4-bit Numeric Representation for LLMs"
+(Elhoushi & Johnson, arXiv 2507.04610):
+  pack / unpack      §2.4.1 and §4.2 (two 4-bit codes per byte; low nibble =
+                     even column is the reading used here, the pages are silent)
+  dequant            §2.5.2 dequant(w_Q) = alpha*w_Q + beta with w_Q = LUT[code];
+                     §2.5.1 group k covers columns k*G .. (k+1)*G-1
+  matmul             §4.1 Eq. 8 and §4.2 (y = x W^T, x is M x K, W is N x K)
+  bits_per_weight    §2.4.1 storage accounting (4.3125 bits at G=128, K=4096)
+
+bf16 values cross this interface as their raw uint16 bit patterns.  The
+arithmetic lives in any4_oracle.c (fp32 fmaf + IEEE round-to-nearest-even to
+bf16 for the dequant, fp64 ascending-k sums for the matmul).
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py.
+The nf4 constant table itself is not printed on the pages; the nf4 pin checks
+the one-table-per-matrix structure for an arbitrary table (parity of the
+table's VALUES with a published nf4 table is unpinned).
+"""
+import contextlib
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    i64 = ctypes.c_int64
+    lib.oracle_bf16_rne.argtypes = [ctypes.c_float]
+    lib.oracle_bf16_rne.restype = ctypes.c_uint16
+    lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_to_f32.restype = ctypes.c_float
+    f32p = ctypes.POINTER(ctypes.c_float)
+    lib.oracle_bf16_rne_array.argtypes = [f32p, u16p, i64]
+    lib.oracle_bf16_rne_array.restype = None
+    lib.oracle_bf16_to_f32_array.argtypes = [u16p, f32p, i64]
+    lib.oracle_bf16_to_f32_array.restype = None
+    lib.oracle_pack.argtypes = [u8p, u8p, i64, i64]
+    lib.oracle_pack.restype = i64
+    lib.oracle_unpack.argtypes = [u8p, u8p, i64, i64]
+    lib.oracle_unpack.restype = None
+    lib.oracle_bits_per_weight.argtypes = [i64, i64, i64, i64]
+    lib.oracle_bits_per_weight.restype = ctypes.c_double
+    lib.oracle_dequant_one.argtypes = [ctypes.c_uint16] * 3
+    lib.oracle_dequant_one.restype = ctypes.c_uint16
+    lib.oracle_dequant.argtypes = [u8p, u16p, i64, u16p, u16p, u16p, i64, i64, i64]
+    lib.oracle_dequant.restype = None
+    lib.oracle_matmul.argtypes = [u16p, u16p, f64p, i64, i64, i64]
+    lib.oracle_matmul.restype = None
+    lib.oracle_matmul_rows.argtypes = [u16p, u8p, u16p, i64, u16p, u16p, i64p, i64,
+                                       f64p, u16p, i64, i64, i64, i64]
+    lib.oracle_matmul_rows.restype = None
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+@contextlib.contextmanager
+def swapped_library(path: str):
+    """Test hook: run the wrappers against another build of the oracle source
+    (the mutation tests plant a mistake in a copy and check that a pin fails)."""
+    global _lib
+    saved = _lib
+    _lib = _bind(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _ptr(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def set_num_threads(t: int) -> None:
+    _load().oracle_set_num_threads(int(t))
+
+
+def bf16_rne(f32: np.ndarray) -> np.ndarray:
+    """Round binary32 values to bfloat16 bit patterns (ties to even)."""
+    f = np.ascontiguousarray(f32, dtype=np.float32)
+    out = np.empty(f.shape, dtype=np.uint16)
+    _load().oracle_bf16_rne_array(_ptr(f, ctypes.c_float), _ptr(out, ctypes.c_uint16), f.size)
+    return out
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns to binary32 (exact)."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float32)
+    _load().oracle_bf16_to_f32_array(_ptr(h, ctypes.c_uint16), _ptr(out, ctypes.c_float), h.size)
+    return out
+
+
+def pack(idx: np.ndarray) -> np.ndarray:
+    """idx uint8 [N, K] (codes 0..15) -> packed uint8 [N, K/2], low nibble = even k.
+
+    Raises ValueError if any code is outside 0..15 or K is odd."""
+    idx = _c(idx, np.uint8)
+    N, K = idx.shape
+    if K % 2:
+        raise ValueError("K must be even")
+    packed = np.empty((N, K // 2), dtype=np.uint8)
+    bad = _load().oracle_pack(_ptr(idx, ctypes.c_uint8), _ptr(packed, ctypes.c_uint8), N, K)
+    if bad:
+        raise ValueError(f"{bad} codes outside 0..15")
+    return packed
+
+
+def unpack(packed: np.ndarray) -> np.ndarray:
+    packed = _c(packed, np.uint8)
+    N, Kh = packed.shape
+    idx = np.empty((N, 2 * Kh), dtype=np.uint8)
+    _load().oracle_unpack(_ptr(packed, ctypes.c_uint8), _ptr(idx, ctypes.c_uint8), N, 2 * Kh)
+    return idx
+
+
+def bits_per_weight(K: int, G: int, lut_bits: int = 16, group_param_bits: int = 16) -> float:
+    return _load().oracle_bits_per_weight(K, G, lut_bits, group_param_bits)
+
+
+def dequant_one(lut_c: int, scale: int, offset: int) -> int:
+    """bf16 bits of bf16_rne(fmaf(LUT[c], scale, offset)) for one weight."""
+    return int(_load().oracle_dequant_one(lut_c, scale, offset))
+
+
+def dequant(packed, lut, scale, offset, G: int, per_tensor_lut: bool = False) -> np.ndarray:
+    """W[n][k] = bf16(fmaf(LUT[n][code], scale[n][k/G], offset[n][k/G])) as uint16 [N, K].
+
+    lut is uint16 [N, 16] (one table per row) or, with per_tensor_lut, [16]
+    (one table for the whole matrix, the nf4/af4 mode)."""
+    packed = _c(packed, np.uint8)
+    lut = _c(lut, np.uint16)
+    scale = _c(scale, np.uint16)
+    offset = _c(offset, np.uint16)
+    N, Kh = packed.shape
+    K = 2 * Kh
+    if K % G:
+        raise ValueError("K must be a multiple of G")
+    if scale.shape != (N, K // G) or offset.shape != (N, K // G):
+        raise ValueError("scale/offset must be [N, K/G]")
+    if per_tensor_lut:
+        if lut.size != 16:
+            raise ValueError("per-tensor LUT must have 16 entries")
+        stride = 0
+    else:
+        if lut.shape != (N, 16):
+            raise ValueError("LUT must be [N, 16]")
+        stride = 16
+    W = np.empty((N, K), dtype=np.uint16)
+    _load().oracle_dequant(_ptr(packed, ctypes.c_uint8), _ptr(lut, ctypes.c_uint16), stride,
+                           _ptr(scale, ctypes.c_uint16), _ptr(offset, ctypes.c_uint16),
+                           _ptr(W, ctypes.c_uint16), N, K, G)
+    return W
+
+
+def matmul(x: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """y = x W^T in fp64 (ascending-k sums).  x uint16 [M, K], W uint16 [N, K]."""
+    x = _c(x, np.uint16)
+    W = _c(W, np.uint16)
+    M, K = x.shape
+    N, K2 = W.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    y = np.empty((M, N), dtype=np.float64)
+    _load().oracle_matmul(_ptr(x, ctypes.c_uint16), _ptr(W, ctypes.c_uint16),
+                          _ptr(y, ctypes.c_double), M, N, K)
+    return y
+
+
+def matmul_rows(x, packed, lut, scale, offset, G: int, rows, per_tensor_lut: bool = False):
+    """fp64 y[:, rows] of y = x dequant(W)^T, dequantising only the chosen rows."""
+    x = _c(x, np.uint16)
+    packed = _c(packed, np.uint8)
+    lut = _c(lut, np.uint16)
+    scale = _c(scale, np.uint16)
+    offset = _c(offset, np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K:
+        raise ValueError("K mismatch")
+    if rows.size and (rows.min() < 0 or rows.max() >= N):
+        raise ValueError("row index out of range")
+    stride = 0 if per_tensor_lut else 16
+    y = np.empty((M, rows.size), dtype=np.float64)
+    wrow = np.empty((rows.size, K), dtype=np.uint16)
+    _load().oracle_matmul_rows(_ptr(x, ctypes.c_uint16), _ptr(packed, ctypes.c_uint8),
+                               _ptr(lut, ctypes.c_uint16), stride,
+                               _ptr(scale, ctypes.c_uint16), _ptr(offset, ctypes.c_uint16),
+                               _ptr(rows, ctypes.c_int64), rows.size,
+                               _ptr(y, ctypes.c_double), _ptr(wrow, ctypes.c_uint16),
+                               M, N, K, G)
+    return y
+
+
+def any4_matmul(x, packed, lut, scale, offset, G: int, per_tensor_lut: bool = False):
+    """Dequant-then-matmul, the full definition: fp64 y [M, N]."""
+    return matmul(x, dequant(packed, lut, scale, offset, G, per_tensor_lut))
+
+
+__all__ = ["bf16_rne", "bf16_to_f32", "pack", "unpack", "bits_per_weight", "dequant_one",
+           "dequant", "matmul", "matmul_rows", "any4_matmul", "num_threads",
+           "set_num_threads"]

@@ -1,0 +1,216 @@
+/*
+ * any4 oracle: a plain, slow, obviously correct CPU statement of what the any4
+ * W4A16 path computes.  TEST INFRASTRUCTURE ONLY: nothing in the product path
+ * (the CUDA library or its Python binding) may include, link or call this file.
+ * It is used by tests/, by __graft_entry__.smoke() and by bench.py's CPU
+ * baseline leg, and by nothing else.  It shares no code with the CUDA path.
+ *
+ * Source of every definition: "any4: Learned 4-bit Numeric Representation for
+ * LLMs" (Elhoushi & Johnson, arXiv 2507.04610):
+ *   - §2.4.1: each row owns a 16-entry table (LUT) of 16-bit values; codes are
+ *     4-bit indices into it; one 16-bit scale and one 16-bit zero point per
+ *     group of g contiguous values of a row; 4.3125 bits/weight at g=128,
+ *     K=4096.  The same section allows ONE table for a whole matrix (nf4/af4).
+ *   - §2.5.1: group-wise scaling along the reduction dimension; group k holds
+ *     columns k*g <= j < (k+1)*g (the printed range has a typo; this is the
+ *     only reading that gives groups of g columns).
+ *   - §2.5.2: dequant(w_Q) = alpha * w_Q + beta.  For any4, w_Q = LUT[code].
+ *   - §4.1 Eq. 8: y_hat_i = sum_j dequant(w_Q[i,j]) * x_j.
+ *   - §4.2: y = x * w^T with x of size M x K and w of size N x K; two any4
+ *     codes share one byte.
+ *
+ * Precision readings (the pages give none for these steps):
+ *   - LUT, scale, offset, x and y are bfloat16; they cross this interface as
+ *     their raw 16-bit patterns (uint16_t).
+ *   - Nibble order: the code of even column k sits in the LOW nibble of byte
+ *     k/2, the code of odd column k in the HIGH nibble.
+ *   - Dequant: W = bf16_rne( fmaf( (float)LUT, (float)scale, (float)offset ) ),
+ *     i.e. one fp32 fused multiply-add (single rounding, C99 fmaf) followed by
+ *     round-to-nearest-even to bfloat16.  No flush-to-zero.
+ *   - Matmul: y[m][n] = sum over k ascending of (double)x[m][k] * (double)W[n][k]
+ *     with W the bf16 dequantised weight, one fp64 accumulator per output.
+ *     Products of two bf16 values are exact in fp64.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -fPIC -shared (no -ffast-math).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------- */
+/* bfloat16 <-> binary32.  bfloat16 is binary32 with the low 16 fraction bits */
+/* dropped: 1 sign bit, 8 exponent bits, 7 fraction bits.                     */
+/* ------------------------------------------------------------------------- */
+
+/* Widening is exact: the bf16 pattern becomes the high half of the binary32. */
+float oracle_bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* Round a binary32 to the nearest bfloat16, ties to the even pattern
+ * (IEEE 754 roundTiesToEven applied at the 7-bit fraction boundary).
+ * Written from the definition: compare the 16 discarded bits with the
+ * halfway point 0x8000.  Overflow past the largest finite value carries
+ * into the exponent and yields infinity, as IEEE 754 requires.  A NaN
+ * stays a NaN (sign kept, quiet bit set).  Subnormals are rounded like
+ * any other value (no flush to zero). */
+uint16_t oracle_bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u) {
+    return (uint16_t)((u >> 16) | 0x0040u); /* NaN: keep it a (quiet) NaN */
+  }
+  uint32_t kept = u >> 16;          /* sign, exponent, 7 fraction bits */
+  uint32_t dropped = u & 0xffffu;   /* the 16 bits rounded away        */
+  if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) {
+    kept += 1u;                     /* may carry into the exponent     */
+  }
+  return (uint16_t)kept;
+}
+
+void oracle_bf16_rne_array(const float* f, uint16_t* h, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) h[i] = oracle_bf16_rne(f[i]);
+}
+
+void oracle_bf16_to_f32_array(const uint16_t* h, float* f, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) f[i] = oracle_bf16_to_f32(h[i]);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Storage layout (§2.4.1, §4.2): two 4-bit codes per byte.                   */
+/* ------------------------------------------------------------------------- */
+
+/* packed[n][j] = idx[n][2j] | idx[n][2j+1] << 4, row-major, K even.
+ * Returns the number of codes outside 0..15 (those are packed masked to
+ * 4 bits; a non-zero return means the input was not a valid code array). */
+int64_t oracle_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K) {
+  int64_t bad = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < K / 2; ++j) {
+      uint8_t lo = idx[n * K + 2 * j];
+      uint8_t hi = idx[n * K + 2 * j + 1];
+      if (lo > 15) ++bad;
+      if (hi > 15) ++bad;
+      packed[n * (K / 2) + j] = (uint8_t)((lo & 15u) | ((hi & 15u) << 4));
+    }
+  }
+  return bad;
+}
+
+/* The code of column k of row n. */
+static unsigned code_at(const uint8_t* packed, int64_t K, int64_t n, int64_t k) {
+  uint8_t byte = packed[n * (K / 2) + k / 2];
+  return (k % 2 == 0) ? (byte & 15u) : (byte >> 4);
+}
+
+void oracle_unpack(const uint8_t* packed, uint8_t* idx, int64_t N, int64_t K) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      idx[n * K + k] = (uint8_t)code_at(packed, K, n, k);
+}
+
+/* Bits stored per weight: the 4-bit code, plus a 16-bit scale and a 16-bit
+ * zero point per group of G, plus a 16-entry table of lut_bits-wide values
+ * per row of K weights (§2.4.1 works this out as 4 + 0.25 + 0.0625 = 4.3125
+ * for G = 128, K = 4096 and 16-bit entries). */
+double oracle_bits_per_weight(int64_t K, int64_t G, int64_t lut_bits, int64_t group_param_bits) {
+  return 4.0 + (2.0 * (double)group_param_bits) / (double)G +
+         (16.0 * (double)lut_bits) / (double)K;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dequant (§2.5.2 with w_Q = LUT[code]).                                     */
+/* ------------------------------------------------------------------------- */
+
+/* One weight: W = bf16_rne(fmaf(LUT[c], scale, offset)). */
+uint16_t oracle_dequant_one(uint16_t lut_c, uint16_t scale, uint16_t offset) {
+  float w = fmaf(oracle_bf16_to_f32(lut_c), oracle_bf16_to_f32(scale),
+                 oracle_bf16_to_f32(offset));
+  return oracle_bf16_rne(w);
+}
+
+/* W[n][k] for the whole matrix.
+ *   lut:          row n's table starts at lut + n * lut_row_stride.
+ *                 lut_row_stride = 16 is any4 (one table per row);
+ *                 lut_row_stride = 0 is one table for the whole matrix
+ *                 (the nf4/af4 mode of §2.4.1).
+ *   scale/offset: [N][K/G], the parameters of group k/G of row n. */
+void oracle_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
+                    const uint16_t* scale, const uint16_t* offset, uint16_t* W,
+                    int64_t N, int64_t K, int64_t G) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      unsigned c = code_at(packed, K, n, k);
+      int64_t g = k / G;
+      W[n * K + k] = oracle_dequant_one(lut[n * lut_row_stride + c],
+                                        scale[n * (K / G) + g],
+                                        offset[n * (K / G) + g]);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Matmul (§4.1 Eq. 8, §4.2 orientation y = x * W^T).                         */
+/* ------------------------------------------------------------------------- */
+
+/* y[m][n] = sum_{k=0..K-1} x[m][k] * W[n][k] in fp64, k ascending.
+ * x: [M][K] bf16, W: [N][K] bf16 (already dequantised), y: [M][N] fp64. */
+void oracle_matmul(const uint16_t* x, const uint16_t* W, double* y,
+                   int64_t M, int64_t N, int64_t K) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        acc += (double)oracle_bf16_to_f32(x[m * K + k]) *
+               (double)oracle_bf16_to_f32(W[n * K + k]);
+      }
+      y[m * N + n] = acc;
+    }
+  }
+}
+
+/* The same outputs for a chosen subset of weight rows, dequantising each
+ * chosen row on the fly (so the full W is never materialised).  Used to
+ * check sampled outputs of full-size problems.
+ *   rows:  the n indices, count of them;  y: [M][count] fp64;
+ *   wrow:  caller scratch of count * K uint16 (receives the dequantised rows). */
+void oracle_matmul_rows(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                        int64_t lut_row_stride, const uint16_t* scale,
+                        const uint16_t* offset, const int64_t* rows, int64_t count,
+                        double* y, uint16_t* wrow, int64_t M, int64_t N, int64_t K,
+                        int64_t G) {
+  (void)N;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < count; ++r) {
+    int64_t n = rows[r];
+    uint16_t* w = wrow + r * K;
+    for (int64_t k = 0; k < K; ++k) {
+      unsigned c = code_at(packed, K, n, k);
+      int64_t g = k / G;
+      w[k] = oracle_dequant_one(lut[n * lut_row_stride + c], scale[n * (K / G) + g],
+                                offset[n * (K / G) + g]);
+    }
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        acc += (double)oracle_bf16_to_f32(x[m * K + k]) * (double)oracle_bf16_to_f32(w[k]);
+      }
+      y[m * count + r] = acc;
+    }
+  }
+}
+
+/* Number of OpenMP threads a parallel region here would use (1 without OpenMP). */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+void oracle_set_num_threads(int t) { omp_set_num_threads(t); }
+#else
+int oracle_num_threads(void) { return 1; }
+void oracle_set_num_threads(int t) { (void)t; }
+#endif

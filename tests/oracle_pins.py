@@ -1,0 +1,419 @@
+"""Pins for the any4 oracle: checks against facts fixed by the pages and by
+mathematics, never against the oracle itself.
+
+Every pin is a plain function that raises AssertionError on failure, so the
+same pins run against the real oracle (tests/test_oracle_pins.py) and against
+copies of the oracle source with a planted mistake (tests/test_oracle_mutants.py,
+which requires that every planted mistake fails at least one pin).
+
+Kinds of pin used (paper: "any4: Learned 4-bit Numeric Representation for
+LLMs", arXiv 2507.04610):
+  * worked examples the pages print (storage accounting, §2.4.1), as fixtures
+    under tests/golden/;
+  * values fixed by the IEEE 754 definition of round-to-nearest-even, and a
+    library routine (torch's fp32 -> bf16 conversion) on a million inputs;
+  * special cases that reduce to a textbook format: the LUT {-8..7} reproduces
+    grouped asymmetric int4 (§2.1, §2.5.1 Eq. 1-2, §2.5.2 Eq. 4 and dequant);
+    one shared table reproduces the nf4/af4 mode (§2.4.1);
+  * exact rational arithmetic (Python fractions) for the fused multiply-add;
+  * invariants (LUT permutation, constant codes, zero scale, one-hot and
+    identity activations, linearity with exactly representable inputs);
+  * brute force with an independent summation (math.fsum, exact) on tiny
+    shapes, within the fp64 error bound of an ascending-k sum.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# --------------------------------------------------------------------------
+# helpers that use only torch / numpy / fractions, never the oracle
+# --------------------------------------------------------------------------
+
+def torch_bf16_bits(f32: np.ndarray) -> np.ndarray:
+    """torch's own fp32 -> bf16 conversion (round to nearest even)."""
+    t = torch.from_numpy(np.ascontiguousarray(f32, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def torch_bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.int16))
+    return t.view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def exact_fma_then_bf16(a: float, b: float, c: float) -> int:
+    """bf16 bits of RNE_bf16(RNE_f32(a*b + c)) with a*b + c formed exactly.
+
+    The exact value is a Fraction; fp64 -> fp32 rounding is done by numpy on a
+    value that is checked to be exact in fp64 first, fp32 -> bf16 by torch."""
+    exact = Fraction(a) * Fraction(b) + Fraction(c)
+    as64 = float(exact)
+    assert Fraction(as64) == exact, "test input not exact in fp64"
+    f32 = np.array([as64], dtype=np.float64).astype(np.float32)
+    return int(torch_bf16_bits(f32)[0])
+
+
+def read_golden(name: str):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append(line)
+    return rows
+
+
+def random_bf16(rng, shape, lo_exp=-12, hi_exp=2):
+    """bf16 bit patterns of random sign, exponent in [lo_exp, hi_exp), 7-bit fraction."""
+    sign = rng.integers(0, 2, size=shape)
+    e = rng.integers(lo_exp, hi_exp, size=shape)
+    frac = rng.integers(0, 128, size=shape)
+    vals = (1 + frac / 128.0) * np.power(2.0, e) * np.where(sign, -1.0, 1.0)
+    return torch_bf16_bits(vals.astype(np.float32))
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding
+# --------------------------------------------------------------------------
+
+def pin_bf16_rne_definition_cases():
+    for row in read_golden("bf16_rne_cases.txt"):
+        src, dst = [s.strip() for s in row.split("->", 1)]
+        dst = dst.split()[0]
+        f = np.array([int(src, 16)], dtype=np.uint32).view(np.float32)
+        got = int(oracle.bf16_rne(f)[0])
+        assert got == int(dst, 16), f"bf16_rne({src}) = {got:04x}, expected {dst}"
+
+
+def pin_bf16_rne_vs_torch():
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 2**32, size=1_000_000, dtype=np.uint64).astype(np.uint32)
+    # force many exact ties and near-ties
+    bits[:200_000] = (bits[:200_000] & 0xFFFF0000) | 0x8000
+    bits[200_000:300_000] = (bits[200_000:300_000] & 0xFFFF0000) | 0x7FFF
+    f = bits.view(np.float32)
+    finite = np.isfinite(f) | np.isinf(f)
+    f = f[finite & ~np.isnan(f)]
+    ours = oracle.bf16_rne(f)
+    ref = torch_bf16_bits(f)
+    bad = np.nonzero(ours != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first f32 bits {f[bad[:3]].view(np.uint32)}"
+    nan = np.array([np.nan, -np.nan], dtype=np.float32)
+    assert np.isnan(oracle.bf16_to_f32(oracle.bf16_rne(nan))).all()
+
+
+def pin_bf16_widen_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        ours = oracle.bf16_to_f32(bits).astype(np.float64)
+    ref = torch_bf16_to_f64(bits)
+    both_nan = np.isnan(ours) & np.isnan(ref)
+    assert np.array_equal(ours[~both_nan], ref[~both_nan])
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+
+
+# --------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------
+
+def pin_pack_worked_examples():
+    for row in read_golden("pack_example.txt"):
+        codes, bytes_ = [s.strip() for s in row.split("->")]
+        idx = np.array([[int(c) for c in codes.split()]], dtype=np.uint8)
+        want = np.array([[int(b, 16) for b in bytes_.split()]], dtype=np.uint8)
+        got = oracle.pack(idx)
+        assert np.array_equal(got, want), f"pack({codes}) = {got}, expected {want}"
+
+
+def pin_pack_roundtrip_exhaustive():
+    # every byte value unpacks to two codes that pack back to the same byte
+    all_bytes = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    codes = oracle.unpack(all_bytes)
+    assert codes.max() <= 15
+    assert np.array_equal(oracle.pack(codes), all_bytes)
+    # every ordered pair of codes packs to a distinct byte and round-trips
+    a, b = np.meshgrid(np.arange(16), np.arange(16), indexing="ij")
+    pairs = np.stack([a.ravel(), b.ravel()], axis=1).astype(np.uint8).reshape(1, 512)
+    packed = oracle.pack(pairs)
+    assert len(set(packed.ravel().tolist())) == 256
+    assert np.array_equal(oracle.unpack(packed), pairs)
+
+
+def pin_pack_rejects_bad_codes():
+    try:
+        oracle.pack(np.array([[3, 16]], dtype=np.uint8))
+    except ValueError:
+        return
+    raise AssertionError("a code of 16 was accepted")
+
+
+def pin_pack_multirow_layout():
+    # row-major [N][K/2]: row n's bytes depend only on row n's codes
+    rng = np.random.default_rng(3)
+    idx = rng.integers(0, 16, size=(5, 64), dtype=np.uint8)
+    full = oracle.pack(idx)
+    for n in range(5):
+        assert np.array_equal(full[n], oracle.pack(idx[n:n + 1])[0])
+    assert full.shape == (5, 32)
+
+
+# --------------------------------------------------------------------------
+# storage accounting (worked example printed in §2.4.1)
+# --------------------------------------------------------------------------
+
+def pin_storage_bits_worked_example():
+    for row in read_golden("storage_bits.txt"):
+        K, G, lb, gb, bits = row.split()
+        got = oracle.bits_per_weight(int(K), int(G), int(lb), int(gb))
+        assert abs(got - float(bits)) < 1e-12, f"{row}: got {got}"
+
+
+def pin_storage_bits_match_array_sizes():
+    # the byte count of an actual any4 weight set matches the accounting
+    N, K, G = 8, 4096, 128
+    idx = np.zeros((N, K), dtype=np.uint8)
+    packed = oracle.pack(idx)
+    lut = np.zeros((N, 16), dtype=np.uint16)
+    scale = np.zeros((N, K // G), dtype=np.uint16)
+    offset = np.zeros((N, K // G), dtype=np.uint16)
+    total_bits = 8 * (packed.nbytes + lut.nbytes + scale.nbytes + offset.nbytes)
+    assert total_bits / (N * K) == oracle.bits_per_weight(K, G)
+
+
+# --------------------------------------------------------------------------
+# dequant
+# --------------------------------------------------------------------------
+
+def pin_dequant_one_exact_fma():
+    """The fused multiply-add rounds once: compare with exact rational arithmetic."""
+    rng = np.random.default_rng(5)
+    a = random_bf16(rng, 4000)
+    b = random_bf16(rng, 4000)
+    c = random_bf16(rng, 4000)
+    av, bv, cv = torch_bf16_to_f64(a), torch_bf16_to_f64(b), torch_bf16_to_f64(c)
+    for i in range(4000):
+        want = exact_fma_then_bf16(av[i], bv[i], cv[i])
+        got = oracle.dequant_one(int(a[i]), int(b[i]), int(c[i]))
+        assert got == want, f"case {i}: {av[i]}*{bv[i]}+{cv[i]}: {got:04x} vs {want:04x}"
+
+
+def pin_dequant_single_rounding_of_fma():
+    """A case where fmaf and a separately rounded multiply then add differ:
+    (1 + 2^-7) * (1 + 2^-7) = 1 + 2^-6 + 2^-14; adding -(1 + 2^-6) leaves
+    2^-14 exactly with one rounding.  A mul-then-add in fp32 would also keep
+    it, so use a product that does not fit fp32: choose values whose product
+    has more than 24 significant bits is impossible for bf16 inputs (8 x 8
+    bits), hence the fp32 fmaf and an exact evaluation always agree before
+    the final bf16 rounding.  Check the zero-offset and zero-scale corners."""
+    one = int(torch_bf16_bits(np.array([1.0], np.float32))[0])
+    zero = 0
+    # LUT * 1 + 0 is the LUT value itself
+    for v in random_bf16(np.random.default_rng(6), 500):
+        assert oracle.dequant_one(int(v), one, zero) == int(v)
+        # LUT * 0 + offset is the offset itself (nonzero offset)
+        assert oracle.dequant_one(one, zero, int(v)) == int(v)
+
+
+def _int4_asymmetric_groups(w, G):
+    """Eq. 2 (asymmetric) scale per group: alpha = (max - min) / (Qmax - Qmin),
+    beta = min, with Qmin = 0 and Qmax = 15 for the 16 codes; Eq. 1 then Eq. 4
+    (round to nearest) give codes 0..15."""
+    N, K = w.shape
+    wg = w.reshape(N, K // G, G)
+    beta = wg.min(axis=2)
+    alpha = (wg.max(axis=2) - beta) / 15.0
+    q = np.rint((wg - beta[..., None]) / alpha[..., None]).clip(0, 15).astype(np.uint8)
+    return q.reshape(N, K), alpha, beta
+
+
+def pin_dequant_int4_special_case():
+    """A LUT of {-8..7} with offset' = beta + 8*alpha reproduces grouped
+    asymmetric int4 dequant alpha*q + beta (§2.1 int4 range -8..7, §2.5.2),
+    bit for bit, where q = code in 0..15 and the int4 value is q - 8."""
+    rng = np.random.default_rng(7)
+    N, K, G = 16, 512, 128
+    w = rng.normal(0, 0.02, size=(N, K))
+    q, alpha, beta = _int4_asymmetric_groups(w, G)
+    a_b = torch_bf16_bits(alpha.astype(np.float32))
+    off_b = torch_bf16_bits((beta + 8 * alpha).astype(np.float32))
+    lut_int4 = torch_bf16_bits(np.arange(-8, 8, dtype=np.float32))
+    lut = np.tile(lut_int4, (N, 1))
+    W = oracle.dequant(oracle.pack(q), lut, a_b, off_b, G)
+    a_v = torch_bf16_to_f64(a_b)
+    o_v = torch_bf16_to_f64(off_b)
+    for n in range(N):
+        for k in range(0, K, 7):
+            g = k // G
+            want = exact_fma_then_bf16(float(int(q[n, k]) - 8), a_v[n, g], o_v[n, g])
+            assert W[n, k] == want, (n, k)
+    # reconstruction error of the int4 round trip is at most alpha/2 plus the
+    # bf16 roundings of alpha, offset and the result
+    Wv = torch_bf16_to_f64(W)
+    err = np.abs(Wv - w).reshape(N, K // G, G).max(axis=2)
+    bound = alpha / 2 + 16 * np.abs(alpha) * 2.0**-8 + np.abs(beta) * 2.0**-7 + 0.05 * 2.0**-7
+    assert (err <= bound).all(), float((err / bound).max())
+
+
+def pin_dequant_shared_table_mode():
+    """One 16-entry table for the whole matrix (the nf4/af4 mode, §2.4.1)
+    equals the per-row mode with that table repeated on every row, and each
+    weight equals T[code]*scale + offset rounded once to fp32 then to bf16.
+    The table here is built like nf4 (asymmetric, an exact zero, in [-1, 1]);
+    the published nf4 constants are not on the pages."""
+    rng = np.random.default_rng(8)
+    N, K, G = 12, 256, 64
+    from statistics import NormalDist
+    nd = NormalDist()
+    neg = [nd.inv_cdf(p) for p in np.linspace(0.02, 0.5, 8)[:-1]]
+    pos = [nd.inv_cdf(p) for p in np.linspace(0.5, 0.98, 9)[1:]]
+    table = np.array(neg + [0.0] + pos)
+    table = table / np.abs(table).max()
+    T = torch_bf16_bits(table.astype(np.float32))
+    assert T.size == 16 and 0 in T.tolist()
+    idx = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    packed = oracle.pack(idx)
+    scale = random_bf16(rng, (N, K // G), -8, -4)
+    offset = random_bf16(rng, (N, K // G), -10, -7)
+    W_shared = oracle.dequant(packed, T, scale, offset, G, per_tensor_lut=True)
+    W_rows = oracle.dequant(packed, np.tile(T, (N, 1)), scale, offset, G)
+    assert np.array_equal(W_shared, W_rows)
+    Tv, sv, ov = torch_bf16_to_f64(T), torch_bf16_to_f64(scale), torch_bf16_to_f64(offset)
+    for n in range(N):
+        for k in range(0, K, 5):
+            want = exact_fma_then_bf16(Tv[idx[n, k]], sv[n, k // G], ov[n, k // G])
+            assert W_shared[n, k] == want
+
+
+def pin_dequant_invariants():
+    rng = np.random.default_rng(9)
+    N, K, G = 6, 384, 128
+    idx = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    lut = random_bf16(rng, (N, 16), -3, 1)
+    scale = random_bf16(rng, (N, K // G), -8, -5)
+    offset = random_bf16(rng, (N, K // G), -10, -8)
+    W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
+    # permuting each row's table and relabelling its codes leaves W unchanged
+    for trial in range(3):
+        perm = np.stack([rng.permutation(16) for _ in range(N)])      # new slot j holds old entry perm[j]
+        inv = np.argsort(perm, axis=1)                                   # old entry c sits at slot inv[c]
+        lut_p = np.take_along_axis(lut, perm, axis=1)
+        idx_p = np.take_along_axis(inv, idx.astype(np.int64), axis=1).astype(np.uint8)
+        assert np.array_equal(oracle.dequant(oracle.pack(idx_p), lut_p, scale, offset, G), W)
+    # constant codes give LUT[c] * scale + offset for every column of a group
+    for c in (0, 5, 15):
+        Wc = oracle.dequant(oracle.pack(np.full((N, K), c, np.uint8)), lut, scale, offset, G)
+        for n in range(N):
+            for g in range(K // G):
+                blk = Wc[n, g * G:(g + 1) * G]
+                assert (blk == blk[0]).all()
+                assert blk[0] == oracle.dequant_one(int(lut[n, c]), int(scale[n, g]),
+                                                    int(offset[n, g]))
+    # zero scale gives the offset everywhere
+    Wz = oracle.dequant(oracle.pack(idx), lut, np.zeros_like(scale), offset, G)
+    assert np.array_equal(Wz, np.repeat(offset, G, axis=1))
+    # each group uses its own parameters: change one group's scale only
+    s2 = scale.copy()
+    s2[2, 1] = torch_bf16_bits(np.array([7.0], np.float32))[0]
+    W2 = oracle.dequant(oracle.pack(idx), lut, s2, offset, G)
+    diff = np.argwhere(W2 != W)
+    assert diff.size and (diff[:, 0] == 2).all()
+    assert (diff[:, 1] >= G).all() and (diff[:, 1] < 2 * G).all()
+
+
+# --------------------------------------------------------------------------
+# matmul
+# --------------------------------------------------------------------------
+
+def _small_problem(rng, M, N, K, G):
+    idx = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    lut = torch_bf16_bits(np.sort(rng.normal(0, 0.5, size=(N, 16)), axis=1).astype(np.float32))
+    scale = torch_bf16_bits((np.abs(rng.normal(0, 0.01, size=(N, K // G))) + 1e-3)
+                            .astype(np.float32))
+    offset = torch_bf16_bits(rng.normal(0, 0.002, size=(N, K // G)).astype(np.float32))
+    x = torch_bf16_bits(rng.normal(0, 1, size=(M, K)).astype(np.float32))
+    return idx, lut, scale, offset, x
+
+
+def pin_matmul_one_hot():
+    rng = np.random.default_rng(12)
+    N, K, G = 24, 256, 64
+    idx, lut, scale, offset, _ = _small_problem(rng, 1, N, K, G)
+    W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
+    Wv = torch_bf16_to_f64(W)
+    one = torch_bf16_bits(np.array([1.0], np.float32))[0]
+    for k in (0, 1, 63, 64, 200, 255):
+        x = np.zeros((1, K), dtype=np.uint16)
+        x[0, k] = one
+        y = oracle.matmul(x, W)
+        assert np.array_equal(y[0], Wv[:, k]), k
+
+
+def pin_matmul_identity():
+    rng = np.random.default_rng(13)
+    N, K, G = 40, 128, 32
+    idx, lut, scale, offset, _ = _small_problem(rng, 1, N, K, G)
+    W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
+    eye = torch_bf16_bits(np.eye(K, dtype=np.float32))
+    y = oracle.matmul(eye, W)
+    assert np.array_equal(y, torch_bf16_to_f64(W).T)
+    assert np.array_equal(oracle.any4_matmul(eye, oracle.pack(idx), lut, scale, offset, G),
+                          torch_bf16_to_f64(W).T)
+
+
+def pin_matmul_brute_force():
+    """Tiny shapes against an exact sum (math.fsum) of the exact products;
+    an ascending fp64 sum of K terms is within K * 2^-53 * sum|terms|."""
+    rng = np.random.default_rng(14)
+    for (M, N, K, G) in [(1, 8, 64, 32), (3, 16, 128, 64), (4, 64, 256, 128)]:
+        idx, lut, scale, offset, x = _small_problem(rng, M, N, K, G)
+        W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
+        y = oracle.matmul(x, W)
+        xv, Wv = torch_bf16_to_f64(x), torch_bf16_to_f64(W)
+        for m in range(M):
+            for n in range(N):
+                terms = xv[m] * Wv[n]           # exact: 8-bit x 8-bit significands
+                exact = math.fsum(terms.tolist())
+                bound = K * 2.0**-53 * float(np.abs(terms).sum()) + 1e-300
+                assert abs(y[m, n] - exact) <= bound, (M, N, K, m, n)
+        # dequant-then-matmul orientation: y = x W^T, not x W
+        assert y.shape == (M, N)
+
+
+def pin_matmul_zero_and_linearity():
+    rng = np.random.default_rng(15)
+    M, N, K, G = 3, 20, 256, 128
+    idx, lut, scale, offset, _ = _small_problem(rng, M, N, K, G)
+    W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
+    assert (oracle.matmul(np.zeros((M, K), np.uint16), W) == 0).all()
+    # small integers are exact in bf16 and the sums below are exact in fp64
+    x1 = rng.integers(-2, 3, size=(M, K)).astype(np.float32)
+    x2 = rng.integers(-2, 3, size=(M, K)).astype(np.float32)
+    y1 = oracle.matmul(torch_bf16_bits(x1), W)
+    y2 = oracle.matmul(torch_bf16_bits(x2), W)
+    y12 = oracle.matmul(torch_bf16_bits(x1 + x2), W)
+    assert np.array_equal(y12, y1 + y2)
+    y3 = oracle.matmul(torch_bf16_bits(3 * x1), W)
+    assert np.array_equal(y3, 3 * y1)
+
+
+def pin_matmul_rows_equals_full():
+    rng = np.random.default_rng(16)
+    M, N, K, G = 2, 33, 192, 64
+    idx, lut, scale, offset, x = _small_problem(rng, M, N, K, G)
+    packed = oracle.pack(idx)
+    full = oracle.any4_matmul(x, packed, lut, scale, offset, G)
+    rows = np.array([0, 5, 32, 7], dtype=np.int64)
+    part = oracle.matmul_rows(x, packed, lut, scale, offset, G, rows)
+    assert np.array_equal(part, full[:, rows])
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,72 @@
+"""Every plausible mistake planted in a copy of the oracle source must fail at
+least one pin (CPU only).  The real oracle source is never modified: each
+mutant is a text substitution compiled into a temporary library."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+from tests import oracle_pins
+
+# (name, original text, planted mistake)
+MUTANTS = [
+    ("nibble_order_unpack", "(k % 2 == 0) ? (byte & 15u) : (byte >> 4)",
+     "(k % 2 == 0) ? (byte >> 4) : (byte & 15u)"),
+    ("nibble_order_pack", "(uint8_t)((lo & 15u) | ((hi & 15u) << 4))",
+     "(uint8_t)((hi & 15u) | ((lo & 15u) << 4))"),
+    ("scale_offset_swapped", "fmaf(oracle_bf16_to_f32(lut_c), oracle_bf16_to_f32(scale),\n"
+     "                 oracle_bf16_to_f32(offset))",
+     "fmaf(oracle_bf16_to_f32(lut_c), oracle_bf16_to_f32(offset),\n"
+     "                 oracle_bf16_to_f32(scale))"),
+    ("offset_dropped", "oracle_bf16_to_f32(offset));\n  return oracle_bf16_rne(w);",
+     "0.0f); (void)offset;\n  return oracle_bf16_rne(w);"),
+    # (a plain multiply-then-add equals fmaf for bf16 operands: the 8x8-bit
+    # product is exact in fp32, so only a perturbed product is a real mistake)
+    ("perturbed_product", "float w = fmaf(oracle_bf16_to_f32(lut_c), oracle_bf16_to_f32(scale),\n"
+     "                 oracle_bf16_to_f32(offset));",
+     "float w = (float)(oracle_bf16_to_f32(lut_c) * oracle_bf16_to_f32(scale));\n"
+     "  w = (float)(w * 1.0009765625f) + oracle_bf16_to_f32(offset);"),
+    ("truncate_not_round", "if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) {",
+     "if (0) {"),
+    ("ties_away", "if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) {",
+     "if (dropped >= 0x8000u) {"),
+    ("group_off_by_one", "      int64_t g = k / G;\n      W[n * K + k]",
+     "      int64_t g = (k + 1) / G; if (g >= K / G) g = K / G - 1;\n      W[n * K + k]"),
+    ("lut_of_row_zero", "lut[n * lut_row_stride + c],\n                                        scale",
+     "lut[c],\n                                        scale"),
+    ("scale_of_row_zero", "scale[n * (K / G) + g],\n                                        offset",
+     "scale[g],\n                                        offset"),
+    ("matmul_drops_last_term", "for (int64_t k = 0; k < K; ++k) {\n        acc += (double)oracle_bf16_to_f32(x[m * K + k]) *\n",
+     "for (int64_t k = 0; k < K - 1; ++k) {\n        acc += (double)oracle_bf16_to_f32(x[m * K + k]) *\n"),
+    ("matmul_sign", "        acc += (double)oracle_bf16_to_f32(x[m * K + k]) *\n               (double)oracle_bf16_to_f32(W[n * K + k]);",
+     "        acc += (double)oracle_bf16_to_f32(x[m * K + k]) *\n               (double)oracle_bf16_to_f32(W[n * K + k]) * (k == 3 ? -1.0 : 1.0);"),
+    ("matmul_fp32_accumulate", "      double acc = 0.0;\n      for (int64_t k = 0; k < K; ++k) {\n        acc += (double)oracle_bf16_to_f32(x[m * K + k])",
+     "      float acc = 0.0f;\n      for (int64_t k = 0; k < K; ++k) {\n        acc += (float)oracle_bf16_to_f32(x[m * K + k])"),
+    ("matmul_rows_wrong_row", "    int64_t n = rows[r];", "    int64_t n = rows[r] + (r > 0);"),
+    ("widen_wrong_shift", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    ("storage_bits_one_param", "4.0 + (2.0 * (double)group_param_bits) / (double)G",
+     "4.0 + (1.0 * (double)group_param_bits) / (double)G"),
+]
+
+
+@pytest.mark.parametrize("name,orig,mutant", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(tmp_path, name, orig, mutant):
+    src = open(oracle_build.SRC).read()
+    assert src.count(orig) >= 1, f"mutation site for {name} not found in the oracle source"
+    bad = src.replace(orig, mutant, 1)
+    c_path = tmp_path / f"{name}.c"
+    so_path = tmp_path / f"lib{name}.so"
+    c_path.write_text(bad)
+    subprocess.run(["gcc", *[f for f in oracle_build.CFLAGS if not f.startswith("-W")],
+                    str(c_path), "-o", str(so_path), "-lm"], check=True)
+    failed = []
+    with oracle.swapped_library(str(so_path)):
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin()
+            except Exception as e:  # AssertionError, or a crash of the wrapper
+                failed.append((pin.__name__, type(e).__name__))
+                break
+    assert failed, f"planted mistake {name!r} passed every pin"
