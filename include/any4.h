@@ -1,0 +1,161 @@
+/*
+ * any4.h -- C ABI of libany4, the B200 (sm_100a) implementation of the any4
+ * weight-only 4-bit matmul.
+ *
+ * Method: "any4: Learned 4-bit Numeric Representation for LLMs" (Elhoushi &
+ * Johnson, arXiv 2507.04610).  Each weight row n owns a learned 16-entry
+ * lookup table LUT[n][0..15]; each weight is a 4-bit code c indexing it; each
+ * group of G consecutive columns of a row shares one scale and one offset
+ * (paper §2.4.1, §2.5.1), and a weight is dequantised as
+ *       W[n][k] = LUT[n][c] * scale[n][k/G] + offset[n][k/G]      (§2.5.2)
+ * The matmul is y = x W^T with x of size M x K and W of size N x K (§4.2,
+ * §4.1 Eq. 8).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - bf16 tensors (x, y, W, LUT, scale, offset) are passed as uint16_t
+ *    pointers to their raw bfloat16 bit patterns.
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or any
+ *    device-accessible allocation), owned by the caller, row-major and
+ *    contiguous.  The library never allocates, frees or keeps them.
+ *  - Every pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream).  The return value reports only host-side argument
+ *    validation and launch errors; nothing is launched when a call returns
+ *    an error.  Errors detected on the device (a code above 15 in any4_pack, a
+ *    pipeline wait that ran out in any4_matmul) are OR-ed into `*dev_status`
+ *    (int32 in device memory, may be NULL), which the caller zeroes before the
+ *    call and reads after synchronising the stream; a non-zero value is one
+ *    of the negative any4_status codes below (their bits OR-ed together).
+ *  - Shape rules: N >= 1, M >= 1, K >= 32, K % 32 == 0, G % 32 == 0,
+ *    K % G == 0.  So every 32-code (16-byte) chunk of a packed row lies in a
+ *    single group.
+ *  - Outputs must not overlap inputs.
+ *  - Results are deterministic: the same inputs, shape and GPU give the same
+ *    bits on every run (no atomics in any reduction).
+ */
+#ifndef ANY4_H
+#define ANY4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Every entry point is exported from the shared library (which is built with
+ * hidden default visibility). */
+#if defined(__GNUC__)
+#define ANY4_API __attribute__((visibility("default")))
+#else
+#define ANY4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum any4_status {
+  ANY4_OK = 0,
+  ANY4_ERR_NULL = -1,        /* a required pointer is NULL                        */
+  ANY4_ERR_SHAPE = -2,       /* a size breaks the shape rules above               */
+  ANY4_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned                  */
+  ANY4_ERR_RANGE = -4,       /* device: a code above 15 was given to any4_pack    */
+  ANY4_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed              */
+  ANY4_ERR_TIMEOUT = -6,     /* device: a bounded pipeline wait gave up           */
+  ANY4_ERR_UNSUPPORTED = -7, /* no kernel for this request (e.g. not an sm_100 GPU)*/
+  ANY4_ERR_WORKSPACE = -8    /* workspace missing or smaller than required        */
+} any4_status;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* any4_stream_t;
+
+/* Which kernel family any4_matmul_ex runs. */
+typedef enum any4_path {
+  ANY4_PATH_AUTO = 0,    /* choose by M (what any4_matmul does)                  */
+  ANY4_PATH_DECODE = 1,  /* CUDA-core LUT-in-registers GEMV / skinny GEMM, M<=16 */
+  ANY4_PATH_PREFILL = 2  /* tcgen05 tensor-core GEMM with dequantised tiles      */
+} any4_path;
+
+/*
+ * any4_pack -- nibble-pack 4-bit codes, two per byte (paper §4.2; §2.4.1).
+ *   idx     [N][K] uint8, each value 0..15           (input)
+ *   packed  [N][K/2] uint8: packed[n][j] = idx[n][2j] | idx[n][2j+1] << 4
+ *           (the even column in the LOW nibble)       (output)
+ * A value above 15 is packed masked to 4 bits and sets ANY4_ERR_RANGE in
+ * *dev_status.  Shape rule: K % 32 == 0 (G plays no part).
+ */
+ANY4_API any4_status any4_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                      int32_t* dev_status, any4_stream_t stream);
+
+/*
+ * any4_dequant -- materialise the bf16 weight (paper §2.5.2 dequant with the
+ * per-row table of §2.4.1):
+ *   W[n][k] = bf16_rne( fmaf( LUT[n][c], scale[n][k/G], offset[n][k/G] ) )
+ * computed in fp32 with one rounding for the fused multiply-add, then rounded
+ * to nearest-even bf16 (no flush to zero).  Bit-exact.
+ *   packed          [N][K/2] uint8 (layout of any4_pack)
+ *   lut             table of row n at lut + n * lut_row_stride, 16 bf16 each;
+ *                   lut_row_stride = 16 for any4 (a table per row) or 0 for
+ *                   one table shared by the whole matrix (the nf4/af4 mode
+ *                   the paper's §2.4.1 describes)
+ *   scale, offset   [N][K/G] bf16
+ *   W               [N][K] bf16 (output)
+ */
+ANY4_API any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
+                         const uint16_t* scale, const uint16_t* offset, uint16_t* W,
+                         int64_t N, int64_t K, int64_t G, any4_stream_t stream);
+
+/*
+ * any4_matmul -- y = x * dequant(W)^T (paper §4.1 Eq. 8, orientation §4.2),
+ * dequantisation fused (W is never written to memory on the decode path).
+ *   x               [M][K] bf16
+ *   packed, lut, lut_row_stride, scale, offset   as for any4_dequant
+ *   y               [M][N] bf16 (output): fp32 accumulation, rounded to
+ *                   nearest-even bf16
+ *   workspace       device scratch of workspace_bytes bytes, at least
+ *                   any4_matmul_workspace_size(M, N, K, G); may be NULL when
+ *                   that size is 0.  Its contents need not be initialised and
+ *                   are undefined afterwards; two calls in flight at the same
+ *                   time must not share one.
+ *   dev_status      see the conventions above (ANY4_ERR_TIMEOUT)
+ * Accuracy: |y - y_ref| <= 1e-2 * rms(y_ref) + ulp_bf16(y_ref) per element,
+ * with y_ref the exact dequant-then-matmul.
+ */
+ANY4_API any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                        int64_t lut_row_stride, const uint16_t* scale,
+                        const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                        int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, any4_stream_t stream);
+
+/* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16).
+ * Same arguments and results otherwise; used to test each path at any M. */
+ANY4_API any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                           int64_t lut_row_stride, const uint16_t* scale,
+                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, any4_path path, any4_stream_t stream);
+
+/* Bytes of workspace any4_matmul needs for this shape (0 if none).  Returns
+ * 0 as well for shapes that break the shape rules (the call then fails). */
+ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+
+/* Same for an explicit path. */
+ANY4_API size_t any4_matmul_workspace_size_ex(int64_t M, int64_t N, int64_t K, int64_t G,
+                                     any4_path path);
+
+/* The path any4_matmul would take for this M (ANY4_PATH_DECODE or _PREFILL). */
+ANY4_API any4_path any4_matmul_choose_path(int64_t M, int64_t N, int64_t K, int64_t G);
+
+/* Static description of an error code; never NULL. */
+ANY4_API const char* any4_status_string(int32_t status);
+
+/* Bits stored per weight for this format: 4 + 32/G + 256/K (16-bit LUT
+ * entries, 16-bit scale and offset), the accounting of paper §2.4.1. */
+ANY4_API double any4_bits_per_weight(int64_t K, int64_t G);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+ANY4_API int32_t any4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ANY4_H */

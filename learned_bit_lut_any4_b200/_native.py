@@ -1,0 +1,213 @@
+"""ctypes binding of libany4.so (argument marshalling only).
+
+Each wrapper checks tensor dtypes/devices/contiguity, passes raw pointers and
+sizes to the C entry point of the same name, on torch's current CUDA stream,
+and raises Any4Error on a non-zero status.  Outputs are allocated with torch
+when not supplied.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libany4.so")
+
+ANY4_OK = 0
+ANY4_ERR_NULL = -1
+ANY4_ERR_SHAPE = -2
+ANY4_ERR_ALIGN = -3
+ANY4_ERR_RANGE = -4
+ANY4_ERR_CUDA = -5
+ANY4_ERR_TIMEOUT = -6
+ANY4_ERR_UNSUPPORTED = -7
+ANY4_ERR_WORKSPACE = -8
+
+PATHS = {"auto": 0, "decode": 1, "prefill": 2}
+
+_lib = None
+
+
+class Any4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: any4 status {status} ({any4_status_string(status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """Load libany4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m learned_bit_lut_any4_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.any4_pack.argtypes = [vp, vp, i64, i64, vp, vp]
+    lib.any4_pack.restype = i32
+    lib.any4_dequant.argtypes = [vp, vp, i64, vp, vp, vp, i64, i64, i64, vp]
+    lib.any4_dequant.restype = i32
+    lib.any4_matmul.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp, vp]
+    lib.any4_matmul.restype = i32
+    lib.any4_matmul_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp,
+                                   i32, vp]
+    lib.any4_matmul_ex.restype = i32
+    lib.any4_matmul_workspace_size.argtypes = [i64, i64, i64, i64]
+    lib.any4_matmul_workspace_size.restype = sz
+    lib.any4_matmul_workspace_size_ex.argtypes = [i64, i64, i64, i64, i32]
+    lib.any4_matmul_workspace_size_ex.restype = sz
+    lib.any4_matmul_choose_path.argtypes = [i64, i64, i64, i64]
+    lib.any4_matmul_choose_path.restype = i32
+    lib.any4_status_string.argtypes = [i32]
+    lib.any4_status_string.restype = ctypes.c_char_p
+    lib.any4_bits_per_weight.argtypes = [i64, i64]
+    lib.any4_bits_per_weight.restype = ctypes.c_double
+    lib.any4_version.argtypes = []
+    lib.any4_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def any4_status_string(status: int) -> str:
+    return library().any4_status_string(int(status)).decode()
+
+
+def any4_version() -> int:
+    return int(library().any4_version())
+
+
+def any4_bits_per_weight(K: int, G: int) -> float:
+    return float(library().any4_bits_per_weight(K, G))
+
+
+def _check(status: int, where: str):
+    if status != ANY4_OK:
+        raise Any4Error(status, where)
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtypes, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must have dtype in {dtypes}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def any4_pack(idx: torch.Tensor, packed: torch.Tensor | None = None,
+              dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """uint8 codes [N, K] (values 0..15) -> uint8 packed [N, K/2] (low nibble = even k).
+
+    A code above 15 sets ANY4_ERR_RANGE in dev_status (int32 CUDA tensor of one
+    element, zeroed by the caller) once the stream has run."""
+    _need(idx, "idx", (torch.uint8,))
+    N, K = idx.shape
+    if packed is None:
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device=idx.device)
+    _need(packed, "packed", (torch.uint8,), idx.device)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", (torch.int32,), idx.device)
+    with torch.cuda.device(idx.device):
+        _check(library().any4_pack(_ptr(idx), _ptr(packed), N, K, _ptr(dev_status),
+                                   _stream(idx.device)), "any4_pack")
+    return packed
+
+
+def _lut_stride(lut: torch.Tensor, N: int) -> int:
+    if lut.dim() == 1 and lut.numel() == 16:
+        return 0
+    if lut.dim() == 2 and tuple(lut.shape) == (N, 16):
+        return 16
+    raise ValueError(f"lut must be [N, 16] or [16], got {tuple(lut.shape)}")
+
+
+def any4_dequant(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
+                 offset: torch.Tensor, G: int, W: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 W[N, K] = bf16(fmaf(LUT[n][code], scale[n][k/G], offset[n][k/G]))."""
+    _need(packed, "packed", (torch.uint8,))
+    dev = packed.device
+    N, Kh = packed.shape
+    K = 2 * Kh
+    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+        _need(t, nm, _BF16, dev)
+    stride = _lut_stride(lut, N)
+    if W is None:
+        W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    _need(W, "W", _BF16, dev)
+    if scale.numel() != N * (K // G if G else 0) or offset.numel() != scale.numel():
+        raise ValueError("scale and offset must hold N * K/G values")
+    with torch.cuda.device(dev):
+        _check(library().any4_dequant(_ptr(packed), _ptr(lut), stride, _ptr(scale),
+                                      _ptr(offset), _ptr(W), N, K, G, _stream(dev)),
+               "any4_dequant")
+    return W
+
+
+def any4_matmul_workspace_size(M: int, N: int, K: int, G: int, path: str = "auto") -> int:
+    return int(library().any4_matmul_workspace_size_ex(M, N, K, G, PATHS[path]))
+
+
+def any4_matmul_choose_path(M: int, N: int, K: int, G: int) -> str:
+    code = int(library().any4_matmul_choose_path(M, N, K, G))
+    return {v: k for k, v in PATHS.items()}[code]
+
+
+def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
+                scale: torch.Tensor, offset: torch.Tensor, G: int,
+                y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                path: str = "auto", dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 y[M, N] = x[M, K] * dequant(W)^T, fp32 accumulation.
+
+    workspace: a CUDA tensor of at least any4_matmul_workspace_size() bytes, or
+    None to have one allocated here when the path needs it."""
+    _need(x, "x", _BF16)
+    dev = x.device
+    _need(packed, "packed", (torch.uint8,), dev)
+    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+        _need(t, nm, _BF16, dev)
+    M, K = x.shape
+    N, Kh = packed.shape
+    if 2 * Kh != K:
+        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
+    stride = _lut_stride(lut, N)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "y", _BF16, dev)
+    lib = library()
+    p = PATHS[path]
+    need = int(lib.any4_matmul_workspace_size_ex(M, N, K, G, p))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), dev)
+        ws_bytes = workspace.numel()
+    if dev_status is not None:
+        _need(dev_status, "dev_status", (torch.int32,), dev)
+    with torch.cuda.device(dev):
+        _check(lib.any4_matmul_ex(_ptr(x), _ptr(packed), _ptr(lut), stride, _ptr(scale),
+                                  _ptr(offset), _ptr(y), M, N, K, G, _ptr(workspace), ws_bytes,
+                                  _ptr(dev_status), p, _stream(dev)), "any4_matmul")
+    return y

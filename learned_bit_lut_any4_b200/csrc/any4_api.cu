@@ -1,0 +1,168 @@
+// The C ABI of libany4: argument validation (before any CUDA call, so a bad
+// call launches nothing) and dispatch to the kernels.
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace any4 {
+
+namespace {
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape rules shared by dequant and matmul (see any4.h).
+bool shape_ok(int64_t N, int64_t K, int64_t G) {
+  if (N < 1 || K < 32 || G < 32) return false;
+  if (K % 32 != 0 || G % 32 != 0 || K % G != 0) return false;
+  // keep every byte offset well inside int64 (N*K*2 bytes of bf16 W)
+  if (N > (int64_t(1) << 40) / K) return false;
+  return true;
+}
+
+bool stride_ok(int64_t lut_row_stride) { return lut_row_stride == 0 || lut_row_stride == 16; }
+
+constexpr int64_t kDecodeMaxM = 16;
+}  // namespace
+
+any4_status current_device(DeviceInfo* info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ANY4_ERR_CUDA;
+  any4_status st = ANY4_OK;
+  std::call_once(g_dev_once[dev], [&] {
+    DeviceInfo d;
+    d.device = dev;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      d.device = -1;
+    }
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess)
+      d.smem_optin = (size_t)optin;
+    g_dev[dev] = d;
+  });
+  if (g_dev[dev].device < 0) return ANY4_ERR_CUDA;
+  // The kernels are built for sm_100a only.
+  if (g_dev[dev].cc_major != 10 || g_dev[dev].cc_minor != 0) st = ANY4_ERR_UNSUPPORTED;
+  *info = g_dev[dev];
+  return st;
+}
+
+}  // namespace any4
+
+using namespace any4;
+
+extern "C" {
+
+int32_t any4_version(void) { return 10000; }
+
+const char* any4_status_string(int32_t s) {
+  switch (s) {
+    case ANY4_OK: return "ok";
+    case ANY4_ERR_NULL: return "a required pointer is NULL";
+    case ANY4_ERR_SHAPE: return "a size breaks the shape rules";
+    case ANY4_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case ANY4_ERR_RANGE: return "a code above 15 was given to any4_pack";
+    case ANY4_ERR_CUDA: return "a CUDA runtime call or launch failed";
+    case ANY4_ERR_TIMEOUT: return "a bounded pipeline wait gave up on the device";
+    case ANY4_ERR_UNSUPPORTED: return "no kernel for this request on this device";
+    case ANY4_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "several device errors (bits OR-ed) or an unknown status";
+  }
+}
+
+double any4_bits_per_weight(int64_t K, int64_t G) {
+  if (K <= 0 || G <= 0) return 0.0;
+  // 4-bit code + (16-bit scale + 16-bit offset) per G + 16 x 16-bit table per K
+  return 4.0 + 32.0 / (double)G + 256.0 / (double)K;
+}
+
+any4_status any4_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                      int32_t* dev_status, any4_stream_t stream) {
+  if (!idx || !packed) return ANY4_ERR_NULL;
+  if (N < 1 || K < 32 || K % 32 != 0 || N > (int64_t(1) << 40) / K) return ANY4_ERR_SHAPE;
+  if (!aligned16(idx) || !aligned16(packed)) return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_pack(idx, packed, N, K, dev_status, (cudaStream_t)stream, dev);
+}
+
+any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
+                         const uint16_t* scale, const uint16_t* offset, uint16_t* W,
+                         int64_t N, int64_t K, int64_t G, any4_stream_t stream) {
+  if (!packed || !lut || !scale || !offset || !W) return ANY4_ERR_NULL;
+  if (!shape_ok(N, K, G) || !stride_ok(lut_row_stride)) return ANY4_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(lut) || !aligned16(scale) || !aligned16(offset) ||
+      !aligned16(W))
+    return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_dequant(packed, lut, lut_row_stride, scale, offset, W, N, K, G,
+                        (cudaStream_t)stream, dev);
+}
+
+any4_path any4_matmul_choose_path(int64_t M, int64_t N, int64_t K, int64_t G) {
+  (void)N; (void)K; (void)G;
+  return M <= kDecodeMaxM ? ANY4_PATH_DECODE : ANY4_PATH_PREFILL;
+}
+
+size_t any4_matmul_workspace_size_ex(int64_t M, int64_t N, int64_t K, int64_t G,
+                                     any4_path path) {
+  if (M < 1 || !shape_ok(N, K, G)) return 0;
+  if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
+  if (path == ANY4_PATH_PREFILL) return prefill_workspace_size(M, N, K, G);
+  return 0;
+}
+
+size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G) {
+  return any4_matmul_workspace_size_ex(M, N, K, G, ANY4_PATH_AUTO);
+}
+
+any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                           int64_t lut_row_stride, const uint16_t* scale,
+                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, any4_path path, any4_stream_t stream) {
+  if (!x || !packed || !lut || !scale || !offset || !y) return ANY4_ERR_NULL;
+  if (M < 1 || !shape_ok(N, K, G) || !stride_ok(lut_row_stride)) return ANY4_ERR_SHAPE;
+  if (M > (int64_t(1) << 40) / K || M > (int64_t(1) << 40) / N) return ANY4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(lut) || !aligned16(scale) ||
+      !aligned16(offset) || !aligned16(y))
+    return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
+  if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
+  if (path == ANY4_PATH_DECODE && M > kDecodeMaxM) return ANY4_ERR_UNSUPPORTED;
+  const size_t need = any4_matmul_workspace_size_ex(M, N, K, G, path);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return ANY4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ANY4_ERR_ALIGN;
+  }
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  if (path == ANY4_PATH_DECODE) {
+    return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
+                         (cudaStream_t)stream, dev);
+  }
+  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
+                        workspace_bytes, dev_status, (cudaStream_t)stream, dev);
+}
+
+any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                        int64_t lut_row_stride, const uint16_t* scale,
+                        const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                        int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, any4_stream_t stream) {
+  return any4_matmul_ex(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
+                        workspace_bytes, dev_status, ANY4_PATH_AUTO, stream);
+}
+
+}  // extern "C"

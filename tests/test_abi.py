@@ -1,0 +1,121 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import learned_bit_lut_any4_b200 as any4
+from learned_bit_lut_any4_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            names += re.findall(r"^ANY4_API\s+[\w\s\*]+?\b(any4_\w+)\s*\(", text, re.M)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for required in ("any4_pack", "any4_dequant", "any4_matmul"):
+        assert required in names
+    assert len(names) == len(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(any4.library_path())
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_version_and_strings():
+    assert any4.any4_version() >= 10000
+    for s in (0, -1, -2, -3, -4, -5, -6, -7, -8, -12345):
+        assert isinstance(any4.any4_status_string(s), str) and any4.any4_status_string(s)
+
+
+@pytest.mark.parametrize("K,G", [(4096, 128), (4096, 64), (1024, 128), (14336, 128),
+                                 (28672, 128), (96, 32)])
+def test_bits_per_weight_matches_oracle(K, G):
+    # the oracle's accounting is pinned to the worked example of the paper (§2.4.1)
+    assert any4.any4_bits_per_weight(K, G) == pytest.approx(oracle.bits_per_weight(K, G), abs=0)
+
+
+FAKE = 0x10000  # an aligned, never dereferenced address (validation runs first)
+
+
+def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, scale=FAKE,
+            offset=FAKE, y=FAKE, ws=None, ws_bytes=0, status=None, path=0):
+    return _native.library().any4_matmul_ex(x, packed, lut, stride, scale, offset, y, M, N, K,
+                                            G, ws, ws_bytes, status, path, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=None), any4.ANY4_ERR_NULL),
+    (dict(packed=None), any4.ANY4_ERR_NULL),
+    (dict(lut=None), any4.ANY4_ERR_NULL),
+    (dict(scale=None), any4.ANY4_ERR_NULL),
+    (dict(offset=None), any4.ANY4_ERR_NULL),
+    (dict(y=None), any4.ANY4_ERR_NULL),
+    (dict(M=0), any4.ANY4_ERR_SHAPE),
+    (dict(N=0), any4.ANY4_ERR_SHAPE),
+    (dict(K=0), any4.ANY4_ERR_SHAPE),
+    (dict(K=48, G=48), any4.ANY4_ERR_SHAPE),
+    (dict(K=128, G=48), any4.ANY4_ERR_SHAPE),
+    (dict(K=96, G=64), any4.ANY4_ERR_SHAPE),
+    (dict(K=16, G=16), any4.ANY4_ERR_SHAPE),
+    (dict(stride=8), any4.ANY4_ERR_SHAPE),
+    (dict(x=FAKE + 2), any4.ANY4_ERR_ALIGN),
+    (dict(packed=FAKE + 8), any4.ANY4_ERR_ALIGN),
+    (dict(y=FAKE + 4), any4.ANY4_ERR_ALIGN),
+    (dict(status=FAKE + 2), any4.ANY4_ERR_ALIGN),
+    (dict(M=17, path=1), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(path=7), any4.ANY4_ERR_UNSUPPORTED),
+])
+def test_matmul_rejects_bad_arguments(kw, expect):
+    assert _matmul(**kw) == expect
+
+
+def test_pack_and_dequant_reject_bad_arguments():
+    lib = _native.library()
+    assert lib.any4_pack(None, FAKE, 4, 64, None, None) == any4.ANY4_ERR_NULL
+    assert lib.any4_pack(FAKE, FAKE, 4, 48, None, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_pack(FAKE, FAKE, 0, 64, None, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_pack(FAKE + 1, FAKE, 4, 64, None, None) == any4.ANY4_ERR_ALIGN
+    assert lib.any4_dequant(FAKE, FAKE, 16, FAKE, FAKE, None, 4, 64, 32, None) == \
+        any4.ANY4_ERR_NULL
+    assert lib.any4_dequant(FAKE, FAKE, 16, FAKE, FAKE, FAKE, 4, 64, 48, None) == \
+        any4.ANY4_ERR_SHAPE
+    assert lib.any4_dequant(FAKE, FAKE, 3, FAKE, FAKE, FAKE, 4, 64, 32, None) == \
+        any4.ANY4_ERR_SHAPE
+    assert lib.any4_dequant(FAKE, FAKE + 6, 16, FAKE, FAKE, FAKE, 4, 64, 32, None) == \
+        any4.ANY4_ERR_ALIGN
+
+
+def test_workspace_size_of_bad_shapes_is_zero():
+    assert any4.any4_matmul_workspace_size(1, 64, 48, 48) == 0
+    assert any4.any4_matmul_workspace_size(0, 64, 64, 32) == 0
+
+
+def test_path_choice():
+    assert any4.any4_matmul_choose_path(1, 4096, 4096, 128) == "decode"
+    assert any4.any4_matmul_choose_path(16, 4096, 4096, 128) == "decode"
+    assert any4.any4_matmul_choose_path(2048, 4096, 4096, 128) == "prefill"
+
+
+def test_product_does_not_import_the_oracle():
+    pkg = os.path.dirname(any4.__file__)
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "any4_oracle" not in text, fn

@@ -1,0 +1,119 @@
+"""Decode-path any4_matmul (M <= 16) on the GPU against the fp64 oracle.
+
+Tolerance: |y - y_ref| <= 1e-2 * rms(y_ref[m, :]) + ulp_bf16(y_ref) per
+element (the stated 1e-2 * rms per output row, plus one bf16 ulp because even
+the correctly rounded bf16 of y_ref exceeds 1e-2 * rms on heavy-tailed rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import learned_bit_lut_any4_b200 as any4
+from tests.gpu_helpers import (DeviceProblem, assert_matmul_close, bits_to_f64, dev_bf16,
+                               dev_u8, host_bits)
+from tests.oracle_pins import torch_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+DECODE_SHAPES = (workloads.TINY + workloads.LLAMA3_8B_DECODE
+                 + [s for s in workloads.SKINNY_SWEEP if s.M <= 16]
+                 + workloads.LLAMA3_70B_DECODE)
+
+
+def _run(d, shape, path="auto"):
+    y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path=path)
+    torch.cuda.synchronize()
+    return host_bits(y)
+
+
+@pytest.mark.parametrize("shape", DECODE_SHAPES, ids=lambda s: s.name)
+def test_decode_full_shapes(shape):
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    assert any4.any4_matmul_choose_path(shape.M, shape.N, shape.K, shape.G) == "decode"
+    y = _run(d, shape)
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    st = assert_matmul_close(y, y_ref, shape.name)
+    print(shape.name, st)
+
+
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_decode_every_m_ragged(M):
+    """Every M the decode path takes, on a shape with a ragged last slice
+    (K = 1056 is not a multiple of the 1024-column slice) and ragged rows."""
+    shape = workloads.Shape(f"ragged_m{M}", M, 1056, 333, 32, 9201, 9700 + M)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    y = _run(d, shape, path="decode")
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    assert_matmul_close(y, y_ref, shape.name)
+
+
+@pytest.mark.parametrize("K,N,G", [(32, 1, 32), (64, 7, 32), (96, 1000, 32), (2048, 5, 64),
+                                   (33792, 40, 128)])
+def test_decode_edge_shapes(K, N, G):
+    shape = workloads.Shape(f"edge_{K}_{N}", 3, K, N, G, 9300 + N, 9800 + K // 32)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    y = _run(d, shape, path="decode")
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    assert_matmul_close(y, y_ref, shape.name)
+
+
+def test_decode_one_hot_is_exact():
+    """x = e_k returns column k of the dequantised weight, bit for bit: the
+    fused group-affine form reduces to fmaf(LUT, scale, offset) rounded once."""
+    shape = workloads.Shape("onehot", 1, 4096, 2000, 128, 9401, 9901)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    W_ref = oracle.dequant(d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    one = torch_bf16_bits(np.array([1.0], np.float32))[0]
+    for k in (0, 1, 31, 32, 1023, 1024, 2047, 4095):
+        x = np.zeros((1, shape.K), np.uint16)
+        x[0, k] = one
+        y = any4.any4_matmul(dev_bf16(x), d.packed, d.lut, d.scale, d.offset, shape.G)
+        torch.cuda.synchronize()
+        got = bits_to_f64(host_bits(y))[0]
+        assert np.array_equal(got, bits_to_f64(W_ref[:, k])), k
+
+
+def test_decode_zero_x_and_determinism():
+    shape = workloads.LLAMA3_8B_DECODE[4]
+    p = workloads.make(shape)
+    d = DeviceProblem(p, check_pack=False)
+    z = torch.zeros_like(d.x)
+    y0 = any4.any4_matmul(z, d.packed, d.lut, d.scale, d.offset, shape.G)
+    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G)
+    y2 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G)
+    torch.cuda.synchronize()
+    assert (bits_to_f64(host_bits(y0)) == 0).all()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_decode_shared_table():
+    shape = workloads.Shape("shared_m4", 4, 4096, 1536, 128, 9501, 9951)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    table = p.lut[3].copy()
+    y = any4.any4_matmul(d.x, d.packed, dev_bf16(table), d.scale, d.offset, shape.G)
+    torch.cuda.synchronize()
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, table, p.scale, p.offset, shape.G,
+                               per_tensor_lut=True)
+    assert_matmul_close(host_bits(y), y_ref, "shared")
+
+
+def test_decode_writes_only_its_output():
+    """Guard bands around y stay untouched."""
+    shape = workloads.Shape("guard", 5, 1024, 999, 64, 9601, 9961)
+    p = workloads.make(shape)
+    d = DeviceProblem(p, check_pack=False)
+    pad = 4096
+    buf = torch.full((pad + shape.M * shape.N + pad,), -7, dtype=torch.int16, device="cuda")
+    y = buf[pad:pad + shape.M * shape.N].view(shape.M, shape.N).view(torch.bfloat16)
+    any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, y=y)
+    torch.cuda.synchronize()
+    assert (buf[:pad] == -7).all() and (buf[pad + shape.M * shape.N:] == -7).all()
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    assert_matmul_close(host_bits(y), y_ref, "guard")
