@@ -125,13 +125,28 @@ ANY4_API any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const
                         int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
                         int32_t* dev_status, any4_stream_t stream);
 
-/* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16).
- * Same arguments and results otherwise; used to test each path at any M. */
+/* Flags of any4_matmul_ex. */
+typedef enum any4_flags {
+  ANY4_FLAG_NONE = 0,
+  /* The caller guarantees that no work still running on `stream` when the
+   * call is issued writes packed, lut, scale or offset (the usual case for
+   * inference weights).  The kernel is then launched as a programmatic
+   * dependent of that work: it may start, and begin streaming the weights,
+   * while the preceding kernel on the stream finishes; x is read and y is
+   * written only after the preceding kernel has completed.  Decode path only;
+   * ignored elsewhere. */
+  ANY4_FLAG_OVERLAP_PRIOR = 1
+} any4_flags;
+
+/* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16)
+ * and flags (a bitwise OR of any4_flags).  Same arguments and results
+ * otherwise; used to test each path at any M and to overlap launches. */
 ANY4_API any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                            int64_t lut_row_stride, const uint16_t* scale,
                            const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
                            int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
-                           int32_t* dev_status, any4_path path, any4_stream_t stream);
+                           int32_t* dev_status, any4_path path, uint32_t flags,
+                           any4_stream_t stream);
 
 /* Bytes of workspace any4_matmul needs for this shape (0 if none).  Returns
  * 0 as well for shapes that break the shape rules (the call then fails). */

@@ -26,6 +26,7 @@ ANY4_ERR_UNSUPPORTED = -7
 ANY4_ERR_WORKSPACE = -8
 
 PATHS = {"auto": 0, "decode": 1, "prefill": 2}
+ANY4_FLAG_OVERLAP_PRIOR = 1
 
 _lib = None
 
@@ -57,7 +58,7 @@ def library() -> ctypes.CDLL:
     lib.any4_matmul.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp, vp]
     lib.any4_matmul.restype = i32
     lib.any4_matmul_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp,
-                                   i32, vp]
+                                   i32, ctypes.c_uint32, vp]
     lib.any4_matmul_ex.restype = i32
     lib.any4_matmul_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.any4_matmul_workspace_size.restype = sz
@@ -177,11 +178,14 @@ def any4_matmul_choose_path(M: int, N: int, K: int, G: int) -> str:
 def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                 scale: torch.Tensor, offset: torch.Tensor, G: int,
                 y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                path: str = "auto", dev_status: torch.Tensor | None = None) -> torch.Tensor:
+                path: str = "auto", dev_status: torch.Tensor | None = None,
+                overlap_prior: bool = False) -> torch.Tensor:
     """bf16 y[M, N] = x[M, K] * dequant(W)^T, fp32 accumulation.
 
     workspace: a CUDA tensor of at least any4_matmul_workspace_size() bytes, or
-    None to have one allocated here when the path needs it."""
+    None to have one allocated here when the path needs it.
+    overlap_prior: ANY4_FLAG_OVERLAP_PRIOR (the weights are not written by
+    work still running on the stream; the decode kernel may then overlap it)."""
     _need(x, "x", _BF16)
     dev = x.device
     _need(packed, "packed", (torch.uint8,), dev)
@@ -209,5 +213,7 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
     with torch.cuda.device(dev):
         _check(lib.any4_matmul_ex(_ptr(x), _ptr(packed), _ptr(lut), stride, _ptr(scale),
                                   _ptr(offset), _ptr(y), M, N, K, G, _ptr(workspace), ws_bytes,
-                                  _ptr(dev_status), p, _stream(dev)), "any4_matmul")
+                                  _ptr(dev_status), p,
+                                  ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0,
+                                  _stream(dev)), "any4_matmul")
     return y

@@ -129,7 +129,8 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
                            int64_t lut_row_stride, const uint16_t* scale,
                            const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
                            int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
-                           int32_t* dev_status, any4_path path, any4_stream_t stream) {
+                           int32_t* dev_status, any4_path path, uint32_t flags,
+                           any4_stream_t stream) {
   if (!x || !packed || !lut || !scale || !offset || !y) return ANY4_ERR_NULL;
   if (M < 1 || !shape_ok(N, K, G) || !stride_ok(lut_row_stride)) return ANY4_ERR_SHAPE;
   if (M > (int64_t(1) << 40) / K || M > (int64_t(1) << 40) / N) return ANY4_ERR_SHAPE;
@@ -139,6 +140,7 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
   if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
   if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
+  if (flags & ~(uint32_t)ANY4_FLAG_OVERLAP_PRIOR) return ANY4_ERR_UNSUPPORTED;
   if (path == ANY4_PATH_DECODE && M > kDecodeMaxM) return ANY4_ERR_UNSUPPORTED;
   const size_t need = any4_matmul_workspace_size_ex(M, N, K, G, path);
   if (need > 0) {
@@ -150,7 +152,7 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (st != ANY4_OK) return st;
   if (path == ANY4_PATH_DECODE) {
     return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
-                         (cudaStream_t)stream, dev);
+                         (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, (cudaStream_t)stream, dev);
   }
   return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
                         workspace_bytes, dev_status, (cudaStream_t)stream, dev);
@@ -162,7 +164,7 @@ any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t
                         int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
                         int32_t* dev_status, any4_stream_t stream) {
   return any4_matmul_ex(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
-                        workspace_bytes, dev_status, ANY4_PATH_AUTO, stream);
+                        workspace_bytes, dev_status, ANY4_PATH_AUTO, ANY4_FLAG_NONE, stream);
 }
 
 }  // extern "C"

@@ -39,7 +39,7 @@ __device__ __forceinline__ float shfl_idx(float v, uint32_t src) {
 // Read-only 16-byte load through the non-coherent path.
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 r;
-  asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
@@ -47,14 +47,14 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 // Streaming 16-byte load: read once, do not keep in L1.
 __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
   uint4 r;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
 __device__ __forceinline__ uint16_t ldg_u16(const uint16_t* p) {
   uint16_t r;
-  asm("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
   return r;
 }
 
@@ -89,7 +89,7 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const DeviceInfo& dev);
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G,
+                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
                           cudaStream_t stream, const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,

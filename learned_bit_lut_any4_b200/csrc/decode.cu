@@ -35,6 +35,7 @@ namespace any4 {
 namespace {
 
 constexpr int kMaxWarps = 8;
+constexpr int kMaxRowsMT = 1024;  // rows_per_block * MT bound (shared memory partials)
 
 template <int KL> struct CodeLoad;
 template <> struct CodeLoad<32> {
@@ -47,14 +48,14 @@ template <> struct CodeLoad<32> {
 template <> struct CodeLoad<16> {
   static constexpr int kWords = 2;
   __device__ __forceinline__ static void load(const uint8_t* p, uint32_t (&w)[2]) {
-    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
                  : "=r"(w[0]), "=r"(w[1]) : "l"(p));
   }
 };
 template <> struct CodeLoad<8> {
   static constexpr int kWords = 1;
   __device__ __forceinline__ static void load(const uint8_t* p, uint32_t (&w)[1]) {
-    asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
   }
 };
 
@@ -77,176 +78,331 @@ __device__ __forceinline__ void fma_bf16x2_f32(float& acc_lo, float& acc_hi, uin
       : "+f"(acc_lo), "+f"(acc_hi) : "r"(w), "r"(xv));
 }
 
-template <int MT, int KL, int R>
+// Sum V = 2^v per-lane values over the 32 lanes, leaving value i's total in
+// the lanes whose bits 4, 3, ... (one per halving step) spell i (most
+// significant first).  V - 1 + 5 - log2(V) shuffles instead of 5 V.
+// D += A * B on the legacy warp-level tensor-core instruction (bf16 inputs,
+// fp32 accumulation): m16n8k16, A row-major 16 x 16, B column-major 16 x 8.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int V>
+__device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
+  int n = V;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & off) != 0;
+      const int half = n / 2;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < half) {
+          const float give = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(kFullMask, give, off);
+        }
+      }
+      n = half;
+    } else {
+      v[0] += __shfl_xor_sync(kFullMask, v[0], off);
+    }
+  }
+  return v[0];
+}
+
+// Which of the V values lane `lane` holds after transpose_reduce<V>.
+template <int V>
+__device__ __forceinline__ int transpose_reduce_index(int lane) {
+  int idx = 0;
+  int n = V;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      idx = 2 * idx + ((lane & off) ? 1 : 0);
+      n /= 2;
+    }
+  }
+  return idx;
+}
+
+// The per-row loads of one lane: its KL codes, the row's table entry for
+// this lane, and the group scale/offset of its chunk.
+template <int KW>
+struct RowRegs {
+  uint32_t code[KW];
+  float lv, sv, ov;
+};
+
+// Where one lane's data of the current row lives; advanced row by row.
+struct RowPtrs {
+  const uint8_t* pk;   // the lane's KL codes
+  const uint16_t* lt;  // table entry lane & 15
+  const uint16_t* sc;  // scale of the chunk's group
+  const uint16_t* of;  // offset of the chunk's group
+};
+
+template <int KL>
+__device__ __forceinline__ void load_row(RowRegs<CodeLoad<KL>::kWords>& rr, const RowPtrs& p,
+                                         bool valid, bool kin) {
+  constexpr int KW = CodeLoad<KL>::kWords;
+  if (valid && kin) {
+    CodeLoad<KL>::load(p.pk, rr.code);
+    rr.sv = bf16_lo_to_f32(ldg_u16(p.sc));
+    rr.ov = bf16_lo_to_f32(ldg_u16(p.of));
+  } else {
+#pragma unroll
+    for (int w = 0; w < KW; ++w) rr.code[w] = 0u;
+    rr.sv = 0.f;
+    rr.ov = 0.f;
+  }
+  rr.lv = valid ? bf16_lo_to_f32(ldg_u16(p.lt)) : 0.f;
+}
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// A block owns a contiguous range of weight rows (sized so that the grid is
+// one wave).  Warp w handles the K-slices w, w + nwarps, ... of every row in
+// the range: it keeps the loads of the next P rows in flight (a row's
+// registers are refilled with the row P further on as soon as it has been
+// consumed) across the whole range, and reduces the lane partials of every P
+// rows with one transposed shuffle reduction.  Slice partials meet in shared
+// memory and are summed in a fixed order.
+//
+// Programmatic dependent launch: the weight-side loads of the first P rows
+// are issued before griddepcontrol.wait, x is read only after it, and y is
+// written only after it.  (When the kernel is launched without the
+// programmatic attribute the wait returns at once.)
+template <int MT, int KL, int P>
 __global__ void __launch_bounds__(kMaxWarps * 32) decode_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-    uint16_t* __restrict__ y, int M, int64_t N, int64_t K, int64_t G, int nslices) {
+    uint16_t* __restrict__ y, int M, int64_t N, int64_t K, int64_t G, int nslices,
+    int rows_per_block) {
   constexpr int KW = CodeLoad<KL>::kWords;
-  __shared__ float s_part[kMaxWarps][R][MT];
+  constexpr int V = P * MT;
+  static_assert(V <= 32 && (V & (V - 1)) == 0, "P * MT must be a power of two <= 32");
+  static_assert(P % 2 == 0 && KL % 8 == 0, "rows go to the tensor core in pairs");
+  extern __shared__ float s_part[];  // [nwarps][RTP][MT]
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   const int64_t groups = K / G;
   const int64_t row_bytes = K / 2;
-  const int64_t nblocks = (N + R - 1) / R;
+  const int RT = rows_per_block;
+  const int RTP = ((RT + P - 1) / P) * P;
+  const int64_t nblocks = (N + RT - 1) / RT;
+  const int my_idx = transpose_reduce_index<V>(lane);
+  const bool writer = (lane & ((32 / V) - 1)) == 0;  // one lane per reduced value
+  bool waited = false;
 
-  uint32_t xw[MT][KL / 2];  // x of the lane's chunk as bf16 pairs (even k low)
-  int cur_slice = -1;
-
-  for (int64_t rb = blockIdx.x; rb < nblocks; rb += gridDim.x) {
-    const int64_t n0 = rb * R;
-    float acc[R][MT][2];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[r][m][0] = acc[r][m][1] = 0.f;
-
+  for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+    const int64_t row0 = blk * RT;
+    const int nrows = (int)((N - row0) < (int64_t)RT ? (N - row0) : (int64_t)RT);
+    bool first_slice = true;
     for (int s = warp; s < nslices; s += nwarps) {
       const int64_t k0 = (int64_t)s * 32 * KL + (int64_t)lane * KL;
       const bool kin = k0 < K;
-
-      // codes, tables and group parameters of the R rows (issued together)
-      uint32_t code[R][KW];
-      float lv[R], sv[R], ov[R];
       const int64_t g = kin ? k0 / G : 0;
+      RowPtrs nxt;  // the row after the ones in flight
+      nxt.pk = packed + row0 * row_bytes + (kin ? k0 / 2 : 0);
+      nxt.lt = lut + row0 * lut_row_stride + (lane & 15);
+      nxt.sc = scale + row0 * groups + g;
+      nxt.of = offset + row0 * groups + g;
+
+      RowRegs<KW> buf[P];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t n = n0 + r;
-        const bool rin = n < N;
-        if (rin && kin) {
-          CodeLoad<KL>::load(packed + n * row_bytes + k0 / 2, code[r]);
-          sv[r] = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
-          ov[r] = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
-        } else {
-#pragma unroll
-          for (int w = 0; w < KW; ++w) code[r][w] = 0u;
-          sv[r] = 0.f;
-          ov[r] = 0.f;
-        }
-        lv[r] = rin ? bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + (lane & 15))) : 0.f;
+      for (int j = 0; j < P; ++j) {
+        load_row<KL>(buf[j], nxt, j < nrows, kin);
+        nxt.pk += row_bytes;
+        nxt.lt += lut_row_stride;
+        nxt.sc += groups;
+        nxt.of += groups;
+      }
+      if (!waited) {  // x (and y) may belong to the preceding kernel
+        grid_dependency_wait();
+        grid_dependents_launch();
+        waited = true;
       }
 
-      if (s != cur_slice) {  // activations of this chunk, reused across rows
-        cur_slice = s;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          if (m < M && kin) {
-            const uint16_t* xp = x + (int64_t)m * K + k0;
-#pragma unroll
-            for (int v = 0; v < KL / 8; ++v) {
-              const uint4 q = ldg_nc_v4(xp + 8 * v);
-              xw[m][4 * v] = q.x;
-              xw[m][4 * v + 1] = q.y;
-              xw[m][4 * v + 2] = q.z;
-              xw[m][4 * v + 3] = q.w;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < KL / 2; ++i) xw[m][i] = 0u;
-          }
-        }
-      }
-
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-#pragma unroll
-        for (int w = 0; w < KW; ++w) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            // byte j of the word: codes of columns k0 + 8w + 2j (low nibble)
-            // and k0 + 8w + 2j + 1 (high nibble)
-            const uint32_t wp = dequant_pair(lv[r], code[r][w] >> (8 * j),
-                                             code[r][w] >> (8 * j + 4), sv[r], ov[r]);
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-              fma_bf16x2_f32(acc[r][m][0], acc[r][m][1], wp, xw[m][4 * w + j]);
-          }
-        }
-      }
-    }
-
-    // reduce over the 32 lanes, then over warps in a fixed order
-#pragma unroll
-    for (int r = 0; r < R; ++r)
+      uint32_t xw[MT][KL / 2];  // activations of this chunk, bf16 pairs (even k low)
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        float v = acc[r][m][0] + acc[r][m][1];
+        if (m < M && kin) {
+          const uint16_t* xp = x + (int64_t)m * K + k0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
-        if (lane == 0) s_part[warp][r][m] = v;
+          for (int v = 0; v < KL / 8; ++v) {
+            const uint4 q = ldg_nc_v4(xp + 8 * v);
+            xw[m][4 * v] = q.x;
+            xw[m][4 * v + 1] = q.y;
+            xw[m][4 * v + 2] = q.z;
+            xw[m][4 * v + 3] = q.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < KL / 2; ++i) xw[m][i] = 0u;
+        }
       }
+
+      for (int i = 0; i < RTP; i += P) {
+        float part[V];
+#pragma unroll
+        for (int j = 0; j < P; j += 2) {
+          // Rows j (A rows 0..7) and j + 1 (A rows 8..15) of this group on the
+          // tensor core.  mma step st covers codes 4st .. 4st+3 of every lane's
+          // chunk: lane (q = lane/4, t = lane%4) supplies A[q][2t, 2t+1, 2t+8,
+          // 2t+9] = W'(its codes 4st..4st+3) of row j, A[q+8][same] = those of
+          // row j+1, and B[2t, 2t+1, 2t+8, 2t+9][q] = x at the same four
+          // columns.  Every product therefore pairs a weight with its own x,
+          // and the diagonals C[q][q], C[q+8][q] (summed over q) are the two
+          // rows' partial dot products; the other entries are not used.
+          float c[MT][4];
+#pragma unroll
+          for (int m = 0; m < MT; ++m) c[m][0] = c[m][1] = c[m][2] = c[m][3] = 0.f;
+          const bool va = i + j < nrows, vb = i + j + 1 < nrows;  // warp-uniform
+          if (va || vb) {
+#pragma unroll
+            for (int st = 0; st < KL / 4; ++st) {
+              const uint32_t ca = buf[j].code[st / 2] >> (16 * (st & 1));
+              const uint32_t cb = buf[j + 1].code[st / 2] >> (16 * (st & 1));
+              const uint32_t a01 = dequant_pair(buf[j].lv, ca, ca >> 4, buf[j].sv, buf[j].ov);
+              const uint32_t a45 = dequant_pair(buf[j].lv, ca >> 8, ca >> 12, buf[j].sv, buf[j].ov);
+              const uint32_t a23 =
+                  dequant_pair(buf[j + 1].lv, cb, cb >> 4, buf[j + 1].sv, buf[j + 1].ov);
+              const uint32_t a67 =
+                  dequant_pair(buf[j + 1].lv, cb >> 8, cb >> 12, buf[j + 1].sv, buf[j + 1].ov);
+#pragma unroll
+              for (int m = 0; m < MT; ++m)
+                mma_16816(c[m], a01, a23, a45, a67, xw[m][2 * st], xw[m][2 * st + 1]);
+            }
+          }
+          const int q = lane >> 2;
+          const bool diag = (lane & 3) == (q >> 1);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float da = (q & 1) ? c[m][1] : c[m][0];
+            const float db = (q & 1) ? c[m][3] : c[m][2];
+            part[j * MT + m] = diag ? da : 0.f;
+            part[(j + 1) * MT + m] = diag ? db : 0.f;
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (i + j + h + P < nrows) {  // refill with the row P further on
+              load_row<KL>(buf[j + h], nxt, true, kin);
+              nxt.pk += row_bytes;
+              nxt.lt += lut_row_stride;
+              nxt.sc += groups;
+              nxt.of += groups;
+            }
+          }
+        }
+        const float tot = transpose_reduce<V>(part, lane);
+        if (writer) {
+          const int r = i + my_idx / MT;
+          const int m = my_idx % MT;
+          float* dst = s_part + ((size_t)warp * RTP + r) * MT + m;
+          *dst = first_slice ? tot : *dst + tot;
+        }
+      }
+      first_slice = false;
+    }
     __syncthreads();
-    if (threadIdx.x < R * MT) {
-      const int r = threadIdx.x / MT;
-      const int m = threadIdx.x % MT;
-      const int64_t n = n0 + r;
-      if (n < N && m < M) {
-        float t = 0.f;
-        for (int w = 0; w < nwarps; ++w) t += s_part[w][r][m];
-        y[(int64_t)m * N + n] = f32_to_bf16_rn(t);
+    const int nw_used = min(nwarps, nslices);
+    for (int t = threadIdx.x; t < nrows * MT; t += blockDim.x) {
+      const int r = t / MT;
+      const int m = t % MT;
+      if (m < M) {
+        float tot = 0.f;
+        for (int w = 0; w < nw_used; ++w) tot += s_part[((size_t)w * RTP + r) * MT + m];
+        y[(int64_t)m * N + row0 + r] = f32_to_bf16_rn(tot);
       }
     }
     __syncthreads();
+  }
+  if (!waited) {
+    grid_dependency_wait();
+    grid_dependents_launch();
   }
 }
 
-struct LaunchCfg {
-  int threads;
-  int grid;
-};
-
-template <int MT, int KL, int R>
+template <int MT, int KL, int P>
 any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                 int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                uint16_t* y, int M, int64_t N, int64_t K, int64_t G, cudaStream_t stream,
-                const DeviceInfo& dev) {
+                uint16_t* y, int M, int64_t N, int64_t K, int64_t G, bool overlap,
+                cudaStream_t stream, const DeviceInfo& dev) {
   const int64_t slice = 32LL * KL;
   const int nslices = (int)((K + slice - 1) / slice);
-  const int nwarps = std::min(nslices, kMaxWarps);
+  // the fewest warps that keep every warp's share of slices equal (<= 8)
+  const int per_warp = (nslices + kMaxWarps - 1) / kMaxWarps;
+  const int nwarps = (nslices + per_warp - 1) / per_warp;
   const int threads = nwarps * 32;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MT, KL, R>, threads,
-                                                    0) != cudaSuccess ||
-      per_sm < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MT, KL, P>, threads,
+                                                    (size_t)kMaxRowsMT * sizeof(float) * nwarps) !=
+          cudaSuccess ||
+      per_sm < 1)
     per_sm = 1;
-  }
-  const int64_t nblocks = (N + R - 1) / R;
-  const int64_t cap = (int64_t)dev.sm_count * per_sm;
-  const int grid = (int)std::min<int64_t>(nblocks, cap);
-  decode_kernel<MT, KL, R><<<grid, threads, 0, stream>>>(x, packed, lut, lut_row_stride, scale,
-                                                         offset, y, M, N, K, G, nslices);
-  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+  // one wave: every resident block owns an equal contiguous range of rows
+  const int64_t wave = (int64_t)dev.sm_count * per_sm;
+  int64_t rt = (N + wave - 1) / wave;
+  rt = std::min<int64_t>(rt, kMaxRowsMT / MT);
+  const int64_t rtp = ((rt + P - 1) / P) * P;
+  const int64_t nblocks = (N + rt - 1) / rt;
+  const int grid = (int)std::min<int64_t>(nblocks, wave);
+  const size_t smem = (size_t)nwarps * rtp * MT * sizeof(float);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, decode_kernel<MT, KL, P>, x, packed, lut,
+                                             lut_row_stride, scale, offset, y, M, N, K, G,
+                                             nslices, (int)rt);
+  return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
 }  // namespace
 
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G,
+                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
                           cudaStream_t stream, const DeviceInfo& dev) {
   // rows of x beyond 8 are handled by further launches over the same weights
   for (int64_t m0 = 0; m0 < M; m0 += 8) {
     const int mb = (int)std::min<int64_t>(M - m0, 8);
     const uint16_t* xb = x + m0 * K;
     uint16_t* yb = y + m0 * N;
+    // only the first launch may overlap the work before it on the stream
+    const bool ov = overlap && m0 == 0;
     any4_status st;
-    const bool few_rows = (N + 7) / 8 < 2LL * dev.sm_count;
     if (mb == 1) {
-      st = few_rows ? run<1, 32, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N,
-                                    K, G, stream, dev)
-                    : run<1, 32, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N,
-                                    K, G, stream, dev);
+      st = run<1, 32, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
+                         stream, dev);
     } else if (mb == 2) {
-      st = run<2, 32, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G,
+      st = run<2, 32, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
                          stream, dev);
     } else if (mb <= 4) {
-      st = run<4, 16, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G,
+      st = run<4, 16, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
                          stream, dev);
     } else {
-      st = run<8, 8, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G,
+      st = run<8, 8, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
                         stream, dev);
     }
     if (st != ANY4_OK) return st;

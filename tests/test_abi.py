@@ -53,9 +53,9 @@ FAKE = 0x10000  # an aligned, never dereferenced address (validation runs first)
 
 
 def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, scale=FAKE,
-            offset=FAKE, y=FAKE, ws=None, ws_bytes=0, status=None, path=0):
+            offset=FAKE, y=FAKE, ws=None, ws_bytes=0, status=None, path=0, flags=0):
     return _native.library().any4_matmul_ex(x, packed, lut, stride, scale, offset, y, M, N, K,
-                                            G, ws, ws_bytes, status, path, None)
+                                            G, ws, ws_bytes, status, path, flags, None)
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -79,6 +79,7 @@ def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, sc
     (dict(status=FAKE + 2), any4.ANY4_ERR_ALIGN),
     (dict(M=17, path=1), any4.ANY4_ERR_UNSUPPORTED),
     (dict(path=7), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(flags=2), any4.ANY4_ERR_UNSUPPORTED),
 ])
 def test_matmul_rejects_bad_arguments(kw, expect):
     assert _matmul(**kw) == expect

@@ -117,3 +117,33 @@ def test_decode_writes_only_its_output():
     assert (buf[:pad] == -7).all() and (buf[pad + shape.M * shape.N:] == -7).all()
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     assert_matmul_close(host_bits(y), y_ref, "guard")
+
+
+def test_decode_overlap_prior_chain():
+    """ANY4_FLAG_OVERLAP_PRIOR: x is produced by the kernel just before each
+    call and y is consumed by the kernel just after; a chain of overlapped
+    calls must match the same chain run without overlap, bit for bit, and the
+    oracle within tolerance."""
+    shape = workloads.Shape("overlap", 1, 4096, 4096, 128, 9701, 9702)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    def chain(overlap):
+        x = d.x.clone()
+        outs = []
+        for i in range(6):
+            x = (x.float() * 0.5 + 0.25).to(torch.bfloat16)      # written by the preceding kernel
+            y = any4.any4_matmul(x, d.packed, d.lut, d.scale, d.offset, shape.G,
+                                 overlap_prior=overlap)
+            outs.append(y.clone())                              # read by the following kernel
+            x = torch.cat([y[:, :shape.K]], dim=1) if shape.N >= shape.K else x
+            x = (x.float() / (x.float().abs().max() + 1)).to(torch.bfloat16)
+        torch.cuda.synchronize()
+        return outs
+    a = chain(False)
+    b = chain(True)
+    for ya, yb in zip(a, b):
+        assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, overlap_prior=True)
+    torch.cuda.synchronize()
+    assert_matmul_close(host_bits(y1), y_ref, "overlap")
