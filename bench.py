@@ -1,0 +1,508 @@
+#!/usr/bin/env python3
+"""Benchmark of the any4 W4A16 matmul on B200: one JSON line.
+
+Metric: any4 matmul HBM GB/s and us at M = 1, TFLOPS at M = 2048, % of roofline.
+
+A step is one pass of the Llama3-8B-shaped decode layer at M = 1: the seven
+any4_matmul calls of one transformer layer (q, k, v, o projections K = 4096;
+gate and up K = 4096, N = 14336; down K = 14336, N = 4096), group size
+G = 128, on seeded synthetic weights (no model weights exist here).  `value`
+is the whole-job algorithmic HBM throughput (packed codes + scales/offsets +
+tables + x + y per call, summed over the seven calls and over all ranks,
+divided by the max-over-ranks device time).  Weights are rotated over enough
+copies that the working set exceeds L2 (every step reads cold weights).
+
+Also reported (same run, not part of the step): the prefill matmuls at
+M = 2048 (TFLOPS), the roofline object of the decode kernel, the CPU oracle
+as a baseline, the end-to-end number through the public API with host
+buffers, and the clocks seen during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 launch under torch.distributed.run; each rank runs an independent
+replica on its own GPU (the path has no exchange step), `scaling` = "weak".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "any4 matmul HBM GB/s & µs (M=1), TFLOPS (M=2048), % of roofline"
+L2_BYTES = 132644864
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash() -> str:
+    """Hash of the decode kernel source: a stored ncu traffic figure is only
+    used while it was taken on this exact source."""
+    h = hashlib.sha256()
+    for fn in ("decode.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "learned_bit_lut_any4_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic():
+    """Per-launch DRAM bytes (read + write) of the decode kernel on this step,
+    from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_llama3_8b_layer_m1.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.]+)", text)
+    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_sum(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                                 else ".", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sms:
+            return None
+        return {"sm_mhz": float(np.median(sms)), "sm_max_mhz": float(max(maxs)),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def _dev_bf16(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def prepare_layer(shapes, copies):
+    """Device copies of each shape's weights (packed on the device by
+    any4_pack), plus x and y buffers."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    sets = []
+    for s in shapes:
+        p = workloads.make(s)
+        packed = any4.any4_pack(torch.from_numpy(p.idx).cuda())
+        lut, sc, of = _dev_bf16(p.lut), _dev_bf16(p.scale), _dev_bf16(p.offset)
+        reps = [(packed, lut, sc, of)] + [(packed.clone(), lut.clone(), sc.clone(), of.clone())
+                                          for _ in range(copies - 1)]
+        x = _dev_bf16(p.x)
+        y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
+        sets.append((s, reps, x, y, p.x))
+    torch.cuda.synchronize()
+    return sets
+
+
+def gpu_arm(args, rank, world):
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+
+    peaks = load_peaks()
+    shapes = workloads.LLAMA3_8B_DECODE
+    layer_weight_bytes = sum(s.N * s.K // 2 + 4 * s.N * (s.K // s.G) + 32 * s.N for s in shapes)
+    copies = max(2, int(np.ceil(3 * L2_BYTES / layer_weight_bytes)))
+    sets = prepare_layer(shapes, copies)
+    step_bytes = sum(s.alg_bytes() for s in shapes)
+    overlap = not args.no_overlap
+    stream = torch.cuda.Stream()
+
+    def step(c):
+        for (s, reps, x, y, _) in sets:
+            w = reps[c % copies]
+            any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+
+    # one graph = `copies` steps (each step on the next weight copy)
+    with torch.cuda.stream(stream):
+        for c in range(copies):
+            step(c)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c in range(copies):
+            step(c)
+    reps_needed = max(1, args.steps // copies)
+    steps_timed = reps_needed * copies
+    warm = max(1, int(np.ceil(args.warmup / copies)))
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            graph.replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first reading before the timed region
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps_needed):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms_local = e0.elapsed_time(e1)
+    ms = allreduce_max(ms_local, world)
+    ms_per_step = ms / steps_timed
+    total_bytes = allreduce_sum(step_bytes * steps_timed, world)
+    value_gbs = total_bytes / (ms * 1e-3) / 1e9
+
+    # per-shape detail (each shape alone, same rotation, events on its stream)
+    detail = {}
+    for (s, reps, x, y, _) in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in range(copies):
+                w = reps[c]
+                any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+        n_rep = max(1, 400 // copies)
+        with torch.cuda.stream(stream):
+            g.replay()
+            stream.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n_rep):
+                g.replay()
+            b.record(stream)
+        b.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (n_rep * copies)
+        gbs = s.alg_bytes() / (us * 1e-6) / 1e9
+        detail[s.name] = {"us": round(us, 3), "GB/s": round(gbs, 1),
+                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del g
+
+    # prefill (M = 2048), TFLOPS against the bf16 peak
+    prefill = {}
+    if not args.skip_prefill:
+        for s in workloads.PREFILL:
+            p = workloads.make(s)
+            packed = any4.any4_pack(torch.from_numpy(p.idx).cuda())
+            lut, sc, of, x = (_dev_bf16(a) for a in (p.lut, p.scale, p.offset, p.x))
+            y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
+            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
+                times = []
+                for _ in range(5):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
+                    b.record(stream)
+                    b.synchronize()
+                    times.append(a.elapsed_time(b) * 1e3)
+            us = float(np.median(times))
+            tf = s.flops() / (us * 1e-6) / 1e12
+            prefill[s.name] = {"us": round(us, 1), "TFLOPS": round(tf, 1),
+                               "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                               "frac_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4)}
+            del packed, lut, sc, of, x, y, flush
+        torch.cuda.synchronize()
+
+    # end to end through the public API with host buffers: every step copies
+    # each call's x from pinned host memory and reads each y back
+    host_x = [torch.from_numpy(np.ascontiguousarray(hx).view(np.int16)).pin_memory()
+              for (_, _, _, _, hx) in sets]
+    host_y = [torch.empty((s.M, s.N), dtype=torch.int16).pin_memory() for (s, *_r) in sets]
+    dev_x = [torch.empty((s.M, s.K), dtype=torch.int16, device="cuda") for (s, *_r) in sets]
+    h2d = sum(t.numel() * 2 for t in host_x)
+    d2h = sum(t.numel() * 2 for t in host_y)
+    e2e_steps = max(copies, min(steps_timed, 400))
+
+    def e2e_step(c):
+        for i, (s, reps, _x, y, _) in enumerate(sets):
+            dev_x[i].copy_(host_x[i], non_blocking=True)
+            w = reps[c % copies]
+            any4.any4_matmul(dev_x[i].view(torch.bfloat16), w[0], w[1], w[2], w[3], s.G, y=y)
+            host_y[i].copy_(y.view(torch.int16), non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for c in range(copies):
+            e2e_step(c)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for c in range(e2e_steps):
+            e2e_step(c)
+        b.record(stream)
+    b.synchronize()
+    barrier(world)
+    e2e_ms = allreduce_max(a.elapsed_time(b), world)
+    e2e_gbs = allreduce_sum(step_bytes * e2e_steps, world) / (e2e_ms * 1e-3) / 1e9
+
+    return {
+        "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
+        "clocks": clocks, "detail": detail, "prefill": prefill, "peaks": peaks,
+        "copies": copies, "step_bytes": step_bytes,
+        "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "launches": len(sets) * steps_timed,
+    }
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_layer_rate(max_seconds: float):
+    """Time the oracle (dequant then fp64 matmul) over whole passes of the
+    decode layer until about max_seconds of CPU work; GB/s on the same
+    algorithmic bytes as the GPU arm."""
+    import oracle
+    shapes = workloads.LLAMA3_8B_DECODE
+    probs = []
+    for s in shapes:
+        p = workloads.make(s)
+        probs.append((s, oracle.pack(p.idx), p))
+    step_bytes = sum(s.alg_bytes() for s in shapes)
+    t0 = time.perf_counter()
+    done_bytes = 0
+    passes = 0
+    while True:
+        for (s, packed, p) in probs:
+            oracle.any4_matmul(p.x, packed, p.lut, p.scale, p.offset, s.G)
+        passes += 1
+        done_bytes += step_bytes
+        if time.perf_counter() - t0 >= max_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{passes} full pass(es) of the 7-matmul Llama3-8B layer at M=1 "
+                      f"(dequant + fp64 matmul), {dt:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    res = oracle_layer_rate(max_seconds=args.reference_seconds)
+    line = {"metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generators, Llama3-8B shapes)",
+            "config": {"workload": "llama3_8b_decode_layer_m1", "M": 1, "G": 128,
+                       "shapes": [[s.name, s.K, s.N] for s in workloads.LLAMA3_8B_DECODE]},
+            "impl": "reference", "cpu_baseline": res,
+            "e2e": {"value": res["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def profile_shape(name: str, calls: int):
+    """Run a few any4_matmul calls (auto path) on one workload shape."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    shape = [s for s in workloads.all_shapes() if s.name == name]
+    if not shape:
+        raise SystemExit(f"unknown shape {name}; known: {[s.name for s in workloads.all_shapes()]}")
+    s = shape[0]
+    p = workloads.make(s)
+    packed = any4.any4_pack(torch.from_numpy(p.idx).cuda())
+    lut, sc, of, x = (_dev_bf16(a) for a in (p.lut, p.scale, p.offset, p.x))
+    y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(calls):
+        any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
+    torch.cuda.synchronize()
+    print(f"profiled {name}: M={s.M} K={s.K} N={s.N} G={s.G}, {calls} calls", flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=40)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the decode kernels without programmatic dependent launch")
+    ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=20.0)
+    ap.add_argument("--profile-shape", default=None,
+                    help="no timing: run --profile-calls any4_matmul calls on one named "
+                         "workload shape (a small, fixed case for ncu captures)")
+    ap.add_argument("--profile-calls", type=int, default=3)
+    args = ap.parse_args()
+    if args.profile_shape:
+        profile_shape(args.profile_shape, args.profile_calls)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank, world, _ = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            reference_arm(args, rank, world)
+            return
+        import torch
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        r = gpu_arm(args, rank, world)
+        if rank != 0:
+            return
+        peaks = r["peaks"]
+        cpu = oracle_layer_rate(max_seconds=args.cpu_seconds) if world == 1 else None
+        achieved = r["value"] / world  # per-GPU decode throughput over the whole step
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": stored_traffic(),
+                    "kernel": "decode_kernel<1,32,8> (the only kernel of the step)",
+                    "peak_source": peaks.get("source", "measured")}
+        line = {
+            "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
+            "steps": r["steps_timed"], "warmup": args.warmup,
+            "ms_per_step": round(r["ms_per_step"], 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generators, Llama3-8B shapes, random any4 weights)",
+            "config": {"workload": "llama3_8b_decode_layer_m1", "M": 1, "G": 128,
+                       "shapes": [[s.name, s.K, s.N] for s in workloads.LLAMA3_8B_DECODE],
+                       "parallelism": f"replicas{world}",
+                       "l2": f"inputs larger than L2: {r['copies']} rotating weight copies",
+                       "overlap_prior": not args.no_overlap},
+            "us_per_layer": round(r["ms_per_step"] * 1e3, 2),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": r["e2e"],
+            "gpu_launches": r["launches"],
+            "clocks": r["clocks"],
+            "detail_m1": r["detail"],
+            "prefill_m2048": r["prefill"],
+        }
+        print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
