@@ -152,7 +152,8 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (st != ANY4_OK) return st;
   if (path == ANY4_PATH_DECODE) {
     return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
-                         (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, (cudaStream_t)stream, dev);
+                         (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, dev_status, (cudaStream_t)stream,
+                         dev);
   }
   return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
                         workspace_bytes, dev_status, (cudaStream_t)stream, dev);

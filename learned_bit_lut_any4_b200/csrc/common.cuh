@@ -90,7 +90,13 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
                           uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          cudaStream_t stream, const DeviceInfo& dev);
+                          int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev);
+bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G);
+any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                              int64_t lut_row_stride, const uint16_t* scale,
+                              const uint16_t* offset, uint16_t* y, int64_t N, int64_t K,
+                              int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
+                              const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                            int64_t lut_row_stride, const uint16_t* scale,

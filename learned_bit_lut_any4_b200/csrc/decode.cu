@@ -383,7 +383,12 @@ any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
                           uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          cudaStream_t stream, const DeviceInfo& dev) {
+                          int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+  // M = 1 with a 1024-column slice holding whole 16-byte runs of scales:
+  // weights streamed by the tensor-memory-access engine (decode_tma.cu)
+  if (decode_tma_supported(M, N, K, G))
+    return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
+                             dev_status, stream, dev);
   // rows of x beyond 8 are handled by further launches over the same weights
   for (int64_t m0 = 0; m0 < M; m0 += 8) {
     const int mb = (int)std::min<int64_t>(M - m0, 8);

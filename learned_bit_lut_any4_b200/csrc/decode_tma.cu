@@ -1,0 +1,481 @@
+// Decode-path any4 matmul at M = 1 with TMA-fed weight streaming.
+//
+// Same arithmetic as decode.cu (paper "any4: Learned 4-bit Numeric
+// Representation for LLMs", §4.1 Eq. 8, §2.5.2, §4.2): exact bf16 W from
+// bf16(fmaf(LUT[c], scale, offset)), table lookup by warp shuffle, products on
+// the tensor core through the diagonal m16n8k16 mapping, fp32 accumulation.
+//
+// What differs is how the weights reach the warps.  Each warp owns one
+// 1024-column slice of K for the rows of its block and streams them through a
+// private ring of S shared-memory stages; one lane issues, per stage of P rows,
+// four cp.async.bulk.tensor.2d loads (packed codes viewed as u32 [N][K/8] with a
+// 128 x P box = 512 bytes a row, the rows' tables [N][16], scales and offsets
+// [N][K/G]), completed on an mbarrier.  The loads run as far ahead as the ring
+// allows without holding registers, so the memory system always has
+// S * P rows queued per warp while the lanes compute, and the block's register
+// footprint stays small enough for several blocks per SM.  Rows past N and
+// columns past K come back as zeros from the tensor loads.
+//
+// Waits on the ring are bounded (about 2 s of %globaltimer); on expiry the
+// kernel sets ANY4_ERR_TIMEOUT in dev_status and every warp stops after
+// waiting (bounded) for the copies it has in flight.
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace any4 {
+namespace {
+
+constexpr int kTmaMaxWarps = 8;
+constexpr int kTmaRows = 8;      // P: rows per stage
+constexpr int kTmaStages = 2;    // S: stages per warp (2 keeps two blocks per SM)
+constexpr unsigned long long kTmaWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init_(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_test_(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_test_(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_(bar, parity)) return true;
+    if ((i & 63u) == 0u && gtimer() - t0 > kTmaWaitNs) return false;
+  }
+}
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                      uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar) : "memory");
+}
+
+struct TmaMaps {
+  CUtensorMap codes;   // u32 [N][K/8], box {128, P}
+  CUtensorMap lut;     // bf16 [N][16], box {16, P}
+  CUtensorMap scale;   // bf16 [N][K/G], box {1024/G, P}
+  CUtensorMap offset;  // bf16 [N][K/G], box {1024/G, P}
+};
+
+// D += A * B, m16n8k16 bf16 -> fp32 (legacy warp-level tensor-core MMA).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two weights of one row: W' = bf16(fmaf(LUT[c], s, o)) for both codes, as one
+// packed fp32x2 fused multiply-add (each half rounded once, exactly like fmaf)
+// and one conversion to bf16x2 (first code in the low half).
+__device__ __forceinline__ uint32_t dq_pair(float lut_lane, uint32_t c_lo, uint32_t c_hi,
+                                           unsigned long long s2, unsigned long long o2) {
+  const float a = shfl_idx(lut_lane, c_lo);
+  const float b = shfl_idx(lut_lane, c_hi);
+  unsigned long long ab, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ab) : "f"(a), "f"(b));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ab), "l"(s2), "l"(o2));
+  float ra, rb;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
+  return pack_bf16x2_rn(ra, rb);
+}
+
+__device__ __forceinline__ unsigned long long dup2(float v) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
+
+// Sum 8 per-lane values over the warp; value i's total ends in the lanes
+// whose bits 4, 3, 2 spell i (lanes 4i .. 4i+3 after the bit reversal below).
+__device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
+  int n = 8;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & off) != 0;
+      const int half = n / 2;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (i < half) {
+          const float give = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(kFullMask, give, off);
+        }
+      }
+      n = half;
+    } else {
+      v[0] += __shfl_xor_sync(kFullMask, v[0], off);
+    }
+  }
+  return v[0];
+}
+
+template <int GPS>  // groups per 1024-column slice (1024 / G)
+__global__ void __launch_bounds__(kTmaMaxWarps * 32) decode_tma_kernel(
+    const __grid_constant__ TmaMaps maps, const uint16_t* __restrict__ x,
+    const uint16_t* __restrict__ lut_shared, uint16_t* __restrict__ y, int N, int K,
+    int nslices, int rows_per_block, int32_t* dev_status) {
+  constexpr int P = kTmaRows;
+  constexpr int S = kTmaStages;
+  constexpr int kCodeBytes = P * 512;
+  constexpr int kLutBytes = P * 32;
+  constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
+  constexpr int kStageBytes = kCodeBytes + kLutBytes + 2 * kGrpBytes;
+  constexpr uint32_t kTx = kCodeBytes + kLutBytes + 2 * P * GPS * 2;
+  static_assert(kStageBytes % 128 == 0, "stage alignment");
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int RT = rows_per_block;
+  const int RTP = ((RT + P - 1) / P) * P;
+  // layout: [rings: nwarps * S * kStageBytes][bars: nwarps * S * 8][partials]
+  const uint32_t base = (smem_addr(smem_raw) + 127u) & ~127u;
+  uint8_t* gbase = smem_raw + (base - smem_addr(smem_raw));
+  const uint32_t ring = base + (uint32_t)(warp * S * kStageBytes);
+  const uint8_t* gring = gbase + warp * S * kStageBytes;
+  const uint32_t bars = base + (uint32_t)(nwarps * S * kStageBytes) + (uint32_t)(warp * S * 8);
+  float* s_part =
+      reinterpret_cast<float*>(gbase + nwarps * S * kStageBytes + nwarps * S * 8 + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + nwarps * S * kStageBytes +
+                                                          nwarps * S * 8);
+  if (threadIdx.x == 0) *s_abort = 0;
+
+  if (lane == 0) {
+    for (int st = 0; st < S; ++st) mbar_init_(bars + 8u * st, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();  // barriers and the abort flag are initialised
+
+  const int64_t nblocks = ((int64_t)N + RT - 1) / RT;
+  uint32_t it_issue = 0, it_use = 0;  // ring positions (issue and consumption order)
+  bool waited = false, ok = true;
+  const int gsub = (lane * 32) / (1024 / GPS);  // this lane's group within the slice
+
+  // Every warp runs the same block loop and reaches the same __syncthreads;
+  // a warp whose wait gave up only stops computing (ok = false) and raises
+  // the block-wide flag so that no result of the block is written.
+  for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+    const int row0 = (int)(blk * RT);
+    const int nrows = (N - row0) < RT ? (N - row0) : RT;
+    const int nstages = (nrows + P - 1) / P;
+    bool first_slice = true;
+    for (int s = warp; s < nslices && ok; s += nwarps) {
+      // producer: the first S stages of this slice
+      auto issue = [&](int stage_idx) {
+        const int st = (int)(it_issue % S);
+        const uint32_t dst = ring + (uint32_t)(st * kStageBytes);
+        const uint32_t bar = bars + 8u * st;
+        const int r = row0 + stage_idx * P;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     :: "r"(bar), "r"(kTx) : "memory");
+        tma2d(dst, &maps.codes, s * 128, r, bar);
+        tma2d(dst + kCodeBytes, &maps.lut, 0, r, bar);
+        tma2d(dst + kCodeBytes + kLutBytes, &maps.scale, s * GPS, r, bar);
+        tma2d(dst + kCodeBytes + kLutBytes + kGrpBytes, &maps.offset, s * GPS, r, bar);
+        ++it_issue;
+      };
+      if (lane == 0) {
+        for (int q = 0; q < S && q < nstages; ++q) issue(q);
+      } else {
+        it_issue += (uint32_t)(S < nstages ? S : nstages);
+      }
+      if (!waited) {  // x (and y) may belong to the preceding kernel
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        waited = true;
+      }
+      const int k0 = s * 1024 + lane * 32;
+      const bool kin = k0 < K;
+      uint32_t xw[16];
+      if (kin) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 q = ldg_nc_v4(x + k0 + 8 * v);
+          xw[4 * v] = q.x; xw[4 * v + 1] = q.y; xw[4 * v + 2] = q.z; xw[4 * v + 3] = q.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xw[i] = 0u;
+      }
+      const float lv_shared =
+          lut_shared ? bf16_lo_to_f32(ldg_u16(lut_shared + (lane & 15))) : 0.f;
+
+      for (int si = 0; si < nstages; ++si) {
+        const int st = (int)(it_use % S);
+        const uint32_t parity = (it_use / S) & 1u;
+        if (!mbar_wait_bounded(bars + 8u * st, parity)) {
+          if (lane == 0) report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
+          ok = false;
+          *s_abort = 1;
+          break;
+        }
+        const uint8_t* sp = gring + st * kStageBytes;
+        const uint4* codes = reinterpret_cast<const uint4*>(sp);
+        const uint16_t* lt = reinterpret_cast<const uint16_t*>(sp + kCodeBytes);
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes);
+        const uint16_t* of =
+            reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes + kGrpBytes);
+        float part[P];
+        // All P rows of the stage, then their P/2 row pairs interleaved step by
+        // step: every pair accumulates in its own registers, so P/2 independent
+        // tensor-core chains are in flight instead of one.
+        constexpr int NP = P / 2;
+        uint4 q[P];
+        float lv[P];
+        unsigned long long sv[P], ov[P];
+#pragma unroll
+        for (int j = 0; j < P; ++j) {
+          const bool rv = si * P + j < nrows;
+          q[j] = rv ? codes[j * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
+          lv[j] = lut_shared ? lv_shared : bf16_lo_to_f32(lt[j * 16 + (lane & 15)]);
+          sv[j] = dup2(bf16_lo_to_f32(sc[j * GPS + gsub]));
+          ov[j] = dup2(bf16_lo_to_f32(of[j * GPS + gsub]));
+        }
+        float c[NP][4];
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp) c[pp][0] = c[pp][1] = c[pp][2] = c[pp][3] = 0.f;
+#pragma unroll
+        for (int stp = 0; stp < 8; ++stp) {
+#pragma unroll
+          for (int pp = 0; pp < NP; ++pp) {
+            // codes 4 stp .. 4 stp + 3 of the lane's 32: A rows 0-7 = row 2pp,
+            // rows 8-15 = row 2pp + 1, B = x at the same four columns; the
+            // diagonals C[q][q], C[q+8][q] are the two rows' partial sums
+            const int ja = 2 * pp, jb = 2 * pp + 1;
+            const uint32_t wa4[4] = {q[ja].x, q[ja].y, q[ja].z, q[ja].w};
+            const uint32_t wb4[4] = {q[jb].x, q[jb].y, q[jb].z, q[jb].w};
+            const uint32_t ca = wa4[stp / 2] >> (16 * (stp & 1));
+            const uint32_t cb = wb4[stp / 2] >> (16 * (stp & 1));
+            const uint32_t a01 = dq_pair(lv[ja], ca, ca >> 4, sv[ja], ov[ja]);
+            const uint32_t a45 = dq_pair(lv[ja], ca >> 8, ca >> 12, sv[ja], ov[ja]);
+            const uint32_t a23 = dq_pair(lv[jb], cb, cb >> 4, sv[jb], ov[jb]);
+            const uint32_t a67 = dq_pair(lv[jb], cb >> 8, cb >> 12, sv[jb], ov[jb]);
+            mma16816(c[pp], a01, a23, a45, a67, xw[2 * stp], xw[2 * stp + 1]);
+          }
+        }
+        {
+          const int qd = lane >> 2;
+          const bool diag = (lane & 3) == (qd >> 1);
+#pragma unroll
+          for (int pp = 0; pp < NP; ++pp) {
+            const float da = (qd & 1) ? c[pp][1] : c[pp][0];
+            const float db = (qd & 1) ? c[pp][3] : c[pp][2];
+            part[2 * pp] = diag ? da : 0.f;
+            part[2 * pp + 1] = diag ? db : 0.f;
+          }
+        }
+        ++it_use;
+        // stage st is consumed: let the tensor loads overwrite it
+        __syncwarp();
+        if (lane == 0 && si + S < nstages) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue(si + S);
+        } else if (si + S < nstages) {
+          ++it_issue;
+        }
+        const float tot = reduce8(part, lane);
+        if ((lane & 3) == 0) {
+          const int idx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+          float* dst = s_part + (size_t)warp * RTP + si * P + idx;
+          *dst = first_slice ? tot : *dst + tot;
+        }
+      }
+      first_slice = false;
+    }
+    __syncthreads();
+    if (*s_abort == 0) {
+      const int nw_used = nwarps < nslices ? nwarps : nslices;
+      for (int t = threadIdx.x; t < nrows; t += blockDim.x) {
+        float tot = 0.f;
+        for (int w = 0; w < nw_used; ++w) tot += s_part[(size_t)w * RTP + t];
+        y[row0 + t] = f32_to_bf16_rn(tot);
+      }
+    }
+    __syncthreads();
+  }
+  if (!waited) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
+  // before leaving, make sure no tensor load of this warp is still writing its ring
+  if (!ok) {
+    while (it_use < it_issue) {
+      const int st = (int)(it_use % S);
+      if (!mbar_wait_bounded(bars + 8u * st, (it_use / S) & 1u)) break;
+      ++it_use;
+    }
+  }
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+bool encode2d(EncodeFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* ptr,
+              uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_inner,
+              uint32_t box_rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int GPS>
+any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                    int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
+                    uint16_t* y, int64_t N, int64_t K, int64_t G, bool overlap,
+                    int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+  constexpr int P = kTmaRows;
+  constexpr int S = kTmaStages;
+  constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
+  constexpr int kStageBytes = P * 512 + P * 32 + 2 * kGrpBytes;
+  EncodeFn enc = get_encode();
+  if (!enc) return ANY4_ERR_UNSUPPORTED;
+  TmaMaps maps;
+  if (!encode2d(enc, &maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, (uint64_t)K / 8,
+                (uint64_t)N, (uint64_t)K / 2, 128, P) ||
+      !encode2d(enc, &maps.scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, scale, (uint64_t)(K / G),
+                (uint64_t)N, (uint64_t)(K / G) * 2, GPS, P) ||
+      !encode2d(enc, &maps.offset, CU_TENSOR_MAP_DATA_TYPE_UINT16, offset, (uint64_t)(K / G),
+                (uint64_t)N, (uint64_t)(K / G) * 2, GPS, P))
+    return ANY4_ERR_CUDA;
+  if (lut_row_stride == 16) {
+    if (!encode2d(enc, &maps.lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, lut, 16, (uint64_t)N, 32, 16,
+                  P))
+      return ANY4_ERR_CUDA;
+  } else {
+    // one table for the matrix: read directly by the kernel; the per-stage
+    // tensor load of the table slot still runs (rows past the first come
+    // back as zeros) so that every stage carries the same byte count
+    if (!encode2d(enc, &maps.lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, lut, 16, 1, 32, 16, P))
+      return ANY4_ERR_CUDA;
+  }
+  const int nslices = (int)((K + 1023) / 1024);
+  const int per_warp = (nslices + kTmaMaxWarps - 1) / kTmaMaxWarps;
+  const int nwarps = (nslices + per_warp - 1) / per_warp;
+  const int threads = nwarps * 32;
+
+  auto kern = decode_tma_kernel<GPS>;
+  const size_t ring_bytes = (size_t)nwarps * S * kStageBytes + (size_t)nwarps * S * 8 + 16 + 128;
+  const int kMaxRT = 512;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)std::min<size_t>(dev.smem_optin, 227 * 1024));
+  });
+  if (attr_err != cudaSuccess) return ANY4_ERR_CUDA;
+  // rows per block from the blocks that fit per SM, which depends (through the
+  // partial sums) on the rows per block: settle it in two passes
+  int per_sm = 2;
+  int64_t rt = 0, rtp = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int64_t wave = (int64_t)dev.sm_count * per_sm;
+    rt = std::min<int64_t>((N + wave - 1) / wave, kMaxRT);
+    rtp = ((rt + P - 1) / P) * P;
+    const size_t smem_try = ring_bytes + (size_t)nwarps * rtp * sizeof(float);
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem_try) !=
+            cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    if (occ == per_sm) break;
+    per_sm = occ;
+  }
+  const int64_t wave = (int64_t)dev.sm_count * per_sm;
+  rt = std::min<int64_t>((N + wave - 1) / wave, kMaxRT);
+  rtp = ((rt + P - 1) / P) * P;
+  const int64_t nblocks = (N + rt - 1) / rt;
+  const int grid = (int)std::min<int64_t>(nblocks, wave);
+  const size_t smem = ring_bytes + (size_t)nwarps * rtp * sizeof(float);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint16_t* lut_shared = lut_row_stride == 0 ? lut : nullptr;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, x, lut_shared, y, (int)N, (int)K,
+                                             nslices, (int)rt, dev_status);
+  return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+}  // namespace
+
+bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G) {
+  if (M != 1) return false;
+  if (G != 32 && G != 64 && G != 128) return false;
+  if ((K / G) % 8 != 0) return false;  // 16-byte row stride of scale/offset
+  if (N > INT32_MAX / 2 || K > INT32_MAX / 2) return false;
+  return true;
+}
+
+any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                              int64_t lut_row_stride, const uint16_t* scale,
+                              const uint16_t* offset, uint16_t* y, int64_t N, int64_t K,
+                              int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
+                              const DeviceInfo& dev) {
+  switch (G) {
+    case 128:
+      return run_tma<8>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
+                        dev_status, stream, dev);
+    case 64:
+      return run_tma<16>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
+                         dev_status, stream, dev);
+    case 32:
+      return run_tma<32>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
+                         dev_status, stream, dev);
+    default:
+      return ANY4_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace any4

@@ -147,3 +147,24 @@ def test_decode_overlap_prior_chain():
     y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, overlap_prior=True)
     torch.cuda.synchronize()
     assert_matmul_close(host_bits(y1), y_ref, "overlap")
+
+
+@pytest.mark.parametrize("K,N,G,shared", [(1024, 1000, 32, False), (1280, 777, 32, False),
+                                          (3072, 300, 64, False), (8192, 2050, 128, False),
+                                          (4096, 1500, 128, True), (2048, 9, 64, True)])
+def test_decode_m1_streamed_variants(K, N, G, shared):
+    """M = 1 shapes of the tensor-memory-streamed decode kernel: every group
+    size it takes, ragged rows, a last 1024-column slice cut short, the one
+    table mode; dev_status must stay clear."""
+    shape = workloads.Shape(f"m1_{K}_{N}_{G}", 1, K, N, G, 9901 + K + N, 9951 + G)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    lut = p.lut[11 % N].copy() if shared else p.lut
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = any4.any4_matmul(d.x, d.packed, dev_bf16(lut), d.scale, d.offset, shape.G,
+                         dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, lut, p.scale, p.offset, shape.G,
+                               per_tensor_lut=shared)
+    assert_matmul_close(host_bits(y), y_ref, shape.name)
