@@ -14,18 +14,20 @@
 //   warp 1      TMEM allocation (512 columns = two 128 x 256 fp32
 //               accumulators) and, from one thread, the tcgen05.mma issue
 //               (M = 128, N = 256, K = 16; both operands K-major in smem)
-//   warps 2..9  the dequant stage: lane l of warp w owns weight row
-//               32 (w - 2) + l of the tile, reads its 32 packed bytes per
-//               stage straight from global memory, looks each code up in a
-//               shared-memory copy of the row's table, applies the group
-//               scale/offset with one fmaf, rounds to bf16 (exactly the
-//               dequant definition) and stores the 128-byte row of the B
-//               tile in the 128-byte-swizzled layout the MMA reads.  After
-//               the last stage of a tile the same warps drain TMEM (tcgen05.ld),
-//               round to bf16 and write y.
-// Table lookups: the table is stored transposed, s_lut[c][row], so the 32
-// lanes of a warp (32 consecutive rows) always hit 32 different banks.
-// Each weight tile is dequantised once per 256 rows of x.
+//   warps 2..17 the dequant stage: two lanes per weight row of the tile, each
+//               owning 32 of the stage's 64 codes; codes, scale and offset are
+//               fetched from global memory three stages ahead into registers,
+//               each code is looked up in the row's table held in registers
+//               (byte permutes, no memory traffic), scaled and offset by a
+//               packed fp32x2 fused multiply-add, rounded to bf16 (exactly the
+//               dequant definition) and stored into the row of the B tile in
+//               the 128-byte-swizzled layout the MMA reads.  After the last
+//               stage of a tile the same warps drain TMEM (tcgen05.ld), round
+//               to bf16 and write y.
+// Shared-memory bandwidth is the scarce resource here (the MMA reads both
+// operands from it, TMA and the dequant warps write them), which is why the
+// table lookups are done in registers.  Each weight tile is dequantised once
+// per 256 rows of x.
 //
 // Synchronisation: mbarriers per stage (x landed / W written / stage free),
 // one for "accumulators ready" and one for "accumulators drained".  Every
@@ -50,18 +52,16 @@ constexpr int kStages = 3;
 constexpr int kATileBytes = kBM * kBK * 2;      // 16 KB
 constexpr int kBTileBytes = kBN * kBK * 2;      // 32 KB
 constexpr int kStageBytes = kNAcc * kATileBytes + kBTileBytes;  // 64 KB
-constexpr int kXformWarps = kBN / 32;           // 8
-constexpr int kThreads = 64 + kXformWarps * 32; // 320
+constexpr int kXformWarps = 2 * kBN / 32;       // 16: two lanes per weight row
+constexpr int kThreads = 64 + kXformWarps * 32; // 576
 constexpr int kTmemCols = kNAcc * kBN;          // 512
-constexpr int kLutBytes = 16 * kBN * 4;         // 16 KB, s_lut[16][256] fp32
-// layout of the dynamic shared memory (offsets from a 16 KB-aligned base)
-constexpr int kLutOff = 0;                      // 16 KB aligned: row/code bits OR in
-constexpr int kStageOff = kLutBytes;            // 1024-byte aligned stages
+// layout of the dynamic shared memory (offsets from a 1 KB-aligned base)
+constexpr int kStageOff = 0;                    // 1024-byte aligned stages
 constexpr int kBarOff = kStageOff + kStages * kStageBytes;
 constexpr int kNumBars = 3 * kStages + 2;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kSmemUsed = kMiscOff + 16;
-constexpr int kSmemAlloc = kSmemUsed + 16384;   // slack to align the base to 16 KB
+constexpr int kSmemAlloc = kSmemUsed + 1024;    // slack to align the base to 1 KB
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -162,6 +162,38 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// The 4-bit code at bit `pos` of w, moved to bits 10..13 (a byte offset of
+// code * 1024 into the transposed table); pos is a compile-time constant.
+__device__ __forceinline__ uint32_t code_at_bit10(uint32_t w, int pos) {
+  return (pos <= 10 ? (w << (10 - pos)) : (w >> (pos - 10))) & 0x3C00u;
+}
+
+// Table lookup in registers, no memory traffic: tl/th are the low/high byte
+// planes of a 16-entry bf16 table (tl[i] holds the low bytes of entries
+// 4i..4i+3).  For the 8 codes of w (code i at bits 4i..4i+3) returns the 8
+// entries as 4 bf16 pairs, pair p = (entry of code 2p) | (entry of code 2p+1) << 16.
+// Per 4 codes: byte permutes pick each byte from entries 0..7 and 8..15 by the
+// code's low 3 bits, a sign-replicating permute turns each code's bit 3 into a
+// byte mask, and a bitwise select keeps the right half-table's byte.
+__device__ __forceinline__ void lookup8(uint32_t w, const uint32_t (&tl)[4],
+                                        const uint32_t (&th)[4], uint32_t (&pair)[4]) {
+  const uint32_t u = w << 4;  // bit 3 of codes 0, 2, 4, 6 into byte sign bits
+#pragma unroll
+  for (int hv = 0; hv < 2; ++hv) {
+    const uint32_t sel = (hv ? (w >> 16) : w) & 0x7777u;
+    // prmt's default mode: a selector nibble with bit 3 set replicates the
+    // sign bit of the chosen byte (the __byte_perm intrinsic ignores bit 3)
+    uint32_t m;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(u), "r"(w), "r"(hv ? 0xFBEAu : 0xD9C8u));
+    const uint32_t x0 = __byte_perm(tl[0], tl[1], sel), x1 = __byte_perm(tl[2], tl[3], sel);
+    const uint32_t y0 = __byte_perm(th[0], th[1], sel), y1 = __byte_perm(th[2], th[3], sel);
+    const uint32_t lo = (x0 & ~m) | (x1 & m);
+    const uint32_t hi = (y0 & ~m) | (y1 & m);
+    pair[2 * hv] = __byte_perm(lo, hi, 0x5140u);
+    pair[2 * hv + 1] = __byte_perm(lo, hi, 0x7362u);
+  }
+}
+
 // Shared-memory matrix descriptor: K-major operand, rows of 128 bytes,
 // 128-byte swizzle, 8-row groups 1024 bytes apart (SBO), base 1024-aligned.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
@@ -185,10 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     uint16_t* __restrict__ y, int M, int N, int K, int G, int vec_store, int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 16383u) & ~16383u;
+  const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
 
-  float* s_lut = reinterpret_cast<float*>(smem + kLutOff);
   auto stage_a = [&](int s, int h) { return base + kStageOff + s * kStageBytes + h * kATileBytes; };
   auto stage_b = [&](int s) { return base + kStageOff + s * kStageBytes + kNAcc * kATileBytes; };
   const uint32_t bars = base + kBarOff;
@@ -277,82 +308,118 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     }
   } else {
     // ------------------------------------------------ dequant + epilogue
-    const int tw = warp - 2;
-    const int rloc = tw * 32 + lane;                 // weight row within the tile
+    const int tw = warp - 2;                         // 0 .. 15
+    const int half = tw >> 3;                        // which 32 codes of a stage
+    const int rloc = (tw & 7) * 32 + lane;           // weight row within the tile
     const int64_t row_bytes = K / 2;
     const int groups = K / G;
-    const float* lrow = s_lut + rloc;              // this row's column of s_lut
     uint32_t it = 0, tcount = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
       const int mt = tile % n_mtiles;
       const int nt = tile / n_mtiles;
       const int n = nt * kBN + rloc;
       const bool rin = n < N;
-      // this row's table, transposed: s_lut[c][rloc] (read back only by this lane)
+      // The row's 16-entry table in registers, split into byte planes:
+      // tl[i] = low bytes of entries 4i..4i+3, th[i] = their high bytes.
+      uint32_t tl[4], th[4];
+      {
+        const uint16_t* lrow = lut + (int64_t)(rin ? n : 0) * lut_row_stride;
+        const uint4 e0 = rin ? ldg_nc_v4(lrow) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 e1 = rin ? ldg_nc_v4(lrow + 8) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        s_lut[c * kBN + rloc] = rin ? bf16_lo_to_f32(ldg_u16(lut + (int64_t)n * lut_row_stride + c))
-                                    : 0.f;
+        for (int i = 0; i < 4; ++i) {
+          tl[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x6420);
+          th[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x7531);
+        }
+      }
       const uint8_t* prow = packed + (int64_t)(rin ? n : 0) * row_bytes;
-      int cur_g = -1;
-      float sv = 0.f, ov = 0.f;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
+      const uint16_t* srow = scale + (int64_t)(rin ? n : 0) * groups;
+      const uint16_t* orow = offset + (int64_t)(rin ? n : 0) * groups;
+
+      // This lane's 32 codes of a stage and their group's scale/offset,
+      // fetched three stages ahead.
+      struct Payload {
+        uint4 q;
+        float s, o;
+      };
+      auto fetch = [&](int kb, Payload& pl) {
+        const int k = kb * kBK + 32 * half;
+        const bool kin = rin && k < K;
+        pl.q = kin ? ldg_stream_v4(prow + k / 2) : make_uint4(0u, 0u, 0u, 0u);
+        pl.s = kin ? bf16_lo_to_f32(ldg_u16(srow + k / G)) : 0.f;
+        pl.o = kin ? bf16_lo_to_f32(ldg_u16(orow + k / G)) : 0.f;
+      };
+      // Dequantise this lane's half of one stage of its row into the B tile.
+      auto xform = [&](int kb, const Payload& pl) -> bool {
         const int s = (int)(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
-        uint4 q[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int k = kb * kBK + 32 * h;
-          q[h] = (rin && k < K) ? ldg_stream_v4(prow + k / 2) : make_uint4(0, 0, 0, 0);
-        }
-        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status)) goto done;
+        ++it;
+        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
         const uint32_t brow = stage_b(s) + (uint32_t)rloc * 128u;
+        const uint32_t words[4] = {pl.q.x, pl.q.y, pl.q.z, pl.q.w};
+        unsigned long long s2, o2;
+        asm("mov.b64 %0, {%1, %1};" : "=l"(s2) : "f"(pl.s));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(o2) : "f"(pl.o));
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int k = kb * kBK + 32 * h;
-          const bool kin = rin && k < K;
-          if (kin) {
-            const int g = k / G;
-            if (g != cur_g) {
-              cur_g = g;
-              sv = bf16_lo_to_f32(ldg_u16(scale + (int64_t)n * groups + g));
-              ov = bf16_lo_to_f32(ldg_u16(offset + (int64_t)n * groups + g));
-            }
+        for (int j = 0; j < 4; ++j) {
+          // the 8 codes of word j (columns k + 8j .. k + 8j + 7), looked up 4 at a time
+          uint32_t lut_pair[4];
+          lookup8(words[j], tl, th, lut_pair);
+          uint32_t out[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            // W' = bf16(fmaf(LUT, s, o)) for both codes of the pair, one packed fp32x2 FMA
+            const float l0 = bf16_lo_to_f32(lut_pair[p]);
+            const float l1 = bf16_hi_to_f32(lut_pair[p]);
+            unsigned long long vv, r;
+            asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(l0), "f"(l1));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(vv), "l"(s2), "l"(o2));
+            float r0, r1;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+            out[p] = pack_bf16x2_rn(r0, r1);  // zeros past K (codes 0, scale 0, offset 0)
           }
-          const uint32_t words[4] = {q[h].x, q[h].y, q[h].z, q[h].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t out[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              // codes of columns k + 8j + 2p (low nibble) and k + 8j + 2p + 1
-              const uint32_t c0 = (words[j] >> (8 * p)) & 15u;
-              const uint32_t c1 = (words[j] >> (8 * p + 4)) & 15u;
-              const float v0 = lrow[c0 * kBN];
-              const float v1 = lrow[c1 * kBN];
-              out[p] = kin ? pack_bf16x2_rn(__fmaf_rn(v0, sv, ov), __fmaf_rn(v1, sv, ov)) : 0u;
-            }
-            // 16-byte chunk (4h + j) of the 128-byte row, 128-byte swizzle
-            const uint32_t chunk = (uint32_t)((4 * h + j) ^ (rloc & 7));
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
-                         :: "r"(brow + chunk * 16u), "r"(out[0]), "r"(out[1]), "r"(out[2]),
-                            "r"(out[3]) : "memory");
-          }
+          // 16-byte chunk (4 half + j) of the 128-byte row, 128-byte swizzle
+          const uint32_t chunk = (uint32_t)((4 * half + j) ^ (rloc & 7));
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
+                       :: "r"(brow + chunk * 16u), "r"(out[0]), "r"(out[1]), "r"(out[2]),
+                          "r"(out[3]) : "memory");
         }
         fence_proxy_async_smem();  // make the generic-proxy stores visible to the MMA
         __syncwarp();
         if (lane == 0) mbar_arrive(full_b(s));
+        return true;
+      };
+
+      Payload pa, pb, pc;
+      fetch(0, pa);
+      if (nkb > 1) fetch(1, pb);
+      if (nkb > 2) fetch(2, pc);
+      bool alive = true;
+      for (int kb = 0; kb < nkb && alive; kb += 3) {
+        alive = xform(kb, pa);
+        if (alive && kb + 3 < nkb) fetch(kb + 3, pa);
+        if (alive && kb + 1 < nkb) {
+          alive = xform(kb + 1, pb);
+          if (alive && kb + 4 < nkb) fetch(kb + 4, pb);
+        }
+        if (alive && kb + 2 < nkb) {
+          alive = xform(kb + 2, pc);
+          if (alive && kb + 5 < nkb) fetch(kb + 5, pc);
+        }
       }
+      if (!alive) goto done;
 
       // epilogue: TMEM -> registers -> bf16 -> y
       if (!mbar_wait(accum_full, tcount & 1u, abort_flag, dev_status)) goto done;
       tc_fence_after();
       {
         const int quad = warp & 3;       // TMEM lanes 32*quad .. 32*quad+31
-        const int hacc = tw >> 2;        // which accumulator
+        const int hacc = (tw >> 2) & 1;  // which accumulator
+        const int cpart = tw >> 3;       // which half of the 256 columns
         const int m = mt * kNAcc * kBM + hacc * kBM + quad * 32 + lane;
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(hacc * kBN);
-        for (int cc = 0; cc < kBN / 32; ++cc) {
+        for (int cc = cpart * (kBN / 64); cc < (cpart + 1) * (kBN / 64); ++cc) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + (uint32_t)(cc * 32), r);
           tmem_wait_ld();
