@@ -19,8 +19,10 @@
 //               fetched from global memory three stages ahead into registers,
 //               each code is looked up in the row's table held in registers
 //               (byte permutes, no memory traffic), scaled and offset by a
-//               packed fp32x2 fused multiply-add, rounded to bf16 (exactly the
-//               dequant definition) and stored into the row of the B tile in
+//               bf16x2 fused multiply-add (the exact LUT*scale+offset rounded
+//               once to bf16: the dequant definition's bf16(fmaf(...)) whenever
+//               the fp32 fmaf is exact, at most one bf16 ulp away otherwise)
+//               and stored into the row of the B tile in
 //               the 128-byte-swizzled layout the MMA reads.  After the last
 //               stage of a tile the same warps drain TMEM (tcgen05.ld), round
 //               to bf16 and write y.
@@ -113,6 +115,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
+// mbar_wait by every lane of a warp, with one verdict for the whole warp (so
+// that no lane is left alone in a later warp-synchronous instruction).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, int32_t* dev_status) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, dev_status)) != 0;
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -145,17 +153,13 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -209,12 +213,37 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
 
+// Walks a block's range [u, ue) of (tile, stage) units as segments: the
+// stages kb0 .. kb1-1 of one tile.
+struct SegIter {
+  int64_t u, ue;
+  int nkb;
+  __device__ __forceinline__ bool next(int& tile, int& kb0, int& kb1) {
+    if (u >= ue) return false;
+    tile = (int)(u / nkb);
+    kb0 = (int)(u - (int64_t)tile * nkb);
+    const int64_t rem = ue - u;
+    kb1 = (int)((int64_t)kb0 + rem < nkb ? (int64_t)kb0 + rem : nkb);
+    u += kb1 - kb0;
+    return true;
+  }
+};
+
+// Stream-K partial sums of one block: 256 x 256 fp32, stored in the order the
+// epilogue threads hold them (block, dequant warp, 16-column chunk, float4 of
+// the chunk, lane) so that every warp-wide store and load is contiguous.  The
+// layout is private to this kernel: the same thread mapping writes and reads it.
+__device__ __forceinline__ size_t partial_index(int blk, int tw, int chunk, int lane) {
+  return ((((size_t)blk * kXformWarps + tw) * (kBN / 32) + chunk) * 4) * 32 + lane;
+}
+
 // ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-    uint16_t* __restrict__ y, int M, int N, int K, int G, int vec_store, int32_t* dev_status) {
+    uint16_t* __restrict__ y, int M, int N, int K, int G, int vec_store, int32_t* dev_status,
+    float* __restrict__ ws_partial, uint32_t* __restrict__ ws_flags) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -230,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const uint32_t accum_empty = bars + 8u * (3 * kStages + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
+  int* partial_done = reinterpret_cast<int*>(smem + kMiscOff + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -243,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     mbar_init(accum_full, 1);
     mbar_init(accum_empty, kXformWarps);
     *abort_flag = 0;
+    *partial_done = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -259,14 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int n_ntiles = (N + kBN - 1) / kBN;
   const int ntiles = n_mtiles * n_ntiles;
   const int nkb = (K + kBK - 1) / kBK;
+  // Stream-K split: the (tile, stage) units are divided evenly over the
+  // blocks; this block owns units [ub, ue).
+  const int64_t U = (int64_t)ntiles * nkb;
+  const int64_t ub = U * blockIdx.x / gridDim.x;
+  const int64_t ue = U * (blockIdx.x + 1) / gridDim.x;
 
   if (warp == 0) {
     // ------------------------------------------------ x tiles via TMA
     if (lane == 0) {
       uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      SegIter seg{ub, ue, nkb};
+      int tile, kb0, kb1;
+      while (seg.next(tile, kb0, kb1)) {
         const int mt = tile % n_mtiles;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % kStages);
           const uint32_t ph = (it / kStages) & 1u;
           if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status)) goto done;
@@ -280,11 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     // ------------------------------------------------ MMA issue (one thread)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+      SegIter seg{ub, ue, nkb};
+      int tile, kb0, kb1;
+      for (; seg.next(tile, kb0, kb1); ++tcount) {
         if (tcount > 0 && !mbar_wait(accum_empty, (tcount - 1) & 1u, abort_flag, dev_status))
           goto done;
         tc_fence_after();
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % kStages);
           const uint32_t ph = (it / kStages) & 1u;
           if (!mbar_wait(full_a(s), ph, abort_flag, dev_status)) goto done;
@@ -298,23 +338,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
               const uint64_t da = smem_desc_sw128(stage_a(s, h));
               // advance 16 columns = 32 bytes = 2 descriptor units
               tc_mma(tmem + (uint32_t)(h * kBN), da + 2u * j, db + 2u * j, kIdesc,
-                     (kb > 0 || j > 0) ? 1u : 0u);
+                     (kb > kb0 || j > 0) ? 1u : 0u);
             }
           }
           tc_commit(empty(s));  // stage s free once these MMAs have read it
         }
-        tc_commit(accum_full);  // accumulators of this tile complete
+        tc_commit(accum_full);  // accumulators of this segment complete
       }
     }
   } else {
     // ------------------------------------------------ dequant + epilogue
     const int tw = warp - 2;                         // 0 .. 15
-    const int half = tw >> 3;                        // which 32 codes of a stage
-    const int rloc = (tw & 7) * 32 + lane;           // weight row within the tile
+    // Lanes 2i and 2i+1 of warp tw share weight row tw * 16 + i: lane parity
+    // `half` picks which 32 of a stage's 64 codes the lane converts, so the
+    // pair's code loads fall in one 32-byte sector.
+    const int half = lane & 1;
+    const int rloc = tw * 16 + (lane >> 1);          // weight row within the tile
     const int64_t row_bytes = K / 2;
     const int groups = K / G;
+    // scale/offset rows are read 8 groups (16 bytes) at a time when every
+    // row starts on a 16-byte boundary
+    const bool oct_vec = (groups & 7) == 0;
     uint32_t it = 0, tcount = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+    SegIter seg{ub, ue, nkb};
+    int tile, kb0, kb1;
+    for (; seg.next(tile, kb0, kb1); ++tcount) {
       const int mt = tile % n_mtiles;
       const int nt = tile / n_mtiles;
       const int n = nt * kBN + rloc;
@@ -334,33 +382,56 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         }
       }
       const uint8_t* prow = packed + (int64_t)(rin ? n : 0) * row_bytes;
-      const uint16_t* srow = scale + (int64_t)(rin ? n : 0) * groups;
-      const uint16_t* orow = offset + (int64_t)(rin ? n : 0) * groups;
+      // the even lane of a pair holds its row's scales, the odd lane its
+      // offsets, 8 groups per register quad
+      const uint16_t* grow = (half ? offset : scale) + (int64_t)(rin ? n : 0) * groups;
+      auto fetch_octet = [&](int o8) -> uint4 {
+        if (!rin || 8 * o8 >= groups) return make_uint4(0u, 0u, 0u, 0u);
+        if (oct_vec) return ldg_nc_v4(grow + 8 * o8);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int g0 = 8 * o8 + 2 * i;
+          const uint32_t lo = g0 < groups ? ldg_u16(grow + g0) : 0u;
+          const uint32_t hi = g0 + 1 < groups ? ldg_u16(grow + g0 + 1) : 0u;
+          w[i] = lo | (hi << 16);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+      };
+      // bf16 bits of group slot j (0..7) of an octet
+      auto pick = [](const uint4& v, int j) -> uint32_t {
+        const uint32_t w = (j & 4) ? ((j & 2) ? v.w : v.z) : ((j & 2) ? v.y : v.x);
+        return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+      };
 
-      // This lane's 32 codes of a stage and their group's scale/offset,
-      // fetched three stages ahead.
-      struct Payload {
-        uint4 q;
-        float s, o;
-      };
-      auto fetch = [&](int kb, Payload& pl) {
+      // This lane's 16 bytes of codes of a stage, fetched three stages ahead.
+      auto fetch = [&](int kb) -> uint4 {
         const int k = kb * kBK + 32 * half;
-        const bool kin = rin && k < K;
-        pl.q = kin ? ldg_stream_v4(prow + k / 2) : make_uint4(0u, 0u, 0u, 0u);
-        pl.s = kin ? bf16_lo_to_f32(ldg_u16(srow + k / G)) : 0.f;
-        pl.o = kin ? bf16_lo_to_f32(ldg_u16(orow + k / G)) : 0.f;
+        return (rin && k < K) ? ldg_stream_v4(prow + k / 2) : make_uint4(0u, 0u, 0u, 0u);
       };
+      int cur8 = (kb0 * kBK) / G >> 3;
+      uint4 oct_cur = fetch_octet(cur8), oct_nxt = fetch_octet(cur8 + 1);
       // Dequantise this lane's half of one stage of its row into the B tile.
-      auto xform = [&](int kb, const Payload& pl) -> bool {
+      auto xform = [&](int kb, const uint4& q) -> bool {
         const int s = (int)(it % kStages);
         const uint32_t ph = (it / kStages) & 1u;
         ++it;
-        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
+        // this lane's group and its partner's (the other half of the row)
+        const int g = (kb * kBK + 32 * half) / G;
+        const int gp = (kb * kBK + 32 * (half ^ 1)) / G;
+        if ((g >> 3) != cur8) {  // both lanes of a pair enter a new octet together
+          cur8 = g >> 3;
+          oct_cur = oct_nxt;
+          oct_nxt = fetch_octet(cur8 + 1);
+        }
+        const uint32_t mine = pick(oct_cur, g & 7);
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, pick(oct_cur, gp & 7), 1);
+        // scale and offset as bf16 pairs (both columns of a pair share a group)
+        const uint32_t s2 = (half ? other : mine) * 0x10001u;
+        const uint32_t o2 = (half ? mine : other) * 0x10001u;
+        if (!mbar_wait_warp(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
         const uint32_t brow = stage_b(s) + (uint32_t)rloc * 128u;
-        const uint32_t words[4] = {pl.q.x, pl.q.y, pl.q.z, pl.q.w};
-        unsigned long long s2, o2;
-        asm("mov.b64 %0, {%1, %1};" : "=l"(s2) : "f"(pl.s));
-        asm("mov.b64 %0, {%1, %1};" : "=l"(o2) : "f"(pl.o));
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           // the 8 codes of word j (columns k + 8j .. k + 8j + 7), looked up 4 at a time
@@ -369,15 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
           uint32_t out[4];
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            // W' = bf16(fmaf(LUT, s, o)) for both codes of the pair, one packed fp32x2 FMA
-            const float l0 = bf16_lo_to_f32(lut_pair[p]);
-            const float l1 = bf16_hi_to_f32(lut_pair[p]);
-            unsigned long long vv, r;
-            asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(l0), "f"(l1));
-            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(vv), "l"(s2), "l"(o2));
-            float r0, r1;
-            asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
-            out[p] = pack_bf16x2_rn(r0, r1);  // zeros past K (codes 0, scale 0, offset 0)
+            // W' = LUT * scale + offset for both codes of the pair with one bf16x2
+            // fused multiply-add (the exact value rounded once to bf16)
+            asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out[p]) : "r"(lut_pair[p]), "r"(s2), "r"(o2));
           }
           // 16-byte chunk (4 half + j) of the 128-byte row, 128-byte swizzle
           const uint32_t chunk = (uint32_t)((4 * half + j) ^ (rloc & 7));
@@ -391,55 +456,118 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         return true;
       };
 
-      Payload pa, pb, pc;
-      fetch(0, pa);
-      if (nkb > 1) fetch(1, pb);
-      if (nkb > 2) fetch(2, pc);
+      uint4 pa = fetch(kb0), pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
+      if (kb0 + 1 < kb1) pb = fetch(kb0 + 1);
+      if (kb0 + 2 < kb1) pc = fetch(kb0 + 2);
       bool alive = true;
-      for (int kb = 0; kb < nkb && alive; kb += 3) {
+      for (int kb = kb0; kb < kb1 && alive; kb += 3) {
         alive = xform(kb, pa);
-        if (alive && kb + 3 < nkb) fetch(kb + 3, pa);
-        if (alive && kb + 1 < nkb) {
+        if (alive && kb + 3 < kb1) pa = fetch(kb + 3);
+        if (alive && kb + 1 < kb1) {
           alive = xform(kb + 1, pb);
-          if (alive && kb + 4 < nkb) fetch(kb + 4, pb);
+          if (alive && kb + 4 < kb1) pb = fetch(kb + 4);
         }
-        if (alive && kb + 2 < nkb) {
+        if (alive && kb + 2 < kb1) {
           alive = xform(kb + 2, pc);
-          if (alive && kb + 5 < nkb) fetch(kb + 5, pc);
+          if (alive && kb + 5 < kb1) pc = fetch(kb + 5);
         }
       }
       if (!alive) goto done;
 
-      // epilogue: TMEM -> registers -> bf16 -> y
-      if (!mbar_wait(accum_full, tcount & 1u, abort_flag, dev_status)) goto done;
+      // epilogue: TMEM -> registers; then either this segment's fp32 partial
+      // sums go to the workspace (a segment that does not start the tile), or
+      // the partials of the tile's later segments are added (in block order)
+      // and the bf16 result is written to y.
+      if (!mbar_wait_warp(accum_full, tcount & 1u, abort_flag, dev_status)) goto done;
       tc_fence_after();
       {
         const int quad = warp & 3;       // TMEM lanes 32*quad .. 32*quad+31
         const int hacc = (tw >> 2) & 1;  // which accumulator
         const int cpart = tw >> 3;       // which half of the 256 columns
-        const int m = mt * kNAcc * kBM + hacc * kBM + quad * 32 + lane;
+        const int mloc = hacc * kBM + quad * 32 + lane;  // row within the 256-row tile
+        const int m = mt * kNAcc * kBM + mloc;
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(hacc * kBN);
-        for (int cc = cpart * (kBN / 64); cc < (cpart + 1) * (kBN / 64); ++cc) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tbase + (uint32_t)(cc * 32), r);
+        const bool first = kb0 == 0;
+        const bool last = kb1 == nkb;
+        // blocks holding the later segments of this tile (stream-K), waited for
+        // once each; they do not depend on this block, so the waits end
+        int c_end = (int)blockIdx.x + 1;
+        if (first && !last) {
+          const int64_t tile_end = (int64_t)(tile + 1) * nkb;
+          while (c_end < (int)gridDim.x && U * c_end / gridDim.x < tile_end) {
+            if (lane == 0) {
+              const unsigned long long t0 = globaltimer();
+              uint32_t f = 0;
+              for (uint32_t i = 0;; ++i) {
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
+                             : "=r"(f) : "l"(ws_flags + c_end) : "memory");
+                if (f != 0u) break;
+                if ((i & 63u) == 0u && (*abort_flag || globaltimer() - t0 > kWaitLimitNs)) {
+                  *abort_flag = 1;
+                  report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
+                  break;
+                }
+              }
+            }
+            __syncwarp();
+            ++c_end;
+          }
+          if (__any_sync(0xffffffffu, *abort_flag != 0)) goto done;
+          __threadfence();  // the partials below are read after their flags
+        }
+        // 16 columns at a time: this warp's 32 rows x 128 columns
+        for (int cc = cpart * (kBN / 32); cc < (cpart + 1) * (kBN / 32); ++cc) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tbase + (uint32_t)(cc * 16), r);
           tmem_wait_ld();
-          const int n0 = nt * kBN + cc * 32;
+          if (!first) {
+            float4* dst = reinterpret_cast<float4*>(ws_partial) +
+                          partial_index(blockIdx.x, tw, cc - cpart * (kBN / 32), lane);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[32 * v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            continue;
+          }
+          float acc[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
+          for (int c = (int)blockIdx.x + 1; c < c_end; ++c) {
+            const float4* src = reinterpret_cast<const float4*>(ws_partial) +
+                                partial_index(c, tw, cc - cpart * (kBN / 32), lane);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 q = __ldcg(src + 32 * v);  // written by another SM: read through L2
+              acc[4 * v] += q.x; acc[4 * v + 1] += q.y; acc[4 * v + 2] += q.z; acc[4 * v + 3] += q.w;
+            }
+          }
+          const int n0 = nt * kBN + cc * 16;
           if (m < M) {
             uint16_t* yr = y + (int64_t)m * N;
-            if (vec_store && n0 + 32 <= N) {
+            if (vec_store && n0 + 16 <= N) {
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const uint4 w = make_uint4(
-                    pack_bf16x2_rn(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                    pack_bf16x2_rn(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                    pack_bf16x2_rn(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                    pack_bf16x2_rn(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+              for (int v = 0; v < 2; ++v) {
+                const uint4 w = make_uint4(pack_bf16x2_rn(acc[8 * v + 0], acc[8 * v + 1]),
+                                           pack_bf16x2_rn(acc[8 * v + 2], acc[8 * v + 3]),
+                                           pack_bf16x2_rn(acc[8 * v + 4], acc[8 * v + 5]),
+                                           pack_bf16x2_rn(acc[8 * v + 6], acc[8 * v + 7]));
                 *reinterpret_cast<uint4*>(yr + n0 + 8 * v) = w;
               }
             } else {
-              for (int i = 0; i < 32; ++i)
-                if (n0 + i < N) yr[n0 + i] = f32_to_bf16_rn(__uint_as_float(r[i]));
+              for (int i = 0; i < 16; ++i)
+                if (n0 + i < N) yr[n0 + i] = f32_to_bf16_rn(acc[i]);
             }
+          }
+        }
+        if (!first) {
+          // this block's partial is complete once all dequant warps have stored
+          // their part: the last one to finish publishes the flag
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && atomicAdd(partial_done, 1) == kXformWarps - 1) {
+            __threadfence();
+            asm volatile("st.release.gpu.global.u32 [%0], %1;"
+                         :: "l"(ws_flags + blockIdx.x), "r"(1u) : "memory");
           }
         }
       }
@@ -480,9 +608,20 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+// Workspace: one fp32 256 x 256 partial tile per block (stream-K) followed by
+// one flag word per block.
+int prefill_slots() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    return sms;
+  return 160;
+}
+
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G) {
   (void)M; (void)N; (void)K; (void)G;
-  return 0;
+  const size_t slots = (size_t)prefill_slots();
+  return slots * (size_t)(kNAcc * kBM) * kBN * sizeof(float) + ((slots * 4 + 255) / 256) * 256;
 }
 
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
@@ -490,7 +629,6 @@ any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint1
                            const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
                            int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
                            int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
-  (void)workspace; (void)workspace_bytes;
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   if (dev.smem_optin < (size_t)kSmemAlloc) return ANY4_ERR_UNSUPPORTED;
   EncodeTiledFn enc = encode_fn();
@@ -515,11 +653,36 @@ any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint1
   if (attr_err != cudaSuccess) return ANY4_ERR_CUDA;
 
   const int64_t tiles = ((M + kNAcc * kBM - 1) / (kNAcc * kBM)) * ((N + kBN - 1) / kBN);
-  const int grid = (int)std::min<int64_t>(tiles, dev.sm_count);
+  const int64_t units = tiles * ((K + kBK - 1) / kBK);
+  // every block keeps at least 4 stages of work
+  const int64_t slots = prefill_slots();
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>({units / 4, (int64_t)dev.sm_count,
+                                                                slots}));
+  const size_t partial_bytes = (size_t)slots * (kNAcc * kBM) * kBN * sizeof(float);
+  if (workspace_bytes < prefill_workspace_size(M, N, K, G) || workspace == nullptr)
+    return ANY4_ERR_WORKSPACE;
+  float* ws_partial = static_cast<float*>(workspace);
+  uint32_t* ws_flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + partial_bytes);
+  if (cudaMemsetAsync(ws_flags, 0, (size_t)grid * sizeof(uint32_t), stream) != cudaSuccess)
+    return ANY4_ERR_CUDA;
   const int vec_store = (N % 8 == 0) ? 1 : 0;
-  prefill_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(map, packed, lut, lut_row_stride, scale,
-                                                         offset, y, (int)M, (int)N, (int)K,
-                                                         (int)G, vec_store, dev_status);
+  // Blocks wait on blocks with larger indices for their partial sums: all
+  // blocks must be resident at once, which the cooperative launch guarantees
+  // (one block fits per SM and the grid is at most the SM count).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, prefill_kernel, map, packed, lut, lut_row_stride, scale, offset, y,
+                         (int)M, (int)N, (int)K, (int)G, vec_store, dev_status, ws_partial,
+                         ws_flags) != cudaSuccess)
+    return ANY4_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
