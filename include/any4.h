@@ -148,6 +148,43 @@ ANY4_API any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, co
                            int32_t* dev_status, any4_path path, uint32_t flags,
                            any4_stream_t stream);
 
+/*
+ * any4_matmul_static_scratch -- any4_matmul on the prefill kernel (the
+ * tensor-core path, any M) with its scratch taken from a fixed array inside
+ * the library instead of a caller-supplied workspace.  The paper has no
+ * counterpart: this is an interface variant for callers that cannot allocate
+ * device memory at the call site (a step that must not call cudaMalloc or
+ * cudaFree, since cudaFree synchronises the whole device; a C caller with no
+ * device allocator of its own).  It allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *   arguments       as for any4_matmul, minus the workspace
+ *   scratch         a file-scope device array of ANY4_STATIC_SCRATCH_BYTES
+ *                   bytes, one per device: 37 MiB + 1 KiB, i.e. one 256 KiB
+ *                   fp32 partial tile per block of a 148-SM grid plus the
+ *                   per-block flags, which each call clears (an async memset
+ *                   on `stream`) before its launch.  If the device needs more
+ *                   (any4_matmul_workspace_size_ex(..., ANY4_PATH_PREFILL)
+ *                   above ANY4_STATIC_SCRATCH_BYTES, e.g. a GPU with more
+ *                   than 148 SMs) the call returns ANY4_ERR_WORKSPACE and
+ *                   launches nothing.
+ *   set-up          the first call on a device looks up the array's device
+ *                   address (cudaGetSymbolAddress, with that device current)
+ *                   and caches it; make that first call before any stream
+ *                   capture.  A failed look-up returns ANY4_ERR_CUDA.
+ *   concurrency     every call on a device uses the same array: calls whose
+ *                   kernels overlap on the GPU (different streams, or several
+ *                   host threads) race on it and give undefined results.
+ *                   Calls issued in order on one stream are safe.
+ * Results are those of any4_matmul_ex(..., ANY4_PATH_PREFILL, ...).
+ */
+#define ANY4_STATIC_SCRATCH_BYTES ((size_t)148 * 262144 + 1024)
+ANY4_API any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t* packed,
+                                                const uint16_t* lut, int64_t lut_row_stride,
+                                                const uint16_t* scale, const uint16_t* offset,
+                                                uint16_t* y, int64_t M, int64_t N, int64_t K,
+                                                int64_t G, int32_t* dev_status,
+                                                any4_stream_t stream);
+
 /* Bytes of workspace any4_matmul needs for this shape (0 if none).  Returns
  * 0 as well for shapes that break the shape rules (the call then fails). */
 ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);

@@ -17,12 +17,14 @@ from ._native import (  # noqa: F401
     ANY4_ERR_TIMEOUT,
     ANY4_ERR_UNSUPPORTED,
     ANY4_ERR_WORKSPACE,
+    ANY4_STATIC_SCRATCH_BYTES,
     PATHS,
     Any4Error,
     any4_bits_per_weight,
     any4_dequant,
     any4_matmul,
     any4_matmul_choose_path,
+    any4_matmul_static_scratch,
     any4_matmul_workspace_size,
     any4_pack,
     any4_status_string,

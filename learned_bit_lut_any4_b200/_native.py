@@ -26,6 +26,8 @@ ANY4_ERR_UNSUPPORTED = -7
 ANY4_ERR_WORKSPACE = -8
 
 PATHS = {"auto": 0, "decode": 1, "prefill": 2}
+# Bytes of the library's fixed scratch array (any4_matmul_static_scratch).
+ANY4_STATIC_SCRATCH_BYTES = 148 * 262144 + 1024
 ANY4_FLAG_OVERLAP_PRIOR = 1
 
 _lib = None
@@ -60,6 +62,9 @@ def library() -> ctypes.CDLL:
     lib.any4_matmul_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp,
                                    i32, ctypes.c_uint32, vp]
     lib.any4_matmul_ex.restype = i32
+    lib.any4_matmul_static_scratch.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64,
+                                               vp, vp]
+    lib.any4_matmul_static_scratch.restype = i32
     lib.any4_matmul_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.any4_matmul_workspace_size.restype = sz
     lib.any4_matmul_workspace_size_ex.argtypes = [i64, i64, i64, i64, i32]
@@ -216,4 +221,39 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                                   _ptr(dev_status), p,
                                   ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0,
                                   _stream(dev)), "any4_matmul")
+    return y
+
+
+def any4_matmul_static_scratch(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
+                               scale: torch.Tensor, offset: torch.Tensor, G: int,
+                               y: torch.Tensor | None = None,
+                               dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """any4_matmul on the prefill kernel with the library's fixed scratch
+    array instead of a workspace (the C entry point allocates nothing).
+
+    For a call that allocates nothing at all, pass y (and dev_status if
+    wanted): only a missing y is allocated here, with torch.  The first call on
+    a device looks up the array's address; make it before any stream capture.
+    Calls whose kernels overlap on the GPU share the array and race."""
+    _need(x, "x", _BF16)
+    dev = x.device
+    _need(packed, "packed", (torch.uint8,), dev)
+    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+        _need(t, nm, _BF16, dev)
+    M, K = x.shape
+    N, Kh = packed.shape
+    if 2 * Kh != K:
+        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
+    stride = _lut_stride(lut, N)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "y", _BF16, dev)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", (torch.int32,), dev)
+    lib = library()
+    with torch.cuda.device(dev):
+        _check(lib.any4_matmul_static_scratch(_ptr(x), _ptr(packed), _ptr(lut), stride,
+                                              _ptr(scale), _ptr(offset), _ptr(y), M, N, K, G,
+                                              _ptr(dev_status), _stream(dev)),
+               "any4_matmul_static_scratch")
     return y

@@ -159,6 +159,31 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
                         workspace_bytes, dev_status, (cudaStream_t)stream, dev);
 }
 
+// The prefill kernel with the library's fixed scratch array (static_scratch.cu)
+// in place of a workspace; same validation as any4_matmul_ex.
+any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t* packed,
+                                       const uint16_t* lut, int64_t lut_row_stride,
+                                       const uint16_t* scale, const uint16_t* offset,
+                                       uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G,
+                                       int32_t* dev_status, any4_stream_t stream) {
+  if (!x || !packed || !lut || !scale || !offset || !y) return ANY4_ERR_NULL;
+  if (M < 1 || !shape_ok(N, K, G) || !stride_ok(lut_row_stride)) return ANY4_ERR_SHAPE;
+  if (M > (int64_t(1) << 40) / K || M > (int64_t(1) << 40) / N) return ANY4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(lut) || !aligned16(scale) ||
+      !aligned16(offset) || !aligned16(y))
+    return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  if (prefill_workspace_size(M, N, K, G) > ANY4_STATIC_SCRATCH_BYTES) return ANY4_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = static_scratch(dev.device, &scratch);
+  if (st != ANY4_OK) return st;
+  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, scratch,
+                        ANY4_STATIC_SCRATCH_BYTES, dev_status, (cudaStream_t)stream, dev);
+}
+
 any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                         int64_t lut_row_stride, const uint16_t* scale,
                         const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,

@@ -98,6 +98,10 @@ any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const ui
                               int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
                               const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+// Device address of the fixed scratch array of any4_matmul_static_scratch on
+// `device` (the current device); resolved on first use per device.
+any4_status static_scratch(int device, void** ptr);
+
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                            int64_t lut_row_stride, const uint16_t* scale,
                            const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
