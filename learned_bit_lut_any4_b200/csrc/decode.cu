@@ -18,10 +18,11 @@
 //    l & 15, so both half-warps hold the full table and `shfl` with the code
 //    word shifted right selects the entry with no masking (the shuffle reads
 //    only the low 5 bits of the source lane).
-//  * Each weight is dequantised exactly as the definition rounds it,
-//      W' = bf16(fmaf(LUT[c], scale, offset)),
-//    two at a time (one cvt.rn.bf16x2), and multiplied with x in fp32 by the
-//    mixed-precision bf16 x bf16 -> f32 FMA of sm_100 (products exact).
+//  * Each weight is dequantised as W' = LUT[c] * scale + offset rounded once
+//    to bf16, two at a time (one bf16x2 fused multiply-add; this equals the
+//    definition's bf16(fmaf(...)) except when that fp32 fmaf is inexact and
+//    lands on a bf16 rounding tie), and the products with x are exact in the
+//    tensor core's fp32 accumulation.
 //    (Factoring the group scale out of the sum -- one FMA per weight --
 //    skips that rounding and misses the tolerance on heavy-tailed tables.)
 //  * Reduction: butterfly shuffles within the warp, then a fixed-order sum
@@ -59,13 +60,18 @@ template <> struct CodeLoad<8> {
   }
 };
 
-// W' = bf16(fmaf(LUT[c], s, o)) for two codes, packed as bf16x2 (first code
-// in the low half): exactly the dequantised weights of the definition.
-__device__ __forceinline__ uint32_t dequant_pair(float lut_lane, uint32_t c_lo, uint32_t c_hi,
-                                                 float s, float o) {
-  const float a = shfl_idx(lut_lane, c_lo);
-  const float b = shfl_idx(lut_lane, c_hi);
-  return pack_bf16x2_rn(__fmaf_rn(a, s, o), __fmaf_rn(b, s, o));
+// W' = LUT[c] * s + o for two codes, packed as bf16x2 (first code in the low
+// half): both table entries (bf16 bits, lane l holding entry l & 15) fetched
+// by shuffle, paired, and one bf16x2 fused multiply-add rounds the exact
+// value once to bf16 -- bf16(fmaf(LUT, s, o)) unless that fp32 fmaf is
+// inexact and lands on a bf16 rounding tie.  s2, o2: scale, offset in both halves.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t lut_lane, uint32_t c_lo, uint32_t c_hi,
+                                                 uint32_t s2, uint32_t o2) {
+  uint32_t a, b, w;
+  asm("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(a) : "r"(lut_lane), "r"(c_lo));
+  asm("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(b) : "r"(lut_lane), "r"(c_hi));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(w) : "r"(__byte_perm(a, b, 0x5410)), "r"(s2), "r"(o2));
+  return w;
 }
 
 // acc_lo += W'.lo * x.lo ; acc_hi += W'.hi * x.hi  -- bf16 x bf16 products
@@ -135,7 +141,8 @@ __device__ __forceinline__ int transpose_reduce_index(int lane) {
 template <int KW>
 struct RowRegs {
   uint32_t code[KW];
-  float lv, sv, ov;
+  uint32_t lv;      // table entry lane & 15 (bf16 bits)
+  uint32_t sv, ov;  // group scale and offset, bf16 bits in both halves
 };
 
 // Where one lane's data of the current row lives; advanced row by row.
@@ -152,15 +159,15 @@ __device__ __forceinline__ void load_row(RowRegs<CodeLoad<KL>::kWords>& rr, cons
   constexpr int KW = CodeLoad<KL>::kWords;
   if (valid && kin) {
     CodeLoad<KL>::load(p.pk, rr.code);
-    rr.sv = bf16_lo_to_f32(ldg_u16(p.sc));
-    rr.ov = bf16_lo_to_f32(ldg_u16(p.of));
+    rr.sv = (uint32_t)ldg_u16(p.sc) * 0x10001u;
+    rr.ov = (uint32_t)ldg_u16(p.of) * 0x10001u;
   } else {
 #pragma unroll
     for (int w = 0; w < KW; ++w) rr.code[w] = 0u;
-    rr.sv = 0.f;
-    rr.ov = 0.f;
+    rr.sv = 0u;
+    rr.ov = 0u;
   }
-  rr.lv = valid ? bf16_lo_to_f32(ldg_u16(p.lt)) : 0.f;
+  rr.lv = valid ? (uint32_t)ldg_u16(p.lt) : 0u;
 }
 
 __device__ __forceinline__ void grid_dependency_wait() {

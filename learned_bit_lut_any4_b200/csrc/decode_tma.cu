@@ -1,9 +1,10 @@
 // Decode-path any4 matmul at M = 1 with TMA-fed weight streaming.
 //
-// Same arithmetic as decode.cu (paper "any4: Learned 4-bit Numeric
-// Representation for LLMs", §4.1 Eq. 8, §2.5.2, §4.2): exact bf16 W from
-// bf16(fmaf(LUT[c], scale, offset)), table lookup by warp shuffle, products on
-// the tensor core through the diagonal m16n8k16 mapping, fp32 accumulation.
+// Paper "any4: Learned 4-bit Numeric Representation for LLMs", §4.1 Eq. 8,
+// §2.5.2, §4.2: bf16 W = LUT[c] * scale + offset rounded once to bf16 (one
+// bf16x2 fused multiply-add per pair of weights), table lookup by warp
+// shuffle, products on the tensor core through the diagonal m16n8k16 mapping,
+// fp32 accumulation.
 //
 // What differs is how the weights reach the warps.  Each warp owns one
 // 1024-column slice of K for the rows of its block and streams them through a
@@ -32,6 +33,15 @@ namespace {
 constexpr int kTmaMaxWarps = 8;
 constexpr int kTmaRows = 8;      // P: rows per stage
 constexpr int kTmaStages = 2;    // S: stages per warp (2 keeps two blocks per SM)
+// Row pairs of a stage (counted from the last) whose table lookups run as
+// byte permutes on the integer pipe instead of warp shuffles, so that the
+// two kinds of lookup proceed on different pipes.
+#ifndef ANY4_DECODE_PRMT_PAIRS
+#define ANY4_DECODE_PRMT_PAIRS 0
+#endif
+constexpr int kTmaPrmtPairs = ANY4_DECODE_PRMT_PAIRS;
+static_assert(kTmaPrmtPairs >= 0 && kTmaPrmtPairs <= kTmaRows / 2, "pairs on the permute path");
+
 constexpr unsigned long long kTmaWaitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -86,26 +96,23 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Two weights of one row: W' = bf16(fmaf(LUT[c], s, o)) for both codes, as one
-// packed fp32x2 fused multiply-add (each half rounded once, exactly like fmaf)
-// and one conversion to bf16x2 (first code in the low half).
-__device__ __forceinline__ uint32_t dq_pair(float lut_lane, uint32_t c_lo, uint32_t c_hi,
-                                           unsigned long long s2, unsigned long long o2) {
-  const float a = shfl_idx(lut_lane, c_lo);
-  const float b = shfl_idx(lut_lane, c_hi);
-  unsigned long long ab, r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ab) : "f"(a), "f"(b));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ab), "l"(s2), "l"(o2));
-  float ra, rb;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
-  return pack_bf16x2_rn(ra, rb);
+// Two weights of one row from the table held in the lanes (lane l: entry
+// l & 15 as bf16 bits): both entries fetched by shuffle, paired into one
+// bf16x2 (first code in the low half) and turned into W' = LUT * s + o by one
+// bf16x2 fused multiply-add: the exact value rounded once to bf16, which is
+// bf16(fmaf(LUT, s, o)) unless that fp32 fmaf is inexact and lands on a bf16
+// rounding tie.  The shuffle reads only the low 5 bits of the code word.
+__device__ __forceinline__ uint32_t dq_pair(uint32_t lut_lane, uint32_t c_lo, uint32_t c_hi,
+                                           uint32_t s2, uint32_t o2) {
+  uint32_t a, b, w;
+  asm("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(a) : "r"(lut_lane), "r"(c_lo));
+  asm("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(b) : "r"(lut_lane), "r"(c_hi));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(w) : "r"(__byte_perm(a, b, 0x5410)), "r"(s2), "r"(o2));
+  return w;
 }
 
-__device__ __forceinline__ unsigned long long dup2(float v) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
-  return r;
-}
+// a bf16 value (bits) in both halves of a bf16x2
+__device__ __forceinline__ uint32_t dup2(uint16_t h) { return (uint32_t)h * 0x10001u; }
 
 // Sum 8 per-lane values over the warp; value i's total ends in the lanes
 // whose bits 4, 3, 2 spell i (lanes 4i .. 4i+3 after the bit reversal below).
@@ -133,7 +140,7 @@ __device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
 }
 
 template <int GPS>  // groups per 1024-column slice (1024 / G)
-__global__ void __launch_bounds__(kTmaMaxWarps * 32) decode_tma_kernel(
+__global__ void __maxnreg__(96) decode_tma_kernel(
     const __grid_constant__ TmaMaps maps, const uint16_t* __restrict__ x,
     const uint16_t* __restrict__ lut_shared, uint16_t* __restrict__ y, int N, int K,
     int nslices, int rows_per_block, int32_t* dev_status) {
@@ -221,8 +228,11 @@ __global__ void __launch_bounds__(kTmaMaxWarps * 32) decode_tma_kernel(
 #pragma unroll
         for (int i = 0; i < 16; ++i) xw[i] = 0u;
       }
-      const float lv_shared =
-          lut_shared ? bf16_lo_to_f32(ldg_u16(lut_shared + (lane & 15))) : 0.f;
+      const uint32_t lv_shared = lut_shared ? (uint32_t)ldg_u16(lut_shared + (lane & 15)) : 0u;
+      // byte planes of the one shared table (pairs on the permute path)
+      uint32_t tls[4] = {0u, 0u, 0u, 0u}, ths[4] = {0u, 0u, 0u, 0u};
+      if (kTmaPrmtPairs > 0 && lut_shared)
+        table_planes(ldg_nc_v4(lut_shared), ldg_nc_v4(lut_shared + 8), tls, ths);
 
       for (int si = 0; si < nstages; ++si) {
         const int st = (int)(it_use % S);
@@ -239,53 +249,83 @@ __global__ void __launch_bounds__(kTmaMaxWarps * 32) decode_tma_kernel(
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes);
         const uint16_t* of =
             reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes + kGrpBytes);
-        float part[P];
-        // All P rows of the stage, then their P/2 row pairs interleaved step by
-        // step: every pair accumulates in its own registers, so P/2 independent
-        // tensor-core chains are in flight instead of one.
+        // The stage's rows a pair at a time (rows 2pp, 2pp+1 share the tensor-core
+        // steps), so that few registers stay live and many warps fit per SM;
+        // each pair accumulates in two chains (even and odd steps) to halve the
+        // dependent-MMA latency.
         constexpr int NP = P / 2;
-        uint4 q[P];
-        float lv[P];
-        unsigned long long sv[P], ov[P];
+        float part[P];
 #pragma unroll
-        for (int j = 0; j < P; ++j) {
-          const bool rv = si * P + j < nrows;
-          q[j] = rv ? codes[j * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
-          lv[j] = lut_shared ? lv_shared : bf16_lo_to_f32(lt[j * 16 + (lane & 15)]);
-          sv[j] = dup2(bf16_lo_to_f32(sc[j * GPS + gsub]));
-          ov[j] = dup2(bf16_lo_to_f32(of[j * GPS + gsub]));
-        }
-        float c[NP][4];
+        for (int j = 0; j < P; ++j) part[j] = 0.f;
+        const int qd = lane >> 2;
+        const bool diag = (lane & 3) == (qd >> 1);
+        // row pairs holding at least one row of the matrix (the last stage of
+        // a block may be partly past its rows)
+        const int rows_left = nrows - si * P;
+        const int npairs = rows_left >= P ? NP : (rows_left + 1) / 2;
+#pragma unroll 1
+        for (int pp = 0; pp < npairs; ++pp) {
+          const int ja = 2 * pp, jb = 2 * pp + 1;
+          const bool va = ja < rows_left, vb = jb < rows_left;
+          const uint4 qa = va ? codes[ja * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 qb = vb ? codes[jb * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t la = lut_shared ? lv_shared : (uint32_t)lt[ja * 16 + (lane & 15)];
+          const uint32_t lb = lut_shared ? lv_shared : (uint32_t)lt[jb * 16 + (lane & 15)];
+          const uint32_t sa = dup2(sc[ja * GPS + gsub]), oa = dup2(of[ja * GPS + gsub]);
+          const uint32_t sb = dup2(sc[jb * GPS + gsub]), ob = dup2(of[jb * GPS + gsub]);
+          const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w};
+          const uint32_t wb4[4] = {qb.x, qb.y, qb.z, qb.w};
+          float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+          // word t = codes 8t .. 8t + 7 of the lane's 32, two mma steps of 4
+          // codes: A rows 0-7 = row ja, rows 8-15 = row jb, B = x at the same
+          // four columns; the diagonals C[q][q], C[q+8][q] are the two rows'
+          // partial sums
+          if (kTmaPrmtPairs > 0 && pp >= NP - kTmaPrmtPairs) {
+            // this pair's lookups as byte permutes on the integer pipe
+            uint32_t tla[4], tha[4], tlb[4], thb[4];
+            if (lut_shared) {
 #pragma unroll
-        for (int pp = 0; pp < NP; ++pp) c[pp][0] = c[pp][1] = c[pp][2] = c[pp][3] = 0.f;
+              for (int i = 0; i < 4; ++i) { tla[i] = tlb[i] = tls[i]; tha[i] = thb[i] = ths[i]; }
+            } else {
+              const uint4* ea = reinterpret_cast<const uint4*>(lt + ja * 16);
+              const uint4* eb = reinterpret_cast<const uint4*>(lt + jb * 16);
+              table_planes(ea[0], ea[1], tla, tha);
+              table_planes(eb[0], eb[1], tlb, thb);
+            }
 #pragma unroll
-        for (int stp = 0; stp < 8; ++stp) {
+            for (int t = 0; t < 4; ++t) {
+              uint32_t A[4], B[4];
+              lookup8(wa4[t], tla, tha, A);
+              lookup8(wb4[t], tlb, thb, B);
 #pragma unroll
-          for (int pp = 0; pp < NP; ++pp) {
-            // codes 4 stp .. 4 stp + 3 of the lane's 32: A rows 0-7 = row 2pp,
-            // rows 8-15 = row 2pp + 1, B = x at the same four columns; the
-            // diagonals C[q][q], C[q+8][q] are the two rows' partial sums
-            const int ja = 2 * pp, jb = 2 * pp + 1;
-            const uint32_t wa4[4] = {q[ja].x, q[ja].y, q[ja].z, q[ja].w};
-            const uint32_t wb4[4] = {q[jb].x, q[jb].y, q[jb].z, q[jb].w};
-            const uint32_t ca = wa4[stp / 2] >> (16 * (stp & 1));
-            const uint32_t cb = wb4[stp / 2] >> (16 * (stp & 1));
-            const uint32_t a01 = dq_pair(lv[ja], ca, ca >> 4, sv[ja], ov[ja]);
-            const uint32_t a45 = dq_pair(lv[ja], ca >> 8, ca >> 12, sv[ja], ov[ja]);
-            const uint32_t a23 = dq_pair(lv[jb], cb, cb >> 4, sv[jb], ov[jb]);
-            const uint32_t a67 = dq_pair(lv[jb], cb >> 8, cb >> 12, sv[jb], ov[jb]);
-            mma16816(c[pp], a01, a23, a45, a67, xw[2 * stp], xw[2 * stp + 1]);
+              for (int p = 0; p < 4; ++p) {
+                A[p] = hfma2_bf16(A[p], sa, oa);
+                B[p] = hfma2_bf16(B[p], sb, ob);
+              }
+              mma16816(c0, A[0], B[0], A[1], B[1], xw[4 * t], xw[4 * t + 1]);
+              mma16816(c1, A[2], B[2], A[3], B[3], xw[4 * t + 2], xw[4 * t + 3]);
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              uint32_t A[4], B[4];
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                A[p] = dq_pair(la, wa4[t] >> (8 * p), wa4[t] >> (8 * p + 4), sa, oa);
+                B[p] = dq_pair(lb, wb4[t] >> (8 * p), wb4[t] >> (8 * p + 4), sb, ob);
+              }
+              mma16816(c0, A[0], B[0], A[1], B[1], xw[4 * t], xw[4 * t + 1]);
+              mma16816(c1, A[2], B[2], A[3], B[3], xw[4 * t + 2], xw[4 * t + 3]);
+            }
           }
-        }
-        {
-          const int qd = lane >> 2;
-          const bool diag = (lane & 3) == (qd >> 1);
+          const float da = (qd & 1) ? c0[1] + c1[1] : c0[0] + c1[0];
+          const float db = (qd & 1) ? c0[3] + c1[3] : c0[2] + c1[2];
 #pragma unroll
-          for (int pp = 0; pp < NP; ++pp) {
-            const float da = (qd & 1) ? c[pp][1] : c[pp][0];
-            const float db = (qd & 1) ? c[pp][3] : c[pp][2];
-            part[2 * pp] = diag ? da : 0.f;
-            part[2 * pp + 1] = diag ? db : 0.f;
+          for (int k = 0; k < NP; ++k) {
+            if (k == pp) {
+              part[2 * k] = diag ? da : 0.f;
+              part[2 * k + 1] = diag ? db : 0.f;
+            }
           }
         }
         ++it_use;

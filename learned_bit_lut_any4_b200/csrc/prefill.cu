@@ -172,32 +172,6 @@ __device__ __forceinline__ uint32_t code_at_bit10(uint32_t w, int pos) {
   return (pos <= 10 ? (w << (10 - pos)) : (w >> (pos - 10))) & 0x3C00u;
 }
 
-// Table lookup in registers, no memory traffic: tl/th are the low/high byte
-// planes of a 16-entry bf16 table (tl[i] holds the low bytes of entries
-// 4i..4i+3).  For the 8 codes of w (code i at bits 4i..4i+3) returns the 8
-// entries as 4 bf16 pairs, pair p = (entry of code 2p) | (entry of code 2p+1) << 16.
-// Per 4 codes: byte permutes pick each byte from entries 0..7 and 8..15 by the
-// code's low 3 bits, a sign-replicating permute turns each code's bit 3 into a
-// byte mask, and a bitwise select keeps the right half-table's byte.
-__device__ __forceinline__ void lookup8(uint32_t w, const uint32_t (&tl)[4],
-                                        const uint32_t (&th)[4], uint32_t (&pair)[4]) {
-  const uint32_t u = w << 4;  // bit 3 of codes 0, 2, 4, 6 into byte sign bits
-#pragma unroll
-  for (int hv = 0; hv < 2; ++hv) {
-    const uint32_t sel = (hv ? (w >> 16) : w) & 0x7777u;
-    // prmt's default mode: a selector nibble with bit 3 set replicates the
-    // sign bit of the chosen byte (the __byte_perm intrinsic ignores bit 3)
-    uint32_t m;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(u), "r"(w), "r"(hv ? 0xFBEAu : 0xD9C8u));
-    const uint32_t x0 = __byte_perm(tl[0], tl[1], sel), x1 = __byte_perm(tl[2], tl[3], sel);
-    const uint32_t y0 = __byte_perm(th[0], th[1], sel), y1 = __byte_perm(th[2], th[3], sel);
-    const uint32_t lo = (x0 & ~m) | (x1 & m);
-    const uint32_t hi = (y0 & ~m) | (y1 & m);
-    pair[2 * hv] = __byte_perm(lo, hi, 0x5140u);
-    pair[2 * hv + 1] = __byte_perm(lo, hi, 0x7362u);
-  }
-}
-
 // Shared-memory matrix descriptor: K-major operand, rows of 128 bytes,
 // 128-byte swizzle, 8-row groups 1024 bytes apart (SBO), base 1024-aligned.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
