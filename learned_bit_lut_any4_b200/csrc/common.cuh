@@ -143,6 +143,13 @@ any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const ui
                               int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
                               const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+// Skinny matmul for 2 <= M <= 16 (standard tensor-core mapping, table
+// lookups by byte permute): skinny.cu.
+any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                          int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
+                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
+                          cudaStream_t stream, const DeviceInfo& dev);
+
 // Device address of the fixed scratch array of any4_matmul_static_scratch on
 // `device` (the current device); resolved on first use per device.
 any4_status static_scratch(int device, void** ptr);

@@ -1,6 +1,12 @@
 // Decode-path any4 matmul, M <= 16: y[m][n] = sum_k x[m][k] * W[n][k] with
 // W[n][k] = LUT[n][c] * scale[n][k/G] + offset[n][k/G] never materialised.
 //
+// launch_decode dispatches: M = 1 goes to the weight-streaming kernel of
+// decode_tma.cu where its shape rules allow (G in {32, 64, 128}, K/G a
+// multiple of 8), else to the kernel below (instantiated for one row of x);
+// 2 <= M <= 16 goes to skinny.cu, which dequantises each weight once for all
+// rows of x.
+//
 // Paper: "any4: Learned 4-bit Numeric Representation for LLMs", §4.1 Eq. 8
 // (y_i = sum_j dequant(w_Q[i,j]) x_j), §2.5.2 (dequant = alpha*w_Q + beta),
 // §4.2 (memory-bound at small M; 16-byte coalesced loads; the 16-entry table
@@ -46,20 +52,6 @@ template <> struct CodeLoad<32> {
     w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
   }
 };
-template <> struct CodeLoad<16> {
-  static constexpr int kWords = 2;
-  __device__ __forceinline__ static void load(const uint8_t* p, uint32_t (&w)[2]) {
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-                 : "=r"(w[0]), "=r"(w[1]) : "l"(p));
-  }
-};
-template <> struct CodeLoad<8> {
-  static constexpr int kWords = 1;
-  __device__ __forceinline__ static void load(const uint8_t* p, uint32_t (&w)[1]) {
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
-  }
-};
-
 // W' = LUT[c] * s + o for two codes, packed as bf16x2 (first code in the low
 // half): both table entries (bf16 bits, lane l holding entry l & 15) fetched
 // by shuffle, paired, and one bf16x2 fused multiply-add rounds the exact
@@ -72,16 +64,6 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t lut_lane, uint32_t c_l
   asm("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(b) : "r"(lut_lane), "r"(c_hi));
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(w) : "r"(__byte_perm(a, b, 0x5410)), "r"(s2), "r"(o2));
   return w;
-}
-
-// acc_lo += W'.lo * x.lo ; acc_hi += W'.hi * x.hi  -- bf16 x bf16 products
-// (exact) accumulated in fp32 by the mixed-precision FMA of sm_100.
-__device__ __forceinline__ void fma_bf16x2_f32(float& acc_lo, float& acc_hi, uint32_t w,
-                                               uint32_t xv) {
-  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-      "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
-      "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
-      : "+f"(acc_lo), "+f"(acc_hi) : "r"(w), "r"(xv));
 }
 
 // Sum V = 2^v per-lane values over the 32 lanes, leaving value i's total in
@@ -396,30 +378,13 @@ any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16
   if (decode_tma_supported(M, N, K, G))
     return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
                              dev_status, stream, dev);
-  // rows of x beyond 8 are handled by further launches over the same weights
-  for (int64_t m0 = 0; m0 < M; m0 += 8) {
-    const int mb = (int)std::min<int64_t>(M - m0, 8);
-    const uint16_t* xb = x + m0 * K;
-    uint16_t* yb = y + m0 * N;
-    // only the first launch may overlap the work before it on the stream
-    const bool ov = overlap && m0 == 0;
-    any4_status st;
-    if (mb == 1) {
-      st = run<1, 32, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
+  // M >= 2: the skinny kernel (one dequantisation of the weights for all rows
+  // of x, standard tensor-core mapping; skinny.cu)
+  if (M >= 2)
+    return launch_skinny(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, overlap,
                          stream, dev);
-    } else if (mb == 2) {
-      st = run<2, 32, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
-                         stream, dev);
-    } else if (mb <= 4) {
-      st = run<4, 16, 8>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
-                         stream, dev);
-    } else {
-      st = run<8, 8, 4>(xb, packed, lut, lut_row_stride, scale, offset, yb, mb, N, K, G, ov,
-                        stream, dev);
-    }
-    if (st != ANY4_OK) return st;
-  }
-  return ANY4_OK;
+  return run<1, 32, 8>(x, packed, lut, lut_row_stride, scale, offset, y, 1, N, K, G, overlap,
+                       stream, dev);
 }
 
 }  // namespace any4

@@ -166,12 +166,6 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// The 4-bit code at bit `pos` of w, moved to bits 10..13 (a byte offset of
-// code * 1024 into the transposed table); pos is a compile-time constant.
-__device__ __forceinline__ uint32_t code_at_bit10(uint32_t w, int pos) {
-  return (pos <= 10 ? (w << (10 - pos)) : (w >> (pos - 10))) & 0x3C00u;
-}
-
 // Shared-memory matrix descriptor: K-major operand, rows of 128 bytes,
 // 128-byte swizzle, 8-row groups 1024 bytes apart (SBO), base 1024-aligned.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {

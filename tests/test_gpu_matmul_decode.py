@@ -51,9 +51,11 @@ def test_decode_every_m_ragged(M):
     assert_matmul_close(y, y_ref, shape.name)
 
 
-@pytest.mark.parametrize("K,N,G", [(32, 1, 32), (64, 7, 32), (96, 1000, 32), (2048, 5, 64),
-                                   (33792, 40, 128)])
+@pytest.mark.parametrize("K,N,G", [(32, 1, 32), (64, 7, 32), (96, 7, 32), (96, 1000, 32),
+                                   (2048, 5, 64), (33792, 40, 128)])
 def test_decode_edge_shapes(K, N, G):
+    """Tiny and ragged shapes; (32, 1, 32) and (96, 7, 32) end the scale and
+    offset tensors on a lone group at an even flat index (N * K/G odd)."""
     shape = workloads.Shape(f"edge_{K}_{N}", 3, K, N, G, 9300 + N, 9800 + K // 32)
     p = workloads.make(shape)
     d = DeviceProblem(p)
@@ -119,12 +121,13 @@ def test_decode_writes_only_its_output():
     assert_matmul_close(host_bits(y), y_ref, "guard")
 
 
-def test_decode_overlap_prior_chain():
+@pytest.mark.parametrize("M", [1, 4, 12])
+def test_decode_overlap_prior_chain(M):
     """ANY4_FLAG_OVERLAP_PRIOR: x is produced by the kernel just before each
     call and y is consumed by the kernel just after; a chain of overlapped
     calls must match the same chain run without overlap, bit for bit, and the
-    oracle within tolerance."""
-    shape = workloads.Shape("overlap", 1, 4096, 4096, 128, 9701, 9702)
+    oracle within tolerance (M = 1: weight-streaming kernel; M > 1: skinny)."""
+    shape = workloads.Shape(f"overlap_m{M}", M, 4096, 4096, 128, 9701, 9702 + M)
     p = workloads.make(shape)
     d = DeviceProblem(p)
     def chain(overlap):
