@@ -59,10 +59,10 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the decode kernel source: a stored ncu traffic figure is only
-    used while it was taken on this exact source."""
+    """Hash of the M = 1 decode kernel source (the only kernel of a step): a
+    stored ncu traffic figure is only used while it was taken on this source."""
     h = hashlib.sha256()
-    for fn in ("decode.cu", "common.cuh"):
+    for fn in ("decode_tma.cu", "common.cuh"):
         with open(os.path.join(ROOT, "learned_bit_lut_any4_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -71,7 +71,7 @@ def kernel_source_hash() -> str:
 def stored_traffic():
     """Per-launch DRAM bytes (read + write) of the decode kernel on this step,
     from the committed ncu summary, if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_llama3_8b_layer_m1.md")
+    path = os.path.join(ROOT, "profiles", "decode_tma_kernel_llama3_8b_layer_m1.md")
     try:
         text = open(path).read()
     except OSError:
@@ -325,6 +325,43 @@ def gpu_arm(args, rank, world):
             del packed, lut, sc, of, x, y, flush
         torch.cuda.synchronize()
 
+    # the batch sweep and the 70B shapes at M = 8 (skinny kernel), each shape
+    # alone on rotating weight copies larger than L2
+    batch = {}
+    if not args.skip_batch:
+        bshapes = [s for s in workloads.SKINNY_SWEEP if 2 <= s.M <= 16] + \
+                  [s for s in workloads.LLAMA3_70B_DECODE if s.M == 8]
+        for s in bshapes:
+            wbytes = s.N * s.K // 2 + 4 * s.N * (s.K // s.G) + 32 * s.N
+            bc = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
+            (_, reps, x, y, _), = prepare_layer([s], bc)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                for c in range(bc):
+                    w = reps[c]
+                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for c in range(bc):
+                    w = reps[c]
+                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+            n_rep = max(2, 200 // bc)
+            with torch.cuda.stream(stream):
+                g.replay()
+                stream.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(n_rep):
+                    g.replay()
+                b.record(stream)
+            b.synchronize()
+            us = a.elapsed_time(b) * 1e3 / (n_rep * bc)
+            gbs = s.alg_bytes() / (us * 1e-6) / 1e9
+            batch[s.name] = {"M": s.M, "us": round(us, 3), "GB/s": round(gbs, 1),
+                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+            del g, reps, x, y
+        torch.cuda.synchronize()
+
     # end to end through the public API with host buffers: every step copies
     # each call's x from pinned host memory and reads each y back
     host_x = [torch.from_numpy(np.ascontiguousarray(hx).view(np.int16)).pin_memory()
@@ -361,7 +398,7 @@ def gpu_arm(args, rank, world):
 
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
-        "clocks": clocks, "detail": detail, "prefill": prefill, "peaks": peaks,
+        "clocks": clocks, "detail": detail, "prefill": prefill, "batch": batch, "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -445,6 +482,8 @@ def main():
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the decode kernels without programmatic dependent launch")
     ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--skip-batch", action="store_true",
+                    help="skip the per-shape timing of the M = 2..16 and 70B M = 8 shapes")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=20.0)
     ap.add_argument("--profile-shape", default=None,
@@ -475,7 +514,7 @@ def main():
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": stored_traffic(),
-                    "kernel": "decode_kernel<1,32,8> (the only kernel of the step)",
+                    "kernel": "decode_tma_kernel<8> (the only kernel of the step)",
                     "peak_source": peaks.get("source", "measured")}
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
@@ -496,6 +535,7 @@ def main():
             "clocks": r["clocks"],
             "detail_m1": r["detail"],
             "prefill_m2048": r["prefill"],
+            "detail_batch": r["batch"],
         }
         print(json.dumps(line), flush=True)
     finally:
