@@ -117,7 +117,12 @@ ANY4_API any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, in
  *                   time must not share one.
  *   dev_status      see the conventions above (ANY4_ERR_TIMEOUT)
  * Accuracy: |y - y_ref| <= 1e-2 * rms(y_ref) + ulp_bf16(y_ref) per element,
- * with y_ref the exact dequant-then-matmul.
+ * with y_ref the exact dequant-then-matmul.  Inside the kernels each weight is
+ * formed as LUT * scale + offset rounded once to bf16 (a bf16x2 fused
+ * multiply-add), which equals any4_dequant's W except when the fp32 fmaf is
+ * inexact and lands exactly on a bf16 rounding tie.
+ * Kernels: M = 1 weight-streaming decode, 2 <= M <= 16 skinny, larger M the
+ * tensor-core prefill (any4_matmul_choose_path).
  */
 ANY4_API any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                         int64_t lut_row_stride, const uint16_t* scale,
