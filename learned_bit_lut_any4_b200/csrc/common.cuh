@@ -79,7 +79,10 @@ __device__ __forceinline__ void lookup8(uint32_t w, const uint32_t (&tl)[4],
     // prmt's default mode: a selector nibble with bit 3 set replicates the
     // sign bit of the chosen byte (the __byte_perm intrinsic ignores bit 3)
     uint32_t m;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(u), "r"(w), "r"(hv ? 0xFBEAu : 0xD9C8u));
+    if (hv)
+      asm("prmt.b32 %0, %1, %2, 0xFBEA;" : "=r"(m) : "r"(u), "r"(w));
+    else
+      asm("prmt.b32 %0, %1, %2, 0xD9C8;" : "=r"(m) : "r"(u), "r"(w));
     const uint32_t x0 = __byte_perm(tl[0], tl[1], sel), x1 = __byte_perm(tl[2], tl[3], sel);
     const uint32_t y0 = __byte_perm(th[0], th[1], sel), y1 = __byte_perm(th[2], th[3], sel);
     const uint32_t lo = (x0 & ~m) | (x1 & m);

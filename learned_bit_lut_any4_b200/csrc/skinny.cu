@@ -6,23 +6,25 @@
 // fused multiply-add), fp32 accumulation, bf16 output.
 //
 // Once M > 1 the decode kernels' diagonal tensor-core mapping needs one MMA
-// per row of x, so this kernel uses the plain m16n8k16 mapping instead, with
-// the dequantised weights as the B operand: A = x (up to 16 rows of x per
-// MMA), B = W^T (8 weight rows x 16 columns).  Every lane owns one weight row
-// of an 8-row group (lane / 4) and 32 consecutive codes of it per 128-column
-// chunk (lane % 4 picks the 32); the MMA's k positions are mapped onto those
-// columns (position 2q + j <-> column 4s + j of lane q's 32, position
-// 2q + 8 + j <-> column 4s + 2 + j, for step s), and x is laid out the same
-// way, so the contraction is unchanged.  Each lane holds its row's 16-entry
-// table in registers as byte planes and looks codes up with byte permutes
-// (lookup8), so the dequantisation cost per weight does not depend on M.
+// per row of x, so this kernel uses the plain m16n8k16 mapping: A = a 16-row
+// tile of dequantised weights, B = x^T (up to 8 rows of x per MMA; two MMAs for
+// M <= 16), so each weight is dequantised once for all rows of x.  Lane l owns
+// weight rows l/4 and l/4 + 8 of the tile and 32 consecutive codes of each per
+// 128-column chunk (q = l % 4 picks the 32); the MMA's k positions are mapped
+// onto those columns (position 2q + j <-> column 4s + j of lane q's 32,
+// position 2q + 8 + j <-> column 4s + 2 + j, for step s) and x is read with the
+// same map, so the contraction is unchanged.  The two rows' dequantised pairs
+// form the A operand directly and x's pairs the B operand, so no operand has
+// to be moved into place.  Each lane holds its two rows' 16-entry tables as
+// byte planes in registers and looks codes up with byte permutes (lookup8).
 //
 // Work split: a block owns a contiguous range of 8-row groups (balanced over
-// the grid); its warps split K into slices of 128 * KC columns; each warp
-// keeps x for its slice in registers, walks the row groups (loads of the next
-// group in flight while the current one is computed) and adds its partial
-// sums into shared memory; the block then sums the warps' partials in a fixed
-// order and writes y.  No atomics: bitwise deterministic.
+// the grid), processed as 16-row tiles (the last may be half empty); its warps
+// split K into slices of 128 * KC columns; each warp keeps x for its slice in
+// registers, streams the tiles' codes, tables and scales through a per-warp
+// ring of asynchronous copies, and adds its partial sums into shared memory;
+// the block then sums the warps' partials in a fixed order and writes y.  No
+// atomics: bitwise deterministic.
 #include <algorithm>
 
 #include "common.cuh"
@@ -31,6 +33,7 @@ namespace any4 {
 namespace {
 
 constexpr int kSkWarps = 8;
+constexpr int kSkStages = 3;  // ring stages per warp (16-row tiles in flight)
 
 __device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1,
                                              uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -39,8 +42,6 @@ __device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-
-constexpr int kSkStages = 4;  // ring stages per warp (8-row groups in flight)
 
 // Asynchronous global -> shared copies (16 or 4 bytes); src_bytes = 0 writes zeros.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -59,32 +60,31 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
 }
 
-// One ring stage (one 8-row group of a warp's slice), in shared memory:
-//   codes  [KC][32 lanes][16 bytes]   each lane's 32 codes of each chunk
-//   table  [8 rows][4 lanes][16 bytes]  the rows' 16-entry tables (the
-//                                     first two 16-byte slots of a row)
-//   so     [8 rows][KC][4 lanes][2][4 bytes]  per lane and chunk: the aligned
-//                                     4-byte words holding the scale, then the
-//                                     offset, of the lane's group
+// One ring stage (one 16-row tile of a warp's slice), in shared memory:
+//   codes  [KC][2 halves][32 lanes][16 bytes]  each lane's 32 codes of rows
+//                                     l/4 (half 0) and l/4 + 8 (half 1) per chunk
+//   table  [16 rows][32 bytes]        the tile rows' 16-entry tables
+//   so     [KC][2 halves][32 lanes][2][4 bytes]  per lane, chunk and row: the
+//                                     aligned 4-byte words holding the scale,
+//                                     then the offset, of the lane's group
 template <int KC>
 struct SkStage {
   static constexpr int kCodes = 0;
-  static constexpr int kTable = KC * 512;
+  static constexpr int kTable = KC * 1024;
   static constexpr int kSo = kTable + 512;
-  static constexpr int kBytes = kSo + 8 * KC * 4 * 8;
+  static constexpr int kBytes = kSo + KC * 512;
 };
 
-// MT: rows of x covered (8 or 16; HI = whether the upper 8 rows of the MMA's
-// 16 are used); KC: 128-column chunks per slice.
+// MT: rows of x covered (8 or 16: one or two MMAs per step); KC: 128-column
+// chunks per slice.
 template <int MT, int KC>
 __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride, const uint16_t* __restrict__ scale,
     const uint16_t* __restrict__ offset, uint16_t* __restrict__ y, int M, int N, int K, int G,
     int groups8, int nslices, int rows_max) {
-  constexpr int MB = MT > 16 ? 2 : 1;
-  constexpr int NA = MB == 1 ? 4 : 2;
-  constexpr bool HI = MT > 8;
+  constexpr int MB = MT / 8;  // 8-row blocks of x (one MMA each per step)
+  constexpr int NA = 2;       // accumulator sets (even / odd steps)
   // dynamic shared memory: [nwarps][kSkStages] ring stages, then the partial
   // sums [nwarps][rows_max][M]
   extern __shared__ __align__(16) uint8_t sk_smem[];
@@ -94,8 +94,11 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
   const int nw_used = nwarps < nslices ? nwarps : nslices;
   const int g0 = (int)((int64_t)groups8 * blockIdx.x / gridDim.x);
   const int g1 = (int)((int64_t)groups8 * (blockIdx.x + 1) / gridDim.x);
-  const int q = lane & 3;        // which 32 columns of a chunk
-  const int r = lane >> 2;       // weight row within the group; x row within a 16-row block
+  const int ngroups = g1 - g0;            // 8-row groups of this block
+  const int ntiles = (ngroups + 1) / 2;   // 16-row tiles (the last may be half empty)
+  const int n_base = g0 * 8;
+  const int q = lane & 3;   // which 32 columns of a chunk
+  const int r = lane >> 2;  // weight rows r and r + 8 of a tile; x row of the B operand
   const int64_t row_bytes = K / 2;
   const int groups = K / G;
   const int64_t so_elems = (int64_t)N * groups;  // elements of scale (and of offset)
@@ -129,48 +132,53 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
       lastq[c] = inq[c] && gq[c] == groups - 1 && (so_elems & 1);
     }
 
-    // Issue the copies of group g into ring stage st: lane (r, q) copies its
-    // codes of each chunk, its half (q < 2) of row r's table (lanes q >= 2
-    // zero-fill spare slots, so that the instruction is uniform), and the
-    // aligned 4-byte words holding its groups' scale and offset.
-    auto issue_group = [&](int g, int st) {
+    // Issue the copies of tile t into ring stage st: lane (r, q) copies its
+    // codes of rows r and r + 8 for each chunk, one 16-byte half of one row's
+    // table (q < 2: row r, else row r + 8), and the aligned 4-byte words
+    // holding its groups' scale and offset.
+    auto issue_tile = [&](int t, int st) {
       const uint32_t sb = ring + (uint32_t)(st * SkStage<KC>::kBytes);
-      const int n = g * 8 + r;
-      const bool rin = n < N;
-      const int nc = rin ? n : 0;
-      const uint8_t* prow = packed + (int64_t)nc * row_bytes;
-      const int64_t srow = (int64_t)nc * groups;
+      const bool upper = 2 * t + 1 < ngroups;  // rows r + 8 belong to this block
 #pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        const bool in = rin && inq[c];
-        cp_async16(sb + SkStage<KC>::kCodes + (uint32_t)((c * 32 + lane) * 16),
-                   prow + (in ? colq[c] / 2 : 0), in ? 16u : 0u);
-      }
-      if (!shared_lut)
-        cp_async16(sb + SkStage<KC>::kTable + (uint32_t)(lane * 16),
-                   lut + (int64_t)nc * lut_row_stride + 8 * (q & 1), (rin && q < 2) ? 16u : 0u);
+      for (int h = 0; h < 2; ++h) {
+        const int n = n_base + 16 * t + r + 8 * h;
+        const bool rin = n < N && (h == 0 || upper);
+        const int nc = rin ? n : 0;
+        const uint8_t* prow = packed + (int64_t)nc * row_bytes;
+        const int64_t srow = (int64_t)nc * groups;
 #pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        const bool in = rin && inq[c];
-        const int64_t gi = srow + gq[c];
-        const uint32_t dst = sb + SkStage<KC>::kSo + (uint32_t)(((r * KC + c) * 4 + q) * 8);
-        if (lastq[c] && n == N - 1) {
-          // the aligned pair would run past the tensors' end: the last group
-          // (even flat index, low half) by plain loads instead
-          const uint32_t sv = ldg_u16(scale + gi), ov = ldg_u16(offset + gi);
-          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" :: "r"(dst), "r"(sv), "r"(ov) : "memory");
-        } else {
-          cp_async4(dst, scale + (gi & ~(int64_t)1), in ? 4u : 0u);
-          cp_async4(dst + 4, offset + (gi & ~(int64_t)1), in ? 4u : 0u);
+        for (int c = 0; c < KC; ++c) {
+          const bool in = rin && inq[c];
+          cp_async16(sb + SkStage<KC>::kCodes + (uint32_t)(((c * 2 + h) * 32 + lane) * 16),
+                     prow + (in ? colq[c] / 2 : 0), in ? 16u : 0u);
+          const int64_t gi = srow + gq[c];
+          const uint32_t dst = sb + SkStage<KC>::kSo + (uint32_t)(((c * 2 + h) * 32 + lane) * 8);
+          if (lastq[c] && n == N - 1) {
+            // the aligned pair would run past the tensors' end: the last group
+            // (even flat index, low half) by plain loads instead
+            const uint32_t sv = ldg_u16(scale + gi), ov = ldg_u16(offset + gi);
+            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" :: "r"(dst), "r"(sv), "r"(ov)
+                         : "memory");
+          } else {
+            cp_async4(dst, scale + (gi & ~(int64_t)1), in ? 4u : 0u);
+            cp_async4(dst + 4, offset + (gi & ~(int64_t)1), in ? 4u : 0u);
+          }
         }
+      }
+      if (!shared_lut) {
+        const int trow = (q < 2 ? r : r + 8);
+        const int n = n_base + 16 * t + trow;
+        const bool rin = n < N && (q < 2 || upper);
+        cp_async16(sb + SkStage<KC>::kTable + (uint32_t)(trow * 32 + (q & 1) * 16),
+                   lut + (int64_t)(rin ? n : 0) * lut_row_stride + 8 * (q & 1), rin ? 16u : 0u);
       }
     };
 
-    // prologue: the first kSkStages - 1 groups in flight (empty commit groups
+    // prologue: the first kSkStages - 1 tiles in flight (empty commit groups
     // past the end keep the group count uniform)
 #pragma unroll
     for (int i = 0; i < kSkStages - 1; ++i) {
-      if (g0 + i < g1) issue_group(g0 + i, i);
+      if (i < ntiles) issue_tile(i, i);
       cp_async_commit();
     }
     if (first_slice) {
@@ -179,52 +187,47 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
       asm volatile("griddepcontrol.wait;" ::: "memory");
       asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     }
-    // x for this slice: rows 16 mb + r and 16 mb + r + 8, the lane's 32
-    // columns of each chunk, as bf16 pairs
-    uint32_t xa[MB][KC][16], xb[MB][KC][16];  // xb: rows + 8 (zero unless HI)
+    // x for this slice as the B operand: rows 8 mb + r, the lane's 32 columns
+    // of each chunk, as bf16 pairs
+    uint32_t xw[MB][KC][16];
 #pragma unroll
     for (int mb = 0; mb < MB; ++mb) {
+      const int m = 8 * mb + r;
 #pragma unroll
       for (int c = 0; c < KC; ++c) {
-        const int col = s * kSliceCols + c * 128 + 32 * q;
-        const int ma = 16 * mb + r, mbr = ma + 8;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const uint4 a = (ma < M && col < K) ? ldg_nc_v4(x + (int64_t)ma * K + col + 8 * v)
-                                              : make_uint4(0u, 0u, 0u, 0u);
-          const uint4 b = (HI && mbr < M && col < K)
-                              ? ldg_nc_v4(x + (int64_t)mbr * K + col + 8 * v)
-                              : make_uint4(0u, 0u, 0u, 0u);
-          xa[mb][c][4 * v] = a.x; xa[mb][c][4 * v + 1] = a.y;
-          xa[mb][c][4 * v + 2] = a.z; xa[mb][c][4 * v + 3] = a.w;
-          xb[mb][c][4 * v] = b.x; xb[mb][c][4 * v + 1] = b.y;
-          xb[mb][c][4 * v + 2] = b.z; xb[mb][c][4 * v + 3] = b.w;
+          const uint4 a = (m < M && inq[c]) ? ldg_nc_v4(x + (int64_t)m * K + colq[c] + 8 * v)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+          xw[mb][c][4 * v] = a.x; xw[mb][c][4 * v + 1] = a.y;
+          xw[mb][c][4 * v + 2] = a.z; xw[mb][c][4 * v + 3] = a.w;
         }
       }
     }
 
     int st = 0, st_issue = kSkStages - 1;
-    for (int g = g0; g < g1; ++g) {
-      if (g + kSkStages - 1 < g1) issue_group(g + kSkStages - 1, st_issue);
+    for (int t = 0; t < ntiles; ++t) {
+      if (t + kSkStages - 1 < ntiles) issue_tile(t + kSkStages - 1, st_issue);
       cp_async_commit();
       st_issue = st_issue + 1 == kSkStages ? 0 : st_issue + 1;
       cp_async_wait<kSkStages - 1>();
-      __syncwarp();  // every lane's copies of group g have landed
+      __syncwarp();  // every lane's copies of tile t have landed
       const uint8_t* sp = ring_g + st * SkStage<KC>::kBytes;
       st = st + 1 == kSkStages ? 0 : st + 1;
-      // parity of the row's first flat scale index (which half of a copied word)
-      const int n_row = g * 8 + r;
-      const int par_row = (n_row & groups) & 1;
-      uint32_t tl[4], th[4];
+      const bool upper = 2 * t + 1 < ngroups;  // warp-uniform
+      // parity of each row's first flat scale index (which half of a copied word)
+      const int nA = n_base + 16 * t + r;
+      const int parA = (nA & groups) & 1, parB = ((nA + 8) & groups) & 1;
+      uint32_t tlA[4], thA[4], tlB[4], thB[4];
       if (shared_lut) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { tl[i] = tls[i]; th[i] = ths[i]; }
+        for (int i = 0; i < 4; ++i) { tlA[i] = tlB[i] = tls[i]; thA[i] = thB[i] = ths[i]; }
       } else {
-        const uint4* e = reinterpret_cast<const uint4*>(sp + SkStage<KC>::kTable + r * 64);
-        table_planes(e[0], e[1], tl, th);
+        const uint4* ea = reinterpret_cast<const uint4*>(sp + SkStage<KC>::kTable + r * 32);
+        const uint4* eb = reinterpret_cast<const uint4*>(sp + SkStage<KC>::kTable + (r + 8) * 32);
+        table_planes(ea[0], ea[1], tlA, thA);
+        table_planes(eb[0], eb[1], tlB, thB);
       }
-      // NA independent accumulator sets (steps taken in turn), so that the
-      // dependent-MMA chain of a group is NA times shorter
       float d[NA][MB][4];
 #pragma unroll
       for (int a = 0; a < NA; ++a)
@@ -232,57 +235,63 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
         for (int mb = 0; mb < MB; ++mb) d[a][mb][0] = d[a][mb][1] = d[a][mb][2] = d[a][mb][3] = 0.f;
 #pragma unroll
       for (int c = 0; c < KC; ++c) {
-        // this chunk's group: its scale and offset sit in the half of the
-        // copied 4-byte words given by the flat index's parity
-        const uint2 sow =
-            *reinterpret_cast<const uint2*>(sp + SkStage<KC>::kSo + ((r * KC + c) * 4 + q) * 8);
-        const uint32_t sh = (uint32_t)((par_row ^ gq[c]) & 1) * 16u;
-        const uint32_t s2 = ((sow.x >> sh) & 0xFFFFu) * 0x10001u;
-        const uint32_t o2 = ((sow.y >> sh) & 0xFFFFu) * 0x10001u;
-        const uint4 qv = *reinterpret_cast<const uint4*>(sp + SkStage<KC>::kCodes + (c * 32 + lane) * 16);
-        const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+        // the rows' group scale and offset sit in the half of the copied
+        // 4-byte words given by the flat index's parity
+        const uint2 swA =
+            *reinterpret_cast<const uint2*>(sp + SkStage<KC>::kSo + ((c * 2 + 0) * 32 + lane) * 8);
+        const uint2 swB =
+            *reinterpret_cast<const uint2*>(sp + SkStage<KC>::kSo + ((c * 2 + 1) * 32 + lane) * 8);
+        const uint32_t shA = (uint32_t)((parA ^ gq[c]) & 1) * 16u;
+        const uint32_t shB = (uint32_t)((parB ^ gq[c]) & 1) * 16u;
+        const uint32_t sA = ((swA.x >> shA) & 0xFFFFu) * 0x10001u;
+        const uint32_t oA = ((swA.y >> shA) & 0xFFFFu) * 0x10001u;
+        const uint32_t sB = ((swB.x >> shB) & 0xFFFFu) * 0x10001u;
+        const uint32_t oB = ((swB.y >> shB) & 0xFFFFu) * 0x10001u;
+        const uint4 qa =
+            *reinterpret_cast<const uint4*>(sp + SkStage<KC>::kCodes + ((c * 2 + 0) * 32 + lane) * 16);
+        const uint4 qb =
+            *reinterpret_cast<const uint4*>(sp + SkStage<KC>::kCodes + ((c * 2 + 1) * 32 + lane) * 16);
+        const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t wb4[4] = {qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          // codes 8t .. 8t + 7 of the lane's 32: W' pairs (8t, 8t+1) .. (8t+6, 8t+7)
-          uint32_t w[4];
-          lookup8(words[t], tl, th, w);
+        for (int w = 0; w < 4; ++w) {
+          // codes 8w .. 8w + 7 of the lane's 32, both rows: W' pairs
+          // (8w, 8w+1) .. (8w+6, 8w+7)
+          uint32_t pa[4], pb[4] = {0u, 0u, 0u, 0u};
+          lookup8(wa4[w], tlA, thA, pa);
 #pragma unroll
-          for (int p = 0; p < 4; ++p) w[p] = hfma2_bf16(w[p], s2, o2);
+          for (int p = 0; p < 4; ++p) pa[p] = hfma2_bf16(pa[p], sA, oA);
+          if (upper) {
+            lookup8(wb4[w], tlB, thB, pb);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) pb[p] = hfma2_bf16(pb[p], sB, oB);
+          }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int stp = 2 * t + h;  // mma step: columns 4 stp .. 4 stp + 3 of the lane's 32
+            const int stp = 2 * w + h;  // mma step: columns 4 stp .. 4 stp + 3 of the lane's 32
 #pragma unroll
             for (int mb = 0; mb < MB; ++mb)
-              mma_m16n8k16(d[(c * 8 + stp) % NA][mb], xa[mb][c][2 * stp], xb[mb][c][2 * stp],
-                           xa[mb][c][2 * stp + 1], xb[mb][c][2 * stp + 1], w[2 * h], w[2 * h + 1]);
+              mma_m16n8k16(d[h][mb], pa[2 * h], pb[2 * h], pa[2 * h + 1], pb[2 * h + 1],
+                           xw[mb][c][2 * stp], xw[mb][c][2 * stp + 1]);
           }
         }
       }
-      __syncwarp();  // stage st may be refilled by the next iteration's copies
+      __syncwarp();  // stage may be refilled by the next iteration's copies
+      // d[.][mb]: D[weight row r (+8)][x row 8 mb + 2q, 2q + 1]
+      const int rowA = 16 * t + r, rowB = rowA + 8;
+      float* base = s_part + (size_t)warp * rows_max * M;
 #pragma unroll
-      for (int a = 1; a < NA; ++a)
+      for (int mb = 0; mb < MB; ++mb) {
+        const float v[4] = {d[0][mb][0] + d[1][mb][0], d[0][mb][1] + d[1][mb][1],
+                            d[0][mb][2] + d[1][mb][2], d[0][mb][3] + d[1][mb][3]};
+        const int m0 = 8 * mb + 2 * q;
 #pragma unroll
-        for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d[0][mb][i] += d[a][mb][i];
-      // d[mb]: D[x row 16 mb + r (+8)][weight row 2q, 2q+1 of the group]
-      {
-        const int row0 = (g - g0) * 8 + 2 * q;
-#pragma unroll
-        for (int mb = 0; mb < MB; ++mb) {
-          const int ma = 16 * mb + r, mbr = ma + 8;
-          float* base = s_part + (size_t)warp * rows_max * M;
-          if (ma < M) {
-            float* p0 = base + (size_t)row0 * M + ma;
-            float* p1 = base + (size_t)(row0 + 1) * M + ma;
-            *p0 = first_slice ? d[0][mb][0] : *p0 + d[0][mb][0];
-            *p1 = first_slice ? d[0][mb][1] : *p1 + d[0][mb][1];
-          }
-          if (HI && mbr < M) {
-            float* p0 = base + (size_t)row0 * M + mbr;
-            float* p1 = base + (size_t)(row0 + 1) * M + mbr;
-            *p0 = first_slice ? d[0][mb][2] : *p0 + d[0][mb][2];
-            *p1 = first_slice ? d[0][mb][3] : *p1 + d[0][mb][3];
+        for (int i = 0; i < 4; ++i) {
+          const int m = m0 + (i & 1);
+          const int row = (i < 2) ? rowA : rowB;
+          if (m < M && (i < 2 || upper)) {
+            float* p = base + (size_t)row * M + m;
+            *p = first_slice ? v[i] : *p + v[i];
           }
         }
       }
@@ -293,14 +302,13 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
   }
   __syncthreads();
   // fixed-order sum over the warps' slices; y written row-contiguously per m
-  const int rows = (g1 - g0) * 8;
-  const int n0 = g0 * 8;
+  const int rows = ngroups * 8;
   for (int i = threadIdx.x; i < rows * M; i += blockDim.x) {
     const int m = i / rows, row = i - m * rows;
-    if (n0 + row >= N) continue;
+    if (n_base + row >= N) continue;
     float tot = 0.f;
     for (int w = 0; w < nw_used; ++w) tot += s_part[((size_t)w * rows_max + row) * M + m];
-    y[(int64_t)m * N + n0 + row] = f32_to_bf16_rn(tot);
+    y[(int64_t)m * N + n_base + row] = f32_to_bf16_rn(tot);
   }
 }
 
