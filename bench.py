@@ -215,6 +215,74 @@ def prepare_layer(shapes, copies):
     return sets
 
 
+def _time_graph(stream, calls, n_rep):
+    """µs per call of `calls` (a list of no-argument callables) captured once in
+    a CUDA graph and replayed n_rep times on `stream` (events on that stream)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for f in calls:
+            f()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for f in calls:
+            f()
+    with torch.cuda.stream(stream):
+        g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_rep):
+            g.replay()
+        b.record(stream)
+    b.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (n_rep * len(calls))
+    del g
+    return us
+
+
+def fig3_square_sweep(stream, overlap):
+    """The paper's speed study (Fig. 3): one row of x times square K x K weights,
+    any4 (a table per row) against the one-table modes through the same kernels
+    (nf4-style table from normal quantiles; int4 as the table {-8..7}) and
+    against torch's dense bf16 matmul of the dequantised W (cuBLAS; context).
+    Every variant cycles over weight copies larger than L2."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    from statistics import NormalDist
+    nd = NormalDist()
+    neg = [-nd.inv_cdf(0.5 + 0.5 * (1 - (i + 0.5) / 8)) for i in range(8)]
+    pos = [nd.inv_cdf(0.5 + 0.5 * (i + 1) / 8.5) for i in range(7)]
+    nf4 = np.array(sorted(neg + [0.0] + pos))
+    nf4 = (nf4 / np.abs(nf4).max()).astype(np.float32)
+    t_nf4 = torch.from_numpy(nf4).cuda().to(torch.bfloat16)
+    t_int4 = torch.arange(-8, 8, dtype=torch.float32, device="cuda").to(torch.bfloat16)
+    out = {}
+    for K in (1024, 2048, 4096, 8192, 16384):
+        s = workloads.Shape(f"fig3_{K}", 1, K, K, 128, 7000 + K, 7100 + K)
+        wbytes = s.N * s.K // 2 + 4 * s.N * (s.K // s.G) + 32 * s.N
+        copies = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
+        (_, reps, x, y, _), = prepare_layer([s], copies)
+        n_rep = max(3, 400 // copies)
+        res = {}
+        for name, table in (("any4", None), ("nf4_style", t_nf4), ("int4", t_int4)):
+            calls = [(lambda w=w, t=table: any4.any4_matmul(
+                x, w[0], w[1] if t is None else t, w[2], w[3], s.G, y=y, overlap_prior=overlap))
+                for w in reps]
+            res[name + "_us"] = round(_time_graph(stream, calls, n_rep), 3)
+        W = any4.any4_dequant(reps[0][0], reps[0][1], reps[0][2], reps[0][3], s.G)
+        dcopies = max(1, int(np.ceil(3 * L2_BYTES / (2 * s.N * s.K))))
+        Ws = [W] + [W.clone() for _ in range(dcopies - 1)]
+        xd = x.clone()
+        calls = [(lambda Wc=Wc: torch.nn.functional.linear(xd, Wc)) for Wc in Ws]
+        res["bf16_dense_us"] = round(_time_graph(stream, calls, max(3, 400 // dcopies)), 3)
+        for name in ("any4", "nf4_style", "int4"):
+            res[name + "_speedup_vs_bf16"] = round(res["bf16_dense_us"] / res[name + "_us"], 2)
+        out[str(K)] = res
+        del reps, x, y, W, Ws, xd
+        torch.cuda.synchronize()
+    return out
+
+
 def gpu_arm(args, rank, world):
     import torch
     import learned_bit_lut_any4_b200 as any4
@@ -362,6 +430,8 @@ def gpu_arm(args, rank, world):
             del g, reps, x, y
         torch.cuda.synchronize()
 
+    fig3 = fig3_square_sweep(stream, overlap) if not args.skip_fig3 else {}
+
     # end to end through the public API with host buffers: every step copies
     # each call's x from pinned host memory and reads each y back
     host_x = [torch.from_numpy(np.ascontiguousarray(hx).view(np.int16)).pin_memory()
@@ -398,7 +468,8 @@ def gpu_arm(args, rank, world):
 
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
-        "clocks": clocks, "detail": detail, "prefill": prefill, "batch": batch, "peaks": peaks,
+        "clocks": clocks, "detail": detail, "prefill": prefill, "batch": batch, "fig3": fig3,
+        "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -482,6 +553,8 @@ def main():
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the decode kernels without programmatic dependent launch")
     ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--skip-fig3", action="store_true",
+                    help="skip the square K = N sweep at M = 1 (any4 / nf4-style / int4 / bf16)")
     ap.add_argument("--skip-batch", action="store_true",
                     help="skip the per-shape timing of the M = 2..16 and 70B M = 8 shapes")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -536,6 +609,7 @@ def main():
             "detail_m1": r["detail"],
             "prefill_m2048": r["prefill"],
             "detail_batch": r["batch"],
+            "fig3_square_m1": r["fig3"],
         }
         print(json.dumps(line), flush=True)
     finally:
