@@ -433,21 +433,30 @@ def gpu_arm(args, rank, world):
     fig3 = fig3_square_sweep(stream, overlap) if not args.skip_fig3 else {}
 
     # end to end through the public API with host buffers: every step copies
-    # each call's x from pinned host memory and reads each y back
-    host_x = [torch.from_numpy(np.ascontiguousarray(hx).view(np.int16)).pin_memory()
-              for (_, _, _, _, hx) in sets]
-    host_y = [torch.empty((s.M, s.N), dtype=torch.int16).pin_memory() for (s, *_r) in sets]
-    dev_x = [torch.empty((s.M, s.K), dtype=torch.int16, device="cuda") for (s, *_r) in sets]
-    h2d = sum(t.numel() * 2 for t in host_x)
-    d2h = sum(t.numel() * 2 for t in host_y)
+    # the step's inputs (every call's x) from pinned host memory in one
+    # transfer and reads the step's results (every call's y) back in one
+    xs = [np.ascontiguousarray(hx).view(np.int16).reshape(-1) for (_, _, _, _, hx) in sets]
+    x_off = np.cumsum([0] + [a.size for a in xs])
+    host_x = torch.from_numpy(np.concatenate(xs)).pin_memory()
+    dev_x = torch.empty(host_x.numel(), dtype=torch.int16, device="cuda")
+    y_sizes = [s.M * s.N for (s, *_r) in sets]
+    y_off = np.cumsum([0] + y_sizes)
+    host_y = torch.empty(int(y_off[-1]), dtype=torch.int16).pin_memory()
+    dev_y = torch.empty(int(y_off[-1]), dtype=torch.int16, device="cuda")
+    x_views = [dev_x[x_off[i]:x_off[i + 1]].view(torch.bfloat16).view(s.M, s.K)
+               for i, (s, *_r) in enumerate(sets)]
+    y_views = [dev_y[y_off[i]:y_off[i + 1]].view(torch.bfloat16).view(s.M, s.N)
+               for i, (s, *_r) in enumerate(sets)]
+    h2d = host_x.numel() * 2
+    d2h = host_y.numel() * 2
     e2e_steps = max(copies, min(steps_timed, 400))
 
     def e2e_step(c):
-        for i, (s, reps, _x, y, _) in enumerate(sets):
-            dev_x[i].copy_(host_x[i], non_blocking=True)
+        dev_x.copy_(host_x, non_blocking=True)
+        for i, (s, reps, _x, _y, _) in enumerate(sets):
             w = reps[c % copies]
-            any4.any4_matmul(dev_x[i].view(torch.bfloat16), w[0], w[1], w[2], w[3], s.G, y=y)
-            host_y[i].copy_(y.view(torch.int16), non_blocking=True)
+            any4.any4_matmul(x_views[i], w[0], w[1], w[2], w[3], s.G, y=y_views[i])
+        host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for c in range(copies):

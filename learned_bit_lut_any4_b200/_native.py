@@ -93,6 +93,29 @@ def any4_bits_per_weight(K: int, G: int) -> float:
     return float(library().any4_bits_per_weight(K, G))
 
 
+# workspace bytes per (device, M, N, K, G, path), asked of the library once
+_WS_NEED: dict = {}
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NULL_CTX = _NullCtx()
+
+
+def _on_device(dev: torch.device):
+    """torch.cuda.device(dev), skipped when dev is already the current device
+    (the C entry points act on the current device)."""
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return _NULL_CTX
+    return torch.cuda.device(dev)
+
+
 def _check(status: int, where: str):
     if status != ANY4_OK:
         raise Any4Error(status, where)
@@ -164,7 +187,7 @@ def any4_dequant(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
     _need(W, "W", _BF16, dev)
     if scale.numel() != N * (K // G if G else 0) or offset.numel() != scale.numel():
         raise ValueError("scale and offset must hold N * K/G values")
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(library().any4_dequant(_ptr(packed), _ptr(lut), stride, _ptr(scale),
                                       _ptr(offset), _ptr(W), N, K, G, _stream(dev)),
                "any4_dequant")
@@ -206,7 +229,10 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
     _need(y, "y", _BF16, dev)
     lib = library()
     p = PATHS[path]
-    need = int(lib.any4_matmul_workspace_size_ex(M, N, K, G, p))
+    key = (dev.index, M, N, K, G, p)
+    need = _WS_NEED.get(key)
+    if need is None:
+        need = _WS_NEED[key] = int(lib.any4_matmul_workspace_size_ex(M, N, K, G, p))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0
@@ -215,7 +241,7 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
         ws_bytes = workspace.numel()
     if dev_status is not None:
         _need(dev_status, "dev_status", (torch.int32,), dev)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib.any4_matmul_ex(_ptr(x), _ptr(packed), _ptr(lut), stride, _ptr(scale),
                                   _ptr(offset), _ptr(y), M, N, K, G, _ptr(workspace), ws_bytes,
                                   _ptr(dev_status), p,
@@ -251,7 +277,7 @@ def any4_matmul_static_scratch(x: torch.Tensor, packed: torch.Tensor, lut: torch
     if dev_status is not None:
         _need(dev_status, "dev_status", (torch.int32,), dev)
     lib = library()
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib.any4_matmul_static_scratch(_ptr(x), _ptr(packed), _ptr(lut), stride,
                                               _ptr(scale), _ptr(offset), _ptr(y), M, N, K, G,
                                               _ptr(dev_status), _stream(dev)),

@@ -1,7 +1,9 @@
 // The C ABI of libany4: argument validation (before any CUDA call, so a bad
 // call launches nothing) and dispatch to the kernels.
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 
@@ -50,6 +52,25 @@ any4_status current_device(DeviceInfo* info) {
   if (g_dev[dev].cc_major != 10 || g_dev[dev].cc_minor != 0) st = ANY4_ERR_UNSUPPORTED;
   *info = g_dev[dev];
   return st;
+}
+
+int cached_occupancy(const void* kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const auto key = std::make_tuple(kernel, threads, smem, dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess)
+    return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = occ;
+  return occ;
 }
 
 }  // namespace any4

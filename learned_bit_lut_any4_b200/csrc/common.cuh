@@ -153,6 +153,12 @@ any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16
                           uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
                           cudaStream_t stream, const DeviceInfo& dev);
 
+// cudaOccupancyMaxActiveBlocksPerMultiprocessor, remembered per (kernel,
+// threads, dynamic shared memory) so that launches after the first of a shape
+// make no occupancy query (it costs microseconds of host time per call).
+// Returns 0 when the query fails.
+int cached_occupancy(const void* kernel, int threads, size_t smem);
+
 // Device address of the fixed scratch array of any4_matmul_static_scratch on
 // `device` (the current device); resolved on first use per device.
 any4_status static_scratch(int device, void** ptr);

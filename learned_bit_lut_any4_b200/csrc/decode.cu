@@ -336,12 +336,9 @@ any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
   const int per_warp = (nslices + kMaxWarps - 1) / kMaxWarps;
   const int nwarps = (nslices + per_warp - 1) / per_warp;
   const int threads = nwarps * 32;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MT, KL, P>, threads,
-                                                    (size_t)kMaxRowsMT * sizeof(float) * nwarps) !=
-          cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(decode_kernel<MT, KL, P>), threads,
+                                (size_t)kMaxRowsMT * sizeof(float) * nwarps);
+  if (per_sm < 1) per_sm = 1;
   // one wave: every resident block owns an equal contiguous range of rows
   const int64_t wave = (int64_t)dev.sm_count * per_sm;
   int64_t rt = (N + wave - 1) / wave;

@@ -457,11 +457,8 @@ any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lu
     rt = std::min<int64_t>((N + wave - 1) / wave, kMaxRT);
     rtp = ((rt + P - 1) / P) * P;
     const size_t smem_try = ring_bytes + (size_t)nwarps * rtp * sizeof(float);
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem_try) !=
-            cudaSuccess ||
-        occ < 1)
-      occ = 1;
+    int occ = cached_occupancy(reinterpret_cast<const void*>(kern), threads, smem_try);
+    if (occ < 1) occ = 1;
     if (occ == per_sm) break;
     per_sm = occ;
   }

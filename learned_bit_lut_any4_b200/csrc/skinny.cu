@@ -66,7 +66,10 @@ __device__ __forceinline__ void cp_async_wait() {
 //   table  [16 rows][32 bytes]        the tile rows' 16-entry tables
 //   so     [KC][2 halves][32 lanes][2][4 bytes]  per lane, chunk and row: the
 //                                     aligned 4-byte words holding the scale,
-//                                     then the offset, of the lane's group
+//                                     then the offset, of the lane's group; or,
+//                                     when the slice's groups fit one aligned
+//                                     8-group window, [16 rows][2][16 bytes]:
+//                                     that window of each row's scales, offsets
 template <int KC>
 struct SkStage {
   static constexpr int kCodes = 0;
@@ -102,6 +105,7 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
   const int64_t row_bytes = K / 2;
   const int groups = K / G;
   const int64_t so_elems = (int64_t)N * groups;  // elements of scale (and of offset)
+  const bool so_vec = (groups & 7) == 0 && (G & (G - 1)) == 0;
   constexpr int kSliceCols = 128 * KC;
   const bool shared_lut = lut_row_stride == 0;
   const int ring_bytes = kSkStages * SkStage<KC>::kBytes;
@@ -118,6 +122,11 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
   }
   bool first_slice = true;
   for (int s = warp; s < nslices; s += nwarps) {
+    // The slice's groups lie in one aligned window of 8 groups (16 bytes of a
+    // scale or offset row) when G is a power of two and every row holds a
+    // multiple of 8 groups: then a tile's scales and offsets are 32 such
+    // windows, one 16-byte copy per lane.
+    const int win = ((s * kSliceCols) / G) & ~7;
     // Per-slice constants of this lane: its column in each chunk, whether it
     // lies inside K, and its group index along the row.
     int colq[KC], gq[KC];
@@ -151,6 +160,7 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
           const bool in = rin && inq[c];
           cp_async16(sb + SkStage<KC>::kCodes + (uint32_t)(((c * 2 + h) * 32 + lane) * 16),
                      prow + (in ? colq[c] / 2 : 0), in ? 16u : 0u);
+          if (so_vec) continue;  // scales and offsets come as whole windows below
           const int64_t gi = srow + gq[c];
           const uint32_t dst = sb + SkStage<KC>::kSo + (uint32_t)(((c * 2 + h) * 32 + lane) * 8);
           if (lastq[c] && n == N - 1) {
@@ -164,6 +174,15 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
             cp_async4(dst + 4, offset + (gi & ~(int64_t)1), in ? 4u : 0u);
           }
         }
+      }
+      if (so_vec) {
+        // lane l: the 16-byte window (8 groups from `win`) of row l & 15 of the
+        // scales (l < 16) or the offsets (l >= 16)
+        const int i = lane & 15, tsr = lane >> 4;
+        const int n = n_base + 16 * t + i;
+        const bool rin = n < N && (i < 8 || upper);
+        cp_async16(sb + SkStage<KC>::kSo + (uint32_t)((i * 2 + tsr) * 16),
+                   (tsr ? offset : scale) + (int64_t)(rin ? n : 0) * groups + win, rin ? 16u : 0u);
       }
       if (!shared_lut) {
         const int trow = (q < 2 ? r : r + 8);
@@ -237,16 +256,26 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
       for (int c = 0; c < KC; ++c) {
         // the rows' group scale and offset sit in the half of the copied
         // 4-byte words given by the flat index's parity
-        const uint2 swA =
-            *reinterpret_cast<const uint2*>(sp + SkStage<KC>::kSo + ((c * 2 + 0) * 32 + lane) * 8);
-        const uint2 swB =
-            *reinterpret_cast<const uint2*>(sp + SkStage<KC>::kSo + ((c * 2 + 1) * 32 + lane) * 8);
-        const uint32_t shA = (uint32_t)((parA ^ gq[c]) & 1) * 16u;
-        const uint32_t shB = (uint32_t)((parB ^ gq[c]) & 1) * 16u;
-        const uint32_t sA = ((swA.x >> shA) & 0xFFFFu) * 0x10001u;
-        const uint32_t oA = ((swA.y >> shA) & 0xFFFFu) * 0x10001u;
-        const uint32_t sB = ((swB.x >> shB) & 0xFFFFu) * 0x10001u;
-        const uint32_t oB = ((swB.y >> shB) & 0xFFFFu) * 0x10001u;
+        uint32_t sA, oA, sB, oB;
+        if (so_vec) {
+          const uint16_t* wv = reinterpret_cast<const uint16_t*>(sp + SkStage<KC>::kSo);
+          const int gw = inq[c] ? gq[c] - win : 0;  // group within the window
+          sA = (uint32_t)wv[(r * 2 + 0) * 8 + gw] * 0x10001u;
+          oA = (uint32_t)wv[(r * 2 + 1) * 8 + gw] * 0x10001u;
+          sB = (uint32_t)wv[((r + 8) * 2 + 0) * 8 + gw] * 0x10001u;
+          oB = (uint32_t)wv[((r + 8) * 2 + 1) * 8 + gw] * 0x10001u;
+        } else {
+          const uint2 swA = *reinterpret_cast<const uint2*>(
+              sp + SkStage<KC>::kSo + ((c * 2 + 0) * 32 + lane) * 8);
+          const uint2 swB = *reinterpret_cast<const uint2*>(
+              sp + SkStage<KC>::kSo + ((c * 2 + 1) * 32 + lane) * 8);
+          const uint32_t shA = (uint32_t)((parA ^ gq[c]) & 1) * 16u;
+          const uint32_t shB = (uint32_t)((parB ^ gq[c]) & 1) * 16u;
+          sA = ((swA.x >> shA) & 0xFFFFu) * 0x10001u;
+          oA = ((swA.y >> shA) & 0xFFFFu) * 0x10001u;
+          sB = ((swB.x >> shB) & 0xFFFFu) * 0x10001u;
+          oB = ((swB.y >> shB) & 0xFFFFu) * 0x10001u;
+        }
         const uint4 qa =
             *reinterpret_cast<const uint4*>(sp + SkStage<KC>::kCodes + ((c * 2 + 0) * 32 + lane) * 16);
         const uint4 qb =
@@ -348,10 +377,8 @@ any4_status run_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t*
       rows_max = ((groups8 + grid - 1) / grid) * 8;
     }
     const size_t smem = ring_total + (size_t)nwarps * rows_max * M * sizeof(float);
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess ||
-        occ < 1)
-      occ = 1;
+    int occ = cached_occupancy(reinterpret_cast<const void*>(kern), threads, smem);
+    if (occ < 1) occ = 1;
     if (occ == per_sm) break;
     per_sm = occ;
   }
