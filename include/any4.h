@@ -190,8 +190,14 @@ ANY4_API any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t
                                                 int64_t G, int32_t* dev_status,
                                                 any4_stream_t stream);
 
-/* Bytes of workspace any4_matmul needs for this shape (0 if none).  Returns
- * 0 as well for shapes that break the shape rules (the call then fails). */
+/* Bytes of workspace any4_matmul needs for this shape (0 if none) to run its
+ * fastest kernel.  Returns 0 as well for shapes that break the shape rules
+ * (the call then fails).  On the prefill path at M >= 1024 the size includes
+ * room for the dequantised weights (N * K * 2 bytes): the call then runs in two
+ * passes (any4_dequant into the workspace, then a tensor-core GEMM that streams
+ * those bf16 weights).  A smaller workspace, down to the one-pass size (the
+ * size this function returns for M < 1024), runs the one-pass kernel, which
+ * dequantises the weights tile by tile. */
 ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 
 /* Same for an explicit path. */

@@ -9,6 +9,17 @@
 
 namespace any4 {
 
+// Two-pass prefill for large M (prefill.cu): the weights dequantised into the
+// workspace, then streamed to the tensor cores by TMA.
+bool prefill_use_two_pass(int64_t M, int64_t N, int64_t K);
+size_t prefill_two_pass_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                                    int64_t lut_row_stride, const uint16_t* scale,
+                                    const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                                    int64_t K, int64_t G, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status,
+                                    cudaStream_t stream, const DeviceInfo& dev);
+
 namespace {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -138,7 +149,9 @@ size_t any4_matmul_workspace_size_ex(int64_t M, int64_t N, int64_t K, int64_t G,
                                      any4_path path) {
   if (M < 1 || !shape_ok(N, K, G)) return 0;
   if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
-  if (path == ANY4_PATH_PREFILL) return prefill_workspace_size(M, N, K, G);
+  if (path == ANY4_PATH_PREFILL)
+    return prefill_use_two_pass(M, N, K) ? prefill_two_pass_workspace_size(M, N, K, G)
+                                         : prefill_workspace_size(M, N, K, G);
   return 0;
 }
 
@@ -163,7 +176,10 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
   if (flags & ~(uint32_t)ANY4_FLAG_OVERLAP_PRIOR) return ANY4_ERR_UNSUPPORTED;
   if (path == ANY4_PATH_DECODE && M > kDecodeMaxM) return ANY4_ERR_UNSUPPORTED;
-  const size_t need = any4_matmul_workspace_size_ex(M, N, K, G, path);
+  // the prefill path runs in one pass with at least prefill_workspace_size
+  // bytes, and in two passes (large M) when the workspace also holds the
+  // dequantised weights
+  const size_t need = path == ANY4_PATH_PREFILL ? prefill_workspace_size(M, N, K, G) : 0;
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return ANY4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ANY4_ERR_ALIGN;
@@ -176,6 +192,11 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
                          (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, dev_status, (cudaStream_t)stream,
                          dev);
   }
+  if (prefill_use_two_pass(M, N, K) &&
+      workspace_bytes >= prefill_two_pass_workspace_size(M, N, K, G))
+    return launch_prefill_two_pass(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
+                                   workspace, workspace_bytes, dev_status, (cudaStream_t)stream,
+                                   dev);
   return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
                         workspace_bytes, dev_status, (cudaStream_t)stream, dev);
 }

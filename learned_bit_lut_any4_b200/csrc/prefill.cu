@@ -206,8 +206,14 @@ __device__ __forceinline__ size_t partial_index(int blk, int tw, int chunk, int 
 }
 
 // ---------------------------------------------------------------- the kernel
+// kWTma = false: the dequant warps build each W tile from the packed codes
+// (one pass).  kWTma = true: W was dequantised to bf16 beforehand (any4_dequant
+// into the workspace) and warp 0 loads its tiles with TMA like the x tiles;
+// the dequant warps only run the epilogue (two passes, for large M).
+template <bool kWTma>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
-    const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
+    const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+    const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
     uint16_t* __restrict__ y, int M, int N, int K, int G, int vec_store, int32_t* dev_status,
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_a(s), 1);
-      mbar_init(full_b(s), kXformWarps);
+      mbar_init(full_b(s), kWTma ? 1 : kXformWarps);
       mbar_init(empty(s), 1);
     }
     mbar_init(accum_full, 1);
@@ -279,6 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
           mbar_arrive_expect_tx(full_a(s), kNAcc * kATileBytes);
           for (int h = 0; h < kNAcc; ++h)
             tma_load_2d(stage_a(s, h), &tmap_x, kb * kBK, mt * kNAcc * kBM + h * kBM, full_a(s));
+          if (kWTma) {
+            // the bf16 W tile: 256 weight rows x 64 columns, same swizzled layout
+            mbar_arrive_expect_tx(full_b(s), kBTileBytes);
+            tma_load_2d(stage_b(s), &tmap_w, kb * kBK, (tile / n_mtiles) * kBN, full_b(s));
+          }
         }
       }
     }
@@ -335,112 +346,114 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       const int nt = tile / n_mtiles;
       const int n = nt * kBN + rloc;
       const bool rin = n < N;
-      // The row's 16-entry table in registers, split into byte planes:
-      // tl[i] = low bytes of entries 4i..4i+3, th[i] = their high bytes.
-      uint32_t tl[4], th[4];
-      {
-        const uint16_t* lrow = lut + (int64_t)(rin ? n : 0) * lut_row_stride;
-        const uint4 e0 = rin ? ldg_nc_v4(lrow) : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 e1 = rin ? ldg_nc_v4(lrow + 8) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          tl[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x6420);
-          th[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x7531);
-        }
-      }
-      const uint8_t* prow = packed + (int64_t)(rin ? n : 0) * row_bytes;
-      // the even lane of a pair holds its row's scales, the odd lane its
-      // offsets, 8 groups per register quad
-      const uint16_t* grow = (half ? offset : scale) + (int64_t)(rin ? n : 0) * groups;
-      auto fetch_octet = [&](int o8) -> uint4 {
-        if (!rin || 8 * o8 >= groups) return make_uint4(0u, 0u, 0u, 0u);
-        if (oct_vec) return ldg_nc_v4(grow + 8 * o8);
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int g0 = 8 * o8 + 2 * i;
-          const uint32_t lo = g0 < groups ? ldg_u16(grow + g0) : 0u;
-          const uint32_t hi = g0 + 1 < groups ? ldg_u16(grow + g0 + 1) : 0u;
-          w[i] = lo | (hi << 16);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
-      };
-      // bf16 bits of group slot j (0..7) of an octet
-      auto pick = [](const uint4& v, int j) -> uint32_t {
-        const uint32_t w = (j & 4) ? ((j & 2) ? v.w : v.z) : ((j & 2) ? v.y : v.x);
-        return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
-      };
-
-      // This lane's 16 bytes of codes of a stage, fetched three stages ahead.
-      auto fetch = [&](int kb) -> uint4 {
-        const int k = kb * kBK + 32 * half;
-        return (rin && k < K) ? ldg_stream_v4(prow + k / 2) : make_uint4(0u, 0u, 0u, 0u);
-      };
-      int cur8 = (kb0 * kBK) / G >> 3;
-      uint4 oct_cur = fetch_octet(cur8), oct_nxt = fetch_octet(cur8 + 1);
-      // Dequantise this lane's half of one stage of its row into the B tile.
-      auto xform = [&](int kb, const uint4& q) -> bool {
-        const int s = (int)(it % kStages);
-        const uint32_t ph = (it / kStages) & 1u;
-        ++it;
-        // this lane's group and its partner's (the other half of the row)
-        const int g = (kb * kBK + 32 * half) / G;
-        const int gp = (kb * kBK + 32 * (half ^ 1)) / G;
-        if ((g >> 3) != cur8) {  // both lanes of a pair enter a new octet together
-          cur8 = g >> 3;
-          oct_cur = oct_nxt;
-          oct_nxt = fetch_octet(cur8 + 1);
-        }
-        const uint32_t mine = pick(oct_cur, g & 7);
-        const uint32_t other = __shfl_xor_sync(0xffffffffu, pick(oct_cur, gp & 7), 1);
-        // scale and offset as bf16 pairs (both columns of a pair share a group)
-        const uint32_t s2 = (half ? other : mine) * 0x10001u;
-        const uint32_t o2 = (half ? mine : other) * 0x10001u;
-        if (!mbar_wait_warp(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
-        const uint32_t brow = stage_b(s) + (uint32_t)rloc * 128u;
-        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // the 8 codes of word j (columns k + 8j .. k + 8j + 7), looked up 4 at a time
-          uint32_t lut_pair[4];
-          lookup8(words[j], tl, th, lut_pair);
-          uint32_t out[4];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            // W' = LUT * scale + offset for both codes of the pair with one bf16x2
-            // fused multiply-add (the exact value rounded once to bf16)
-            asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out[p]) : "r"(lut_pair[p]), "r"(s2), "r"(o2));
+      if constexpr (!kWTma) {
+        // The row's 16-entry table in registers, split into byte planes:
+        // tl[i] = low bytes of entries 4i..4i+3, th[i] = their high bytes.
+        uint32_t tl[4], th[4];
+        {
+          const uint16_t* lrow = lut + (int64_t)(rin ? n : 0) * lut_row_stride;
+          const uint4 e0 = rin ? ldg_nc_v4(lrow) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 e1 = rin ? ldg_nc_v4(lrow + 8) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t e[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            tl[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x6420);
+            th[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x7531);
           }
-          // 16-byte chunk (4 half + j) of the 128-byte row, 128-byte swizzle
-          const uint32_t chunk = (uint32_t)((4 * half + j) ^ (rloc & 7));
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
-                       :: "r"(brow + chunk * 16u), "r"(out[0]), "r"(out[1]), "r"(out[2]),
-                          "r"(out[3]) : "memory");
         }
-        fence_proxy_async_smem();  // make the generic-proxy stores visible to the MMA
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full_b(s));
-        return true;
-      };
+        const uint8_t* prow = packed + (int64_t)(rin ? n : 0) * row_bytes;
+        // the even lane of a pair holds its row's scales, the odd lane its
+        // offsets, 8 groups per register quad
+        const uint16_t* grow = (half ? offset : scale) + (int64_t)(rin ? n : 0) * groups;
+        auto fetch_octet = [&](int o8) -> uint4 {
+          if (!rin || 8 * o8 >= groups) return make_uint4(0u, 0u, 0u, 0u);
+          if (oct_vec) return ldg_nc_v4(grow + 8 * o8);
+          uint32_t w[4];
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int g0 = 8 * o8 + 2 * i;
+            const uint32_t lo = g0 < groups ? ldg_u16(grow + g0) : 0u;
+            const uint32_t hi = g0 + 1 < groups ? ldg_u16(grow + g0 + 1) : 0u;
+            w[i] = lo | (hi << 16);
+          }
+          return make_uint4(w[0], w[1], w[2], w[3]);
+        };
+        // bf16 bits of group slot j (0..7) of an octet
+        auto pick = [](const uint4& v, int j) -> uint32_t {
+          const uint32_t w = (j & 4) ? ((j & 2) ? v.w : v.z) : ((j & 2) ? v.y : v.x);
+          return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+        };
 
-      uint4 pa = fetch(kb0), pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
-      if (kb0 + 1 < kb1) pb = fetch(kb0 + 1);
-      if (kb0 + 2 < kb1) pc = fetch(kb0 + 2);
-      bool alive = true;
-      for (int kb = kb0; kb < kb1 && alive; kb += 3) {
-        alive = xform(kb, pa);
-        if (alive && kb + 3 < kb1) pa = fetch(kb + 3);
-        if (alive && kb + 1 < kb1) {
-          alive = xform(kb + 1, pb);
-          if (alive && kb + 4 < kb1) pb = fetch(kb + 4);
+        // This lane's 16 bytes of codes of a stage, fetched three stages ahead.
+        auto fetch = [&](int kb) -> uint4 {
+          const int k = kb * kBK + 32 * half;
+          return (rin && k < K) ? ldg_stream_v4(prow + k / 2) : make_uint4(0u, 0u, 0u, 0u);
+        };
+        int cur8 = (kb0 * kBK) / G >> 3;
+        uint4 oct_cur = fetch_octet(cur8), oct_nxt = fetch_octet(cur8 + 1);
+        // Dequantise this lane's half of one stage of its row into the B tile.
+        auto xform = [&](int kb, const uint4& q) -> bool {
+          const int s = (int)(it % kStages);
+          const uint32_t ph = (it / kStages) & 1u;
+          ++it;
+          // this lane's group and its partner's (the other half of the row)
+          const int g = (kb * kBK + 32 * half) / G;
+          const int gp = (kb * kBK + 32 * (half ^ 1)) / G;
+          if ((g >> 3) != cur8) {  // both lanes of a pair enter a new octet together
+            cur8 = g >> 3;
+            oct_cur = oct_nxt;
+            oct_nxt = fetch_octet(cur8 + 1);
+          }
+          const uint32_t mine = pick(oct_cur, g & 7);
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, pick(oct_cur, gp & 7), 1);
+          // scale and offset as bf16 pairs (both columns of a pair share a group)
+          const uint32_t s2 = (half ? other : mine) * 0x10001u;
+          const uint32_t o2 = (half ? mine : other) * 0x10001u;
+          if (!mbar_wait_warp(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
+          const uint32_t brow = stage_b(s) + (uint32_t)rloc * 128u;
+          const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // the 8 codes of word j (columns k + 8j .. k + 8j + 7), looked up 4 at a time
+            uint32_t lut_pair[4];
+            lookup8(words[j], tl, th, lut_pair);
+            uint32_t out[4];
+  #pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              // W' = LUT * scale + offset for both codes of the pair with one bf16x2
+              // fused multiply-add (the exact value rounded once to bf16)
+              asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out[p]) : "r"(lut_pair[p]), "r"(s2), "r"(o2));
+            }
+            // 16-byte chunk (4 half + j) of the 128-byte row, 128-byte swizzle
+            const uint32_t chunk = (uint32_t)((4 * half + j) ^ (rloc & 7));
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
+                         :: "r"(brow + chunk * 16u), "r"(out[0]), "r"(out[1]), "r"(out[2]),
+                            "r"(out[3]) : "memory");
+          }
+          fence_proxy_async_smem();  // make the generic-proxy stores visible to the MMA
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_b(s));
+          return true;
+        };
+
+        uint4 pa = fetch(kb0), pb = make_uint4(0u, 0u, 0u, 0u), pc = pb;
+        if (kb0 + 1 < kb1) pb = fetch(kb0 + 1);
+        if (kb0 + 2 < kb1) pc = fetch(kb0 + 2);
+        bool alive = true;
+        for (int kb = kb0; kb < kb1 && alive; kb += 3) {
+          alive = xform(kb, pa);
+          if (alive && kb + 3 < kb1) pa = fetch(kb + 3);
+          if (alive && kb + 1 < kb1) {
+            alive = xform(kb + 1, pb);
+            if (alive && kb + 4 < kb1) pb = fetch(kb + 4);
+          }
+          if (alive && kb + 2 < kb1) {
+            alive = xform(kb + 2, pc);
+            if (alive && kb + 5 < kb1) pc = fetch(kb + 5);
+          }
         }
-        if (alive && kb + 2 < kb1) {
-          alive = xform(kb + 2, pc);
-          if (alive && kb + 5 < kb1) pc = fetch(kb + 5);
-        }
+        if (!alive) goto done;
       }
-      if (!alive) goto done;
 
       // epilogue: TMEM -> registers; then either this segment's fp32 partial
       // sums go to the workspace (a segment that does not start the tile), or
@@ -592,31 +605,51 @@ size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G) {
   return slots * (size_t)(kNAcc * kBM) * kBN * sizeof(float) + ((slots * 4 + 255) / 256) * 256;
 }
 
-any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
-                           int64_t lut_row_stride, const uint16_t* scale,
-                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
-                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
-                           int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+namespace {
+
+// Shared launcher of both kernel modes; w_bf16 is the dequantised weight
+// matrix (kWTma) or unused.
+template <bool kWTma>
+any4_status launch_prefill_impl(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                                int64_t lut_row_stride, const uint16_t* scale,
+                                const uint16_t* offset, const uint16_t* w_bf16, uint16_t* y,
+                                int64_t M, int64_t N, int64_t K, int64_t G, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream,
+                                const DeviceInfo& dev) {
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   if (dev.smem_optin < (size_t)kSmemAlloc) return ANY4_ERR_UNSUPPORTED;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return ANY4_ERR_UNSUPPORTED;
 
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+  // x [M][K] in 128 x 64 boxes; W [N][K] (bf16, two-pass mode) in 256 x 64
+  // boxes; both 128-byte swizzled, the layout the MMA descriptors read
+  CUtensorMap map, map_w;
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
-          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return ANY4_ERR_CUDA;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ANY4_ERR_CUDA;
+  }
+  map_w = map;
+  if (kWTma) {
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBN};
+    if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(w_bf16), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ANY4_ERR_CUDA;
+  }
 
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kSmemAlloc);
+    attr_err = cudaFuncSetAttribute(prefill_kernel<kWTma>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return ANY4_ERR_CUDA;
 
@@ -647,11 +680,52 @@ any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint1
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, prefill_kernel, map, packed, lut, lut_row_stride, scale, offset, y,
-                         (int)M, (int)N, (int)K, (int)G, vec_store, dev_status, ws_partial,
-                         ws_flags) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, prefill_kernel<kWTma>, map, map_w, packed, lut, lut_row_stride,
+                         scale, offset, y, (int)M, (int)N, (int)K, (int)G, vec_store, dev_status,
+                         ws_partial, ws_flags) != cudaSuccess)
     return ANY4_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+}  // namespace
+
+any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                           int64_t lut_row_stride, const uint16_t* scale,
+                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_prefill_impl<false>(x, packed, lut, lut_row_stride, scale, offset, nullptr, y, M,
+                                    N, K, G, workspace, workspace_bytes, dev_status, stream, dev);
+}
+
+// Two passes for large M: the weights are dequantised once into the
+// workspace (bf16, bit-exact with any4_dequant) and the tensor-core kernel
+// streams them with TMA, so every weight is dequantised once instead of once
+// per 256 rows of x.
+bool prefill_use_two_pass(int64_t M, int64_t N, int64_t K) {
+  (void)N; (void)K;
+  return M >= 1024;
+}
+
+size_t prefill_two_pass_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G) {
+  return prefill_workspace_size(M, N, K, G) + (((size_t)N * K * 2 + 255) / 256) * 256;
+}
+
+any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                                    int64_t lut_row_stride, const uint16_t* scale,
+                                    const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
+                                    int64_t K, int64_t G, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status,
+                                    cudaStream_t stream, const DeviceInfo& dev) {
+  if (workspace == nullptr || workspace_bytes < prefill_two_pass_workspace_size(M, N, K, G))
+    return ANY4_ERR_WORKSPACE;
+  const size_t fused = prefill_workspace_size(M, N, K, G);
+  uint16_t* w = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + fused);
+  any4_status st = launch_dequant(packed, lut, lut_row_stride, scale, offset, w, N, K, G, stream,
+                                  dev);
+  if (st != ANY4_OK) return st;
+  return launch_prefill_impl<true>(x, packed, lut, lut_row_stride, scale, offset, w, y, M, N, K, G,
+                                   workspace, fused, dev_status, stream, dev);
 }
 
 }  // namespace any4

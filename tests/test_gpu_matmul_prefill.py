@@ -108,3 +108,23 @@ def test_prefill_deterministic_and_shared_table():
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, table, p.scale, p.offset, shape.G,
                                per_tensor_lut=True)
     assert_matmul_close(host_bits(y1), y_ref, "shared")
+
+
+def test_prefill_one_pass_with_small_workspace():
+    """At M >= 1024 the full workspace selects the two-pass kernel (weights
+    dequantised into it first); a workspace of only the one-pass size must
+    run the one-pass kernel instead, with the same accuracy."""
+    shape = workloads.Shape("pf_onepass", 1024, 2048, 1100, 128, 9971, 9972)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    one_pass = any4.any4_matmul_workspace_size(300, shape.N, shape.K, shape.G)
+    full = any4.any4_matmul_workspace_size(shape.M, shape.N, shape.K, shape.G)
+    assert full >= one_pass + shape.N * shape.K * 2
+    ws = torch.empty(one_pass, dtype=torch.uint8, device="cuda")
+    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, workspace=ws,
+                          path="prefill")
+    y2 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path="prefill")
+    torch.cuda.synchronize()
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+    assert_matmul_close(host_bits(y1), y_ref, "one pass")
+    assert_matmul_close(host_bits(y2), y_ref, "two passes")
