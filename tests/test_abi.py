@@ -106,6 +106,21 @@ def test_workspace_size_of_bad_shapes_is_zero():
     assert any4.any4_matmul_workspace_size(0, 64, 64, 32) == 0
 
 
+def test_workspace_sizes_by_path():
+    """Decode needs no workspace; prefill below M = 1024 needs the one-pass
+    stream-K scratch (independent of the shape); from M = 1024 the size adds
+    room for the dequantised bf16 weights, N * K * 2 bytes rounded to 256."""
+    N, K, G = 1100, 2048, 128
+    assert any4.any4_matmul_workspace_size(16, N, K, G) == 0
+    one = any4.any4_matmul_workspace_size(17, N, K, G)
+    assert one > 0 and one == any4.any4_matmul_workspace_size(1023, N, K, G)
+    assert one == any4.any4_matmul_workspace_size(300, 64, 64, 32)
+    two = any4.any4_matmul_workspace_size(1024, N, K, G)
+    assert two - one == ((N * K * 2 + 255) // 256) * 256
+    # an explicit prefill path at small M still uses the one-pass size
+    assert any4.any4_matmul_workspace_size(4, N, K, G, path="prefill") == one
+
+
 def test_path_choice():
     assert any4.any4_matmul_choose_path(1, 4096, 4096, 128) == "decode"
     assert any4.any4_matmul_choose_path(16, 4096, 4096, 128) == "decode"
