@@ -128,3 +128,23 @@ def test_prefill_one_pass_with_small_workspace():
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     assert_matmul_close(host_bits(y1), y_ref, "one pass")
     assert_matmul_close(host_bits(y2), y_ref, "two passes")
+
+
+@pytest.mark.parametrize("M,K,N,G,shared", [(1030, 1056, 777, 32, False),
+                                            (1024, 2080, 300, 32, True),
+                                            (1500, 1024, 513, 64, False)])
+def test_prefill_two_pass_edges(M, K, N, G, shared):
+    """The two-pass kernel (M >= 1024, full workspace) with a ragged last
+    K stage (K % 64 == 32), ragged M and N, the one-table mode and G = 32."""
+    shape = workloads.Shape(f"pf2_{M}_{K}_{N}", M, K, N, G, 9981 + N, 9982 + M)
+    p = workloads.make(shape)
+    d = DeviceProblem(p)
+    lut = p.lut[7 % N].copy() if shared else p.lut
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = any4.any4_matmul(d.x, d.packed, dev_bf16(lut), d.scale, d.offset, shape.G,
+                         path="prefill", dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    y_ref = oracle.any4_matmul(p.x, d.packed_ref, lut, p.scale, p.offset, shape.G,
+                               per_tensor_lut=shared)
+    assert_matmul_close(host_bits(y), y_ref, shape.name)
