@@ -13,6 +13,12 @@ Every function follows "any4: Learned 4-bit Numeric Representation for LLMs"
                      §2.5.1 group k covers columns k*G .. (k+1)*G-1
   matmul             §4.1 Eq. 8 and §4.2 (y = x W^T, x is M x K, W is N x K)
   bits_per_weight    §2.4.1 storage accounting (4.3125 bits at G=128, K=4096)
+  group_scale        §2.5.1 Eq. 1-2 (alpha = (max - min) / 15, beta = min)
+  scaled_weights     §2.5.1 Eq. 1 (w_S = (w - beta) / alpha)
+  kmeans_row         §4.1 E-step (Eq. 18) and M-step (Eq. 23), weighted Lloyd
+                     iteration from a quantile initialisation
+  quantize           §4.1 and Appendix A.1 (Alg. 1): scaling, then k-means per
+                     row with sample weight alpha * E|x|; bf16 table and codes
 
 bf16 values cross this interface as their raw uint16 bit patterns.  The
 arithmetic lives in any4_oracle.c (fp32 fmaf + IEEE round-to-nearest-even to
@@ -64,6 +70,15 @@ def _bind(lib):
     lib.oracle_matmul_rows.argtypes = [u16p, u8p, u16p, i64, u16p, u16p, i64p, i64,
                                        f64p, u16p, i64, i64, i64, i64]
     lib.oracle_matmul_rows.restype = None
+    lib.oracle_group_scale.argtypes = [u16p, i64, i64, i64, u16p, u16p]
+    lib.oracle_group_scale.restype = None
+    lib.oracle_scaled_weights.argtypes = [u16p, u16p, u16p, i64, i64, i64, f64p]
+    lib.oracle_scaled_weights.restype = None
+    lib.oracle_kmeans_row.argtypes = [f64p, f64p, i64, i64, f64p, u8p]
+    lib.oracle_kmeans_row.restype = i64
+    lib.oracle_any4_quantize.argtypes = [u16p, f32p, i64, i64, i64, i64, u8p, u16p, u16p, u16p,
+                                         i64p]
+    lib.oracle_any4_quantize.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -233,6 +248,84 @@ def any4_matmul(x, packed, lut, scale, offset, G: int, per_tensor_lut: bool = Fa
     return matmul(x, dequant(packed, lut, scale, offset, G, per_tensor_lut))
 
 
+def _check_weight(w, G):
+    w = _c(w, np.uint16)
+    if w.ndim != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    if N < 1 or K < 1 or G < 1 or K % G:
+        raise ValueError("need N, K, G >= 1 and K a multiple of G")
+    return w, N, K
+
+
+def group_scale(w, G: int):
+    """§2.5.1 Eq. 1-2 per group of G columns: (scale, offset) as bf16 bits [N, K/G],
+    scale = bf16((max - min) / 15 in fp32), offset = min."""
+    w, N, K = _check_weight(w, G)
+    scale = np.empty((N, K // G), dtype=np.uint16)
+    offset = np.empty((N, K // G), dtype=np.uint16)
+    _load().oracle_group_scale(_ptr(w, ctypes.c_uint16), N, K, G, _ptr(scale, ctypes.c_uint16),
+                               _ptr(offset, ctypes.c_uint16))
+    return scale, offset
+
+
+def scaled_weights(w, scale, offset, G: int):
+    """fp64 w_S = (w - offset) / scale [N, K] (0 in a group whose scale is 0)."""
+    w, N, K = _check_weight(w, G)
+    scale = _c(scale, np.uint16)
+    offset = _c(offset, np.uint16)
+    if scale.shape != (N, K // G) or offset.shape != (N, K // G):
+        raise ValueError("scale/offset must be [N, K/G]")
+    ws = np.empty((N, K), dtype=np.float64)
+    _load().oracle_scaled_weights(_ptr(w, ctypes.c_uint16), _ptr(scale, ctypes.c_uint16),
+                                  _ptr(offset, ctypes.c_uint16), N, K, G,
+                                  _ptr(ws, ctypes.c_double))
+    return ws
+
+
+def kmeans_row(xs, u, max_iter: int):
+    """Weighted Lloyd iteration (§4.1 Eq. 18 / Eq. 23) on one row from the
+    quantile initialisation: (fp64 centroids [16], codes uint8 [K], M-steps run)."""
+    xs = _c(xs, np.float64)
+    u = _c(u, np.float64)
+    if xs.ndim != 1 or u.shape != xs.shape or xs.size < 1:
+        raise ValueError("xs and u must be equal-length non-empty vectors")
+    if max_iter < 0:
+        raise ValueError("max_iter must be >= 0")
+    c = np.empty(16, dtype=np.float64)
+    code = np.empty(xs.size, dtype=np.uint8)
+    it = _load().oracle_kmeans_row(_ptr(xs, ctypes.c_double), _ptr(u, ctypes.c_double), xs.size,
+                                   int(max_iter), _ptr(c, ctypes.c_double),
+                                   _ptr(code, ctypes.c_uint8))
+    return c, code, int(it)
+
+
+def quantize(w, ex, G: int, max_iter: int):
+    """The whole any4 quantiser (§2.5.1 scaling, then §4.1 weighted k-means per
+    row): w bf16 bits [N, K], ex = E|x| fp32 [K] (finite, >= 0).
+
+    Returns (codes uint8 [N, K], lut bf16 bits [N, 16], scale [N, K/G],
+    offset [N, K/G], iters int64 [N])."""
+    w, N, K = _check_weight(w, G)
+    ex = _c(ex, np.float32)
+    if ex.shape != (K,):
+        raise ValueError("ex must be [K]")
+    if not np.all(np.isfinite(ex)) or np.any(ex < 0):
+        raise ValueError("ex must be finite and >= 0")
+    if max_iter < 0:
+        raise ValueError("max_iter must be >= 0")
+    codes = np.empty((N, K), dtype=np.uint8)
+    lut = np.empty((N, 16), dtype=np.uint16)
+    scale = np.empty((N, K // G), dtype=np.uint16)
+    offset = np.empty((N, K // G), dtype=np.uint16)
+    iters = np.empty(N, dtype=np.int64)
+    _load().oracle_any4_quantize(_ptr(w, ctypes.c_uint16), _ptr(ex, ctypes.c_float), N, K, G,
+                                 int(max_iter), _ptr(codes, ctypes.c_uint8),
+                                 _ptr(lut, ctypes.c_uint16), _ptr(scale, ctypes.c_uint16),
+                                 _ptr(offset, ctypes.c_uint16), _ptr(iters, ctypes.c_int64))
+    return codes, lut, scale, offset, iters
+
+
 __all__ = ["bf16_rne", "bf16_to_f32", "pack", "unpack", "bits_per_weight", "dequant_one",
            "dequant", "matmul", "matmul_rows", "any4_matmul", "num_threads",
-           "set_num_threads"]
+           "set_num_threads", "group_scale", "scaled_weights", "kmeans_row", "quantize"]

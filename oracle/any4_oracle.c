@@ -35,6 +35,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ------------------------------------------------------------------------- */
@@ -214,3 +215,155 @@ void oracle_set_num_threads(int t) { omp_set_num_threads(t); }
 int oracle_num_threads(void) { return 1; }
 void oracle_set_num_threads(int t) { (void)t; }
 #endif
+
+/* ------------------------------------------------------------------------- */
+/* Learning the table of each row.
+ *
+ * Follows the quantisation procedure of the same paper:
+ *   - §2.5.1 Eq. 1-2: per group of G columns, alpha = (max - min) / (Qmax - Qmin)
+ *     with Qmax - Qmin = 15 for 4 bits, beta = min, and the scaled weight
+ *     w_S = (w - beta) / alpha;
+ *   - §4.1 E-step (Eq. 18): each scaled weight takes the nearest table entry;
+ *   - §4.1 M-step (Eq. 23): each entry becomes the mean of its cluster's
+ *     scaled weights, weighted by alpha_{i,j} * E|x_j|;
+ *   - §4.1 / Appendix A.1 (Alg. 1): rows are independent; the steps
+ *     alternate until the table stops changing.
+ * Readings where the pages leave a step open:
+ *   - w is bf16 (its -0 is read as +0); E|x_j| is fp32, >= 0, one per column.
+ *   - alpha is the bf16 rounding of the fp32 quotient (max - min) / 15 (both
+ *     fp32 operations correctly rounded) and beta = min (exact in bf16); the
+ *     k-means runs on w_S formed with these stored values, in fp64:
+ *     w_S = ((double)w - beta) / alpha, or 0 for every column of a group
+ *     whose stored alpha is 0.
+ *   - Sample weight u_j = alpha_{g(j)} * E|x_j| in fp64 (exact: 8 x 24 bits).
+ *   - Initial table: the quantiles of the row's sorted w_S, entry q at
+ *     position floor(q (K - 1) / 15) (deterministic; scikit-learn's k-means++
+ *     seeding draws random numbers).
+ *   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q.
+ *   - M-step: numerator and denominator summed in fp64 over ascending column
+ *     index, each product rounded before its add; a cluster whose weights
+ *     sum to 0 (empty, or all weights 0) keeps its entry.
+ *   - Stop after max_iter M-steps, or as soon as an E-step changes no code.
+ *   - Table: LUT_q = bf16_rne((float)c_q); the returned codes are a final
+ *     E-step against these stored bf16 entries (the values dequant uses).
+ */
+
+static float canon_bf16(uint16_t h) { return oracle_bf16_to_f32(h) + 0.0f; }
+
+/* Eq. 1-2 on every group: scale = bf16(alpha), offset = bf16(beta) = min. */
+void oracle_group_scale(const uint16_t* w, int64_t N, int64_t K, int64_t G, uint16_t* scale,
+                        uint16_t* offset) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < K / G; ++g) {
+      float mn = canon_bf16(w[n * K + g * G]);
+      float mx = mn;
+      for (int64_t k = g * G; k < (g + 1) * G; ++k) {
+        float v = canon_bf16(w[n * K + k]);
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+      }
+      float alpha = (mx - mn) / 15.0f;
+      scale[n * (K / G) + g] = oracle_bf16_rne(alpha);
+      offset[n * (K / G) + g] = oracle_bf16_rne(mn);
+    }
+  }
+}
+
+/* w_S = (w - beta) / alpha for one row, with the stored bf16 alpha and beta
+ * (0 where alpha is 0). */
+static void scaled_row(const uint16_t* w, const uint16_t* scale, const uint16_t* offset,
+                       int64_t K, int64_t G, double* ws) {
+  for (int64_t k = 0; k < K; ++k) {
+    double alpha = (double)oracle_bf16_to_f32(scale[k / G]);
+    double beta = (double)oracle_bf16_to_f32(offset[k / G]);
+    ws[k] = alpha > 0.0 ? ((double)canon_bf16(w[k]) - beta) / alpha : 0.0;
+  }
+}
+
+void oracle_scaled_weights(const uint16_t* w, const uint16_t* scale, const uint16_t* offset,
+                           int64_t N, int64_t K, int64_t G, double* ws) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    scaled_row(w + n * K, scale + n * (K / G), offset + n * (K / G), K, G, ws + n * K);
+}
+
+static int cmp_double(const void* a, const void* b) {
+  double x = *(const double*)a, y = *(const double*)b;
+  return (x > y) - (x < y);
+}
+
+/* E-step (Eq. 18): nearest of the 16 entries, ties to the lowest index.
+ * Returns how many codes changed. */
+static int64_t assign_nearest(const double* xs, int64_t K, const double* c, uint8_t* code) {
+  int64_t changed = 0;
+  for (int64_t j = 0; j < K; ++j) {
+    int best_q = 0;
+    double best = fabs(xs[j] - c[0]);
+    for (int q = 1; q < 16; ++q) {
+      double d = fabs(xs[j] - c[q]);
+      if (d < best) {
+        best = d;
+        best_q = q;
+      }
+    }
+    if (code[j] != (uint8_t)best_q) ++changed;
+    code[j] = (uint8_t)best_q;
+  }
+  return changed;
+}
+
+/* Weighted Lloyd iteration on one row: samples xs[0..K), weights u[0..K).
+ * Out: c[16] (fp64 centroids) and code[K] (the E-step matching c).  Returns
+ * the number of M-steps run. */
+int64_t oracle_kmeans_row(const double* xs, const double* u, int64_t K, int64_t max_iter,
+                          double* c, uint8_t* code) {
+  double* sorted = (double*)malloc((size_t)K * sizeof(double));
+  memcpy(sorted, xs, (size_t)K * sizeof(double));
+  qsort(sorted, (size_t)K, sizeof(double), cmp_double);
+  for (int q = 0; q < 16; ++q) c[q] = sorted[(q * (K - 1)) / 15];
+  free(sorted);
+
+  memset(code, 0, (size_t)K);
+  assign_nearest(xs, K, c, code);
+  int64_t it = 0;
+  while (it < max_iter) {
+    double num[16], den[16];
+    for (int q = 0; q < 16; ++q) num[q] = den[q] = 0.0;
+    for (int64_t j = 0; j < K; ++j) {           /* M-step (Eq. 23) */
+      num[code[j]] += u[j] * xs[j];
+      den[code[j]] += u[j];
+    }
+    for (int q = 0; q < 16; ++q)
+      if (den[q] > 0.0) c[q] = num[q] / den[q];
+    ++it;
+    if (assign_nearest(xs, K, c, code) == 0) break;
+  }
+  return it;
+}
+
+/* The whole quantiser for an [N][K] bf16 weight: scale, offset, LUT and codes.
+ * iters[n] (may be NULL) receives the M-steps run on row n. */
+void oracle_any4_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
+                          int64_t max_iter, uint8_t* code, uint16_t* lut, uint16_t* scale,
+                          uint16_t* offset, int64_t* iters) {
+  oracle_group_scale(w, N, K, G, scale, offset);
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t n = 0; n < N; ++n) {
+    double* xs = (double*)malloc((size_t)K * sizeof(double));
+    double* u = (double*)malloc((size_t)K * sizeof(double));
+    scaled_row(w + n * K, scale + n * (K / G), offset + n * (K / G), K, G, xs);
+    for (int64_t k = 0; k < K; ++k)
+      u[k] = (double)oracle_bf16_to_f32(scale[n * (K / G) + k / G]) * (double)ex[k];
+    double c[16], table[16];
+    int64_t it = oracle_kmeans_row(xs, u, K, max_iter, c, code + n * K);
+    if (iters) iters[n] = it;
+    for (int q = 0; q < 16; ++q) {
+      lut[n * 16 + q] = oracle_bf16_rne((float)c[q]);
+      table[q] = (double)oracle_bf16_to_f32(lut[n * 16 + q]);
+    }
+    assign_nearest(xs, K, table, code + n * K);
+    free(xs);
+    free(u);
+  }
+}

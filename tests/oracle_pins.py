@@ -416,4 +416,243 @@ def pin_matmul_rows_equals_full():
     assert np.array_equal(part, full[:, rows])
 
 
+# --------------------------------------------------------------------------
+# learning the table: §2.5.1 Eq. 1-2 scaling, §4.1 E-step (Eq. 18) and M-step
+# (Eq. 23), Appendix A.1 Alg. 1 (k-means per row, sample weight alpha * E|x|)
+# --------------------------------------------------------------------------
+
+def _quantile_init(xs):
+    """The initial table read from the pages: entry q is the element at
+    position floor(q (K - 1) / 15) of the row sorted by numpy."""
+    s = np.sort(np.asarray(xs, dtype=np.float64))
+    return s[[(q * (xs.size - 1)) // 15 for q in range(16)]]
+
+
+def _nearest(xs, table):
+    """Eq. 18 by brute force: numpy's argmin returns the first (lowest) index on a tie."""
+    return np.argmin(np.abs(xs[:, None] - table[None, :]), axis=1).astype(np.uint8)
+
+
+def _numpy_scale(w_bits, G):
+    """Eq. 1-2 with numpy fp32 (each operation correctly rounded) and torch's bf16 rounding."""
+    N, K = w_bits.shape
+    wf = torch_bf16_to_f64(w_bits).astype(np.float32).reshape(N, K // G, G) + np.float32(0)
+    mn, mx = wf.min(axis=2), wf.max(axis=2)
+    return torch_bf16_bits((mx - mn) / np.float32(15)), torch_bf16_bits(mn)
+
+
+def _sklearn_kmeans(xs, u, max_iter=500):
+    """scikit-learn's weighted Lloyd k-means (the library Appendix C.2 names),
+    started from the quantile table."""
+    from sklearn.cluster import KMeans
+    km = KMeans(n_clusters=16, init=_quantile_init(xs)[:, None], n_init=1, max_iter=max_iter,
+                tol=0.0, algorithm="lloyd").fit(xs[:, None], sample_weight=u)
+    return km.cluster_centers_[:, 0], km.labels_.astype(np.uint8)
+
+
+def _levels_problem(rng, N, K, G, levels):
+    """Groups holding exactly beta_g + alpha_g * levels (each level G/16 times,
+    shuffled), alpha_g a power of two: every value is exact in bf16."""
+    w = np.empty((N, K), dtype=np.float64)
+    for n in range(N):
+        for g in range(K // G):
+            alpha = 2.0 ** -(5 + (n + g) % 3)
+            beta = -(1 + (n * 7 + g) % 5) / 32.0
+            vals = beta + alpha * np.repeat(levels, G // 16)
+            w[n, g * G:(g + 1) * G] = rng.permutation(vals)
+    bits = torch_bf16_bits(w.astype(np.float32))
+    assert np.array_equal(torch_bf16_to_f64(bits), w), "levels not exact in bf16"
+    return bits
+
+
+def pin_group_scale_closed_form():
+    rng = np.random.default_rng(101)
+    N, K, G = 6, 256, 64
+    w = random_bf16(rng, (N, K), lo_exp=-9, hi_exp=-3)
+    scale, offset = oracle.group_scale(w, G)
+    s_ref, o_ref = _numpy_scale(w, G)
+    assert np.array_equal(scale, s_ref) and np.array_equal(offset, o_ref)
+    # a constant group has scale 0; a group of zeros signed either way has offset +0
+    w2 = w.copy()
+    w2[0, :G] = w2[0, 5]
+    w2[1, G:2 * G] = 0x8000
+    w2[1, G + 3] = 0x0000
+    scale2, offset2 = oracle.group_scale(w2, G)
+    assert scale2[0, 0] == 0 and offset2[0, 0] == w2[0, 5]
+    assert scale2[1, 1] == 0 and offset2[1, 1] == 0x0000
+
+
+def pin_scaled_weights_range_and_reconstruction():
+    rng = np.random.default_rng(102)
+    N, K, G = 5, 384, 128
+    w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    scale, offset = oracle.group_scale(w, G)
+    ws = oracle.scaled_weights(w, scale, offset, G)
+    a = torch_bf16_to_f64(scale).repeat(G, axis=1)
+    b = torch_bf16_to_f64(offset).repeat(G, axis=1)
+    wf = torch_bf16_to_f64(w)
+    g = ws.reshape(N, K // G, G)
+    assert np.all(g.min(axis=2) == 0.0)               # the minimum maps to 0 exactly
+    assert np.allclose(g.max(axis=2), 15.0, rtol=2 ** -7, atol=0)
+    assert np.all(np.abs(a * ws + b - wf) <= 2 ** -50 * (np.abs(wf) + np.abs(b)))
+    # groups on the int4 grid: w = beta + alpha * k gives w_S = k exactly
+    levels = np.arange(16, dtype=np.float64)
+    w3 = _levels_problem(rng, 2, 256, 64, levels)
+    s3, o3 = oracle.group_scale(w3, 64)
+    ws3 = oracle.scaled_weights(w3, s3, o3, 64)
+    assert np.array_equal(ws3, np.round(ws3)) and ws3.min() == 0 and ws3.max() == 15
+
+
+def pin_kmeans_initial_table_and_nearest():
+    rng = np.random.default_rng(103)
+    xs = rng.uniform(0, 15, 300)
+    c, code, it = oracle.kmeans_row(xs, np.ones(300), 0)
+    assert it == 0
+    assert np.array_equal(c, _quantile_init(xs))
+    assert np.array_equal(code, _nearest(xs, c))
+
+
+def pin_kmeans_ties_go_to_lowest_entry():
+    # 16 levels 0..15 (8 copies each) and the 15 midpoints between them: the
+    # quantile table is exactly 0..15 and every midpoint is a tie.
+    mids = np.arange(15) + 0.5
+    xs = np.sort(np.concatenate([np.repeat(np.arange(16.0), 8), mids]))
+    c, code, _ = oracle.kmeans_row(xs, np.ones(xs.size), 0)
+    assert np.array_equal(c, np.arange(16.0))
+    for m in range(15):
+        assert code[np.searchsorted(xs, m + 0.5)] == m
+    assert np.array_equal(code, _nearest(xs, c))
+
+
+def _pairs_problem():
+    """Cluster q holds 10q (weight 3) and 10q + 1 (weight 1); entry 15 starts at 151."""
+    xs = np.array([v for q in range(16) for v in (10.0 * q, 10.0 * q + 1)])
+    u = np.tile([3.0, 1.0], 16)
+    return xs, u
+
+
+def pin_kmeans_weighted_mean_closed_form():
+    xs, u = _pairs_problem()
+    c, code, it = oracle.kmeans_row(xs, u, 20)
+    assert np.array_equal(code, np.repeat(np.arange(16), 2))
+    assert np.array_equal(c, 10.0 * np.arange(16) + 0.25)   # (3 * 10q + (10q + 1)) / 4
+    assert it == 1
+
+
+def pin_kmeans_zero_weight_cluster_keeps_entry():
+    xs, u = _pairs_problem()
+    u[10:12] = 0.0                                           # cluster 5 weighs nothing
+    c, _, _ = oracle.kmeans_row(xs, u, 20)
+    init = _quantile_init(xs)
+    assert c[5] == init[5] == 50.0
+    assert np.array_equal(np.delete(c, 5), np.delete(10.0 * np.arange(16) + 0.25, 5))
+
+
+def pin_kmeans_matches_scikit_learn():
+    rng = np.random.default_rng(104)
+    for K in (400, 1024):
+        xs = np.clip(rng.normal(7.5, 2.5, K), 0, 15)
+        u = rng.gamma(2.0, 1.0, K)
+        c, code, it = oracle.kmeans_row(xs, u, 500)
+        c_ref, code_ref = _sklearn_kmeans(xs, u)
+        assert 0 < it < 500
+        assert np.allclose(c, c_ref, rtol=1e-12, atol=1e-12)
+        assert np.array_equal(code, code_ref)
+
+
+def pin_kmeans_objective_never_increases():
+    rng = np.random.default_rng(105)
+    xs = rng.uniform(0, 15, 700) ** 1.5 / 15 ** 0.5
+    u = rng.gamma(1.5, 1.0, 700)
+    prev = None
+    for t in range(12):
+        c, code, _ = oracle.kmeans_row(xs, u, t)
+        obj = math.fsum(u * (xs - c[code]) ** 2)
+        if prev is not None:
+            assert obj <= prev * (1 + 1e-12)
+        prev = obj
+
+
+def pin_quantize_matches_scikit_learn_pipeline():
+    rng = np.random.default_rng(106)
+    N, K, G = 3, 256, 64
+    w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    ex = np.abs(rng.normal(0, 1, K)).astype(np.float32) + np.float32(0.05)
+    codes, lut, scale, offset, _ = oracle.quantize(w, ex, G, 300)
+    s_ref, o_ref = _numpy_scale(w, G)
+    assert np.array_equal(scale, s_ref) and np.array_equal(offset, o_ref)
+    a = torch_bf16_to_f64(s_ref).repeat(G, axis=1)
+    b = torch_bf16_to_f64(o_ref).repeat(G, axis=1)
+    ws = (torch_bf16_to_f64(w) - b) / a
+    for n in range(N):
+        u = a[n] * ex.astype(np.float64)
+        c_ref, _ = _sklearn_kmeans(ws[n], u, 300)
+        lut_ref = torch_bf16_bits(c_ref.astype(np.float32))
+        assert np.array_equal(lut[n], lut_ref)
+        assert np.array_equal(codes[n], _nearest(ws[n], torch_bf16_to_f64(lut_ref)))
+
+
+def pin_quantize_recovers_exact_levels():
+    rng = np.random.default_rng(107)
+    levels = np.array([0, 0.5, 1.25, 2, 3.5, 4, 5.75, 6, 7.5, 8.25, 9, 10.5, 11.75, 13, 14.25,
+                       15])
+    N, K, G = 3, 512, 128
+    w = _levels_problem(rng, N, K, G, levels)
+    ex = rng.uniform(0.1, 2.0, K).astype(np.float32)
+    codes, lut, scale, offset, _ = oracle.quantize(w, ex, G, 50)
+    assert np.array_equal(torch_bf16_to_f64(lut), np.tile(levels, (N, 1)))
+    a = torch_bf16_to_f64(scale).repeat(G, axis=1)
+    b = torch_bf16_to_f64(offset).repeat(G, axis=1)
+    assert np.array_equal(a * levels[codes] + b, torch_bf16_to_f64(w))
+
+
+def pin_quantize_invariant_to_power_of_two_activation_scale():
+    rng = np.random.default_rng(108)
+    w = torch_bf16_bits(rng.normal(0, 0.02, (4, 512)).astype(np.float32))
+    ex = rng.lognormal(0, 1, 512).astype(np.float32)
+    r1 = oracle.quantize(w, ex, 128, 40)
+    r2 = oracle.quantize(w, ex * np.float32(8), 128, 40)
+    for a, b in zip(r1, r2):
+        assert np.array_equal(a, b)
+
+
+def pin_quantize_degenerate_rows():
+    rng = np.random.default_rng(109)
+    N, K, G = 3, 256, 64
+    w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    w[0, :] = torch_bf16_bits(np.array([0.125], dtype=np.float32))[0]   # constant row
+    w[1, G:2 * G] = w[1, G]                                             # one constant group
+    ex = np.abs(rng.normal(0, 1, K)).astype(np.float32)
+    codes, lut, scale, offset, _ = oracle.quantize(w, ex, G, 30)
+    assert np.all(scale[0] == 0) and np.all(lut[0] == 0) and np.all(codes[0] == 0)
+    assert np.all(offset[0] == w[0, 0])
+    assert scale[1, 1] == 0 and offset[1, 1] == w[1, G]
+    # no activation weight anywhere: every cluster keeps its entry of the quantile table
+    codes2, lut2, scale2, offset2, it2 = oracle.quantize(w, np.zeros(K, np.float32), G, 30)
+    ws = (torch_bf16_to_f64(w[2]) - torch_bf16_to_f64(offset2[2]).repeat(G)) / \
+        torch_bf16_to_f64(scale2[2]).repeat(G)
+    assert np.array_equal(lut2[2], torch_bf16_bits(_quantile_init(ws).astype(np.float32)))
+    assert it2[2] == 1
+
+
+def pin_quantize_beats_int4_rounding():
+    """The paper's premise (§4.1) at toy scale: on Gaussian rows the learned
+    table has a lower weighted error than the int4 grid on the same scaling,
+    by more when a group spans the whole row (G = K) than at G = 128."""
+    rng = np.random.default_rng(110)
+    N, K = 6, 1024
+    for G, bound in ((128, 0.9), (K, 0.75)):
+        w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+        ex = rng.lognormal(0, 1, K).astype(np.float32)
+        codes, lut, scale, offset, _ = oracle.quantize(w, ex, G, 100)
+        a = torch_bf16_to_f64(scale).repeat(G, axis=1)
+        b = torch_bf16_to_f64(offset).repeat(G, axis=1)
+        ws = (torch_bf16_to_f64(w) - b) / a
+        u = a * ex.astype(np.float64)
+        rec = np.take_along_axis(torch_bf16_to_f64(lut), codes.astype(np.int64), 1)
+        err_any4 = math.fsum((u * (ws - rec) ** 2).ravel())
+        err_int4 = math.fsum((u * (ws - np.clip(np.round(ws), 0, 15)) ** 2).ravel())
+        assert err_any4 < bound * err_int4, (G, err_any4 / err_int4)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

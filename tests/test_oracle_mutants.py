@@ -46,6 +46,25 @@ MUTANTS = [
      "      float acc = 0.0f;\n      for (int64_t k = 0; k < K; ++k) {\n        acc += (float)oracle_bf16_to_f32(x[m * K + k])"),
     ("matmul_rows_wrong_row", "    int64_t n = rows[r];", "    int64_t n = rows[r] + (r > 0);"),
     ("widen_wrong_shift", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    ("alpha_over_16", "float alpha = (mx - mn) / 15.0f;", "float alpha = (mx - mn) / 16.0f;"),
+    ("beta_is_max", "offset[n * (K / G) + g] = oracle_bf16_rne(mn);",
+     "offset[n * (K / G) + g] = oracle_bf16_rne(mx);"),
+    ("scaled_without_offset", "ws[k] = alpha > 0.0 ? ((double)canon_bf16(w[k]) - beta) / alpha : 0.0;",
+     "ws[k] = alpha > 0.0 ? (double)canon_bf16(w[k]) / alpha : 0.0; (void)beta;"),
+    ("quantile_off_by_one", "c[q] = sorted[(q * (K - 1)) / 15];", "c[q] = sorted[(q * K) / 16];"),
+    ("ties_to_highest", "      if (d < best) {", "      if (d <= best) {"),
+    ("mstep_unweighted", "      num[code[j]] += u[j] * xs[j];\n      den[code[j]] += u[j];",
+     "      num[code[j]] += xs[j];\n      den[code[j]] += 1.0;"),
+    ("mstep_weight_squared", "      num[code[j]] += u[j] * xs[j];\n      den[code[j]] += u[j];",
+     "      num[code[j]] += u[j] * u[j] * xs[j];\n      den[code[j]] += u[j] * u[j];"),
+    ("empty_cluster_zeroed", "if (den[q] > 0.0) c[q] = num[q] / den[q];",
+     "c[q] = den[q] > 0.0 ? num[q] / den[q] : 0.0;"),
+    ("sample_weight_without_alpha",
+     "u[k] = (double)oracle_bf16_to_f32(scale[n * (K / G) + k / G]) * (double)ex[k];",
+     "u[k] = (double)ex[k];"),
+    ("codes_from_unrounded_centroids", "    assign_nearest(xs, K, table, code + n * K);\n", "\n"),
+    ("one_lloyd_step_only", "    if (assign_nearest(xs, K, c, code) == 0) break;",
+     "    assign_nearest(xs, K, c, code);\n    break;"),
     ("storage_bits_one_param", "4.0 + (2.0 * (double)group_param_bits) / (double)G",
      "4.0 + (1.0 * (double)group_param_bits) / (double)G"),
 ]
