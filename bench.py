@@ -535,6 +535,54 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def quantize_detail(max_iter: int, cpu_seconds: float):
+    """Time any4_quantize (learning the tables) on the Llama3-8B layer matrices
+    with CUDA events on the launching stream, and the oracle beside it on a
+    bounded sample of rows of each matrix; one JSON line."""
+    import torch
+    import oracle
+    import learned_bit_lut_any4_b200 as any4
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    out = []
+    for s in workloads.QUANTIZE_LLAMA3_8B:
+        w_bits = workloads.draw_dense_weight(s)
+        ex_np = workloads.draw_abs_act_mean(s)
+        w = _dev_bf16(w_bits)
+        ex = torch.from_numpy(ex_np).cuda()
+        any4.any4_quantize(w, ex, s.G, max_iter)            # warm-up (module load, attributes)
+        torch.cuda.synchronize()
+        reps = 3
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            _, _, _, _, iters = any4.any4_quantize(w, ex, s.G, max_iter, return_iters=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / reps
+        it = iters.cpu().numpy().astype(np.int64)
+        # algorithmic bytes: read w and E|x|, write codes, scale/offset and tables
+        alg = 2 * s.N * s.K + 4 * s.K + s.N * s.K // 2 + 4 * s.N * (s.K // s.G) + 32 * s.N
+        rows = 1
+        t = time.perf_counter()
+        while True:
+            oracle.quantize(w_bits[:rows], ex_np, s.G, max_iter)
+            dt = time.perf_counter() - t
+            if dt >= cpu_seconds / len(workloads.QUANTIZE_LLAMA3_8B) or rows >= s.N:
+                break
+            rows = min(s.N, rows * 4)
+            t = time.perf_counter()
+        out.append({"shape": s.name, "N": s.N, "K": s.K, "G": s.G, "max_iter": max_iter,
+                    "gpu_ms": round(ms, 3), "gpu_rows_per_s": round(s.N / ms * 1e3, 1),
+                    "mean_m_steps": round(float(it.mean()), 2), "max_m_steps": int(it.max()),
+                    "alg_bytes": alg, "gb_per_s": round(alg / ms / 1e6, 2),
+                    "hbm_frac": round(alg / ms / 1e6 / peaks["hbm_gbs"], 5),
+                    "mstep_columns_per_s": round(float(it.sum() * s.K) / ms * 1e3, 1),
+                    "oracle_rows": rows, "oracle_rows_per_s": round(rows / dt, 2),
+                    "oracle_cores": oracle.num_threads()})
+    print(json.dumps({"detail": "quantize", "shapes": out}), flush=True)
+
+
 def profile_shape(name: str, calls: int):
     """Run a few any4_matmul calls (auto path) on one workload shape."""
     import torch
@@ -572,9 +620,16 @@ def main():
                     help="no timing: run --profile-calls any4_matmul calls on one named "
                          "workload shape (a small, fixed case for ncu captures)")
     ap.add_argument("--profile-calls", type=int, default=3)
+    ap.add_argument("--quantize-detail", action="store_true",
+                    help="no step: time any4_quantize on the Llama3-8B matrices (and the "
+                         "oracle on a sample of rows) and print one JSON line")
+    ap.add_argument("--quantize-iters", type=int, default=100)
     args = ap.parse_args()
     if args.profile_shape:
         profile_shape(args.profile_shape, args.profile_calls)
+        return
+    if args.quantize_detail:
+        quantize_detail(args.quantize_iters, args.cpu_seconds)
         return
     if args.warmup < 3:
         args.warmup = 3

@@ -86,6 +86,43 @@ ANY4_API any4_status any4_pack(const uint8_t* idx, uint8_t* packed, int64_t N, i
                       int32_t* dev_status, any4_stream_t stream);
 
 /*
+ * any4_quantize -- learn the any4 representation of a bf16 weight matrix: per
+ * group scaling (paper §2.5.1 Eq. 1-2), then per row a weighted k-means on the
+ * scaled weights (§4.1: E-step Eq. 18, M-step Eq. 23; Appendix A.1 Alg. 1).
+ * Its outputs are the inputs of any4_dequant and any4_matmul (one table per
+ * row, lut_row_stride 16).
+ *   w          [N][K] bf16 weight                                    (input)
+ *   ex_abs     [K] fp32, E|x_j|: the mean absolute calibration activation of
+ *              input column j; finite and >= 0                       (input)
+ *   max_iter   M-steps at most, 0 <= max_iter <= ANY4_QUANTIZE_MAX_ITER
+ *   packed     [N][K/2] uint8 codes (layout of any4_pack)            (output)
+ *   lut        [N][16] bf16 table                                     (output)
+ *   scale      [N][K/G] bf16 alpha                                    (output)
+ *   offset     [N][K/G] bf16 beta                                     (output)
+ *   iters      [N] int32, M-steps run per row; may be NULL (4-byte aligned)
+ * Steps, each floating-point operation correctly rounded, in this order:
+ *   alpha = bf16(fp32(max - min) / 15) and beta = min over each group of G
+ *   columns (-0 read as +0); w_S = (w - beta) / alpha in fp64 (0 where alpha
+ *   is 0); the starting table holds the elements at positions
+ *   floor(q (K - 1) / 15), q = 0..15, of the row's sorted w_S; E-step: nearest
+ *   entry by |w_S - c_q|, ties to the lowest q; M-step: c_q = sum(u_j w_S_j) /
+ *   sum(u_j) over the columns of cluster q in ascending order, fp64, with
+ *   u_j = alpha_{g(j)} * E|x_j|; a cluster whose u_j sum to 0 keeps its entry;
+ *   stop after max_iter M-steps or when an E-step changes no code;
+ *   LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
+ *   LUT.  The results are bit-identical on every run and GPU.
+ * Shape rules as above, plus K <= ANY4_QUANTIZE_MAX_K (the row and its sort
+ * buffer live in one block's shared memory).  NaN or infinite weights or
+ * activation statistics give unspecified results.  One thread block per row.
+ */
+#define ANY4_QUANTIZE_MAX_K 16384
+#define ANY4_QUANTIZE_MAX_ITER 100000
+ANY4_API any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64_t N, int64_t K,
+                                   int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                                   uint16_t* scale, uint16_t* offset, int32_t* iters,
+                                   any4_stream_t stream);
+
+/*
  * any4_dequant -- materialise the bf16 weight (paper §2.5.2 dequant with the
  * per-row table of §2.4.1):
  *   W[n][k] = bf16_rne( fmaf( LUT[n][c], scale[n][k/G], offset[n][k/G] ) )

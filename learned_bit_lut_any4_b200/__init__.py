@@ -1,7 +1,7 @@
 """any4 on B200: Python binding of libany4 (the sm_100a CUDA library).
 
-This module only marshals arguments: every step of the any4 path (pack,
-dequant, matmul) runs in the CUDA kernels of libany4.so, reached through its
+This module only marshals arguments: every step of the any4 path (quantize,
+pack, dequant, matmul) runs in the CUDA kernels of libany4.so, reached through its
 C ABI (include/any4.h).  PyTorch provides device memory and the current
 stream.  There is no CPU fallback: if the library is missing or the device is
 not an sm_100 GPU, the calls raise.
@@ -17,6 +17,8 @@ from ._native import (  # noqa: F401
     ANY4_ERR_TIMEOUT,
     ANY4_ERR_UNSUPPORTED,
     ANY4_ERR_WORKSPACE,
+    ANY4_QUANTIZE_MAX_ITER,
+    ANY4_QUANTIZE_MAX_K,
     ANY4_STATIC_SCRATCH_BYTES,
     PATHS,
     Any4Error,
@@ -27,6 +29,7 @@ from ._native import (  # noqa: F401
     any4_matmul_static_scratch,
     any4_matmul_workspace_size,
     any4_pack,
+    any4_quantize,
     any4_status_string,
     any4_version,
     library,

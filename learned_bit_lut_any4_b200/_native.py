@@ -29,6 +29,9 @@ PATHS = {"auto": 0, "decode": 1, "prefill": 2}
 # Bytes of the library's fixed scratch array (any4_matmul_static_scratch).
 ANY4_STATIC_SCRATCH_BYTES = 148 * 262144 + 1024
 ANY4_FLAG_OVERLAP_PRIOR = 1
+# Limits of any4_quantize (the row lives in one block's shared memory).
+ANY4_QUANTIZE_MAX_K = 16384
+ANY4_QUANTIZE_MAX_ITER = 100000
 
 _lib = None
 
@@ -55,6 +58,8 @@ def library() -> ctypes.CDLL:
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     lib.any4_pack.argtypes = [vp, vp, i64, i64, vp, vp]
     lib.any4_pack.restype = i32
+    lib.any4_quantize.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
+    lib.any4_quantize.restype = i32
     lib.any4_dequant.argtypes = [vp, vp, i64, vp, vp, vp, i64, i64, i64, vp]
     lib.any4_dequant.restype = i32
     lib.any4_matmul.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp, vp]
@@ -162,6 +167,36 @@ def any4_pack(idx: torch.Tensor, packed: torch.Tensor | None = None,
         _check(library().any4_pack(_ptr(idx), _ptr(packed), N, K, _ptr(dev_status),
                                    _stream(idx.device)), "any4_pack")
     return packed
+
+
+def any4_quantize(w: torch.Tensor, ex_abs: torch.Tensor, G: int, max_iter: int = 100,
+                  return_iters: bool = False):
+    """Learn the any4 representation of a bf16 weight w [N, K]: group scaling,
+    then a weighted k-means per row with sample weight alpha * E|x| (ex_abs,
+    fp32 [K], finite and >= 0).  Returns (packed [N, K/2] uint8, lut [N, 16],
+    scale [N, K/G], offset [N, K/G]) in bf16, plus the int32 M-steps per row
+    when return_iters."""
+    _need(w, "w", _BF16)
+    dev = w.device
+    _need(ex_abs, "ex_abs", (torch.float32,), dev)
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    if ex_abs.numel() != K:
+        raise ValueError(f"ex_abs must hold K={K} values")
+    ng = K // G if G > 0 else 0
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    lut = torch.empty((N, 16), dtype=torch.bfloat16, device=dev)
+    scale = torch.empty((N, ng), dtype=torch.bfloat16, device=dev)
+    offset = torch.empty((N, ng), dtype=torch.bfloat16, device=dev)
+    iters = torch.empty(N, dtype=torch.int32, device=dev) if return_iters else None
+    with _on_device(dev):
+        _check(library().any4_quantize(_ptr(w), _ptr(ex_abs), N, K, G, int(max_iter),
+                                       _ptr(packed), _ptr(lut), _ptr(scale), _ptr(offset),
+                                       _ptr(iters), _stream(dev)), "any4_quantize")
+    if return_iters:
+        return packed, lut, scale, offset, iters
+    return packed, lut, scale, offset
 
 
 def _lut_stride(lut: torch.Tensor, N: int) -> int:

@@ -20,6 +20,13 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
                                     size_t workspace_bytes, int32_t* dev_status,
                                     cudaStream_t stream, const DeviceInfo& dev);
 
+// Table learning (quantize.cu): one thread block per weight row.
+size_t quantize_smem_bytes(int64_t K, int64_t G);
+any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
+                            int32_t max_iter, uint8_t* packed, uint16_t* lut, uint16_t* scale,
+                            uint16_t* offset, int32_t* iters, cudaStream_t stream,
+                            const DeviceInfo& dev);
+
 namespace {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -123,6 +130,25 @@ any4_status any4_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
   any4_status st = current_device(&dev);
   if (st != ANY4_OK) return st;
   return launch_pack(idx, packed, N, K, dev_status, (cudaStream_t)stream, dev);
+}
+
+any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64_t N, int64_t K,
+                          int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                          uint16_t* scale, uint16_t* offset, int32_t* iters,
+                          any4_stream_t stream) {
+  if (!w || !ex_abs || !packed || !lut || !scale || !offset) return ANY4_ERR_NULL;
+  if (!shape_ok(N, K, G) || K > ANY4_QUANTIZE_MAX_K || N > INT32_MAX || max_iter < 0 ||
+      max_iter > ANY4_QUANTIZE_MAX_ITER)
+    return ANY4_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(ex_abs) || !aligned16(packed) || !aligned16(lut) ||
+      !aligned16(scale) || !aligned16(offset))
+    return ANY4_ERR_ALIGN;
+  if (iters && (reinterpret_cast<uintptr_t>(iters) & 3u)) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_quantize(w, ex_abs, N, K, G, max_iter, packed, lut, scale, offset, iters,
+                         (cudaStream_t)stream, dev);
 }
 
 any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,

@@ -1,0 +1,249 @@
+// Learning the table of each row: the quantiser that produces the packed codes,
+// tables, scales and offsets the matmul consumes.
+//
+// "any4: Learned 4-bit Numeric Representation for LLMs":
+//   §2.5.1 Eq. 1-2   group-wise scaling: alpha = (max - min) / 15, beta = min,
+//                    scaled weight w_S = (w - beta) / alpha;
+//   §4.1 Eq. 18      E-step: each scaled weight takes its nearest table entry;
+//   §4.1 Eq. 23      M-step: an entry becomes the mean of its cluster's scaled
+//                    weights, weighted by alpha_{i,j} * E|x_j|;
+//   Appendix A.1     rows are independent (Alg. 1 runs k-means row by row).
+//
+// One thread block per row, the row held in shared memory.  Every floating-point
+// step is one correctly rounded IEEE operation written with an explicit-rounding
+// intrinsic (nothing is contracted into a fused multiply-add), taken in the order
+// of a sequential loop, so the results are bit-identical to a plain sequential
+// statement of the same steps:
+//   - alpha = bf16(fp32(fp32(max - min) / 15)), beta = min (exact in bf16);
+//     w is read with -0 as +0;
+//   - w_S = ((double)w - beta) / alpha in fp64, 0 in a group whose alpha is 0;
+//   - initial table: entry q = the element at position floor(q (K - 1) / 15)
+//     of the sorted row (a bitonic sort in shared memory);
+//   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q;
+//   - M-step: sample weight u_j = alpha_{g(j)} * E|x_j| (exact in fp64);
+//     numerator sum(u_j * w_S_j) and denominator sum(u_j) over ascending j,
+//     one lane of warp 0 per cluster and per sum, so the rounding order is the
+//     sequential one; a cluster whose weights sum to 0 keeps its entry;
+//   - stop after max_iter M-steps, or when an E-step changes no code;
+//   - LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
+//     LUT, packed two per byte (even column in the low nibble).
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace any4 {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantWarps = kQuantThreads / 32;
+
+// Shared-memory layout of one row (K columns, NG = K / G groups, P = the
+// power of two >= K the sort runs over).
+struct QuantSmem {
+  size_t xs, ex, alpha, beta, cent, table, code, total;
+};
+
+__host__ __device__ inline int64_t pow2_at_least(int64_t K) {
+  int64_t p = 32;
+  while (p < K) p <<= 1;
+  return p;
+}
+
+__host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G) {
+  QuantSmem s;
+  const int64_t NG = K / G;
+  s.xs = 0;                                            // double [P]
+  s.cent = s.xs + 8 * (size_t)pow2_at_least(K);        // double [16]
+  s.table = s.cent + 8 * 16;                           // double [16]
+  s.ex = s.table + 8 * 16;                             // float [K]
+  s.alpha = s.ex + 4 * (size_t)K;                      // float [NG]
+  s.beta = s.alpha + 4 * (size_t)NG;                   // float [NG]
+  s.code = s.beta + 4 * (size_t)NG;                    // uint8 [K]
+  s.total = (s.code + (size_t)K + 15) & ~(size_t)15;
+  return s;
+}
+
+// bf16 value with -0 read as +0 (x + 0 rounds -0 to +0 and leaves all else).
+__device__ __forceinline__ float bf16_canon(uint16_t h) {
+  return __fadd_rn(__uint_as_float((uint32_t)h << 16), 0.0f);
+}
+
+__device__ __forceinline__ double scaled_weight(float w, float alpha, float beta) {
+  return alpha > 0.0f ? __ddiv_rn(__dsub_rn((double)w, (double)beta), (double)alpha) : 0.0;
+}
+
+// E-step over the row: nearest entry of c (ties to the lowest index).  Returns
+// (uniformly across the block) whether any code changed.
+__device__ __forceinline__ bool estep(const double* xs, int K, const double* c, uint8_t* code) {
+  double cr[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) cr[q] = c[q];
+  int changed = 0;
+  for (int j = threadIdx.x; j < K; j += kQuantThreads) {
+    const double x = xs[j];
+    double best = fabs(__dsub_rn(x, cr[0]));
+    int bq = 0;
+#pragma unroll
+    for (int q = 1; q < 16; ++q) {
+      const double d = fabs(__dsub_rn(x, cr[q]));
+      if (d < best) {
+        best = d;
+        bq = q;
+      }
+    }
+    if (code[j] != (uint8_t)bq) changed = 1;
+    code[j] = (uint8_t)bq;
+  }
+  return __syncthreads_or(changed) != 0;
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, int K, int G,
+                int max_iter, uint8_t* __restrict__ packed, uint16_t* __restrict__ lut,
+                uint16_t* __restrict__ scale, uint16_t* __restrict__ offset,
+                int32_t* __restrict__ iters) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const QuantSmem L = quant_smem_layout(K, G);
+  double* xs = reinterpret_cast<double*>(smem + L.xs);
+  double* cent = reinterpret_cast<double*>(smem + L.cent);
+  double* table = reinterpret_cast<double*>(smem + L.table);
+  float* ex_s = reinterpret_cast<float*>(smem + L.ex);
+  float* alpha_s = reinterpret_cast<float*>(smem + L.alpha);
+  float* beta_s = reinterpret_cast<float*>(smem + L.beta);
+  uint8_t* code = smem + L.code;
+
+  const int64_t n = blockIdx.x;
+  const int NG = K / G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint16_t* wrow = w + n * (int64_t)K;
+
+  for (int j = tid; j < K; j += kQuantThreads) {
+    ex_s[j] = ex[j];
+    code[j] = 0;
+  }
+
+  // Eq. 1-2: one warp per group; min and max are exact, so their order is free.
+  for (int g = warp; g < NG; g += kQuantWarps) {
+    float mn = bf16_canon(wrow[g * G + lane]);
+    float mx = mn;
+    for (int j = g * G + 32 + lane; j < (g + 1) * G; j += 32) {
+      const float v = bf16_canon(wrow[j]);
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(kFullMask, mn, s));
+      mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, s));
+    }
+    if (lane == 0) {
+      const uint16_t a = f32_to_bf16_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+      const uint16_t b = (uint16_t)(__float_as_uint(mn) >> 16);   // mn is a bf16 value
+      scale[n * NG + g] = a;
+      offset[n * NG + g] = b;
+      alpha_s[g] = __uint_as_float((uint32_t)a << 16);
+      beta_s[g] = mn;
+    }
+  }
+  __syncthreads();
+
+  // Initial table: quantiles of the sorted w_S (+inf pads the sort to P).
+  const int P = (int)pow2_at_least(K);
+  for (int j = tid; j < P; j += kQuantThreads)
+    xs[j] = j < K ? scaled_weight(bf16_canon(wrow[j]), alpha_s[j / G], beta_s[j / G])
+                  : __longlong_as_double(0x7ff0000000000000LL);
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < P; i += kQuantThreads) {
+        const int l = i ^ jj;
+        if (l > i) {
+          const double a = xs[i], b = xs[l];
+          if ((i & k) == 0 ? (a > b) : (a < b)) {
+            xs[i] = b;
+            xs[l] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (tid < 16) cent[tid] = xs[(int)(((int64_t)tid * (K - 1)) / 15)];
+  __syncthreads();
+  for (int j = tid; j < K; j += kQuantThreads)
+    xs[j] = scaled_weight(bf16_canon(wrow[j]), alpha_s[j / G], beta_s[j / G]);
+  __syncthreads();
+
+  estep(xs, K, cent, code);
+  int it = 0;
+  while (it < max_iter) {
+    if (warp == 0) {
+      // Eq. 23: lane q sums u_j * w_S_j, lane 16 + q sums u_j, over the
+      // columns of cluster q in ascending order.
+      const int q = lane & 15;
+      const bool den = lane >= 16;
+      double acc = 0.0;
+      for (int g = 0; g < NG; ++g) {
+        const double a = (double)alpha_s[g];
+        const int j1 = (g + 1) * G;
+#pragma unroll 4
+        for (int j = g * G; j < j1; ++j) {
+          const double u = __dmul_rn(a, (double)ex_s[j]);
+          const double t = den ? u : __dmul_rn(u, xs[j]);
+          if (code[j] == q) acc = __dadd_rn(acc, t);
+        }
+      }
+      const double d = __shfl_down_sync(kFullMask, acc, 16);
+      if (lane < 16 && d > 0.0) cent[q] = __ddiv_rn(acc, d);
+    }
+    __syncthreads();
+    ++it;
+    if (!estep(xs, K, cent, code)) break;
+  }
+
+  if (tid < 16) {
+    const uint16_t b = f32_to_bf16_rn(__double2float_rn(cent[tid]));
+    lut[n * 16 + tid] = b;
+    table[tid] = (double)__uint_as_float((uint32_t)b << 16);
+  }
+  if (tid == 0 && iters) iters[n] = it;
+  __syncthreads();
+  estep(xs, K, table, code);
+
+  // Pack 32 codes (16 bytes) per thread step; K % 32 == 0.
+  uint4* prow = reinterpret_cast<uint4*>(packed + n * (int64_t)(K / 2));
+  for (int c = tid; c < K / 32; c += kQuantThreads) {
+    uint32_t v[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int j = c * 32 + b * 8 + h * 2;
+        word |= (uint32_t)(code[j] | (code[j + 1] << 4)) << (8 * h);
+      }
+      v[b] = word;
+    }
+    prow[c] = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+}  // namespace
+
+size_t quantize_smem_bytes(int64_t K, int64_t G) { return quant_smem_layout(K, G).total; }
+
+any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
+                            int32_t max_iter, uint8_t* packed, uint16_t* lut, uint16_t* scale,
+                            uint16_t* offset, int32_t* iters, cudaStream_t stream,
+                            const DeviceInfo& dev) {
+  const size_t smem = quantize_smem_bytes(K, G);
+  if (smem > dev.smem_optin) return ANY4_ERR_SHAPE;
+  if (cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ANY4_ERR_CUDA;
+  quantize_kernel<<<(unsigned)N, kQuantThreads, smem, stream>>>(
+      w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
+  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+}  // namespace any4

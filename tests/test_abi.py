@@ -101,6 +101,29 @@ def test_pack_and_dequant_reject_bad_arguments():
         any4.ANY4_ERR_ALIGN
 
 
+@pytest.mark.parametrize("kw,expect", [
+    (dict(w=None), any4.ANY4_ERR_NULL),
+    (dict(ex=None), any4.ANY4_ERR_NULL),
+    (dict(offset=None), any4.ANY4_ERR_NULL),
+    (dict(K=48), any4.ANY4_ERR_SHAPE),
+    (dict(G=48), any4.ANY4_ERR_SHAPE),
+    (dict(N=0), any4.ANY4_ERR_SHAPE),
+    (dict(K=any4.ANY4_QUANTIZE_MAX_K + 32, G=32), any4.ANY4_ERR_SHAPE),
+    (dict(max_iter=-1), any4.ANY4_ERR_SHAPE),
+    (dict(max_iter=any4.ANY4_QUANTIZE_MAX_ITER + 1), any4.ANY4_ERR_SHAPE),
+    (dict(ex=FAKE + 4), any4.ANY4_ERR_ALIGN),
+    (dict(packed=FAKE + 8), any4.ANY4_ERR_ALIGN),
+    (dict(iters=FAKE + 2), any4.ANY4_ERR_ALIGN),
+])
+def test_quantize_rejects_bad_arguments(kw, expect):
+    a = dict(w=FAKE, ex=FAKE, N=4, K=256, G=64, max_iter=10, packed=FAKE, lut=FAKE, scale=FAKE,
+             offset=FAKE, iters=None)
+    a.update(kw)
+    assert _native.library().any4_quantize(a["w"], a["ex"], a["N"], a["K"], a["G"],
+                                           a["max_iter"], a["packed"], a["lut"], a["scale"],
+                                           a["offset"], a["iters"], None) == expect
+
+
 def test_workspace_size_of_bad_shapes_is_zero():
     assert any4.any4_matmul_workspace_size(1, 64, 48, 48) == 0
     assert any4.any4_matmul_workspace_size(0, 64, 64, 32) == 0

@@ -149,3 +149,47 @@ CONFIGS = {
 def all_shapes():
     for group in CONFIGS.values():
         yield from group
+
+
+# --------------------------------------------------------------------------
+# Inputs of the quantiser (learning the tables): a dense bf16 weight and the
+# mean absolute activation of each input column, E|x_j| (the statistic the
+# paper's §4.1 Eq. 23 weights the M-step with, taken from a calibration
+# prompt; here drawn, since no model or prompt is run).
+#   w        normal(0, 0.02) -> bf16, [N, K] (the spread of Llama-sized
+#            linear weights)
+#   E|x_j|   lognormal(-0.5, 0.8), then 1 column in 200 (seeded choice)
+#            multiplied by 20: the few outlier channels LLM activations have;
+#            fp32 [K]
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class QuantShape:
+    """One weight matrix to quantise: W[N, K] with groups of G columns."""
+    name: str
+    N: int
+    K: int
+    G: int
+    seed: int
+
+
+def draw_dense_weight(s: QuantShape) -> np.ndarray:
+    rng = np.random.default_rng(np.random.SeedSequence(s.seed))
+    return _to_bf16_bits(rng.normal(0.0, 0.02, size=(s.N, s.K)).astype(np.float32))
+
+
+def draw_abs_act_mean(s: QuantShape) -> np.ndarray:
+    rng = np.random.default_rng(np.random.SeedSequence(s.seed + 1_000_000))
+    ex = rng.lognormal(-0.5, 0.8, size=s.K)
+    outliers = rng.choice(s.K, size=max(1, s.K // 200), replace=False)
+    ex[outliers] *= 20.0
+    return ex.astype(np.float32)
+
+
+# The Llama3-8B linear layers (§5) as matrices to quantise.
+QUANTIZE_LLAMA3_8B = [
+    QuantShape("8b_q", 4096, 4096, 128, 4501),
+    QuantShape("8b_k", 1024, 4096, 128, 4502),
+    QuantShape("8b_gate", 14336, 4096, 128, 4505),
+    QuantShape("8b_down", 4096, 14336, 128, 4507),
+]
