@@ -19,6 +19,10 @@ Every function follows "any4: Learned 4-bit Numeric Representation for LLMs"
                      iteration from a quantile initialisation
   quantize           §4.1 and Appendix A.1 (Alg. 1): scaling, then k-means per
                      row with sample weight alpha * E|x|; bf16 table and codes
+  *_bits             the same for n-bit codes, n in {2, 3, 4} (§4.1 Eq. 9: 2^n
+                     values per row; §5: any3, any2), with the storage reading
+                     "one little-endian bit stream per row" (the pages give no
+                     layout below 4 bits)
 
 bf16 values cross this interface as their raw uint16 bit patterns.  The
 arithmetic lives in any4_oracle.c (fp32 fmaf + IEEE round-to-nearest-even to
@@ -79,6 +83,22 @@ def _bind(lib):
     lib.oracle_any4_quantize.argtypes = [u16p, f32p, i64, i64, i64, i64, u8p, u16p, u16p, u16p,
                                          i64p]
     lib.oracle_any4_quantize.restype = None
+    ci = ctypes.c_int
+    lib.oracle_group_scale_bits.argtypes = [u16p, i64, i64, i64, ci, u16p, u16p]
+    lib.oracle_group_scale_bits.restype = None
+    lib.oracle_kmeans_row_bits.argtypes = [f64p, f64p, i64, ci, i64, f64p, u8p]
+    lib.oracle_kmeans_row_bits.restype = i64
+    lib.oracle_quantize_bits.argtypes = [u16p, f32p, i64, i64, i64, ci, i64, u8p, u16p, u16p,
+                                         u16p, i64p]
+    lib.oracle_quantize_bits.restype = None
+    lib.oracle_pack_bits.argtypes = [u8p, u8p, i64, i64, ci]
+    lib.oracle_pack_bits.restype = i64
+    lib.oracle_unpack_bits.argtypes = [u8p, u8p, i64, i64, ci]
+    lib.oracle_unpack_bits.restype = None
+    lib.oracle_dequant_bits.argtypes = [u8p, u16p, i64, u16p, u16p, u16p, i64, i64, i64, ci]
+    lib.oracle_dequant_bits.restype = None
+    lib.oracle_bits_per_weight_n.argtypes = [i64, i64, ci]
+    lib.oracle_bits_per_weight_n.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -326,6 +346,133 @@ def quantize(w, ex, G: int, max_iter: int):
     return codes, lut, scale, offset, iters
 
 
+# --------------------------------------------------------------------------
+# n-bit variants (any3, any2; n = 4 is any4): §4.1 Eq. 9 (2^n values per row),
+# §5 (any3 / any2 evaluated).  Storage reading: a row's codes form one
+# little-endian bit stream, code k in bits [n k, n k + n).
+# --------------------------------------------------------------------------
+
+_BITS = (2, 3, 4)
+
+
+def _check_bits(bits):
+    if bits not in _BITS:
+        raise ValueError(f"bits must be one of {_BITS}")
+    return int(bits)
+
+
+def pack_bits(idx: np.ndarray, bits: int) -> np.ndarray:
+    """idx uint8 [N, K] (codes 0 .. 2^bits - 1) -> packed uint8 [N, bits*K/8]."""
+    bits = _check_bits(bits)
+    idx = _c(idx, np.uint8)
+    N, K = idx.shape
+    if K % 8:
+        raise ValueError("K must be a multiple of 8")
+    packed = np.empty((N, bits * K // 8), dtype=np.uint8)
+    bad = _load().oracle_pack_bits(_ptr(idx, ctypes.c_uint8), _ptr(packed, ctypes.c_uint8), N, K,
+                                   bits)
+    if bad:
+        raise ValueError(f"{bad} codes outside 0..{(1 << bits) - 1}")
+    return packed
+
+
+def unpack_bits(packed: np.ndarray, bits: int, K: int) -> np.ndarray:
+    bits = _check_bits(bits)
+    packed = _c(packed, np.uint8)
+    N = packed.shape[0]
+    if K % 8 or packed.shape[1] != bits * K // 8:
+        raise ValueError("packed must be [N, bits*K/8] with K a multiple of 8")
+    idx = np.empty((N, K), dtype=np.uint8)
+    _load().oracle_unpack_bits(_ptr(packed, ctypes.c_uint8), _ptr(idx, ctypes.c_uint8), N, K, bits)
+    return idx
+
+
+def dequant_bits(packed, lut, scale, offset, G: int, bits: int, K: int,
+                 per_tensor_lut: bool = False) -> np.ndarray:
+    """W[n][k] = bf16(fmaf(LUT[n][code], scale[n][k/G], offset[n][k/G])) for
+    n-bit codes; lut is [N, 2^bits] or, with per_tensor_lut, [2^bits]."""
+    bits = _check_bits(bits)
+    packed = _c(packed, np.uint8)
+    lut = _c(lut, np.uint16)
+    scale = _c(scale, np.uint16)
+    offset = _c(offset, np.uint16)
+    N = packed.shape[0]
+    nq = 1 << bits
+    if K % 8 or K % G or packed.shape[1] != bits * K // 8:
+        raise ValueError("bad K, G or packed shape")
+    if scale.shape != (N, K // G) or offset.shape != (N, K // G):
+        raise ValueError("scale/offset must be [N, K/G]")
+    if per_tensor_lut:
+        if lut.size != nq:
+            raise ValueError(f"per-tensor LUT must have {nq} entries")
+        stride = 0
+    else:
+        if lut.shape != (N, nq):
+            raise ValueError(f"LUT must be [N, {nq}]")
+        stride = nq
+    W = np.empty((N, K), dtype=np.uint16)
+    _load().oracle_dequant_bits(_ptr(packed, ctypes.c_uint8), _ptr(lut, ctypes.c_uint16), stride,
+                                _ptr(scale, ctypes.c_uint16), _ptr(offset, ctypes.c_uint16),
+                                _ptr(W, ctypes.c_uint16), N, K, G, bits)
+    return W
+
+
+def bits_per_weight_n(K: int, G: int, bits: int) -> float:
+    return _load().oracle_bits_per_weight_n(K, G, _check_bits(bits))
+
+
+def group_scale_bits(w, G: int, bits: int):
+    """Eq. 1-2 with Qmax - Qmin = 2^bits - 1: (scale, offset) bf16 bits [N, K/G]."""
+    bits = _check_bits(bits)
+    w, N, K = _check_weight(w, G)
+    scale = np.empty((N, K // G), dtype=np.uint16)
+    offset = np.empty((N, K // G), dtype=np.uint16)
+    _load().oracle_group_scale_bits(_ptr(w, ctypes.c_uint16), N, K, G, bits,
+                                    _ptr(scale, ctypes.c_uint16), _ptr(offset, ctypes.c_uint16))
+    return scale, offset
+
+
+def kmeans_row_bits(xs, u, bits: int, max_iter: int):
+    """kmeans_row with 2^bits entries."""
+    bits = _check_bits(bits)
+    xs = _c(xs, np.float64)
+    u = _c(u, np.float64)
+    if xs.ndim != 1 or u.shape != xs.shape or xs.size < 1 or max_iter < 0:
+        raise ValueError("bad arguments")
+    c = np.empty(1 << bits, dtype=np.float64)
+    code = np.empty(xs.size, dtype=np.uint8)
+    it = _load().oracle_kmeans_row_bits(_ptr(xs, ctypes.c_double), _ptr(u, ctypes.c_double),
+                                        xs.size, bits, int(max_iter), _ptr(c, ctypes.c_double),
+                                        _ptr(code, ctypes.c_uint8))
+    return c, code, int(it)
+
+
+def quantize_bits(w, ex, G: int, bits: int, max_iter: int):
+    """quantize for n-bit codes: (codes [N, K], lut [N, 2^bits], scale, offset, iters)."""
+    bits = _check_bits(bits)
+    w, N, K = _check_weight(w, G)
+    ex = _c(ex, np.float32)
+    if ex.shape != (K,):
+        raise ValueError("ex must be [K]")
+    if not np.all(np.isfinite(ex)) or np.any(ex < 0):
+        raise ValueError("ex must be finite and >= 0")
+    if max_iter < 0:
+        raise ValueError("max_iter must be >= 0")
+    nq = 1 << bits
+    codes = np.empty((N, K), dtype=np.uint8)
+    lut = np.empty((N, nq), dtype=np.uint16)
+    scale = np.empty((N, K // G), dtype=np.uint16)
+    offset = np.empty((N, K // G), dtype=np.uint16)
+    iters = np.empty(N, dtype=np.int64)
+    _load().oracle_quantize_bits(_ptr(w, ctypes.c_uint16), _ptr(ex, ctypes.c_float), N, K, G,
+                                 bits, int(max_iter), _ptr(codes, ctypes.c_uint8),
+                                 _ptr(lut, ctypes.c_uint16), _ptr(scale, ctypes.c_uint16),
+                                 _ptr(offset, ctypes.c_uint16), _ptr(iters, ctypes.c_int64))
+    return codes, lut, scale, offset, iters
+
+
 __all__ = ["bf16_rne", "bf16_to_f32", "pack", "unpack", "bits_per_weight", "dequant_one",
            "dequant", "matmul", "matmul_rows", "any4_matmul", "num_threads",
-           "set_num_threads", "group_scale", "scaled_weights", "kmeans_row", "quantize"]
+           "set_num_threads", "group_scale", "scaled_weights", "kmeans_row", "quantize",
+           "pack_bits", "unpack_bits", "dequant_bits", "bits_per_weight_n", "group_scale_bits",
+           "kmeans_row_bits", "quantize_bits"]

@@ -219,9 +219,11 @@ void oracle_set_num_threads(int t) { (void)t; }
 /* ------------------------------------------------------------------------- */
 /* Learning the table of each row.
  *
- * Follows the quantisation procedure of the same paper:
+ * Follows the quantisation procedure of the same paper, for n-bit codes
+ * (§4.1 Eq. 9: a set of 2^n values per row, "any n"; n = 4 is any4, and §5
+ * evaluates any3 and any2):
  *   - §2.5.1 Eq. 1-2: per group of G columns, alpha = (max - min) / (Qmax - Qmin)
- *     with Qmax - Qmin = 15 for 4 bits, beta = min, and the scaled weight
+ *     with Qmax - Qmin = 2^n - 1, beta = min, and the scaled weight
  *     w_S = (w - beta) / alpha;
  *   - §4.1 E-step (Eq. 18): each scaled weight takes the nearest table entry;
  *   - §4.1 M-step (Eq. 23): each entry becomes the mean of its cluster's
@@ -230,15 +232,15 @@ void oracle_set_num_threads(int t) { (void)t; }
  *     alternate until the table stops changing.
  * Readings where the pages leave a step open:
  *   - w is bf16 (its -0 is read as +0); E|x_j| is fp32, >= 0, one per column.
- *   - alpha is the bf16 rounding of the fp32 quotient (max - min) / 15 (both
- *     fp32 operations correctly rounded) and beta = min (exact in bf16); the
- *     k-means runs on w_S formed with these stored values, in fp64:
+ *   - alpha is the bf16 rounding of the fp32 quotient (max - min) / (2^n - 1)
+ *     (both fp32 operations correctly rounded) and beta = min (exact in
+ *     bf16); the k-means runs on w_S formed with these stored values, in fp64:
  *     w_S = ((double)w - beta) / alpha, or 0 for every column of a group
  *     whose stored alpha is 0.
  *   - Sample weight u_j = alpha_{g(j)} * E|x_j| in fp64 (exact: 8 x 24 bits).
  *   - Initial table: the quantiles of the row's sorted w_S, entry q at
- *     position floor(q (K - 1) / 15) (deterministic; scikit-learn's k-means++
- *     seeding draws random numbers).
+ *     position floor(q (K - 1) / (2^n - 1)) (deterministic; scikit-learn's
+ *     k-means++ seeding draws random numbers).
  *   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q.
  *   - M-step: numerator and denominator summed in fp64 over ascending column
  *     index, each product rounded before its add; a cluster whose weights
@@ -251,8 +253,9 @@ void oracle_set_num_threads(int t) { (void)t; }
 static float canon_bf16(uint16_t h) { return oracle_bf16_to_f32(h) + 0.0f; }
 
 /* Eq. 1-2 on every group: scale = bf16(alpha), offset = bf16(beta) = min. */
-void oracle_group_scale(const uint16_t* w, int64_t N, int64_t K, int64_t G, uint16_t* scale,
-                        uint16_t* offset) {
+void oracle_group_scale_bits(const uint16_t* w, int64_t N, int64_t K, int64_t G, int bits,
+                             uint16_t* scale, uint16_t* offset) {
+  const float levels = (float)((1 << bits) - 1);
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t g = 0; g < K / G; ++g) {
@@ -263,11 +266,16 @@ void oracle_group_scale(const uint16_t* w, int64_t N, int64_t K, int64_t G, uint
         if (v < mn) mn = v;
         if (v > mx) mx = v;
       }
-      float alpha = (mx - mn) / 15.0f;
+      float alpha = (mx - mn) / levels;
       scale[n * (K / G) + g] = oracle_bf16_rne(alpha);
       offset[n * (K / G) + g] = oracle_bf16_rne(mn);
     }
   }
+}
+
+void oracle_group_scale(const uint16_t* w, int64_t N, int64_t K, int64_t G, uint16_t* scale,
+                        uint16_t* offset) {
+  oracle_group_scale_bits(w, N, K, G, 4, scale, offset);
 }
 
 /* w_S = (w - beta) / alpha for one row, with the stored bf16 alpha and beta
@@ -293,14 +301,15 @@ static int cmp_double(const void* a, const void* b) {
   return (x > y) - (x < y);
 }
 
-/* E-step (Eq. 18): nearest of the 16 entries, ties to the lowest index.
+/* E-step (Eq. 18): nearest of the nq entries, ties to the lowest index.
  * Returns how many codes changed. */
-static int64_t assign_nearest(const double* xs, int64_t K, const double* c, uint8_t* code) {
+static int64_t assign_nearest(const double* xs, int64_t K, const double* c, int nq,
+                              uint8_t* code) {
   int64_t changed = 0;
   for (int64_t j = 0; j < K; ++j) {
     int best_q = 0;
     double best = fabs(xs[j] - c[0]);
-    for (int q = 1; q < 16; ++q) {
+    for (int q = 1; q < nq; ++q) {
       double d = fabs(xs[j] - c[q]);
       if (d < best) {
         best = d;
@@ -313,41 +322,53 @@ static int64_t assign_nearest(const double* xs, int64_t K, const double* c, uint
   return changed;
 }
 
-/* Weighted Lloyd iteration on one row: samples xs[0..K), weights u[0..K).
- * Out: c[16] (fp64 centroids) and code[K] (the E-step matching c).  Returns
- * the number of M-steps run. */
-int64_t oracle_kmeans_row(const double* xs, const double* u, int64_t K, int64_t max_iter,
-                          double* c, uint8_t* code) {
+/* Weighted Lloyd iteration on one row with nq entries: samples xs[0..K),
+ * weights u[0..K).  Out: c[nq] (fp64 centroids) and code[K] (the E-step
+ * matching c).  Returns the number of M-steps run. */
+static int64_t kmeans_row(const double* xs, const double* u, int64_t K, int nq,
+                          int64_t max_iter, double* c, uint8_t* code) {
   double* sorted = (double*)malloc((size_t)K * sizeof(double));
   memcpy(sorted, xs, (size_t)K * sizeof(double));
   qsort(sorted, (size_t)K, sizeof(double), cmp_double);
-  for (int q = 0; q < 16; ++q) c[q] = sorted[(q * (K - 1)) / 15];
+  for (int q = 0; q < nq; ++q) c[q] = sorted[(q * (K - 1)) / (nq - 1)];
   free(sorted);
 
   memset(code, 0, (size_t)K);
-  assign_nearest(xs, K, c, code);
+  assign_nearest(xs, K, c, nq, code);
   int64_t it = 0;
   while (it < max_iter) {
     double num[16], den[16];
-    for (int q = 0; q < 16; ++q) num[q] = den[q] = 0.0;
+    for (int q = 0; q < nq; ++q) num[q] = den[q] = 0.0;
     for (int64_t j = 0; j < K; ++j) {           /* M-step (Eq. 23) */
       num[code[j]] += u[j] * xs[j];
       den[code[j]] += u[j];
     }
-    for (int q = 0; q < 16; ++q)
+    for (int q = 0; q < nq; ++q)
       if (den[q] > 0.0) c[q] = num[q] / den[q];
     ++it;
-    if (assign_nearest(xs, K, c, code) == 0) break;
+    if (assign_nearest(xs, K, c, nq, code) == 0) break;
   }
   return it;
 }
 
-/* The whole quantiser for an [N][K] bf16 weight: scale, offset, LUT and codes.
- * iters[n] (may be NULL) receives the M-steps run on row n. */
-void oracle_any4_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
-                          int64_t max_iter, uint8_t* code, uint16_t* lut, uint16_t* scale,
-                          uint16_t* offset, int64_t* iters) {
-  oracle_group_scale(w, N, K, G, scale, offset);
+int64_t oracle_kmeans_row_bits(const double* xs, const double* u, int64_t K, int bits,
+                               int64_t max_iter, double* c, uint8_t* code) {
+  return kmeans_row(xs, u, K, 1 << bits, max_iter, c, code);
+}
+
+int64_t oracle_kmeans_row(const double* xs, const double* u, int64_t K, int64_t max_iter,
+                          double* c, uint8_t* code) {
+  return kmeans_row(xs, u, K, 16, max_iter, c, code);
+}
+
+/* The whole quantiser for an [N][K] bf16 weight and n-bit codes: scale,
+ * offset, LUT [N][2^n] and codes [N][K].  iters[n] (may be NULL) receives the
+ * M-steps run on row n. */
+void oracle_quantize_bits(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
+                          int bits, int64_t max_iter, uint8_t* code, uint16_t* lut,
+                          uint16_t* scale, uint16_t* offset, int64_t* iters) {
+  const int nq = 1 << bits;
+  oracle_group_scale_bits(w, N, K, G, bits, scale, offset);
 #pragma omp parallel for schedule(dynamic)
   for (int64_t n = 0; n < N; ++n) {
     double* xs = (double*)malloc((size_t)K * sizeof(double));
@@ -356,14 +377,87 @@ void oracle_any4_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t
     for (int64_t k = 0; k < K; ++k)
       u[k] = (double)oracle_bf16_to_f32(scale[n * (K / G) + k / G]) * (double)ex[k];
     double c[16], table[16];
-    int64_t it = oracle_kmeans_row(xs, u, K, max_iter, c, code + n * K);
+    int64_t it = kmeans_row(xs, u, K, nq, max_iter, c, code + n * K);
     if (iters) iters[n] = it;
-    for (int q = 0; q < 16; ++q) {
-      lut[n * 16 + q] = oracle_bf16_rne((float)c[q]);
-      table[q] = (double)oracle_bf16_to_f32(lut[n * 16 + q]);
+    for (int q = 0; q < nq; ++q) {
+      lut[n * nq + q] = oracle_bf16_rne((float)c[q]);
+      table[q] = (double)oracle_bf16_to_f32(lut[n * nq + q]);
     }
-    assign_nearest(xs, K, table, code + n * K);
+    assign_nearest(xs, K, table, nq, code + n * K);
     free(xs);
     free(u);
   }
+}
+
+void oracle_any4_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
+                          int64_t max_iter, uint8_t* code, uint16_t* lut, uint16_t* scale,
+                          uint16_t* offset, int64_t* iters) {
+  oracle_quantize_bits(w, ex, N, K, G, 4, max_iter, code, lut, scale, offset, iters);
+}
+
+/* ------------------------------------------------------------------------- */
+/* n-bit storage (any3, any2; any4 is n = 4).  The pages give no layout below
+ * 4 bits.  Reading: the codes of a row form one little-endian bit stream,
+ * code k in bits [n k, n k + n) (bit i of the stream is bit i % 8 of byte
+ * i / 8); for n = 4 this is the nibble order above.  A row of K codes takes
+ * n K / 8 bytes (K % 8 == 0).  The table of a row has 2^n bf16 entries.      */
+/* ------------------------------------------------------------------------- */
+
+/* Returns how many codes were >= 2^bits (they are packed masked). */
+int64_t oracle_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K, int bits) {
+  const int64_t row_bytes = bits * K / 8;
+  const unsigned mask = (1u << bits) - 1u;
+  int64_t bad = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    uint8_t* row = packed + n * row_bytes;
+    memset(row, 0, (size_t)row_bytes);
+    for (int64_t k = 0; k < K; ++k) {
+      unsigned c = idx[n * K + k];
+      if (c > mask) ++bad;
+      for (int b = 0; b < bits; ++b) {
+        int64_t bit = (int64_t)bits * k + b;
+        if ((c >> b) & 1u) row[bit / 8] |= (uint8_t)(1u << (bit % 8));
+      }
+    }
+  }
+  return bad;
+}
+
+static unsigned code_at_bits(const uint8_t* row, int64_t k, int bits) {
+  unsigned c = 0;
+  for (int b = 0; b < bits; ++b) {
+    int64_t bit = (int64_t)bits * k + b;
+    c |= (unsigned)((row[bit / 8] >> (bit % 8)) & 1u) << b;
+  }
+  return c;
+}
+
+void oracle_unpack_bits(const uint8_t* packed, uint8_t* idx, int64_t N, int64_t K, int bits) {
+  const int64_t row_bytes = bits * K / 8;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      idx[n * K + k] = (uint8_t)code_at_bits(packed + n * row_bytes, k, bits);
+}
+
+/* W[n][k] = bf16_rne(fmaf(LUT[n][c], scale, offset)) with c the n-bit code;
+ * lut_row_stride is 2^bits (a table per row) or 0 (one table). */
+void oracle_dequant_bits(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
+                         const uint16_t* scale, const uint16_t* offset, uint16_t* W, int64_t N,
+                         int64_t K, int64_t G, int bits) {
+  const int64_t row_bytes = bits * K / 8;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      unsigned c = code_at_bits(packed + n * row_bytes, k, bits);
+      int64_t g = k / G;
+      W[n * K + k] = oracle_dequant_one(lut[n * lut_row_stride + c], scale[n * (K / G) + g],
+                                        offset[n * (K / G) + g]);
+    }
+  }
+}
+
+/* Storage per weight for n-bit codes: n + (2 x 16-bit group parameters) / G +
+ * 2^n x 16-bit table entries / K (the §2.4.1 accounting for any n). */
+double oracle_bits_per_weight_n(int64_t K, int64_t G, int bits) {
+  return (double)bits + 32.0 / (double)G + (16.0 * (double)(1 << bits)) / (double)K;
 }

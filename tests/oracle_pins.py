@@ -421,11 +421,11 @@ def pin_matmul_rows_equals_full():
 # (Eq. 23), Appendix A.1 Alg. 1 (k-means per row, sample weight alpha * E|x|)
 # --------------------------------------------------------------------------
 
-def _quantile_init(xs):
+def _quantile_init(xs, nq=16):
     """The initial table read from the pages: entry q is the element at
-    position floor(q (K - 1) / 15) of the row sorted by numpy."""
+    position floor(q (K - 1) / (nq - 1)) of the row sorted by numpy."""
     s = np.sort(np.asarray(xs, dtype=np.float64))
-    return s[[(q * (xs.size - 1)) // 15 for q in range(16)]]
+    return s[[(q * (xs.size - 1)) // (nq - 1) for q in range(nq)]]
 
 
 def _nearest(xs, table):
@@ -433,32 +433,33 @@ def _nearest(xs, table):
     return np.argmin(np.abs(xs[:, None] - table[None, :]), axis=1).astype(np.uint8)
 
 
-def _numpy_scale(w_bits, G):
+def _numpy_scale(w_bits, G, levels=15):
     """Eq. 1-2 with numpy fp32 (each operation correctly rounded) and torch's bf16 rounding."""
     N, K = w_bits.shape
     wf = torch_bf16_to_f64(w_bits).astype(np.float32).reshape(N, K // G, G) + np.float32(0)
     mn, mx = wf.min(axis=2), wf.max(axis=2)
-    return torch_bf16_bits((mx - mn) / np.float32(15)), torch_bf16_bits(mn)
+    return torch_bf16_bits((mx - mn) / np.float32(levels)), torch_bf16_bits(mn)
 
 
-def _sklearn_kmeans(xs, u, max_iter=500):
+def _sklearn_kmeans(xs, u, max_iter=500, nq=16):
     """scikit-learn's weighted Lloyd k-means (the library Appendix C.2 names),
     started from the quantile table."""
     from sklearn.cluster import KMeans
-    km = KMeans(n_clusters=16, init=_quantile_init(xs)[:, None], n_init=1, max_iter=max_iter,
-                tol=0.0, algorithm="lloyd").fit(xs[:, None], sample_weight=u)
+    km = KMeans(n_clusters=nq, init=_quantile_init(xs, nq)[:, None], n_init=1,
+                max_iter=max_iter, tol=0.0, algorithm="lloyd").fit(xs[:, None], sample_weight=u)
     return km.cluster_centers_[:, 0], km.labels_.astype(np.uint8)
 
 
 def _levels_problem(rng, N, K, G, levels):
-    """Groups holding exactly beta_g + alpha_g * levels (each level G/16 times,
-    shuffled), alpha_g a power of two: every value is exact in bf16."""
+    """Groups holding exactly beta_g + alpha_g * levels (each level
+    G / len(levels) times, shuffled), alpha_g a power of two: every value is
+    exact in bf16."""
     w = np.empty((N, K), dtype=np.float64)
     for n in range(N):
         for g in range(K // G):
             alpha = 2.0 ** -(5 + (n + g) % 3)
             beta = -(1 + (n * 7 + g) % 5) / 32.0
-            vals = beta + alpha * np.repeat(levels, G // 16)
+            vals = beta + alpha * np.repeat(levels, G // len(levels))
             w[n, g * G:(g + 1) * G] = rng.permutation(vals)
     bits = torch_bf16_bits(w.astype(np.float32))
     assert np.array_equal(torch_bf16_to_f64(bits), w), "levels not exact in bf16"
@@ -653,6 +654,135 @@ def pin_quantize_beats_int4_rounding():
         err_any4 = math.fsum((u * (ws - rec) ** 2).ravel())
         err_int4 = math.fsum((u * (ws - np.clip(np.round(ws), 0, 15)) ** 2).ravel())
         assert err_any4 < bound * err_int4, (G, err_any4 / err_int4)
+
+
+# --------------------------------------------------------------------------
+# n-bit variants: any3 and any2 (§4.1 Eq. 9: 2^n values per row; §5).  The
+# storage reading (the pages give none below 4 bits): a row's codes form one
+# little-endian bit stream, code k in bits [n k, n k + n).
+# --------------------------------------------------------------------------
+
+def pin_pack_bits_worked_examples():
+    # any3, codes 1..7 then 0: the 24-bit little-endian word sum(c_k << 3k)
+    # = 1 + 2*8 + 3*64 + 4*512 + 5*4096 + 6*32768 + 7*262144 = 0x1F58D1
+    assert oracle.pack_bits(np.array([[1, 2, 3, 4, 5, 6, 7, 0]], np.uint8), 3).tolist() == \
+        [[0xD1, 0x58, 0x1F]]
+    # any2, codes 0 1 2 3 | 3 2 1 0: bytes 0b11100100 and 0b00011011
+    assert oracle.pack_bits(np.array([[0, 1, 2, 3, 3, 2, 1, 0]], np.uint8), 2).tolist() == \
+        [[0xE4, 0x1B]]
+
+
+def pin_pack_bits_is_a_little_endian_bit_stream():
+    rng = np.random.default_rng(120)
+    for bits in (2, 3, 4):
+        idx = rng.integers(0, 1 << bits, size=(5, 64), dtype=np.uint8)
+        packed = oracle.pack_bits(idx, bits)
+        assert packed.shape == (5, bits * 64 // 8)
+        stream = np.unpackbits(packed, axis=1, bitorder="little").reshape(5, 64, bits)
+        assert np.array_equal((stream << np.arange(bits)).sum(axis=2), idx)   # numpy's decoder
+        assert np.array_equal(oracle.unpack_bits(packed, bits, 64), idx)
+        if bits == 4:
+            assert np.array_equal(packed, oracle.pack(idx))          # the any4 nibble order
+        bad = idx.copy()
+        bad[2, 7] = 1 << bits
+        try:
+            oracle.pack_bits(bad, bits)
+        except ValueError:
+            pass
+        else:
+            raise AssertionError("out-of-range code accepted")
+
+
+def pin_dequant_bits_reduces_to_any4():
+    """n-bit codes with a 2^n-entry table equal any4 codes with the table
+    padded to 16 entries (the padding is never indexed)."""
+    rng = np.random.default_rng(121)
+    N, K, G = 6, 256, 64
+    for bits in (2, 3):
+        nq = 1 << bits
+        idx = rng.integers(0, nq, size=(N, K), dtype=np.uint8)
+        lut = random_bf16(rng, (N, nq))
+        pad = random_bf16(rng, (N, 16 - nq))
+        scale = random_bf16(rng, (N, K // G), -8, -4)
+        offset = random_bf16(rng, (N, K // G), -10, -6)
+        W = oracle.dequant_bits(oracle.pack_bits(idx, bits), lut, scale, offset, G, bits, K)
+        W4 = oracle.dequant(oracle.pack(idx), np.concatenate([lut, pad], axis=1), scale, offset, G)
+        assert np.array_equal(W, W4)
+        one = lut[0]
+        Ws = oracle.dequant_bits(oracle.pack_bits(idx, bits), one, scale, offset, G, bits, K,
+                                 per_tensor_lut=True)
+        W4s = oracle.dequant(oracle.pack(idx), np.concatenate([one, pad[0]]), scale, offset, G,
+                             per_tensor_lut=True)
+        assert np.array_equal(Ws, W4s)
+
+
+def pin_bits_per_weight_n_accounting():
+    # the §2.4.1 accounting with 2^n table entries: any4 4.3125 (the paper's
+    # worked example), any3 3 + 0.25 + 0.03125, any2 2 + 0.25 + 0.015625
+    for bits, expect in ((4, 4.3125), (3, 3.28125), (2, 2.265625)):
+        assert oracle.bits_per_weight_n(4096, 128, bits) == expect
+    N, K, G = 3, 512, 64
+    for bits in (2, 3, 4):
+        nbytes = N * bits * K // 8 + 2 * 2 * N * (K // G) + 2 * N * (1 << bits)
+        assert oracle.bits_per_weight_n(K, G, bits) == 8 * nbytes / (N * K)
+
+
+def pin_quantize_bits_matches_scikit_learn_pipeline():
+    rng = np.random.default_rng(122)
+    N, K, G = 3, 256, 64
+    for bits in (2, 3):
+        nq = 1 << bits
+        w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+        ex = np.abs(rng.normal(0, 1, K)).astype(np.float32) + np.float32(0.05)
+        codes, lut, scale, offset, _ = oracle.quantize_bits(w, ex, G, bits, 300)
+        s_ref, o_ref = _numpy_scale(w, G, levels=nq - 1)
+        assert np.array_equal(scale, s_ref) and np.array_equal(offset, o_ref)
+        a = torch_bf16_to_f64(s_ref).repeat(G, axis=1)
+        b = torch_bf16_to_f64(o_ref).repeat(G, axis=1)
+        ws = (torch_bf16_to_f64(w) - b) / a
+        for n in range(N):
+            c_ref, _ = _sklearn_kmeans(ws[n], a[n] * ex.astype(np.float64), 300, nq)
+            lut_ref = torch_bf16_bits(c_ref.astype(np.float32))
+            assert np.array_equal(lut[n], lut_ref)
+            assert np.array_equal(codes[n], _nearest(ws[n], torch_bf16_to_f64(lut_ref)))
+
+
+def pin_quantize_bits_four_is_any4():
+    rng = np.random.default_rng(123)
+    w = torch_bf16_bits(rng.normal(0, 0.02, (5, 512)).astype(np.float32))
+    ex = rng.lognormal(0, 1, 512).astype(np.float32)
+    for a, b in zip(oracle.quantize_bits(w, ex, 128, 4, 60), oracle.quantize(w, ex, 128, 60)):
+        assert np.array_equal(a, b)
+
+
+def pin_quantize_bits_recovers_exact_levels():
+    rng = np.random.default_rng(124)
+    levels = np.array([0, 1, 2.5, 3, 4.25, 5.5, 6, 7])
+    N, K, G = 3, 256, 64
+    w = _levels_problem(rng, N, K, G, levels)
+    codes, lut, scale, offset, _ = oracle.quantize_bits(w, rng.uniform(0.1, 2, K).astype(np.float32),
+                                                        G, 3, 50)
+    assert np.array_equal(torch_bf16_to_f64(lut), np.tile(levels, (N, 1)))
+    a = torch_bf16_to_f64(scale).repeat(G, axis=1)
+    b = torch_bf16_to_f64(offset).repeat(G, axis=1)
+    assert np.array_equal(a * levels[codes] + b, torch_bf16_to_f64(w))
+
+
+def pin_quantize_bits_error_falls_with_more_bits():
+    """Weighted reconstruction error of w (weights E|x|): any2 > any3 > any4."""
+    rng = np.random.default_rng(125)
+    N, K, G = 4, 1024, 128
+    w = torch_bf16_bits(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    ex = rng.lognormal(0, 1, K).astype(np.float32)
+    wf = torch_bf16_to_f64(w)
+    errs = []
+    for bits in (2, 3, 4):
+        codes, lut, scale, offset, _ = oracle.quantize_bits(w, ex, G, bits, 100)
+        rec = (np.take_along_axis(torch_bf16_to_f64(lut), codes.astype(np.int64), 1)
+               * torch_bf16_to_f64(scale).repeat(G, axis=1)
+               + torch_bf16_to_f64(offset).repeat(G, axis=1))
+        errs.append(math.fsum((ex.astype(np.float64) * (wf - rec) ** 2).ravel()))
+    assert errs[0] > 2 * errs[1] > 4 * errs[2], errs
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -46,12 +46,12 @@ MUTANTS = [
      "      float acc = 0.0f;\n      for (int64_t k = 0; k < K; ++k) {\n        acc += (float)oracle_bf16_to_f32(x[m * K + k])"),
     ("matmul_rows_wrong_row", "    int64_t n = rows[r];", "    int64_t n = rows[r] + (r > 0);"),
     ("widen_wrong_shift", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
-    ("alpha_over_16", "float alpha = (mx - mn) / 15.0f;", "float alpha = (mx - mn) / 16.0f;"),
+    ("alpha_over_16", "float alpha = (mx - mn) / levels;", "float alpha = (mx - mn) / (levels + 1.0f);"),
     ("beta_is_max", "offset[n * (K / G) + g] = oracle_bf16_rne(mn);",
      "offset[n * (K / G) + g] = oracle_bf16_rne(mx);"),
     ("scaled_without_offset", "ws[k] = alpha > 0.0 ? ((double)canon_bf16(w[k]) - beta) / alpha : 0.0;",
      "ws[k] = alpha > 0.0 ? (double)canon_bf16(w[k]) / alpha : 0.0; (void)beta;"),
-    ("quantile_off_by_one", "c[q] = sorted[(q * (K - 1)) / 15];", "c[q] = sorted[(q * K) / 16];"),
+    ("quantile_off_by_one", "c[q] = sorted[(q * (K - 1)) / (nq - 1)];", "c[q] = sorted[(q * K) / nq];"),
     ("ties_to_highest", "      if (d < best) {", "      if (d <= best) {"),
     ("mstep_unweighted", "      num[code[j]] += u[j] * xs[j];\n      den[code[j]] += u[j];",
      "      num[code[j]] += xs[j];\n      den[code[j]] += 1.0;"),
@@ -62,9 +62,21 @@ MUTANTS = [
     ("sample_weight_without_alpha",
      "u[k] = (double)oracle_bf16_to_f32(scale[n * (K / G) + k / G]) * (double)ex[k];",
      "u[k] = (double)ex[k];"),
-    ("codes_from_unrounded_centroids", "    assign_nearest(xs, K, table, code + n * K);\n", "\n"),
-    ("one_lloyd_step_only", "    if (assign_nearest(xs, K, c, code) == 0) break;",
-     "    assign_nearest(xs, K, c, code);\n    break;"),
+    ("codes_from_unrounded_centroids", "    assign_nearest(xs, K, table, nq, code + n * K);\n", "\n"),
+    ("one_lloyd_step_only", "    if (assign_nearest(xs, K, c, nq, code) == 0) break;",
+     "    assign_nearest(xs, K, c, nq, code);\n    break;"),
+    ("pack_bits_msb_first", "if ((c >> b) & 1u) row[bit / 8] |= (uint8_t)(1u << (bit % 8));",
+     "if ((c >> b) & 1u) row[bit / 8] |= (uint8_t)(0x80u >> (bit % 8));"),
+    ("unpack_bits_reversed", "c |= (unsigned)((row[bit / 8] >> (bit % 8)) & 1u) << b;",
+     "c |= (unsigned)((row[bit / 8] >> (bit % 8)) & 1u) << (bits - 1 - b);"),
+    ("dequant_bits_row_zero_table",
+     "W[n * K + k] = oracle_dequant_one(lut[n * lut_row_stride + c], scale[n * (K / G) + g],",
+     "W[n * K + k] = oracle_dequant_one(lut[c], scale[n * (K / G) + g],"),
+    ("levels_is_two_to_the_n", "const float levels = (float)((1 << bits) - 1);",
+     "const float levels = (float)(1 << bits);"),
+    ("bits_per_weight_n_sixteen_entries",
+     "return (double)bits + 32.0 / (double)G + (16.0 * (double)(1 << bits)) / (double)K;",
+     "return (double)bits + 32.0 / (double)G + (16.0 * 16.0) / (double)K;"),
     ("storage_bits_one_param", "4.0 + (2.0 * (double)group_param_bits) / (double)G",
      "4.0 + (1.0 * (double)group_param_bits) / (double)G"),
 ]
