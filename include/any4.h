@@ -123,6 +123,40 @@ ANY4_API any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64
                                    any4_stream_t stream);
 
 /*
+ * n-bit variants: any3 and any2 (and any4 again as bits = 4).  The paper states
+ * the learned table for any bit width n (§4.1 Eq. 9: 2^n values per row) and
+ * evaluates 3 and 2 bits (§5); it gives no storage layout below 4 bits.
+ * Layout here: the codes of a row form one little-endian bit stream, code k in
+ * bits [n k, n k + n) (bit i of the stream is bit i % 8 of byte i / 8), so a
+ * packed row holds n K / 8 bytes; for n = 4 this is any4_pack's layout.  A
+ * row's table holds 2^n bf16 entries.  Shape rules and conventions as above;
+ * bits is 2, 3 or 4 (4 runs the any4 call of the same name).
+ *
+ * any4_pack_bits     idx [N][K] uint8 (codes 0 .. 2^n - 1) -> packed
+ *                    [N][n K / 8]; a larger code is packed masked to n bits
+ *                    and sets ANY4_ERR_RANGE in *dev_status.
+ * any4_dequant_bits  W[n][k] = bf16_rne(fmaf(LUT[n][c], scale[n][k/G],
+ *                    offset[n][k/G])) for the n-bit code c; lut_row_stride is
+ *                    2^n (a table per row) or 0 (one table).  Bit-exact.
+ * any4_quantize_bits any4_quantize with 2^n table entries: alpha =
+ *                    bf16(fp32(max - min) / (2^n - 1)), the quantile start at
+ *                    positions floor(q (K - 1) / (2^n - 1)), lut [N][2^n],
+ *                    packed [N][n K / 8]; otherwise the steps of
+ *                    any4_quantize.  The results are bit-identical on every
+ *                    run and GPU.
+ */
+ANY4_API any4_status any4_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                                    int32_t bits, int32_t* dev_status, any4_stream_t stream);
+ANY4_API any4_status any4_dequant_bits(const uint8_t* packed, const uint16_t* lut,
+                                       int64_t lut_row_stride, const uint16_t* scale,
+                                       const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
+                                       int64_t G, int32_t bits, any4_stream_t stream);
+ANY4_API any4_status any4_quantize_bits(const uint16_t* w, const float* ex_abs, int64_t N,
+                                        int64_t K, int64_t G, int32_t bits, int32_t max_iter,
+                                        uint8_t* packed, uint16_t* lut, uint16_t* scale,
+                                        uint16_t* offset, int32_t* iters, any4_stream_t stream);
+
+/*
  * any4_dequant -- materialise the bf16 weight (paper §2.5.2 dequant with the
  * per-row table of §2.4.1):
  *   W[n][k] = bf16_rne( fmaf( LUT[n][c], scale[n][k/G], offset[n][k/G] ) )

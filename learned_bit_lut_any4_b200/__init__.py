@@ -24,12 +24,15 @@ from ._native import (  # noqa: F401
     Any4Error,
     any4_bits_per_weight,
     any4_dequant,
+    any4_dequant_bits,
     any4_matmul,
     any4_matmul_choose_path,
     any4_matmul_static_scratch,
     any4_matmul_workspace_size,
     any4_pack,
+    any4_pack_bits,
     any4_quantize,
+    any4_quantize_bits,
     any4_status_string,
     any4_version,
     library,

@@ -60,6 +60,12 @@ def library() -> ctypes.CDLL:
     lib.any4_pack.restype = i32
     lib.any4_quantize.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
     lib.any4_quantize.restype = i32
+    lib.any4_quantize_bits.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.any4_quantize_bits.restype = i32
+    lib.any4_pack_bits.argtypes = [vp, vp, i64, i64, i32, vp, vp]
+    lib.any4_pack_bits.restype = i32
+    lib.any4_dequant_bits.argtypes = [vp, vp, i64, vp, vp, vp, i64, i64, i64, i32, vp]
+    lib.any4_dequant_bits.restype = i32
     lib.any4_dequant.argtypes = [vp, vp, i64, vp, vp, vp, i64, i64, i64, vp]
     lib.any4_dequant.restype = i32
     lib.any4_matmul.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp, vp]
@@ -197,6 +203,86 @@ def any4_quantize(w: torch.Tensor, ex_abs: torch.Tensor, G: int, max_iter: int =
     if return_iters:
         return packed, lut, scale, offset, iters
     return packed, lut, scale, offset
+
+
+def any4_quantize_bits(w: torch.Tensor, ex_abs: torch.Tensor, G: int, bits: int,
+                       max_iter: int = 100, return_iters: bool = False):
+    """any4_quantize with 2^bits table entries (bits 2, 3 or 4): packed
+    [N, bits*K/8] uint8 (one little-endian bit stream per row), lut [N, 2^bits],
+    scale and offset [N, K/G] in bf16 (+ int32 M-steps per row)."""
+    _need(w, "w", _BF16)
+    dev = w.device
+    _need(ex_abs, "ex_abs", (torch.float32,), dev)
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    if ex_abs.numel() != K:
+        raise ValueError(f"ex_abs must hold K={K} values")
+    if bits not in (2, 3, 4):
+        raise ValueError("bits must be 2, 3 or 4")
+    ng = K // G if G > 0 else 0
+    packed = torch.empty((N, bits * K // 8), dtype=torch.uint8, device=dev)
+    lut = torch.empty((N, 1 << bits), dtype=torch.bfloat16, device=dev)
+    scale = torch.empty((N, ng), dtype=torch.bfloat16, device=dev)
+    offset = torch.empty((N, ng), dtype=torch.bfloat16, device=dev)
+    iters = torch.empty(N, dtype=torch.int32, device=dev) if return_iters else None
+    with _on_device(dev):
+        _check(library().any4_quantize_bits(_ptr(w), _ptr(ex_abs), N, K, G, bits, int(max_iter),
+                                            _ptr(packed), _ptr(lut), _ptr(scale), _ptr(offset),
+                                            _ptr(iters), _stream(dev)), "any4_quantize_bits")
+    if return_iters:
+        return packed, lut, scale, offset, iters
+    return packed, lut, scale, offset
+
+
+def any4_pack_bits(idx: torch.Tensor, bits: int, packed: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """uint8 codes [N, K] (0 .. 2^bits - 1) -> packed [N, bits*K/8]: one
+    little-endian bit stream per row, code k in bits [bits*k, bits*k + bits)."""
+    _need(idx, "idx", (torch.uint8,))
+    N, K = idx.shape
+    if bits not in (2, 3, 4):
+        raise ValueError("bits must be 2, 3 or 4")
+    if packed is None:
+        packed = torch.empty((N, bits * K // 8), dtype=torch.uint8, device=idx.device)
+    _need(packed, "packed", (torch.uint8,), idx.device)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", (torch.int32,), idx.device)
+    with _on_device(idx.device):
+        _check(library().any4_pack_bits(_ptr(idx), _ptr(packed), N, K, bits, _ptr(dev_status),
+                                        _stream(idx.device)), "any4_pack_bits")
+    return packed
+
+
+def any4_dequant_bits(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
+                      offset: torch.Tensor, G: int, bits: int,
+                      W: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 W[N, K] from n-bit codes; lut is [N, 2^bits] or [2^bits] (one table)."""
+    _need(packed, "packed", (torch.uint8,))
+    dev = packed.device
+    if bits not in (2, 3, 4):
+        raise ValueError("bits must be 2, 3 or 4")
+    N, nb = packed.shape
+    K = nb * 8 // bits
+    nq = 1 << bits
+    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+        _need(t, nm, _BF16, dev)
+    if lut.dim() == 1 and lut.numel() == nq:
+        stride = 0
+    elif lut.dim() == 2 and tuple(lut.shape) == (N, nq):
+        stride = nq
+    else:
+        raise ValueError(f"lut must be [N, {nq}] or [{nq}], got {tuple(lut.shape)}")
+    if W is None:
+        W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    _need(W, "W", _BF16, dev)
+    if scale.numel() != N * (K // G if G else 0) or offset.numel() != scale.numel():
+        raise ValueError("scale and offset must hold N * K/G values")
+    with _on_device(dev):
+        _check(library().any4_dequant_bits(_ptr(packed), _ptr(lut), stride, _ptr(scale),
+                                           _ptr(offset), _ptr(W), N, K, G, bits, _stream(dev)),
+               "any4_dequant_bits")
+    return W
 
 
 def _lut_stride(lut: torch.Tensor, N: int) -> int:

@@ -20,12 +20,20 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
                                     size_t workspace_bytes, int32_t* dev_status,
                                     cudaStream_t stream, const DeviceInfo& dev);
 
-// Table learning (quantize.cu): one thread block per weight row.
+// Table learning (quantize.cu): one thread block per weight row; bits = 2, 3, 4.
 size_t quantize_smem_bytes(int64_t K, int64_t G);
 any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
-                            int32_t max_iter, uint8_t* packed, uint16_t* lut, uint16_t* scale,
-                            uint16_t* offset, int32_t* iters, cudaStream_t stream,
-                            const DeviceInfo& dev);
+                            int bits, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                            uint16_t* scale, uint16_t* offset, int32_t* iters,
+                            cudaStream_t stream, const DeviceInfo& dev);
+// n-bit storage below 4 bits (nbit.cu): bits = 2 or 3.
+any4_status launch_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                             int bits, int32_t* dev_status, cudaStream_t stream,
+                             const DeviceInfo& dev);
+any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
+                                int64_t lut_row_stride, const uint16_t* scale,
+                                const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
+                                int64_t G, int bits, cudaStream_t stream, const DeviceInfo& dev);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -136,7 +144,16 @@ any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64_t N, int
                           int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
                           uint16_t* scale, uint16_t* offset, int32_t* iters,
                           any4_stream_t stream) {
+  return any4_quantize_bits(w, ex_abs, N, K, G, 4, max_iter, packed, lut, scale, offset, iters,
+                            stream);
+}
+
+any4_status any4_quantize_bits(const uint16_t* w, const float* ex_abs, int64_t N, int64_t K,
+                               int64_t G, int32_t bits, int32_t max_iter, uint8_t* packed,
+                               uint16_t* lut, uint16_t* scale, uint16_t* offset, int32_t* iters,
+                               any4_stream_t stream) {
   if (!w || !ex_abs || !packed || !lut || !scale || !offset) return ANY4_ERR_NULL;
+  if (bits < 2 || bits > 4) return ANY4_ERR_SHAPE;
   if (!shape_ok(N, K, G) || K > ANY4_QUANTIZE_MAX_K || N > INT32_MAX || max_iter < 0 ||
       max_iter > ANY4_QUANTIZE_MAX_ITER)
     return ANY4_ERR_SHAPE;
@@ -147,8 +164,42 @@ any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64_t N, int
   DeviceInfo dev;
   any4_status st = current_device(&dev);
   if (st != ANY4_OK) return st;
-  return launch_quantize(w, ex_abs, N, K, G, max_iter, packed, lut, scale, offset, iters,
+  return launch_quantize(w, ex_abs, N, K, G, bits, max_iter, packed, lut, scale, offset, iters,
                          (cudaStream_t)stream, dev);
+}
+
+any4_status any4_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                           int32_t bits, int32_t* dev_status, any4_stream_t stream) {
+  if (bits == 4) return any4_pack(idx, packed, N, K, dev_status, stream);
+  if (!idx || !packed) return ANY4_ERR_NULL;
+  if (bits < 2 || bits > 3 || N < 1 || K < 32 || K % 32 != 0 || N > (int64_t(1) << 40) / K)
+    return ANY4_ERR_SHAPE;
+  if (!aligned16(idx) || !aligned16(packed)) return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_pack_bits(idx, packed, N, K, bits, dev_status, (cudaStream_t)stream, dev);
+}
+
+any4_status any4_dequant_bits(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
+                              const uint16_t* scale, const uint16_t* offset, uint16_t* W,
+                              int64_t N, int64_t K, int64_t G, int32_t bits,
+                              any4_stream_t stream) {
+  if (bits == 4)
+    return any4_dequant(packed, lut, lut_row_stride, scale, offset, W, N, K, G, stream);
+  if (!packed || !lut || !scale || !offset || !W) return ANY4_ERR_NULL;
+  if (bits < 2 || bits > 3 || !shape_ok(N, K, G) ||
+      (lut_row_stride != 0 && lut_row_stride != (int64_t(1) << bits)))
+    return ANY4_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(lut) || !aligned16(scale) || !aligned16(offset) ||
+      !aligned16(W))
+    return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_dequant_bits(packed, lut, lut_row_stride, scale, offset, W, N, K, G, bits,
+                             (cudaStream_t)stream, dev);
 }
 
 any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,

@@ -1,0 +1,182 @@
+// n-bit storage below 4 bits (any3, any2): pack and dequant kernels (sm_100a).
+//
+// "any4: Learned 4-bit Numeric Representation for LLMs" states the table for
+// any bit width (§4.1 Eq. 9: 2^n values per row) and evaluates any3 and any2
+// (§5); it gives no storage layout below 4 bits.  Layout here: the codes of a
+// row form one little-endian bit stream, code k in bits [n k, n k + n), so a
+// row of K codes takes n K / 8 bytes (for n = 4 this is any4's nibble order,
+// which any4_pack / any4_dequant already serve).  A thread handles one chunk
+// of 32 codes: n 32-bit words, inside one row (K % 32 == 0) and one group
+// (G % 32 == 0).  Both kernels are streaming and HBM-bound; grids are a
+// multiple of the SM count and loop over the chunks.
+#include "common.cuh"
+
+namespace any4 {
+namespace {
+
+constexpr int kNbThreads = 256;
+
+template <int BITS>
+__device__ __forceinline__ void load_chunk(const uint8_t* p, uint32_t (&v)[BITS]) {
+  if constexpr (BITS == 2) {
+    const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = t.x;
+    v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int b = 0; b < BITS; ++b) v[b] = __ldg(reinterpret_cast<const uint32_t*>(p) + b);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_chunk(uint8_t* p, const uint32_t (&v)[BITS]) {
+  if constexpr (BITS == 2) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int b = 0; b < BITS; ++b) reinterpret_cast<uint32_t*>(p)[b] = v[b];
+  }
+}
+
+// Code k (0..31) of a chunk held in BITS words.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_of(const uint32_t (&v)[BITS], int k) {
+  const int bit = BITS * k, w = bit >> 5, off = bit & 31;
+  uint32_t c = v[w] >> off;
+  if (off + BITS > 32) c |= v[w + 1] << (32 - off);
+  return c & ((1u << BITS) - 1u);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kNbThreads)
+pack_bits_kernel(const uint8_t* __restrict__ idx, uint8_t* __restrict__ packed, int64_t chunks,
+                 int32_t* dev_status) {
+  constexpr uint32_t kMask = (1u << BITS) - 1u;
+  constexpr uint32_t kHigh = (~kMask & 0xffu) * 0x01010101u;  // bits no code may set
+  uint32_t bad = 0;
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 a = ldg_stream_v4(idx + c * 32);
+    const uint4 b = ldg_stream_v4(idx + c * 32 + 16);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t v[BITS];
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) v[i] = 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const uint32_t cd = (in[k >> 2] >> (8 * (k & 3))) & kMask;
+      const int bit = BITS * k, w = bit >> 5, off = bit & 31;
+      v[w] |= cd << off;
+      if (off + BITS > 32) v[w + 1] |= cd >> (32 - off);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bad |= in[i] & kHigh;
+    store_chunk<BITS>(packed + c * (4 * BITS), v);
+  }
+  if (__any_sync(kFullMask, bad != 0u)) {
+    if ((threadIdx.x & 31) == 0) report_status(dev_status, (int32_t)ANY4_ERR_RANGE);
+  }
+}
+
+// Table entry `code` of a row table held as bf16 pairs in registers: t0..t3
+// hold entries (0,1) (2,3) (4,5) (6,7); with 4 entries only t0, t1 are used.
+template <int BITS>
+__device__ __forceinline__ float table_entry(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
+                                             uint32_t code) {
+  const uint32_t e = code & 3u;
+  const uint32_t sel = (2u * e) | ((2u * e + 1u) << 4);   // bytes 2e, 2e+1 of the pair
+  uint32_t v;
+  if constexpr (BITS == 3) {
+    v = (code & 4u) ? __byte_perm(t2, t3, sel) : __byte_perm(t0, t1, sel);
+  } else {
+    v = __byte_perm(t0, t1, sel);
+  }
+  return __uint_as_float(v << 16);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kNbThreads)
+dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut,
+                    int64_t lut_row_stride, const uint16_t* __restrict__ scale,
+                    const uint16_t* __restrict__ offset, uint16_t* __restrict__ W, int64_t N,
+                    int64_t K, int64_t G) {
+  const int64_t chunks_per_row = K / 32;
+  const int64_t chunks = N * chunks_per_row;
+  const int64_t groups = K / G;
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = c / chunks_per_row;
+    const int64_t k0 = (c - n * chunks_per_row) * 32;
+    const int64_t g = k0 / G;
+    const float s = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
+    const float o = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
+    uint32_t t0, t1, t2 = 0, t3 = 0;
+    if constexpr (BITS == 3) {
+      const uint4 t = __ldg(reinterpret_cast<const uint4*>(lut + n * lut_row_stride));
+      t0 = t.x;
+      t1 = t.y;
+      t2 = t.z;
+      t3 = t.w;
+    } else {
+      const uint2 t = __ldg(reinterpret_cast<const uint2*>(lut + n * lut_row_stride));
+      t0 = t.x;
+      t1 = t.y;
+    }
+    uint32_t v[BITS];
+    load_chunk<BITS>(packed + c * (4 * BITS), v);
+    uint32_t out[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const float lo = __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(v, 2 * p)), s, o);
+      const float hi =
+          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(v, 2 * p + 1)), s, o);
+      out[p] = pack_bf16x2_rn(lo, hi);
+    }
+    uint16_t* dst = W + n * K + k0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      stg_stream_v4(dst + 8 * q, make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2],
+                                            out[4 * q + 3]));
+  }
+}
+
+int nb_grid(int64_t chunks, const DeviceInfo& dev) {
+  const int64_t want = (chunks + kNbThreads - 1) / kNbThreads;
+  const int64_t cap = (int64_t)dev.sm_count * 8;
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+any4_status launch_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
+                             int bits, int32_t* dev_status, cudaStream_t stream,
+                             const DeviceInfo& dev) {
+  const int64_t chunks = N * K / 32;
+  if (bits == 3)
+    pack_bits_kernel<3><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(idx, packed, chunks,
+                                                                          dev_status);
+  else if (bits == 2)
+    pack_bits_kernel<2><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(idx, packed, chunks,
+                                                                          dev_status);
+  else
+    return ANY4_ERR_SHAPE;
+  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
+                                int64_t lut_row_stride, const uint16_t* scale,
+                                const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
+                                int64_t G, int bits, cudaStream_t stream, const DeviceInfo& dev) {
+  const int64_t chunks = N * K / 32;
+  if (bits == 3)
+    dequant_bits_kernel<3><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(
+        packed, lut, lut_row_stride, scale, offset, W, N, K, G);
+  else if (bits == 2)
+    dequant_bits_kernel<2><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(
+        packed, lut, lut_row_stride, scale, offset, W, N, K, G);
+  else
+    return ANY4_ERR_SHAPE;
+  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+}  // namespace any4

@@ -1,9 +1,11 @@
 // Learning the table of each row: the quantiser that produces the packed codes,
 // tables, scales and offsets the matmul consumes.
 //
-// "any4: Learned 4-bit Numeric Representation for LLMs":
-//   §2.5.1 Eq. 1-2   group-wise scaling: alpha = (max - min) / 15, beta = min,
-//                    scaled weight w_S = (w - beta) / alpha;
+// "any4: Learned 4-bit Numeric Representation for LLMs", for n-bit codes
+// (§4.1 Eq. 9: 2^n table entries per row; n = 4 is any4, §5 evaluates any3
+// and any2):
+//   §2.5.1 Eq. 1-2   group-wise scaling: alpha = (max - min) / (2^n - 1),
+//                    beta = min, scaled weight w_S = (w - beta) / alpha;
 //   §4.1 Eq. 18      E-step: each scaled weight takes its nearest table entry;
 //   §4.1 Eq. 23      M-step: an entry becomes the mean of its cluster's scaled
 //                    weights, weighted by alpha_{i,j} * E|x_j|;
@@ -14,11 +16,12 @@
 // intrinsic (nothing is contracted into a fused multiply-add), taken in the order
 // of a sequential loop, so the results are bit-identical to a plain sequential
 // statement of the same steps:
-//   - alpha = bf16(fp32(fp32(max - min) / 15)), beta = min (exact in bf16);
+//   - alpha = bf16(fp32(fp32(max - min) / (2^n - 1))), beta = min (exact in bf16);
 //     w is read with -0 as +0;
 //   - w_S = ((double)w - beta) / alpha in fp64, 0 in a group whose alpha is 0;
-//   - initial table: entry q = the element at position floor(q (K - 1) / 15)
-//     of the sorted row (a bitonic sort in shared memory);
+//   - initial table: entry q = the element at position
+//     floor(q (K - 1) / (2^n - 1)) of the sorted row (a bitonic sort in
+//     shared memory);
 //   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q;
 //   - M-step: sample weight u_j = alpha_{g(j)} * E|x_j| (exact in fp64);
 //     numerator sum(u_j * w_S_j) and denominator sum(u_j) over ascending j,
@@ -26,7 +29,8 @@
 //     sequential one; a cluster whose weights sum to 0 keeps its entry;
 //   - stop after max_iter M-steps, or when an E-step changes no code;
 //   - LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
-//     LUT, packed two per byte (even column in the low nibble).
+//     LUT, packed as one little-endian bit stream per row (code k in bits
+//     [n k, n k + n); for n = 4 two per byte, even column in the low nibble).
 #include <cstdint>
 
 #include "common.cuh"
@@ -72,19 +76,20 @@ __device__ __forceinline__ double scaled_weight(float w, float alpha, float beta
   return alpha > 0.0f ? __ddiv_rn(__dsub_rn((double)w, (double)beta), (double)alpha) : 0.0;
 }
 
-// E-step over the row: nearest entry of c (ties to the lowest index).  Returns
-// (uniformly across the block) whether any code changed.
+// E-step over the row: nearest of the NQ entries of c (ties to the lowest
+// index).  Returns (uniformly across the block) whether any code changed.
+template <int NQ>
 __device__ __forceinline__ bool estep(const double* xs, int K, const double* c, uint8_t* code) {
-  double cr[16];
+  double cr[NQ];
 #pragma unroll
-  for (int q = 0; q < 16; ++q) cr[q] = c[q];
+  for (int q = 0; q < NQ; ++q) cr[q] = c[q];
   int changed = 0;
   for (int j = threadIdx.x; j < K; j += kQuantThreads) {
     const double x = xs[j];
     double best = fabs(__dsub_rn(x, cr[0]));
     int bq = 0;
 #pragma unroll
-    for (int q = 1; q < 16; ++q) {
+    for (int q = 1; q < NQ; ++q) {
       const double d = fabs(__dsub_rn(x, cr[q]));
       if (d < best) {
         best = d;
@@ -97,6 +102,8 @@ __device__ __forceinline__ bool estep(const double* xs, int K, const double* c, 
   return __syncthreads_or(changed) != 0;
 }
 
+// NQ = 2^n table entries (4, 8 or 16); the packed row has n K / 8 bytes.
+template <int NQ>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, int K, int G,
                 int max_iter, uint8_t* __restrict__ packed, uint16_t* __restrict__ lut,
@@ -137,7 +144,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
       mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, s));
     }
     if (lane == 0) {
-      const uint16_t a = f32_to_bf16_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+      const uint16_t a = f32_to_bf16_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)(NQ - 1)));
       const uint16_t b = (uint16_t)(__float_as_uint(mn) >> 16);   // mn is a bf16 value
       scale[n * NG + g] = a;
       offset[n * NG + g] = b;
@@ -168,20 +175,21 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
       __syncthreads();
     }
   }
-  if (tid < 16) cent[tid] = xs[(int)(((int64_t)tid * (K - 1)) / 15)];
+  if (tid < NQ) cent[tid] = xs[(int)(((int64_t)tid * (K - 1)) / (NQ - 1))];
   __syncthreads();
   for (int j = tid; j < K; j += kQuantThreads)
     xs[j] = scaled_weight(bf16_canon(wrow[j]), alpha_s[j / G], beta_s[j / G]);
   __syncthreads();
 
-  estep(xs, K, cent, code);
+  estep<NQ>(xs, K, cent, code);
   int it = 0;
   while (it < max_iter) {
     if (warp == 0) {
-      // Eq. 23: lane q sums u_j * w_S_j, lane 16 + q sums u_j, over the
-      // columns of cluster q in ascending order.
-      const int q = lane & 15;
-      const bool den = lane >= 16;
+      // Eq. 23: lane q sums u_j * w_S_j, lane NQ + q sums u_j, over the
+      // columns of cluster q in ascending order (lanes from 2 NQ up repeat
+      // that work and write nothing).
+      const int q = lane & (NQ - 1);
+      const bool den = (lane & NQ) != 0;
       double acc = 0.0;
       for (int g = 0; g < NG; ++g) {
         const double a = (double)alpha_s[g];
@@ -193,39 +201,59 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
           if (code[j] == q) acc = __dadd_rn(acc, t);
         }
       }
-      const double d = __shfl_down_sync(kFullMask, acc, 16);
-      if (lane < 16 && d > 0.0) cent[q] = __ddiv_rn(acc, d);
+      const double d = __shfl_down_sync(kFullMask, acc, NQ);
+      if (lane < NQ && d > 0.0) cent[q] = __ddiv_rn(acc, d);
     }
     __syncthreads();
     ++it;
-    if (!estep(xs, K, cent, code)) break;
+    if (!estep<NQ>(xs, K, cent, code)) break;
   }
 
-  if (tid < 16) {
+  if (tid < NQ) {
     const uint16_t b = f32_to_bf16_rn(__double2float_rn(cent[tid]));
-    lut[n * 16 + tid] = b;
+    lut[n * NQ + tid] = b;
     table[tid] = (double)__uint_as_float((uint32_t)b << 16);
   }
   if (tid == 0 && iters) iters[n] = it;
   __syncthreads();
-  estep(xs, K, table, code);
+  estep<NQ>(xs, K, table, code);
 
-  // Pack 32 codes (16 bytes) per thread step; K % 32 == 0.
-  uint4* prow = reinterpret_cast<uint4*>(packed + n * (int64_t)(K / 2));
+  // Pack 32 codes (BITS words) per thread step; K % 32 == 0.
+  constexpr int BITS = NQ == 16 ? 4 : (NQ == 8 ? 3 : 2);
+  uint32_t* prow = reinterpret_cast<uint32_t*>(packed + n * (int64_t)(K / 8 * BITS));
   for (int c = tid; c < K / 32; c += kQuantThreads) {
-    uint32_t v[4];
+    uint32_t v[BITS];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      uint32_t word = 0;
+    for (int b = 0; b < BITS; ++b) v[b] = 0;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int j = c * 32 + b * 8 + h * 2;
-        word |= (uint32_t)(code[j] | (code[j + 1] << 4)) << (8 * h);
-      }
-      v[b] = word;
+    for (int k = 0; k < 32; ++k) {
+      const uint32_t cd = code[c * 32 + k];
+      const int bit = BITS * k, w = bit >> 5, off = bit & 31;
+      v[w] |= cd << off;
+      if (off + BITS > 32) v[w + 1] |= cd >> (32 - off);
     }
-    prow[c] = make_uint4(v[0], v[1], v[2], v[3]);
+    if constexpr (BITS == 4) {
+      reinterpret_cast<uint4*>(prow)[c] = make_uint4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (BITS == 2) {
+      reinterpret_cast<uint2*>(prow)[c] = make_uint2(v[0], v[1]);
+    } else {
+#pragma unroll
+      for (int b = 0; b < BITS; ++b) prow[c * BITS + b] = v[b];
+    }
   }
+}
+
+template <int NQ>
+any4_status launch_quantize_nq(const uint16_t* w, const float* ex, int64_t N, int64_t K,
+                               int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                               uint16_t* scale, uint16_t* offset, int32_t* iters, size_t smem,
+                               cudaStream_t stream) {
+  if (cudaFuncSetAttribute(quantize_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ANY4_ERR_CUDA;
+  quantize_kernel<NQ><<<(unsigned)N, kQuantThreads, smem, stream>>>(
+      w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
+  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
 }  // namespace
@@ -233,17 +261,24 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
 size_t quantize_smem_bytes(int64_t K, int64_t G) { return quant_smem_layout(K, G).total; }
 
 any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
-                            int32_t max_iter, uint8_t* packed, uint16_t* lut, uint16_t* scale,
-                            uint16_t* offset, int32_t* iters, cudaStream_t stream,
-                            const DeviceInfo& dev) {
+                            int bits, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                            uint16_t* scale, uint16_t* offset, int32_t* iters,
+                            cudaStream_t stream, const DeviceInfo& dev) {
   const size_t smem = quantize_smem_bytes(K, G);
   if (smem > dev.smem_optin) return ANY4_ERR_SHAPE;
-  if (cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return ANY4_ERR_CUDA;
-  quantize_kernel<<<(unsigned)N, kQuantThreads, smem, stream>>>(
-      w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
-  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+  switch (bits) {
+    case 4:
+      return launch_quantize_nq<16>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
+                                    smem, stream);
+    case 3:
+      return launch_quantize_nq<8>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
+                                   smem, stream);
+    case 2:
+      return launch_quantize_nq<4>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
+                                   smem, stream);
+    default:
+      return ANY4_ERR_SHAPE;
+  }
 }
 
 }  // namespace any4

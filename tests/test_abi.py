@@ -124,6 +124,38 @@ def test_quantize_rejects_bad_arguments(kw, expect):
                                            a["offset"], a["iters"], None) == expect
 
 
+def test_nbit_calls_reject_bad_arguments():
+    lib = _native.library()
+    E = any4
+    # pack: bits outside 2..4, shapes, alignment
+    assert lib.any4_pack_bits(FAKE, FAKE, 4, 64, 5, None, None) == E.ANY4_ERR_SHAPE
+    assert lib.any4_pack_bits(FAKE, FAKE, 4, 64, 1, None, None) == E.ANY4_ERR_SHAPE
+    assert lib.any4_pack_bits(None, FAKE, 4, 64, 3, None, None) == E.ANY4_ERR_NULL
+    assert lib.any4_pack_bits(FAKE, FAKE, 4, 48, 3, None, None) == E.ANY4_ERR_SHAPE
+    assert lib.any4_pack_bits(FAKE, FAKE + 4, 4, 64, 2, None, None) == E.ANY4_ERR_ALIGN
+    assert lib.any4_pack_bits(FAKE + 1, FAKE, 4, 64, 4, None, None) == E.ANY4_ERR_ALIGN
+    # dequant: the table stride must be 2^bits or 0
+    assert lib.any4_dequant_bits(FAKE, FAKE, 16, FAKE, FAKE, FAKE, 4, 64, 32, 3, None) == \
+        E.ANY4_ERR_SHAPE
+    assert lib.any4_dequant_bits(FAKE, FAKE, 8, FAKE, FAKE, FAKE, 4, 64, 48, 3, None) == \
+        E.ANY4_ERR_SHAPE
+    assert lib.any4_dequant_bits(FAKE, FAKE, 4, FAKE, FAKE, None, 4, 64, 32, 2, None) == \
+        E.ANY4_ERR_NULL
+    assert lib.any4_dequant_bits(FAKE, FAKE + 2, 4, FAKE, FAKE, FAKE, 4, 64, 32, 2, None) == \
+        E.ANY4_ERR_ALIGN
+    assert lib.any4_dequant_bits(FAKE, FAKE, 8, FAKE, FAKE, FAKE, 4, 64, 32, 6, None) == \
+        E.ANY4_ERR_SHAPE
+    # quantize: bits, and the any4 limits
+    q = lib.any4_quantize_bits
+    assert q(FAKE, FAKE, 4, 256, 64, 1, 10, FAKE, FAKE, FAKE, FAKE, None, None) == E.ANY4_ERR_SHAPE
+    assert q(FAKE, FAKE, 4, 256, 64, 5, 10, FAKE, FAKE, FAKE, FAKE, None, None) == E.ANY4_ERR_SHAPE
+    assert q(FAKE, FAKE, 4, 256, 48, 3, 10, FAKE, FAKE, FAKE, FAKE, None, None) == E.ANY4_ERR_SHAPE
+    assert q(FAKE, None, 4, 256, 64, 2, 10, FAKE, FAKE, FAKE, FAKE, None, None) == E.ANY4_ERR_NULL
+    assert q(FAKE, FAKE, 4, 256, 64, 3, -1, FAKE, FAKE, FAKE, FAKE, None, None) == E.ANY4_ERR_SHAPE
+    assert q(FAKE, FAKE, 4, 256, 64, 2, 10, FAKE, FAKE + 8, FAKE, FAKE, None, None) == \
+        E.ANY4_ERR_ALIGN
+
+
 def test_workspace_size_of_bad_shapes_is_zero():
     assert any4.any4_matmul_workspace_size(1, 64, 48, 48) == 0
     assert any4.any4_matmul_workspace_size(0, 64, 64, 32) == 0
