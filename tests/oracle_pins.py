@@ -303,8 +303,8 @@ def pin_dequant_invariants():
     W = oracle.dequant(oracle.pack(idx), lut, scale, offset, G)
     # permuting each row's table and relabelling its codes leaves W unchanged
     for trial in range(3):
-        perm = np.stack([rng.permutation(16) for _ in range(N)])      # new slot j holds old entry perm[j]
-        inv = np.argsort(perm, axis=1)                                   # old entry c sits at slot inv[c]
+        perm = np.stack([rng.permutation(16) for _ in range(N)])  # slot j holds old entry perm[j]
+        inv = np.argsort(perm, axis=1)                              # old entry c sits at slot inv[c]
         lut_p = np.take_along_axis(lut, perm, axis=1)
         idx_p = np.take_along_axis(inv, idx.astype(np.int64), axis=1).astype(np.uint8)
         assert np.array_equal(oracle.dequant(oracle.pack(idx_p), lut_p, scale, offset, G), W)
@@ -760,8 +760,8 @@ def pin_quantize_bits_recovers_exact_levels():
     levels = np.array([0, 1, 2.5, 3, 4.25, 5.5, 6, 7])
     N, K, G = 3, 256, 64
     w = _levels_problem(rng, N, K, G, levels)
-    codes, lut, scale, offset, _ = oracle.quantize_bits(w, rng.uniform(0.1, 2, K).astype(np.float32),
-                                                        G, 3, 50)
+    ex = rng.uniform(0.1, 2, K).astype(np.float32)
+    codes, lut, scale, offset, _ = oracle.quantize_bits(w, ex, G, 3, 50)
     assert np.array_equal(torch_bf16_to_f64(lut), np.tile(levels, (N, 1)))
     a = torch_bf16_to_f64(scale).repeat(G, axis=1)
     b = torch_bf16_to_f64(offset).repeat(G, axis=1)
