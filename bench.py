@@ -15,7 +15,8 @@ copies that the working set exceeds L2 (every step reads cold weights).
 Also reported (same run, not part of the step): the prefill matmuls at
 M = 2048 (TFLOPS), the roofline object of the decode kernel, the CPU oracle
 as a baseline, the end-to-end number through the public API with host
-buffers, and the clocks seen during the timed region.
+buffers, the clocks seen during the timed region, and the time any4_quantize
+takes to learn the tables of the Llama3-8B matrices, beside the oracle.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -535,10 +536,10 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def quantize_detail(max_iter: int, cpu_seconds: float):
+def table_learning_detail(max_iter: int, cpu_seconds: float, reps: int = 3):
     """Time any4_quantize (learning the tables) on the Llama3-8B layer matrices
     with CUDA events on the launching stream, and the oracle beside it on a
-    bounded sample of rows of each matrix; one JSON line."""
+    bounded sample of rows of each matrix (about cpu_seconds in all)."""
     import torch
     import oracle
     import learned_bit_lut_any4_b200 as any4
@@ -552,7 +553,6 @@ def quantize_detail(max_iter: int, cpu_seconds: float):
         ex = torch.from_numpy(ex_np).cuda()
         any4.any4_quantize(w, ex, s.G, max_iter)            # warm-up (module load, attributes)
         torch.cuda.synchronize()
-        reps = 3
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(reps):
@@ -580,7 +580,7 @@ def quantize_detail(max_iter: int, cpu_seconds: float):
                     "mstep_columns_per_s": round(float(it.sum() * s.K) / ms * 1e3, 1),
                     "oracle_rows": rows, "oracle_rows_per_s": round(rows / dt, 2),
                     "oracle_cores": oracle.num_threads()})
-    print(json.dumps({"detail": "quantize", "shapes": out}), flush=True)
+    return out
 
 
 def profile_shape(name: str, calls: int):
@@ -624,12 +624,16 @@ def main():
                     help="no step: time any4_quantize on the Llama3-8B matrices (and the "
                          "oracle on a sample of rows) and print one JSON line")
     ap.add_argument("--quantize-iters", type=int, default=100)
+    ap.add_argument("--skip-table-learning", action="store_true",
+                    help="leave the any4_quantize timing out of the JSON line")
     args = ap.parse_args()
     if args.profile_shape:
         profile_shape(args.profile_shape, args.profile_calls)
         return
     if args.quantize_detail:
-        quantize_detail(args.quantize_iters, args.cpu_seconds)
+        print(json.dumps({"detail": "quantize",
+                          "shapes": table_learning_detail(args.quantize_iters, args.cpu_seconds)}),
+              flush=True)
         return
     if args.warmup < 3:
         args.warmup = 3
@@ -647,6 +651,13 @@ def main():
             return
         peaks = r["peaks"]
         cpu = oracle_layer_rate(max_seconds=args.cpu_seconds) if world == 1 else None
+        table = None
+        if world == 1 and not args.skip_table_learning:
+            try:  # a detail beside the step: its failure is reported, not fatal
+                table = {"max_iter": args.quantize_iters,
+                         "matrices": table_learning_detail(args.quantize_iters, 4.0, reps=2)}
+            except Exception as e:  # pragma: no cover - only on a GPU machine
+                table = {"error": f"{type(e).__name__}: {e}"}
         achieved = r["value"] / world  # per-GPU decode throughput over the whole step
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -674,6 +685,7 @@ def main():
             "prefill_m2048": r["prefill"],
             "detail_batch": r["batch"],
             "fig3_square_m1": r["fig3"],
+            "table_learning": table,
         }
         print(json.dumps(line), flush=True)
     finally:
