@@ -190,3 +190,24 @@ def test_product_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "any4_oracle" not in text, fn
+
+
+def test_bindings_refuse_host_tensors_and_wrong_dtypes():
+    """The Python binding checks dtype and device before any library call; a
+    host tensor is refused (there is no CPU path)."""
+    import torch
+    w = torch.zeros((4, 256), dtype=torch.bfloat16)
+    ex = torch.zeros(256, dtype=torch.float32)
+    idx = torch.zeros((4, 256), dtype=torch.uint8)
+    for call in (lambda: any4.any4_quantize(w, ex, 64),
+                 lambda: any4.any4_quantize_bits(w, ex, 64, 3),
+                 lambda: any4.any4_pack_bits(idx, 3),
+                 lambda: any4.any4_pack(idx)):
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+    with pytest.raises(TypeError):
+        any4.any4_quantize(w.float(), ex, 64)
+    with pytest.raises(TypeError):
+        any4.any4_pack_bits(idx.to(torch.int32), 2)
+    with pytest.raises(TypeError):
+        any4.any4_dequant_bits(idx.float(), w, w, w, 64, 3)
