@@ -365,6 +365,31 @@ def gpu_arm(args, rank, world):
                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
         del g
 
+    # single-call latency of each M = 1 shape: one launch between an event
+    # pair, after a write of twice the L2 size (cold caches); 3 discarded, 20 kept
+    single = {}
+    try:  # a detail beside the step: its failure is reported, not fatal
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+        for (s, reps, x, y, _) in sets:
+            w = reps[0]
+            times = []
+            with torch.cuda.stream(stream):
+                for i in range(23):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y)
+                    b.record(stream)
+                    b.synchronize()
+                    if i >= 3:
+                        times.append(a.elapsed_time(b) * 1e3)
+            single[s.name] = {"us_median": round(float(np.median(times)), 2),
+                              "us_best": round(float(min(times)), 2)}
+        del flush
+        torch.cuda.synchronize()
+    except Exception as e:  # pragma: no cover - only on a GPU machine
+        single = {"error": f"{type(e).__name__}: {e}"}
+
     # prefill (M = 2048), TFLOPS against the bf16 peak
     prefill = {}
     if not args.skip_prefill:
@@ -478,7 +503,8 @@ def gpu_arm(args, rank, world):
 
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
-        "clocks": clocks, "detail": detail, "prefill": prefill, "batch": batch, "fig3": fig3,
+        "clocks": clocks, "detail": detail, "single": single, "prefill": prefill,
+        "batch": batch, "fig3": fig3,
         "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -682,6 +708,7 @@ def main():
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
             "detail_m1": r["detail"],
+            "single_call_m1": r["single"],
             "prefill_m2048": r["prefill"],
             "detail_batch": r["batch"],
             "fig3_square_m1": r["fig3"],
