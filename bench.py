@@ -15,8 +15,9 @@ copies that the working set exceeds L2 (every step reads cold weights).
 Also reported (same run, not part of the step): the prefill matmuls at
 M = 2048 (TFLOPS), the roofline object of the decode kernel, the CPU oracle
 as a baseline, the end-to-end number through the public API with host
-buffers, the clocks seen during the timed region, and the time any4_quantize
-takes to learn the tables of the Llama3-8B matrices, beside the oracle.
+buffers, the clocks seen during the timed region, the single-call latency of
+each M = 1 shape, the time any4_quantize takes to learn the tables of the
+Llama3-8B matrices (beside the oracle), and the any3 / any2 / any4 dequant rate.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -609,6 +610,48 @@ def table_learning_detail(max_iter: int, cpu_seconds: float, reps: int = 3):
     return out
 
 
+def nbit_dequant_detail(reps: int = 10):
+    """Time any4_dequant_bits for n = 2, 3, 4 on the Llama3-8B gate matrix
+    (4096 -> 14336, G = 128), L2 flushed before each call: HBM GB/s of the
+    algorithmic bytes (codes, scales, offsets and tables read, bf16 W written)."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    peaks = load_peaks()
+    N, K, G = 14336, 4096, 128
+    rng = np.random.default_rng(4600)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    W = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    out = {"N": N, "K": K, "G": G}
+    for bits in (2, 3, 4):
+        nq = 1 << bits
+        packed = torch.from_numpy(rng.integers(0, 256, size=(N, bits * K // 8),
+                                               dtype=np.uint8)).cuda()
+        lut = _dev_bf16(workloads._to_bf16_bits(rng.normal(0, 0.5, (N, nq)).astype(np.float32)))
+        scale = _dev_bf16(workloads._to_bf16_bits(
+            (np.abs(rng.normal(0, 0.01, (N, K // G))) + 1e-3).astype(np.float32)))
+        offset = _dev_bf16(workloads._to_bf16_bits(
+            rng.normal(0, 0.002, (N, K // G)).astype(np.float32)))
+        any4.any4_dequant_bits(packed, lut, scale, offset, G, bits, W=W)
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            any4.any4_dequant_bits(packed, lut, scale, offset, G, bits, W=W)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b) * 1e3)
+        us = float(np.median(times))
+        alg = N * K * bits // 8 + 4 * N * (K // G) + 2 * nq * N + 2 * N * K
+        out[f"any{bits}"] = {"us": round(us, 2), "GB/s": round(alg / us / 1e3, 1),
+                             "frac_hbm": round(alg / us / 1e3 / peaks["hbm_gbs"], 4)}
+        del packed, lut, scale, offset
+    del flush, W
+    torch.cuda.synchronize()
+    return out
+
+
 def profile_shape(name: str, calls: int):
     """Run a few any4_matmul calls (auto path) on one workload shape."""
     import torch
@@ -684,6 +727,12 @@ def main():
                          "matrices": table_learning_detail(args.quantize_iters, 4.0, reps=2)}
             except Exception as e:  # pragma: no cover - only on a GPU machine
                 table = {"error": f"{type(e).__name__}: {e}"}
+        nbit = None
+        if world == 1:
+            try:  # a detail beside the step: its failure is reported, not fatal
+                nbit = nbit_dequant_detail()
+            except Exception as e:  # pragma: no cover - only on a GPU machine
+                nbit = {"error": f"{type(e).__name__}: {e}"}
         achieved = r["value"] / world  # per-GPU decode throughput over the whole step
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -713,6 +762,7 @@ def main():
             "detail_batch": r["batch"],
             "fig3_square_m1": r["fig3"],
             "table_learning": table,
+            "nbit_dequant": nbit,
         }
         print(json.dumps(line), flush=True)
     finally:
