@@ -62,10 +62,10 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the M = 1 decode kernel source (the only kernel of a step): a
+    """Hash of the M = 1 pair-table decode kernel source (the only kernel of a step): a
     stored ncu traffic figure is only used while it was taken on this source."""
     h = hashlib.sha256()
-    for fn in ("decode_tma.cu", "common.cuh"):
+    for fn in ("decode_pair.cu", "common.cuh"):
         with open(os.path.join(ROOT, "learned_bit_lut_any4_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -74,7 +74,7 @@ def kernel_source_hash() -> str:
 def stored_traffic():
     """Per-launch DRAM bytes (read + write) of the decode kernel on this step,
     from the committed ncu summary, if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_tma_kernel_llama3_8b_layer_m1.md")
+    path = os.path.join(ROOT, "profiles", "decode_pair_kernel_llama3_8b_layer_m1.md")
     try:
         text = open(path).read()
     except OSError:
@@ -198,6 +198,24 @@ def _dev_bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
 
 
+_WS = {}
+
+
+def ws_for(s):
+    """One decode workspace shared by every call of this process (calls on one
+    stream run in order, and the kernels touch it only after their
+    predecessor has finished), grown to the largest size asked for."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    need = any4.any4_matmul_workspace_size(s.M, s.N, s.K, s.G)
+    if s.M > 16:
+        return None  # prefill: the binding allocates its workspace
+    cur = _WS.get("decode")
+    if cur is None or cur.numel() < need:
+        cur = _WS["decode"] = torch.empty(max(need, 1 << 16), dtype=torch.uint8, device="cuda")
+    return cur
+
+
 def prepare_layer(shapes, copies):
     """Device copies of each shape's weights (packed on the device by
     any4_pack), plus x and y buffers."""
@@ -268,7 +286,8 @@ def fig3_square_sweep(stream, overlap):
         res = {}
         for name, table in (("any4", None), ("nf4_style", t_nf4), ("int4", t_int4)):
             calls = [(lambda w=w, t=table: any4.any4_matmul(
-                x, w[0], w[1] if t is None else t, w[2], w[3], s.G, y=y, overlap_prior=overlap))
+                x, w[0], w[1] if t is None else t, w[2], w[3], s.G, y=y, overlap_prior=overlap,
+                workspace=ws_for(s)))
                 for w in reps]
             res[name + "_us"] = round(_time_graph(stream, calls, n_rep), 3)
         W = any4.any4_dequant(reps[0][0], reps[0][1], reps[0][2], reps[0][3], s.G)
@@ -282,6 +301,37 @@ def fig3_square_sweep(stream, overlap):
         out[str(K)] = res
         del reps, x, y, W, Ws, xd
         torch.cuda.synchronize()
+    return out
+
+
+def time_weight_set(shapes, stream, overlap, peaks):
+    """Time any4_matmul on one weight set (the shapes share a weight seed and
+    differ in M and x) on rotating weight copies larger than L2, replayed in
+    a CUDA graph; per shape µs per call, GB/s of its algorithmic bytes and the
+    fraction of the HBM peak (+ TFLOPS for M > 16)."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    s0 = shapes[0]
+    wbytes = s0.N * s0.K // 2 + 4 * s0.N * (s0.K // s0.G) + 32 * s0.N
+    bc = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
+    (_, reps, _, _, _), = prepare_layer([s0], bc)
+    out = {}
+    for s in shapes:
+        x = _dev_bf16(workloads.draw_x(s))
+        y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
+        ws = ws_for(s)
+        calls = [(lambda w=w: any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y,
+                                               overlap_prior=overlap, workspace=ws))
+                 for w in reps]
+        us = _time_graph(stream, calls, max(2, 200 // bc))
+        gbs = s.alg_bytes() / (us * 1e-6) / 1e9
+        r = {"M": s.M, "K": s.K, "N": s.N, "G": s.G, "us": round(us, 3), "GB/s": round(gbs, 1),
+             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        if s.M > 16:
+            r["TFLOPS"] = round(s.flops() / (us * 1e-6) / 1e12, 2)
+        out[s.name] = r
+        del x, y
+    del reps
     return out
 
 
@@ -301,7 +351,8 @@ def gpu_arm(args, rank, world):
     def step(c):
         for (s, reps, x, y, _) in sets:
             w = reps[c % copies]
-            any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+            any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap,
+                             workspace=ws_for(s))
 
     # one graph = `copies` steps (each step on the next weight copy)
     with torch.cuda.stream(stream):
@@ -349,7 +400,8 @@ def gpu_arm(args, rank, world):
         with torch.cuda.graph(g, stream=stream):
             for c in range(copies):
                 w = reps[c]
-                any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
+                any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap,
+                             workspace=ws_for(s))
         n_rep = max(1, 400 // copies)
         with torch.cuda.stream(stream):
             g.replay()
@@ -379,7 +431,7 @@ def gpu_arm(args, rank, world):
                     flush.zero_()
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record(stream)
-                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y)
+                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, workspace=ws_for(s))
                     b.record(stream)
                     b.synchronize()
                     if i >= 3:
@@ -420,41 +472,19 @@ def gpu_arm(args, rank, world):
             del packed, lut, sc, of, x, y, flush
         torch.cuda.synchronize()
 
-    # the batch sweep and the 70B shapes at M = 8 (skinny kernel), each shape
-    # alone on rotating weight copies larger than L2
-    batch = {}
+    # the other M = 1 targets (tiny, the G = 64 variant, the 70B-shaped
+    # matrices) and the batch sweep (M = 2 .. 32, 70B at M = 8): each weight set
+    # once on rotating copies larger than L2, timed at every M it is used with
+    more_m1, batch = {}, {}
     if not args.skip_batch:
-        bshapes = [s for s in workloads.SKINNY_SWEEP if 2 <= s.M <= 16] + \
-                  [s for s in workloads.LLAMA3_70B_DECODE if s.M == 8]
-        for s in bshapes:
-            wbytes = s.N * s.K // 2 + 4 * s.N * (s.K // s.G) + 32 * s.N
-            bc = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
-            (_, reps, x, y, _), = prepare_layer([s], bc)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(stream):
-                for c in range(bc):
-                    w = reps[c]
-                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
-            stream.synchronize()
-            with torch.cuda.graph(g, stream=stream):
-                for c in range(bc):
-                    w = reps[c]
-                    any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap)
-            n_rep = max(2, 200 // bc)
-            with torch.cuda.stream(stream):
-                g.replay()
-                stream.synchronize()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                for _ in range(n_rep):
-                    g.replay()
-                b.record(stream)
-            b.synchronize()
-            us = a.elapsed_time(b) * 1e3 / (n_rep * bc)
-            gbs = s.alg_bytes() / (us * 1e-6) / 1e9
-            batch[s.name] = {"M": s.M, "us": round(us, 3), "GB/s": round(gbs, 1),
-                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-            del g, reps, x, y
+        groups = [workloads.TINY, [s for s in workloads.SKINNY_SWEEP if s.G == 64]]
+        groups.append([s for s in workloads.SKINNY_SWEEP if s.G == 128])
+        for nm in ("gate", "up", "down"):
+            groups.append([s for s in workloads.LLAMA3_70B_DECODE if s.name.startswith(f"70b_{nm}_")])
+        for grp in groups:
+            res = time_weight_set(grp, stream, overlap, peaks)
+            for s in grp:
+                (more_m1 if s.M == 1 and s.name != "sweep_m1" else batch)[s.name] = res[s.name]
         torch.cuda.synchronize()
 
     fig3 = fig3_square_sweep(stream, overlap) if not args.skip_fig3 else {}
@@ -482,7 +512,8 @@ def gpu_arm(args, rank, world):
         dev_x.copy_(host_x, non_blocking=True)
         for i, (s, reps, _x, _y, _) in enumerate(sets):
             w = reps[c % copies]
-            any4.any4_matmul(x_views[i], w[0], w[1], w[2], w[3], s.G, y=y_views[i])
+            any4.any4_matmul(x_views[i], w[0], w[1], w[2], w[3], s.G, y=y_views[i],
+                             workspace=ws_for(s))
         host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -505,7 +536,7 @@ def gpu_arm(args, rank, world):
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
         "clocks": clocks, "detail": detail, "single": single, "prefill": prefill,
-        "batch": batch, "fig3": fig3,
+        "batch": batch, "more_m1": more_m1, "fig3": fig3,
         "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -737,7 +768,7 @@ def main():
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": stored_traffic(),
-                    "kernel": "decode_tma_kernel<8> (the only kernel of the step)",
+                    "kernel": "decode_pair_kernel<1, 4> (the only kernel of the step)",
                     "peak_source": peaks.get("source", "measured")}
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
@@ -756,13 +787,16 @@ def main():
             "e2e": r["e2e"],
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
-            "detail_m1": r["detail"],
-            "single_call_m1": r["single"],
-            "prefill_m2048": r["prefill"],
-            "detail_batch": r["batch"],
+            # bulky details first; the target numbers (per-shape M = 1 and the
+            # prefill fractions) close the line, where its tail is kept
             "fig3_square_m1": r["fig3"],
             "table_learning": table,
             "nbit_dequant": nbit,
+            "single_call_m1": r["single"],
+            "detail_batch": r["batch"],
+            "detail_m1": r["detail"],
+            "detail_m1_more": r["more_m1"],
+            "prefill_m2048": r["prefill"],
         }
         print(json.dumps(line), flush=True)
     finally:

@@ -185,15 +185,22 @@ ANY4_API any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, in
  *                   any4_matmul_workspace_size(M, N, K, G); may be NULL when
  *                   that size is 0.  Its contents need not be initialised and
  *                   are undefined afterwards; two calls in flight at the same
- *                   time must not share one.
+ *                   time must not share one.  At M <= 2 the size is that of
+ *                   the pair-table decode kernel (tens of KiB); a NULL
+ *                   or smaller workspace there runs the slower decode kernels
+ *                   that need none.  After a call that reported
+ *                   ANY4_ERR_TIMEOUT, zero the workspace (or take another)
+ *                   before its next use: the aborted call may have left a
+ *                   block's "partial sums published" marker in it.
  *   dev_status      see the conventions above (ANY4_ERR_TIMEOUT)
  * Accuracy: |y - y_ref| <= 1e-2 * rms(y_ref) + ulp_bf16(y_ref) per element,
  * with y_ref the exact dequant-then-matmul.  Inside the kernels each weight is
  * formed as LUT * scale + offset rounded once to bf16 (a bf16x2 fused
  * multiply-add), which equals any4_dequant's W except when the fp32 fmaf is
  * inexact and lands exactly on a bf16 rounding tie.
- * Kernels: M = 1 weight-streaming decode, 2 <= M <= 16 skinny, larger M the
- * tensor-core prefill (any4_matmul_choose_path).
+ * Kernels: M <= 2 the pair-table decode (given its workspace; else M = 1
+ * weight-streaming decode), 2 <= M <= 16 skinny, larger M the tensor-core
+ * prefill (any4_matmul_choose_path).
  */
 ANY4_API any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                         int64_t lut_row_stride, const uint16_t* scale,
@@ -211,7 +218,20 @@ typedef enum any4_flags {
    * while the preceding kernel on the stream finishes; x is read and y is
    * written only after the preceding kernel has completed.  Decode path only;
    * ignored elsewhere. */
-  ANY4_FLAG_OVERLAP_PRIOR = 1
+  ANY4_FLAG_OVERLAP_PRIOR = 1,
+  /* y is an fp32 [M][N] array (still 16-byte aligned) and receives the fp32
+   * sums before their rounding to bf16: the kernels' accumulation can then be
+   * compared with the exact result on its own.  Every path. */
+  ANY4_FLAG_FP32_OUT = 2,
+  /* Test hook for the failure handling, not for production calls: block 0 of
+   * the kernel stops its weight (or x) stream after the first stage and every
+   * bounded wait gives up after 1 ms instead of about 2 s.  The call then ends
+   * with ANY4_ERR_TIMEOUT in *dev_status, its y undefined, no memory outside
+   * y and the workspace written, the kernel's own copies drained and its
+   * tensor memory released, so the device and stream stay usable.  Kernels
+   * with bounded waits only: the pair-table and weight-streaming decode
+   * kernels and the prefill kernel (others ignore it). */
+  ANY4_FLAG_TEST_STALL = 4
 } any4_flags;
 
 /* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16)
@@ -238,20 +258,30 @@ ANY4_API any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, co
  *                   bytes, one per device: 37 MiB + 1 KiB, i.e. one 256 KiB
  *                   fp32 partial tile per block of a 148-SM grid plus the
  *                   per-block flags, which each call clears (an async memset
- *                   on `stream`) before its launch.  If the device needs more
+ *                   on `stream`) before its launch.  The array is reserved on
+ *                   every device where the library's module is loaded, in
+ *                   every process that loads libany4, whether or not this
+ *                   entry point is ever called.  If the device needs more
  *                   (any4_matmul_workspace_size_ex(..., ANY4_PATH_PREFILL)
  *                   above ANY4_STATIC_SCRATCH_BYTES, e.g. a GPU with more
  *                   than 148 SMs) the call returns ANY4_ERR_WORKSPACE and
  *                   launches nothing.
  *   set-up          the first call on a device looks up the array's device
  *                   address (cudaGetSymbolAddress, with that device current)
- *                   and caches it; make that first call before any stream
- *                   capture.  A failed look-up returns ANY4_ERR_CUDA.
+ *                   and caches it per device, keyed by the identity of the
+ *                   current context: after a device reset (or a released and
+ *                   re-created primary context) the next call looks it up
+ *                   again.  Make the first call on a device, and the first
+ *                   after a reset, before any stream capture.  A failed
+ *                   look-up returns ANY4_ERR_CUDA.
  *   concurrency     every call on a device uses the same array: calls whose
  *                   kernels overlap on the GPU (different streams, or several
  *                   host threads) race on it and give undefined results.
  *                   Calls issued in order on one stream are safe.
- * Results are those of any4_matmul_ex(..., ANY4_PATH_PREFILL, ...).
+ * Results are those of the one-pass prefill kernel (what
+ * any4_matmul_ex(..., ANY4_PATH_PREFILL, ...) runs below M = 1024 or with a
+ * workspace of only the one-pass size); at larger M they agree with the
+ * two-pass route within the matmul tolerance above, not bit for bit.
  */
 #define ANY4_STATIC_SCRATCH_BYTES ((size_t)148 * 262144 + 1024)
 ANY4_API any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t* packed,

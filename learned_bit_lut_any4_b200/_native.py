@@ -29,6 +29,8 @@ PATHS = {"auto": 0, "decode": 1, "prefill": 2}
 # Bytes of the library's fixed scratch array (any4_matmul_static_scratch).
 ANY4_STATIC_SCRATCH_BYTES = 148 * 262144 + 1024
 ANY4_FLAG_OVERLAP_PRIOR = 1
+ANY4_FLAG_FP32_OUT = 2
+ANY4_FLAG_TEST_STALL = 4
 # Limits of any4_quantize (the row lives in one block's shared memory).
 ANY4_QUANTIZE_MAX_K = 16384
 ANY4_QUANTIZE_MAX_ITER = 100000
@@ -162,13 +164,16 @@ def any4_pack(idx: torch.Tensor, packed: torch.Tensor | None = None,
 
     A code above 15 sets ANY4_ERR_RANGE in dev_status (int32 CUDA tensor of one
     element, zeroed by the caller) once the stream has run."""
-    _need(idx, "idx", (torch.uint8,))
+    if not isinstance(idx, torch.Tensor) or idx.dim() != 2:
+        raise ValueError("idx must be a [N, K] tensor")
     N, K = idx.shape
+    if packed is not None:
+        _need_shape(packed, "packed", (N, K // 2))
+    _need(idx, "idx", (torch.uint8,))
     if packed is None:
         packed = torch.empty((N, K // 2), dtype=torch.uint8, device=idx.device)
     _need(packed, "packed", (torch.uint8,), idx.device)
-    if dev_status is not None:
-        _need(dev_status, "dev_status", (torch.int32,), idx.device)
+    _need_status(dev_status, idx.device)
     with torch.cuda.device(idx.device):
         _check(library().any4_pack(_ptr(idx), _ptr(packed), N, K, _ptr(dev_status),
                                    _stream(idx.device)), "any4_pack")
@@ -246,8 +251,8 @@ def any4_pack_bits(idx: torch.Tensor, bits: int, packed: torch.Tensor | None = N
     if packed is None:
         packed = torch.empty((N, bits * K // 8), dtype=torch.uint8, device=idx.device)
     _need(packed, "packed", (torch.uint8,), idx.device)
-    if dev_status is not None:
-        _need(dev_status, "dev_status", (torch.int32,), idx.device)
+    _need_shape(packed, "packed", (N, bits * K // 8))
+    _need_status(dev_status, idx.device)
     with _on_device(idx.device):
         _check(library().any4_pack_bits(_ptr(idx), _ptr(packed), N, K, bits, _ptr(dev_status),
                                         _stream(idx.device)), "any4_pack_bits")
@@ -276,6 +281,7 @@ def any4_dequant_bits(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tens
     if W is None:
         W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
     _need(W, "W", _BF16, dev)
+    _need_shape(W, "W", (N, K))
     if scale.numel() != N * (K // G if G else 0) or offset.numel() != scale.numel():
         raise ValueError("scale and offset must hold N * K/G values")
     with _on_device(dev):
@@ -283,6 +289,58 @@ def any4_dequant_bits(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tens
                                            _ptr(offset), _ptr(W), N, K, G, bits, _stream(dev)),
                "any4_dequant_bits")
     return W
+
+
+def _need_shape(t: torch.Tensor, name: str, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need_status(dev_status, dev):
+    """dev_status: None, or an int32 CUDA tensor of at least one element."""
+    if dev_status is None:
+        return
+    if isinstance(dev_status, torch.Tensor) and dev_status.numel() < 1:
+        raise ValueError("dev_status must hold at least one int32")
+    _need(dev_status, "dev_status", (torch.int32,), dev)
+
+
+def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_out=False):
+    """Validate the operands of a matmul call on the host, before any launch:
+    the C ABI sees bare pointers and cannot check that a buffer is large
+    enough, so a short y, scale or offset is caught here.  Sizes are checked
+    before devices, so the checks hold for any tensor.  Returns
+    (M, N, K, lut_row_stride, y), allocating y when it is None."""
+    for t, nm, dts in ((x, "x", _BF16), (packed, "packed", (torch.uint8,)), (lut, "lut", _BF16),
+                       (scale, "scale", _BF16), (offset, "offset", _BF16)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{nm} must be a torch.Tensor")
+        if t.dtype not in dts:
+            raise TypeError(f"{nm} must have dtype in {dts}, got {t.dtype}")
+    if x.dim() != 2 or packed.dim() != 2:
+        raise ValueError("x must be [M, K] and packed [N, K/2]")
+    M, K = x.shape
+    N, Kh = packed.shape
+    if 2 * Kh != K:
+        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
+    if G <= 0 or K % G != 0:
+        raise ValueError(f"G={G} must be positive and divide K={K}")
+    stride = _lut_stride(lut, N)
+    if scale.numel() != N * (K // G) or offset.numel() != N * (K // G):
+        raise ValueError(f"scale and offset must hold N * K/G = {N * (K // G)} values")
+    if y is not None:
+        _need_shape(y, "y", (M, N))
+    if isinstance(dev_status, torch.Tensor) and dev_status.numel() < 1:
+        raise ValueError("dev_status must hold at least one int32")
+    dev = x.device
+    _need(x, "x", _BF16)
+    _need(packed, "packed", (torch.uint8,), dev)
+    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+        _need(t, nm, _BF16, dev)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if fp32_out else torch.bfloat16, device=dev)
+    _need(y, "y", (torch.float32,) if fp32_out else _BF16, dev)
+    return M, N, K, stride, y
 
 
 def _lut_stride(lut: torch.Tensor, N: int) -> int:
@@ -306,6 +364,7 @@ def any4_dequant(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
     if W is None:
         W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
     _need(W, "W", _BF16, dev)
+    _need_shape(W, "W", (N, K))
     if scale.numel() != N * (K // G if G else 0) or offset.numel() != scale.numel():
         raise ValueError("scale and offset must hold N * K/G values")
     with _on_device(dev):
@@ -328,26 +387,21 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                 scale: torch.Tensor, offset: torch.Tensor, G: int,
                 y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 path: str = "auto", dev_status: torch.Tensor | None = None,
-                overlap_prior: bool = False) -> torch.Tensor:
+                overlap_prior: bool = False, fp32_out: bool = False,
+                test_stall: bool = False) -> torch.Tensor:
     """bf16 y[M, N] = x[M, K] * dequant(W)^T, fp32 accumulation.
 
     workspace: a CUDA tensor of at least any4_matmul_workspace_size() bytes, or
-    None to have one allocated here when the path needs it.
+    None to have one allocated here when the path needs it (an empty tensor
+    passes none: the decode path then runs its kernels that need none).
     overlap_prior: ANY4_FLAG_OVERLAP_PRIOR (the weights are not written by
-    work still running on the stream; the decode kernel may then overlap it)."""
-    _need(x, "x", _BF16)
+    work still running on the stream; the decode kernel may then overlap it).
+    fp32_out: ANY4_FLAG_FP32_OUT, y is fp32 and holds the sums unrounded.
+    test_stall: ANY4_FLAG_TEST_STALL, a test of the failure handling (one
+    block's stream stops, the call ends with ANY4_ERR_TIMEOUT in dev_status)."""
+    M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y,
+                                             dev_status, fp32_out)
     dev = x.device
-    _need(packed, "packed", (torch.uint8,), dev)
-    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
-        _need(t, nm, _BF16, dev)
-    M, K = x.shape
-    N, Kh = packed.shape
-    if 2 * Kh != K:
-        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
-    stride = _lut_stride(lut, N)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    _need(y, "y", _BF16, dev)
     lib = library()
     p = PATHS[path]
     key = (dev.index, M, N, K, G, p)
@@ -360,13 +414,16 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
     if workspace is not None:
         _need(workspace, "workspace", (torch.uint8,), dev)
         ws_bytes = workspace.numel()
-    if dev_status is not None:
-        _need(dev_status, "dev_status", (torch.int32,), dev)
+        if ws_bytes == 0:
+            workspace = None
+    _need_status(dev_status, dev)
     with _on_device(dev):
         _check(lib.any4_matmul_ex(_ptr(x), _ptr(packed), _ptr(lut), stride, _ptr(scale),
                                   _ptr(offset), _ptr(y), M, N, K, G, _ptr(workspace), ws_bytes,
                                   _ptr(dev_status), p,
-                                  ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0,
+                                  (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
+                                  | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
+                                  | (ANY4_FLAG_TEST_STALL if test_stall else 0),
                                   _stream(dev)), "any4_matmul")
     return y
 
@@ -382,21 +439,10 @@ def any4_matmul_static_scratch(x: torch.Tensor, packed: torch.Tensor, lut: torch
     wanted): only a missing y is allocated here, with torch.  The first call on
     a device looks up the array's address; make it before any stream capture.
     Calls whose kernels overlap on the GPU share the array and race."""
-    _need(x, "x", _BF16)
+    M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y,
+                                             dev_status)
     dev = x.device
-    _need(packed, "packed", (torch.uint8,), dev)
-    for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
-        _need(t, nm, _BF16, dev)
-    M, K = x.shape
-    N, Kh = packed.shape
-    if 2 * Kh != K:
-        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
-    stride = _lut_stride(lut, N)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    _need(y, "y", _BF16, dev)
-    if dev_status is not None:
-        _need(dev_status, "dev_status", (torch.int32,), dev)
+    _need_status(dev_status, dev)
     lib = library()
     with _on_device(dev):
         _check(lib.any4_matmul_static_scratch(_ptr(x), _ptr(packed), _ptr(lut), stride,

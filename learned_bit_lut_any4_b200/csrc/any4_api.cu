@@ -15,9 +15,9 @@ bool prefill_use_two_pass(int64_t M, int64_t N, int64_t K);
 size_t prefill_two_pass_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                                     int64_t lut_row_stride, const uint16_t* scale,
-                                    const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
-                                    int64_t K, int64_t G, void* workspace,
-                                    size_t workspace_bytes, int32_t* dev_status,
+                                    const uint16_t* offset, uint16_t* y, float* y32, int64_t M,
+                                    int64_t N, int64_t K, int64_t G, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, bool test_stall,
                                     cudaStream_t stream, const DeviceInfo& dev);
 
 // Table learning (quantize.cu): one thread block per weight row; bits = 2, 3, 4.
@@ -97,6 +97,24 @@ int cached_occupancy(const void* kernel, int threads, size_t smem) {
   std::lock_guard<std::mutex> lock(mu);
   cache[key] = occ;
   return occ;
+}
+
+any4_status ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> opted;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ANY4_ERR_CUDA;
+  const auto key = std::make_pair(kernel, dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = opted.find(key);
+  if (it != opted.end() && it->second >= bytes) return ANY4_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return ANY4_ERR_CUDA;
+  }
+  opted[key] = bytes;
+  return ANY4_OK;
 }
 
 }  // namespace any4
@@ -229,7 +247,14 @@ size_t any4_matmul_workspace_size_ex(int64_t M, int64_t N, int64_t K, int64_t G,
   if (path == ANY4_PATH_PREFILL)
     return prefill_use_two_pass(M, N, K) ? prefill_two_pass_workspace_size(M, N, K, G)
                                          : prefill_workspace_size(M, N, K, G);
-  return 0;
+  // decode: the pair-table kernel's stream-K exchange (M <= 2); sized for the
+  // current device, or for a 160-SM grid where there is none
+  DeviceInfo dev;
+  if (current_device(&dev) != ANY4_OK) {
+    dev = DeviceInfo();
+    dev.sm_count = 160;
+  }
+  return decode_pair_workspace_size(M, N, K, G, dev);
 }
 
 size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G) {
@@ -249,9 +274,13 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
       !aligned16(offset) || !aligned16(y))
     return ANY4_ERR_ALIGN;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  if (workspace && !aligned16(workspace)) return ANY4_ERR_ALIGN;
   if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
   if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
-  if (flags & ~(uint32_t)ANY4_FLAG_OVERLAP_PRIOR) return ANY4_ERR_UNSUPPORTED;
+  if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL))
+    return ANY4_ERR_UNSUPPORTED;
+  float* y32 = (flags & ANY4_FLAG_FP32_OUT) ? reinterpret_cast<float*>(y) : nullptr;
+  const bool test_stall = (flags & ANY4_FLAG_TEST_STALL) != 0;
   if (path == ANY4_PATH_DECODE && M > kDecodeMaxM) return ANY4_ERR_UNSUPPORTED;
   // the prefill path runs in one pass with at least prefill_workspace_size
   // bytes, and in two passes (large M) when the workspace also holds the
@@ -265,17 +294,18 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   any4_status st = current_device(&dev);
   if (st != ANY4_OK) return st;
   if (path == ANY4_PATH_DECODE) {
-    return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
-                         (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, dev_status, (cudaStream_t)stream,
-                         dev);
+    return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                         workspace, workspace_bytes, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,
+                         dev_status, test_stall, (cudaStream_t)stream, dev);
   }
   if (prefill_use_two_pass(M, N, K) &&
       workspace_bytes >= prefill_two_pass_workspace_size(M, N, K, G))
-    return launch_prefill_two_pass(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
-                                   workspace, workspace_bytes, dev_status, (cudaStream_t)stream,
-                                   dev);
-  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, workspace,
-                        workspace_bytes, dev_status, (cudaStream_t)stream, dev);
+    return launch_prefill_two_pass(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K,
+                                   G, workspace, workspace_bytes, dev_status, test_stall,
+                                   (cudaStream_t)stream, dev);
+  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                        workspace, workspace_bytes, dev_status, test_stall, (cudaStream_t)stream,
+                        dev);
 }
 
 // The prefill kernel with the library's fixed scratch array (static_scratch.cu)
@@ -299,8 +329,9 @@ any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t* packed,
   void* scratch = nullptr;
   st = static_scratch(dev.device, &scratch);
   if (st != ANY4_OK) return st;
-  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, scratch,
-                        ANY4_STATIC_SCRATCH_BYTES, dev_status, (cudaStream_t)stream, dev);
+  return launch_prefill(x, packed, lut, lut_row_stride, scale, offset, y, nullptr, M, N, K, G,
+                        scratch, ANY4_STATIC_SCRATCH_BYTES, dev_status, false,
+                        (cudaStream_t)stream, dev);
 }
 
 any4_status any4_matmul(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,

@@ -135,23 +135,39 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const uint16_t* scale, const uint16_t* offset, uint16_t* W,
                            int64_t N, int64_t K, int64_t G, cudaStream_t stream,
                            const DeviceInfo& dev);
+// The decode path (M <= 16).  y32, when not NULL, receives the fp32 sums
+// instead of y (the unrounded results).  A workspace of at least
+// decode_pair_workspace_size bytes selects the pair-table kernel for M <= 2.
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev);
+                          uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                          void* workspace, size_t workspace_bytes, bool overlap,
+                          int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                          const DeviceInfo& dev);
+// Pair-table decode for M <= 2 (decode_pair.cu): workspace bytes it needs on
+// `dev` (0 when the shape is not supported).
+bool decode_pair_supported(int64_t M, int64_t N, int64_t K, int64_t G);
+size_t decode_pair_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G,
+                                  const DeviceInfo& dev);
+any4_status launch_decode_pair(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                               int64_t lut_row_stride, const uint16_t* scale,
+                               const uint16_t* offset, uint16_t* y, float* y32, int64_t M,
+                               int64_t N, int64_t K, int64_t G, void* workspace, bool overlap,
+                               int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                               const DeviceInfo& dev);
 bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G);
 any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                               int64_t lut_row_stride, const uint16_t* scale,
-                              const uint16_t* offset, uint16_t* y, int64_t N, int64_t K,
-                              int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
-                              const DeviceInfo& dev);
+                              const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
+                              int64_t K, int64_t G, bool overlap, int32_t* dev_status,
+                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 // Skinny matmul for 2 <= M <= 16 (standard tensor-core mapping, table
 // lookups by byte permute): skinny.cu.
 any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          cudaStream_t stream, const DeviceInfo& dev);
+                          uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                          bool overlap, cudaStream_t stream, const DeviceInfo& dev);
 
 // cudaOccupancyMaxActiveBlocksPerMultiprocessor, remembered per (kernel,
 // threads, dynamic shared memory) so that launches after the first of a shape
@@ -159,13 +175,21 @@ any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16
 // Returns 0 when the query fails.
 int cached_occupancy(const void* kernel, int threads, size_t smem);
 
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) on the
+// current device, skipped when that device already allows `kernel` at least
+// `bytes`.  Function attributes belong to a device, so a process that
+// launches on several GPUs opts each one in; the cache is keyed per (kernel,
+// device) and guarded by a mutex (callers may be on several host threads).
+any4_status ensure_dynamic_smem(const void* kernel, size_t bytes);
+
 // Device address of the fixed scratch array of any4_matmul_static_scratch on
 // `device` (the current device); resolved on first use per device.
 any4_status static_scratch(int device, void** ptr);
 
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                            int64_t lut_row_stride, const uint16_t* scale,
-                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
-                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
-                           int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev);
+                           const uint16_t* offset, uint16_t* y, float* y32, int64_t M,
+                           int64_t N, int64_t K, int64_t G, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, bool test_stall,
+                           cudaStream_t stream, const DeviceInfo& dev);
 }  // namespace any4

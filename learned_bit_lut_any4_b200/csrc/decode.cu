@@ -176,8 +176,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32) decode_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-    uint16_t* __restrict__ y, int M, int64_t N, int64_t K, int64_t G, int nslices,
-    int rows_per_block) {
+    uint16_t* __restrict__ y, float* __restrict__ y32, int M, int64_t N, int64_t K, int64_t G,
+    int nslices, int rows_per_block) {
   constexpr int KW = CodeLoad<KL>::kWords;
   constexpr int V = P * MT;
   static_assert(V <= 32 && (V & (V - 1)) == 0, "P * MT must be a power of two <= 32");
@@ -314,7 +314,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) decode_kernel(
       if (m < M) {
         float tot = 0.f;
         for (int w = 0; w < nw_used; ++w) tot += s_part[((size_t)w * RTP + r) * MT + m];
-        y[(int64_t)m * N + row0 + r] = f32_to_bf16_rn(tot);
+        if (y32 != nullptr)
+          y32[(int64_t)m * N + row0 + r] = tot;
+        else
+          y[(int64_t)m * N + row0 + r] = f32_to_bf16_rn(tot);
       }
     }
     __syncthreads();
@@ -328,7 +331,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) decode_kernel(
 template <int MT, int KL, int P>
 any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                 int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                uint16_t* y, int M, int64_t N, int64_t K, int64_t G, bool overlap,
+                uint16_t* y, float* y32, int M, int64_t N, int64_t K, int64_t G, bool overlap,
                 cudaStream_t stream, const DeviceInfo& dev) {
   const int64_t slice = 32LL * KL;
   const int nslices = (int)((K + slice - 1) / slice);
@@ -359,8 +362,8 @@ any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t err = cudaLaunchKernelEx(&cfg, decode_kernel<MT, KL, P>, x, packed, lut,
-                                             lut_row_stride, scale, offset, y, M, N, K, G,
-                                             nslices, (int)rt);
+                                             lut_row_stride, scale, offset, y, y32, M, N, K,
+                                             G, nslices, (int)rt);
   return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
@@ -368,19 +371,27 @@ any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
 
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+                          uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                          void* workspace, size_t workspace_bytes, bool overlap,
+                          int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                          const DeviceInfo& dev) {
+  // M <= 2 with its workspace: pair-table lookups, stream-K over 64-row sets
+  // (decode_pair.cu)
+  const size_t pair_ws = decode_pair_workspace_size(M, N, K, G, dev);
+  if (pair_ws > 0 && workspace != nullptr && workspace_bytes >= pair_ws)
+    return launch_decode_pair(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                              workspace, overlap, dev_status, test_stall, stream, dev);
   // M = 1 with a 1024-column slice holding whole 16-byte runs of scales:
   // weights streamed by the tensor-memory-access engine (decode_tma.cu)
   if (decode_tma_supported(M, N, K, G))
-    return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
-                             dev_status, stream, dev);
+    return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G,
+                             overlap, dev_status, test_stall, stream, dev);
   // M >= 2: the skinny kernel (one dequantisation of the weights for all rows
   // of x, standard tensor-core mapping; skinny.cu)
   if (M >= 2)
-    return launch_skinny(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, overlap,
-                         stream, dev);
-  return run<1, 32, 8>(x, packed, lut, lut_row_stride, scale, offset, y, 1, N, K, G, overlap,
+    return launch_skinny(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                         overlap, stream, dev);
+  return run<1, 32, 8>(x, packed, lut, lut_row_stride, scale, offset, y, y32, 1, N, K, G, overlap,
                        stream, dev);
 }
 

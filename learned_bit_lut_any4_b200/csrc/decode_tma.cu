@@ -43,6 +43,7 @@ constexpr int kTmaPrmtPairs = ANY4_DECODE_PRMT_PAIRS;
 static_assert(kTmaPrmtPairs >= 0 && kTmaPrmtPairs <= kTmaRows / 2, "pairs on the permute path");
 
 constexpr unsigned long long kTmaWaitNs = 2000000000ull;
+constexpr unsigned long long kTmaTestWaitNs = 1000000ull;  // the test-stall mode's limit
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -64,12 +65,13 @@ __device__ __forceinline__ bool mbar_test_(uint32_t bar, uint32_t parity) {
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit) {
   if (mbar_test_(bar, parity)) return true;
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_(bar, parity)) return true;
-    if ((i & 63u) == 0u && gtimer() - t0 > kTmaWaitNs) return false;
+    if ((i & 63u) == 0u && gtimer() - t0 > limit) return false;
   }
 }
 __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -142,8 +144,11 @@ __device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
 template <int GPS>  // groups per 1024-column slice (1024 / G)
 __global__ void __maxnreg__(96) decode_tma_kernel(
     const __grid_constant__ TmaMaps maps, const uint16_t* __restrict__ x,
-    const uint16_t* __restrict__ lut_shared, uint16_t* __restrict__ y, int N, int K,
-    int nslices, int rows_per_block, int32_t* dev_status) {
+    const uint16_t* __restrict__ lut_shared, uint16_t* __restrict__ y, float* __restrict__ y32,
+    int N, int K, int nslices, int rows_per_block, int32_t* dev_status, int test_stall) {
+  // test_stall: warp 0 of block 0 stops its weight stream after one stage,
+  // so its next wait runs out (1 ms limit) and the kernel ends cleanly
+  const unsigned long long wait_ns = test_stall ? kTmaTestWaitNs : kTmaWaitNs;
   constexpr int P = kTmaRows;
   constexpr int S = kTmaStages;
   constexpr int kCodeBytes = P * 512;
@@ -192,7 +197,13 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
     bool first_slice = true;
     for (int s = warp; s < nslices && ok; s += nwarps) {
       // producer: the first S stages of this slice
+      // (every lane counts the issues; lane 0 issues the tensor loads)
       auto issue = [&](int stage_idx) {
+        if (test_stall && blockIdx.x == 0 && warp == 0 && it_issue >= 1) return;
+        if (lane != 0) {
+          ++it_issue;
+          return;
+        }
         const int st = (int)(it_issue % S);
         const uint32_t dst = ring + (uint32_t)(st * kStageBytes);
         const uint32_t bar = bars + 8u * st;
@@ -205,11 +216,7 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         tma2d(dst + kCodeBytes + kLutBytes + kGrpBytes, &maps.offset, s * GPS, r, bar);
         ++it_issue;
       };
-      if (lane == 0) {
-        for (int q = 0; q < S && q < nstages; ++q) issue(q);
-      } else {
-        it_issue += (uint32_t)(S < nstages ? S : nstages);
-      }
+      for (int q = 0; q < S && q < nstages; ++q) issue(q);
       if (!waited) {  // x (and y) may belong to the preceding kernel
         asm volatile("griddepcontrol.wait;" ::: "memory");
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -237,7 +244,7 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
       for (int si = 0; si < nstages; ++si) {
         const int st = (int)(it_use % S);
         const uint32_t parity = (it_use / S) & 1u;
-        if (!mbar_wait_bounded(bars + 8u * st, parity)) {
+        if (!mbar_wait_bounded(bars + 8u * st, parity, wait_ns)) {
           if (lane == 0) report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
           ok = false;
           *s_abort = 1;
@@ -331,11 +338,9 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         ++it_use;
         // stage st is consumed: let the tensor loads overwrite it
         __syncwarp();
-        if (lane == 0 && si + S < nstages) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (si + S < nstages) {
+          if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           issue(si + S);
-        } else if (si + S < nstages) {
-          ++it_issue;
         }
         const float tot = reduce8(part, lane);
         if ((lane & 3) == 0) {
@@ -352,7 +357,10 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
       for (int t = threadIdx.x; t < nrows; t += blockDim.x) {
         float tot = 0.f;
         for (int w = 0; w < nw_used; ++w) tot += s_part[(size_t)w * RTP + t];
-        y[row0 + t] = f32_to_bf16_rn(tot);
+        if (y32 != nullptr)
+          y32[row0 + t] = tot;
+        else
+          y[row0 + t] = f32_to_bf16_rn(tot);
       }
     }
     __syncthreads();
@@ -365,7 +373,7 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
   if (!ok) {
     while (it_use < it_issue) {
       const int st = (int)(it_use % S);
-      if (!mbar_wait_bounded(bars + 8u * st, (it_use / S) & 1u)) break;
+      if (!mbar_wait_bounded(bars + 8u * st, (it_use / S) & 1u, wait_ns)) break;
       ++it_use;
     }
   }
@@ -406,8 +414,9 @@ bool encode2d(EncodeFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* 
 template <int GPS>
 any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                     int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                    uint16_t* y, int64_t N, int64_t K, int64_t G, bool overlap,
-                    int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+                    uint16_t* y, float* y32, int64_t N, int64_t K, int64_t G, bool overlap,
+                    int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                    const DeviceInfo& dev) {
   constexpr int P = kTmaRows;
   constexpr int S = kTmaStages;
   constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
@@ -441,13 +450,9 @@ any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lu
   auto kern = decode_tma_kernel<GPS>;
   const size_t ring_bytes = (size_t)nwarps * S * kStageBytes + (size_t)nwarps * S * 8 + 16 + 128;
   const int kMaxRT = 512;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)std::min<size_t>(dev.smem_optin, 227 * 1024));
-  });
-  if (attr_err != cudaSuccess) return ANY4_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern),
+                          std::min<size_t>(dev.smem_optin, 227 * 1024)) != ANY4_OK)
+    return ANY4_ERR_CUDA;
   // rows per block from the blocks that fit per SM, which depends (through the
   // partial sums) on the rows per block: settle it in two passes
   int per_sm = 2;
@@ -480,8 +485,8 @@ any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lu
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const uint16_t* lut_shared = lut_row_stride == 0 ? lut : nullptr;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, x, lut_shared, y, (int)N, (int)K,
-                                             nslices, (int)rt, dev_status);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, x, lut_shared, y, y32, (int)N, (int)K,
+                                             nslices, (int)rt, dev_status, test_stall ? 1 : 0);
   return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
@@ -497,19 +502,19 @@ bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G) {
 
 any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                               int64_t lut_row_stride, const uint16_t* scale,
-                              const uint16_t* offset, uint16_t* y, int64_t N, int64_t K,
-                              int64_t G, bool overlap, int32_t* dev_status, cudaStream_t stream,
-                              const DeviceInfo& dev) {
+                              const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
+                              int64_t K, int64_t G, bool overlap, int32_t* dev_status,
+                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev) {
   switch (G) {
     case 128:
-      return run_tma<8>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
-                        dev_status, stream, dev);
+      return run_tma<8>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
+                        dev_status, test_stall, stream, dev);
     case 64:
-      return run_tma<16>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
-                         dev_status, stream, dev);
+      return run_tma<16>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
+                         dev_status, test_stall, stream, dev);
     case 32:
-      return run_tma<32>(x, packed, lut, lut_row_stride, scale, offset, y, N, K, G, overlap,
-                         dev_status, stream, dev);
+      return run_tma<32>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
+                         dev_status, test_stall, stream, dev);
     default:
       return ANY4_ERR_UNSUPPORTED;
   }

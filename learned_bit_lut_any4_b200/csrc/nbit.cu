@@ -8,7 +8,10 @@
 // which any4_pack / any4_dequant already serve).  A thread handles one chunk
 // of 32 codes: n 32-bit words, inside one row (K % 32 == 0) and one group
 // (G % 32 == 0).  Both kernels are streaming and HBM-bound; grids are a
-// multiple of the SM count and loop over the chunks.
+// multiple of the SM count and loop over the chunks (pack) or over 1024-column
+// segments of rows (dequant, a warp per segment).
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace any4 {
@@ -94,22 +97,36 @@ __device__ __forceinline__ float table_entry(uint32_t t0, uint32_t t1, uint32_t 
   return __uint_as_float(v << 16);
 }
 
+// dequant: one warp per 1024-column segment of a row, lane l on the segment's
+// 32-code chunk l (its n words are the n * 4 bytes after lane l - 1's, so the
+// warp's code loads are contiguous).  The 64 output bytes of a lane go to a
+// shared-memory copy of the segment's bf16 row, 16 bytes at a time in a
+// lane-rotated order (lanes 2i and 2i + 1 start at the 16-byte unit i mod 4
+// of their 64 bytes), which keeps every phase of 8 lanes on 8 distinct bank
+// groups; one bulk copy then writes the 2 KiB segment while the warp moves on
+// (two staging buffers per warp).
+constexpr int kNbWarps = 8;
+constexpr int kNbSeg = 1024;
+
 template <int BITS>
-__global__ void __launch_bounds__(kNbThreads)
+__global__ void __launch_bounds__(kNbWarps * 32)
 dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut,
                     int64_t lut_row_stride, const uint16_t* __restrict__ scale,
                     const uint16_t* __restrict__ offset, uint16_t* __restrict__ W, int64_t N,
                     int64_t K, int64_t G) {
-  const int64_t chunks_per_row = K / 32;
-  const int64_t chunks = N * chunks_per_row;
+  __shared__ __align__(128) uint16_t s_out[kNbWarps][2][kNbSeg];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t segs_per_row = (K + kNbSeg - 1) / kNbSeg;
+  const int64_t nseg = N * segs_per_row;
   const int64_t groups = K / G;
-  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
-       c += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = c / chunks_per_row;
-    const int64_t k0 = (c - n * chunks_per_row) * 32;
-    const int64_t g = k0 / G;
-    const float s = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
-    const float o = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
+  int buf = 0;
+  for (int64_t sg = (int64_t)blockIdx.x * kNbWarps + warp; sg < nseg;
+       sg += (int64_t)gridDim.x * kNbWarps) {
+    const int64_t n = sg / segs_per_row;
+    const int64_t col0 = (sg - n * segs_per_row) * kNbSeg;
+    const int cols = (int)min((int64_t)kNbSeg, K - col0);  // a multiple of 32
+    const int64_t k0 = col0 + 32 * lane;
+    const bool on = 32 * lane < cols;
     uint32_t t0, t1, t2 = 0, t3 = 0;
     if constexpr (BITS == 3) {
       const uint4 t = __ldg(reinterpret_cast<const uint4*>(lut + n * lut_row_stride));
@@ -122,8 +139,16 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
       t0 = t.x;
       t1 = t.y;
     }
+    float s = 0.f, o = 0.f;
     uint32_t v[BITS];
-    load_chunk<BITS>(packed + c * (4 * BITS), v);
+#pragma unroll
+    for (int b = 0; b < BITS; ++b) v[b] = 0u;
+    if (on) {
+      const int64_t g = k0 / G;
+      s = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
+      o = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
+      load_chunk<BITS>(packed + (n * K + k0) / 8 * BITS, v);
+    }
     uint32_t out[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
@@ -132,12 +157,34 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
           __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(v, 2 * p + 1)), s, o);
       out[p] = pack_bf16x2_rn(lo, hi);
     }
-    uint16_t* dst = W + n * K + k0;
+    // the bulk copy that last read this buffer (two segments ago) must be done
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    __syncwarp();
+    uint16_t* seg_out = s_out[warp][buf];
+    if (on) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      stg_stream_v4(dst + 8 * q, make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2],
-                                            out[4 * q + 3]));
+      for (int step = 0; step < 4; ++step) {
+        const int q = (step + (lane >> 1)) & 3;  // 16-byte unit of this lane's 64 bytes
+        const uint4 val = q == 0 ? make_uint4(out[0], out[1], out[2], out[3])
+                        : q == 1 ? make_uint4(out[4], out[5], out[6], out[7])
+                        : q == 2 ? make_uint4(out[8], out[9], out[10], out[11])
+                                 : make_uint4(out[12], out[13], out[14], out[15]);
+        *reinterpret_cast<uint4*>(seg_out + 32 * lane + 8 * q) = val;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                   :: "l"(W + n * K + col0), "r"((uint32_t)__cvta_generic_to_shared(seg_out)),
+                      "r"((uint32_t)cols * 2u) : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    buf ^= 1;
   }
+  // every bulk copy of this warp has finished before the block's shared memory goes
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  __syncwarp();
 }
 
 int nb_grid(int64_t chunks, const DeviceInfo& dev) {
@@ -167,15 +214,16 @@ any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
                                 int64_t lut_row_stride, const uint16_t* scale,
                                 const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
                                 int64_t G, int bits, cudaStream_t stream, const DeviceInfo& dev) {
-  const int64_t chunks = N * K / 32;
-  if (bits == 3)
-    dequant_bits_kernel<3><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(
-        packed, lut, lut_row_stride, scale, offset, W, N, K, G);
-  else if (bits == 2)
-    dequant_bits_kernel<2><<<nb_grid(chunks, dev), kNbThreads, 0, stream>>>(
-        packed, lut, lut_row_stride, scale, offset, W, N, K, G);
-  else
-    return ANY4_ERR_SHAPE;
+  // a warp per 1024-column segment; 8 warps per block
+  const int64_t segs = N * ((K + kNbSeg - 1) / kNbSeg);
+  auto kern = bits == 3 ? dequant_bits_kernel<3> : dequant_bits_kernel<2>;
+  if (bits != 3 && bits != 2) return ANY4_ERR_SHAPE;
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(kern), kNbWarps * 32, 0);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t want = (segs + kNbWarps - 1) / kNbWarps;
+  const int64_t cap = (int64_t)dev.sm_count * per_sm;
+  kern<<<(unsigned)std::max<int64_t>(1, std::min(want, cap)), kNbWarps * 32, 0, stream>>>(
+      packed, lut, lut_row_stride, scale, offset, W, N, K, G);
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 

@@ -62,11 +62,15 @@ constexpr int kStageOff = 0;                    // 1024-byte aligned stages
 constexpr int kBarOff = kStageOff + kStages * kStageBytes;
 constexpr int kNumBars = 3 * kStages + 2;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
-constexpr int kSmemUsed = kMiscOff + 16;
+constexpr int kSmemUsed = kMiscOff + 32;
 constexpr int kSmemAlloc = kSmemUsed + 1024;    // slack to align the base to 1 KB
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
+// Every wait on a barrier or a flag gives up after this long (about 2 s of
+// %globaltimer), or after 1 ms in the test mode that stops one block's x
+// stream on purpose.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr unsigned long long kTestWaitLimitNs = 1000000ull;
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -100,14 +104,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // false (after flagging the error and the CTA-wide abort) if it does not
 // complete within the limit or another role has aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* dev_status) {
+                                          int32_t* dev_status, unsigned long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit) {
         *abort_flag = 1;
         report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
         return false;
@@ -118,8 +122,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // mbar_wait by every lane of a warp, with one verdict for the whole warp (so
 // that no lane is left alone in a later warp-synchronous instruction).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int32_t* dev_status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, dev_status)) != 0;
+                                               volatile int* abort_flag, int32_t* dev_status,
+                                               unsigned long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, dev_status, limit)) != 0;
 }
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -127,12 +132,25 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Tensor load with an L2 eviction policy (from createpolicy): x tiles are
+// read by every block that works on their rows, so they are kept in L2
+// (evict_last) while the weight stream, read once, goes first (evict_first).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
+                                            uint32_t bar, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];"
-      :: "r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar) : "memory");
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;"
+      :: "r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar), "l"(policy) : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -216,8 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-    uint16_t* __restrict__ y, int M, int N, int K, int G, int vec_store, int32_t* dev_status,
-    float* __restrict__ ws_partial, uint32_t* __restrict__ ws_flags) {
+    uint16_t* __restrict__ y, float* __restrict__ y32, int M, int N, int K, int G, int vec_store,
+    int32_t* dev_status, float* __restrict__ ws_partial, uint32_t* __restrict__ ws_flags,
+    int test_stall) {
+  // test_stall: block 0's x stream stops after its first stage, so a wait of
+  // the MMA issuer runs out (1 ms limit); the kernel must end cleanly
+  const unsigned long long wait_ns = test_stall ? kTestWaitLimitNs : kWaitLimitNs;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -234,6 +256,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
   int* partial_done = reinterpret_cast<int*>(smem + kMiscOff + 8);
+  // stages of x (and W) the producer issued and the MMA issuer saw complete:
+  // on an abort, the copies between the two are drained before the exit
+  volatile uint32_t* n_issued = reinterpret_cast<volatile uint32_t*>(smem + kMiscOff + 12);
+  volatile uint32_t* n_landed = reinterpret_cast<volatile uint32_t*>(smem + kMiscOff + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -248,6 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     mbar_init(accum_empty, kXformWarps);
     *abort_flag = 0;
     *partial_done = 0;
+    *n_issued = 0;
+    *n_landed = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -273,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   if (warp == 0) {
     // ------------------------------------------------ x tiles via TMA
     if (lane == 0) {
+      const uint64_t pol_x = l2_policy_evict_last(), pol_w = l2_policy_evict_first();
       uint32_t it = 0;
       SegIter seg{ub, ue, nkb};
       int tile, kb0, kb1;
@@ -281,14 +310,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % kStages);
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status)) goto done;
+          if (test_stall && blockIdx.x == 0 && it >= 1) goto done;  // the stream stops here
+          if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, dev_status, wait_ns)) goto done;
+          *n_issued = it + 1;
           mbar_arrive_expect_tx(full_a(s), kNAcc * kATileBytes);
           for (int h = 0; h < kNAcc; ++h)
-            tma_load_2d(stage_a(s, h), &tmap_x, kb * kBK, mt * kNAcc * kBM + h * kBM, full_a(s));
+            tma_load_2d(stage_a(s, h), &tmap_x, kb * kBK, mt * kNAcc * kBM + h * kBM, full_a(s),
+                        pol_x);
           if (kWTma) {
             // the bf16 W tile: 256 weight rows x 64 columns, same swizzled layout
             mbar_arrive_expect_tx(full_b(s), kBTileBytes);
-            tma_load_2d(stage_b(s), &tmap_w, kb * kBK, (tile / n_mtiles) * kBN, full_b(s));
+            tma_load_2d(stage_b(s), &tmap_w, kb * kBK, (tile / n_mtiles) * kBN, full_b(s),
+                        pol_w);
           }
         }
       }
@@ -300,14 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       SegIter seg{ub, ue, nkb};
       int tile, kb0, kb1;
       for (; seg.next(tile, kb0, kb1); ++tcount) {
-        if (tcount > 0 && !mbar_wait(accum_empty, (tcount - 1) & 1u, abort_flag, dev_status))
+        if (tcount > 0 && !mbar_wait(accum_empty, (tcount - 1) & 1u, abort_flag, dev_status, wait_ns))
           goto done;
         tc_fence_after();
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % kStages);
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(full_a(s), ph, abort_flag, dev_status)) goto done;
-          if (!mbar_wait(full_b(s), ph, abort_flag, dev_status)) goto done;
+          if (!mbar_wait(full_a(s), ph, abort_flag, dev_status, wait_ns)) goto done;
+          if (!mbar_wait(full_b(s), ph, abort_flag, dev_status, wait_ns)) goto done;
+          *n_landed = it + 1;
           tc_fence_after();
           const uint64_t db = smem_desc_sw128(stage_b(s));
 #pragma unroll
@@ -409,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
           // scale and offset as bf16 pairs (both columns of a pair share a group)
           const uint32_t s2 = (half ? other : mine) * 0x10001u;
           const uint32_t o2 = (half ? mine : other) * 0x10001u;
-          if (!mbar_wait_warp(empty(s), ph ^ 1u, abort_flag, dev_status)) return false;
+          if (!mbar_wait_warp(empty(s), ph ^ 1u, abort_flag, dev_status, wait_ns)) return false;
           const uint32_t brow = stage_b(s) + (uint32_t)rloc * 128u;
           const uint32_t words[4] = {q.x, q.y, q.z, q.w};
   #pragma unroll
@@ -459,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       // sums go to the workspace (a segment that does not start the tile), or
       // the partials of the tile's later segments are added (in block order)
       // and the bf16 result is written to y.
-      if (!mbar_wait_warp(accum_full, tcount & 1u, abort_flag, dev_status)) goto done;
+      if (!mbar_wait_warp(accum_full, tcount & 1u, abort_flag, dev_status, wait_ns)) goto done;
       tc_fence_after();
       {
         const int quad = warp & 3;       // TMEM lanes 32*quad .. 32*quad+31
@@ -483,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
                 asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
                              : "=r"(f) : "l"(ws_flags + c_end) : "memory");
                 if (f != 0u) break;
-                if ((i & 63u) == 0u && (*abort_flag || globaltimer() - t0 > kWaitLimitNs)) {
+                if ((i & 63u) == 0u && (*abort_flag || globaltimer() - t0 > wait_ns)) {
                   *abort_flag = 1;
                   report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
                   break;
@@ -523,7 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
             }
           }
           const int n0 = nt * kBN + cc * 16;
-          if (m < M) {
+          if (m < M && y32 != nullptr) {
+            // the unrounded fp32 sums
+            float* yr = y32 + (int64_t)m * N;
+            for (int i = 0; i < 16; ++i)
+              if (n0 + i < N) yr[n0 + i] = acc[i];
+          } else if (m < M) {
             uint16_t* yr = y + (int64_t)m * N;
             if (vec_store && n0 + 16 <= N) {
 #pragma unroll
@@ -559,6 +598,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   }
 done:
   tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // tensor loads issued but never seen complete may still be writing the
+    // stages: wait for them (bounded) before the block's shared memory is freed
+    for (uint32_t it = *n_landed; it < *n_issued; ++it) {
+      const int s = (int)(it % kStages);
+      const uint32_t ph = (it / kStages) & 1u;
+      const unsigned long long t0 = globaltimer();
+      while (!(mbar_try_wait(full_a(s), ph) && (!kWTma || mbar_try_wait(full_b(s), ph))))
+        if (globaltimer() - t0 > kWaitLimitNs) break;
+    }
+  }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -613,9 +664,9 @@ template <bool kWTma>
 any4_status launch_prefill_impl(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                                 int64_t lut_row_stride, const uint16_t* scale,
                                 const uint16_t* offset, const uint16_t* w_bf16, uint16_t* y,
-                                int64_t M, int64_t N, int64_t K, int64_t G, void* workspace,
-                                size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream,
-                                const DeviceInfo& dev) {
+                                float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                bool test_stall, cudaStream_t stream, const DeviceInfo& dev) {
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   if (dev.smem_optin < (size_t)kSmemAlloc) return ANY4_ERR_UNSUPPORTED;
   EncodeTiledFn enc = encode_fn();
@@ -645,13 +696,9 @@ any4_status launch_prefill_impl(const uint16_t* x, const uint8_t* packed, const 
       return ANY4_ERR_CUDA;
   }
 
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_kernel<kWTma>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-  });
-  if (attr_err != cudaSuccess) return ANY4_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_kernel<kWTma>), kSmemAlloc) !=
+      ANY4_OK)
+    return ANY4_ERR_CUDA;
 
   const int64_t tiles = ((M + kNAcc * kBM - 1) / (kNAcc * kBM)) * ((N + kBN - 1) / kBN);
   const int64_t units = tiles * ((K + kBK - 1) / kBK);
@@ -681,8 +728,9 @@ any4_status launch_prefill_impl(const uint16_t* x, const uint8_t* packed, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, prefill_kernel<kWTma>, map, map_w, packed, lut, lut_row_stride,
-                         scale, offset, y, (int)M, (int)N, (int)K, (int)G, vec_store, dev_status,
-                         ws_partial, ws_flags) != cudaSuccess)
+                         scale, offset, y, y32, (int)M, (int)N, (int)K, (int)G, vec_store,
+                         dev_status,
+                         ws_partial, ws_flags, test_stall ? 1 : 0) != cudaSuccess)
     return ANY4_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
@@ -691,11 +739,13 @@ any4_status launch_prefill_impl(const uint16_t* x, const uint8_t* packed, const 
 
 any4_status launch_prefill(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                            int64_t lut_row_stride, const uint16_t* scale,
-                           const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
-                           int64_t K, int64_t G, void* workspace, size_t workspace_bytes,
-                           int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
-  return launch_prefill_impl<false>(x, packed, lut, lut_row_stride, scale, offset, nullptr, y, M,
-                                    N, K, G, workspace, workspace_bytes, dev_status, stream, dev);
+                           const uint16_t* offset, uint16_t* y, float* y32, int64_t M,
+                           int64_t N, int64_t K, int64_t G, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, bool test_stall,
+                           cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_prefill_impl<false>(x, packed, lut, lut_row_stride, scale, offset, nullptr, y,
+                                    y32, M, N, K, G, workspace, workspace_bytes, dev_status,
+                                    test_stall, stream, dev);
 }
 
 // Two passes for large M: the weights are dequantised once into the
@@ -713,9 +763,9 @@ size_t prefill_two_pass_workspace_size(int64_t M, int64_t N, int64_t K, int64_t 
 
 any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                                     int64_t lut_row_stride, const uint16_t* scale,
-                                    const uint16_t* offset, uint16_t* y, int64_t M, int64_t N,
-                                    int64_t K, int64_t G, void* workspace,
-                                    size_t workspace_bytes, int32_t* dev_status,
+                                    const uint16_t* offset, uint16_t* y, float* y32, int64_t M,
+                                    int64_t N, int64_t K, int64_t G, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, bool test_stall,
                                     cudaStream_t stream, const DeviceInfo& dev) {
   if (workspace == nullptr || workspace_bytes < prefill_two_pass_workspace_size(M, N, K, G))
     return ANY4_ERR_WORKSPACE;
@@ -724,8 +774,8 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
   any4_status st = launch_dequant(packed, lut, lut_row_stride, scale, offset, w, N, K, G, stream,
                                   dev);
   if (st != ANY4_OK) return st;
-  return launch_prefill_impl<true>(x, packed, lut, lut_row_stride, scale, offset, w, y, M, N, K, G,
-                                   workspace, fused, dev_status, stream, dev);
+  return launch_prefill_impl<true>(x, packed, lut, lut_row_stride, scale, offset, w, y, y32, M, N,
+                                   K, G, workspace, fused, dev_status, test_stall, stream, dev);
 }
 
 }  // namespace any4

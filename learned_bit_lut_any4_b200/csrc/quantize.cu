@@ -248,8 +248,7 @@ any4_status launch_quantize_nq(const uint16_t* w, const float* ex, int64_t N, in
                                int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
                                uint16_t* scale, uint16_t* offset, int32_t* iters, size_t smem,
                                cudaStream_t stream) {
-  if (cudaFuncSetAttribute(quantize_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(quantize_kernel<NQ>), smem) != ANY4_OK)
     return ANY4_ERR_CUDA;
   quantize_kernel<NQ><<<(unsigned)N, kQuantThreads, smem, stream>>>(
       w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);

@@ -84,8 +84,8 @@ template <int MT, int KC>
 __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
     const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed,
     const uint16_t* __restrict__ lut, int64_t lut_row_stride, const uint16_t* __restrict__ scale,
-    const uint16_t* __restrict__ offset, uint16_t* __restrict__ y, int M, int N, int K, int G,
-    int groups8, int nslices, int rows_max) {
+    const uint16_t* __restrict__ offset, uint16_t* __restrict__ y, float* __restrict__ y32,
+    int M, int N, int K, int G, int groups8, int nslices, int rows_max) {
   constexpr int MB = MT / 8;  // 8-row blocks of x (one MMA each per step)
   constexpr int NA = 2;       // accumulator sets (even / odd steps)
   // dynamic shared memory: [nwarps][kSkStages] ring stages, then the partial
@@ -337,15 +337,18 @@ __global__ void __launch_bounds__(kSkWarps * 32, 2) skinny_kernel(
     if (n_base + row >= N) continue;
     float tot = 0.f;
     for (int w = 0; w < nw_used; ++w) tot += s_part[((size_t)w * rows_max + row) * M + m];
-    y[(int64_t)m * N + n_base + row] = f32_to_bf16_rn(tot);
+    if (y32 != nullptr)
+      y32[(int64_t)m * N + n_base + row] = tot;
+    else
+      y[(int64_t)m * N + n_base + row] = f32_to_bf16_rn(tot);
   }
 }
 
 template <int MT, int KC>
 any4_status run_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                        int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                       uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                       cudaStream_t stream, const DeviceInfo& dev) {
+                       uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                       bool overlap, cudaStream_t stream, const DeviceInfo& dev) {
   auto kern = skinny_kernel<MT, KC>;
   const int nslices = (int)((K + 128 * KC - 1) / (128 * KC));
   const int nwarps = std::min(kSkWarps, nslices);
@@ -359,13 +362,8 @@ any4_status run_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t*
       512, (int64_t)((smem_max - ring_total) / ((size_t)nwarps * M * sizeof(float))) / 8 * 8);
   if (rows_cap < 8) return ANY4_ERR_UNSUPPORTED;
   int per_sm = 0;
-  static bool attr_done = false;  // one per template instance
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) !=
-        cudaSuccess)
-      return ANY4_ERR_CUDA;
-    attr_done = true;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem_max) != ANY4_OK)
+    return ANY4_ERR_CUDA;
   // balanced 8-row-group ranges, one resident wave
   int64_t grid = 0, rows_max = 0;
   for (int pass = 0; pass < 2; ++pass) {
@@ -394,7 +392,7 @@ any4_status run_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t*
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, x, packed, lut, lut_row_stride, scale,
-                                             offset, y, (int)M, (int)N, (int)K, (int)G,
+                                             offset, y, y32, (int)M, (int)N, (int)K, (int)G,
                                              (int)groups8, nslices, (int)rows_max);
   return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
@@ -403,14 +401,14 @@ any4_status run_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t*
 
 any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                          uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t G, bool overlap,
-                          cudaStream_t stream, const DeviceInfo& dev) {
+                          uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
+                          bool overlap, cudaStream_t stream, const DeviceInfo& dev) {
   if (M < 1 || M > 16 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return ANY4_ERR_UNSUPPORTED;
   if (M <= 8)
-    return run_skinny<8, 2>(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, overlap,
-                            stream, dev);
-  return run_skinny<16, 1>(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G, overlap,
-                           stream, dev);
+    return run_skinny<8, 2>(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                            overlap, stream, dev);
+  return run_skinny<16, 1>(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
+                           overlap, stream, dev);
 }
 
 }  // namespace any4

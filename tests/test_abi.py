@@ -79,7 +79,9 @@ def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, sc
     (dict(status=FAKE + 2), any4.ANY4_ERR_ALIGN),
     (dict(M=17, path=1), any4.ANY4_ERR_UNSUPPORTED),
     (dict(path=7), any4.ANY4_ERR_UNSUPPORTED),
-    (dict(flags=2), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(flags=8), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(ws=FAKE + 8, ws_bytes=1 << 20), any4.ANY4_ERR_ALIGN),
 ])
 def test_matmul_rejects_bad_arguments(kw, expect):
     assert _matmul(**kw) == expect
@@ -161,12 +163,28 @@ def test_workspace_size_of_bad_shapes_is_zero():
     assert any4.any4_matmul_workspace_size(0, 64, 64, 32) == 0
 
 
+def _sm_count():
+    import torch
+    return (torch.cuda.get_device_properties(0).multi_processor_count
+            if torch.cuda.is_available() else 160)
+
+
 def test_workspace_sizes_by_path():
-    """Decode needs no workspace; prefill below M = 1024 needs the one-pass
-    stream-K scratch (independent of the shape); from M = 1024 the size adds
-    room for the dequantised bf16 weights, N * K * 2 bytes rounded to 256."""
+    """Decode at M <= 2 takes the pair-table kernel's stream-K exchange (one
+    64 x M fp32 partial and one 8-byte flag per block of an SM-count grid,
+    rounded to 256 bytes) where its shape rules hold, and nothing otherwise;
+    prefill below M = 1024 needs the one-pass stream-K scratch (independent of
+    the shape); from M = 1024 the size adds room for the dequantised bf16
+    weights, N * K * 2 bytes rounded to 256."""
     N, K, G = 1100, 2048, 128
-    assert any4.any4_matmul_workspace_size(16, N, K, G) == 0
+    sms = _sm_count()
+    for M in (1, 2):
+        assert any4.any4_matmul_workspace_size(M, N, K, G) == \
+            ((sms * M * 64 * 4 + sms * 8 + 255) // 256) * 256
+    assert any4.any4_matmul_workspace_size(1, N, K, 256) == 0       # G outside {32, 64, 128}
+    assert any4.any4_matmul_workspace_size(1, N, 1024 + 64, 64) == 0  # K/G not a multiple of 8
+    for M in (3, 8, 16):
+        assert any4.any4_matmul_workspace_size(M, N, K, G) == 0
     one = any4.any4_matmul_workspace_size(17, N, K, G)
     assert one > 0 and one == any4.any4_matmul_workspace_size(1023, N, K, G)
     assert one == any4.any4_matmul_workspace_size(300, 64, 64, 32)
@@ -211,3 +229,62 @@ def test_bindings_refuse_host_tensors_and_wrong_dtypes():
         any4.any4_pack_bits(idx.to(torch.int32), 2)
     with pytest.raises(TypeError):
         any4.any4_dequant_bits(idx.float(), w, w, w, 64, 3)
+
+
+def test_matmul_bindings_check_sizes_before_launch():
+    """The C ABI sees bare pointers and cannot tell a short buffer; the Python
+    matmul wrappers check every size against M, N, K and G before any library
+    call, so an undersized y, scale, offset or dev_status never reaches a
+    kernel (sizes are checked before the device, so host tensors show it)."""
+    import torch
+    M, N, K, G = 2, 16, 256, 64
+    x = torch.zeros((M, K), dtype=torch.bfloat16)
+    packed = torch.zeros((N, K // 2), dtype=torch.uint8)
+    lut = torch.zeros((N, 16), dtype=torch.bfloat16)
+    so = torch.zeros((N, K // G), dtype=torch.bfloat16)
+    short = torch.zeros((N, K // G - 1), dtype=torch.bfloat16)
+    for fn in (any4.any4_matmul, any4.any4_matmul_static_scratch):
+        with pytest.raises(ValueError, match="y must have shape"):
+            fn(x, packed, lut, so, so, G, y=torch.zeros((M, N - 1), dtype=torch.bfloat16))
+        with pytest.raises(ValueError, match="y must have shape"):
+            fn(x, packed, lut, so, so, G, y=torch.zeros((M * N,), dtype=torch.bfloat16))
+        with pytest.raises(ValueError, match="scale and offset"):
+            fn(x, packed, lut, short, so, G)
+        with pytest.raises(ValueError, match="scale and offset"):
+            fn(x, packed, lut, so, short, G)
+        with pytest.raises(ValueError, match="divide K"):
+            fn(x, packed, lut, so, so, 96)
+        with pytest.raises(ValueError, match="packed holds"):
+            fn(x, packed[:, :64], lut, so, so, G)
+        with pytest.raises(ValueError, match="lut must be"):
+            fn(x, packed, lut[:8], so, so, G)
+        with pytest.raises(ValueError, match="dev_status"):
+            fn(x, packed, lut, so, so, G, y=torch.zeros((M, N), dtype=torch.bfloat16),
+               dev_status=torch.zeros(0, dtype=torch.int32))
+        # right sizes on host tensors: refused for the device, not the sizes
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            fn(x, packed, lut, so, so, G)
+    with pytest.raises(ValueError, match="packed must have shape"):
+        any4.any4_pack(torch.zeros((N, K), dtype=torch.uint8),
+                       packed=torch.zeros((N, K // 2 - 16), dtype=torch.uint8))
+
+
+def _prefill_one_pass_bytes(slots):
+    """The one-pass prefill workspace: one fp32 256 x 256 partial tile per
+    block of the stream-K grid, then one flag word per block rounded up to
+    256 bytes."""
+    return slots * 256 * 256 * 4 + (slots * 4 + 255) // 256 * 256
+
+
+def test_static_scratch_holds_a_148_sm_grid_and_no_more():
+    """ANY4_STATIC_SCRATCH_BYTES covers the one-pass prefill workspace of a
+    148-SM B200 and refuses a grid of one more block (the entry point then
+    returns ANY4_ERR_WORKSPACE).  The library's own size (the SM count of the
+    current device, or 160 blocks where there is no device) pins the formula."""
+    import torch
+    slots = (torch.cuda.get_device_properties(0).multi_processor_count
+             if torch.cuda.is_available() else 160)
+    assert any4.any4_matmul_workspace_size(16, 1024, 1024, 128, path="prefill") == \
+        _prefill_one_pass_bytes(slots)
+    assert _prefill_one_pass_bytes(148) <= any4.ANY4_STATIC_SCRATCH_BYTES
+    assert _prefill_one_pass_bytes(149) > any4.ANY4_STATIC_SCRATCH_BYTES

@@ -22,8 +22,17 @@ DECODE_SHAPES = (workloads.TINY + workloads.LLAMA3_8B_DECODE
                  + workloads.LLAMA3_70B_DECODE)
 
 
-def _run(d, shape, path="auto"):
-    y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path=path)
+NO_WORKSPACE = "no_workspace"
+
+
+def _run(d, shape, path="auto", workspace=None):
+    """workspace None: the binding allocates what the path asks for (the
+    pair-table kernel at M <= 2); NO_WORKSPACE: none is passed, so M <= 2
+    runs the decode kernels that need none."""
+    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE \
+        else workspace
+    y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path=path,
+                         workspace=ws)
     torch.cuda.synchronize()
     return host_bits(y)
 
@@ -37,6 +46,11 @@ def test_decode_full_shapes(shape):
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     st = assert_matmul_close(y, y_ref, shape.name)
     print(shape.name, st)
+    if shape.M <= 2:
+        # the same shape on the kernels that need no workspace
+        y = _run(d, shape, workspace=NO_WORKSPACE)
+        st = assert_matmul_close(y, y_ref, shape.name + " without workspace")
+        print(shape.name, "without workspace", st)
 
 
 @pytest.mark.parametrize("M", list(range(1, 17)))
@@ -46,9 +60,10 @@ def test_decode_every_m_ragged(M):
     shape = workloads.Shape(f"ragged_m{M}", M, 1056, 333, 32, 9201, 9700 + M)
     p = workloads.make(shape)
     d = DeviceProblem(p)
-    y = _run(d, shape, path="decode")
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
-    assert_matmul_close(y, y_ref, shape.name)
+    for ws in (None, NO_WORKSPACE):
+        y = _run(d, shape, path="decode", workspace=ws)
+        assert_matmul_close(y, y_ref, f"{shape.name} {ws}")
 
 
 @pytest.mark.parametrize("K,N,G", [(32, 1, 32), (64, 7, 32), (96, 7, 32), (96, 1000, 32),
@@ -56,26 +71,32 @@ def test_decode_every_m_ragged(M):
 def test_decode_edge_shapes(K, N, G):
     """Tiny and ragged shapes; (32, 1, 32) and (96, 7, 32) end the scale and
     offset tensors on a lone group at an even flat index (N * K/G odd)."""
-    shape = workloads.Shape(f"edge_{K}_{N}", 3, K, N, G, 9300 + N, 9800 + K // 32)
-    p = workloads.make(shape)
-    d = DeviceProblem(p)
-    y = _run(d, shape, path="decode")
-    y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
-    assert_matmul_close(y, y_ref, shape.name)
+    for M in (1, 2, 3):
+        shape = workloads.Shape(f"edge_{K}_{N}_m{M}", M, K, N, G, 9300 + N, 9800 + K // 32)
+        p = workloads.make(shape)
+        d = DeviceProblem(p)
+        y = _run(d, shape, path="decode")
+        y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
+        assert_matmul_close(y, y_ref, shape.name)
 
 
-def test_decode_one_hot_is_exact():
+@pytest.mark.parametrize("workspace", [None, NO_WORKSPACE])
+def test_decode_one_hot_is_exact(workspace):
     """x = e_k returns column k of the dequantised weight, bit for bit: the
-    fused group-affine form reduces to fmaf(LUT, scale, offset) rounded once."""
+    fused group-affine form reduces to fmaf(LUT, scale, offset) rounded once.
+    Both M = 1 kernels (pair table with its workspace, weight streaming
+    without)."""
     shape = workloads.Shape("onehot", 1, 4096, 2000, 128, 9401, 9901)
     p = workloads.make(shape)
     d = DeviceProblem(p)
     W_ref = oracle.dequant(d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     one = torch_bf16_bits(np.array([1.0], np.float32))[0]
-    for k in (0, 1, 31, 32, 1023, 1024, 2047, 4095):
+    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE else None
+    for k in (0, 1, 31, 32, 127, 128, 1023, 1024, 2047, 4095):
         x = np.zeros((1, shape.K), np.uint16)
         x[0, k] = one
-        y = any4.any4_matmul(dev_bf16(x), d.packed, d.lut, d.scale, d.offset, shape.G)
+        y = any4.any4_matmul(dev_bf16(x), d.packed, d.lut, d.scale, d.offset, shape.G,
+                             workspace=ws)
         torch.cuda.synchronize()
         got = bits_to_f64(host_bits(y))[0]
         assert np.array_equal(got, bits_to_f64(W_ref[:, k])), k
@@ -106,9 +127,10 @@ def test_decode_shared_table():
     assert_matmul_close(host_bits(y), y_ref, "shared")
 
 
-def test_decode_writes_only_its_output():
+@pytest.mark.parametrize("M", [1, 2, 5])
+def test_decode_writes_only_its_output(M):
     """Guard bands around y stay untouched."""
-    shape = workloads.Shape("guard", 5, 1024, 999, 64, 9601, 9961)
+    shape = workloads.Shape(f"guard_m{M}", M, 1024, 999, 64, 9601, 9961)
     p = workloads.make(shape)
     d = DeviceProblem(p, check_pack=False)
     pad = 4096
@@ -121,22 +143,25 @@ def test_decode_writes_only_its_output():
     assert_matmul_close(host_bits(y), y_ref, "guard")
 
 
-@pytest.mark.parametrize("M", [1, 4, 12])
-def test_decode_overlap_prior_chain(M):
+@pytest.mark.parametrize("M,workspace", [(1, None), (2, None), (1, NO_WORKSPACE), (4, None),
+                                         (12, None)])
+def test_decode_overlap_prior_chain(M, workspace):
     """ANY4_FLAG_OVERLAP_PRIOR: x is produced by the kernel just before each
     call and y is consumed by the kernel just after; a chain of overlapped
     calls must match the same chain run without overlap, bit for bit, and the
-    oracle within tolerance (M = 1: weight-streaming kernel; M > 1: skinny)."""
+    oracle within tolerance (M <= 2: pair-table kernel, or weight streaming
+    without a workspace; M > 2: skinny)."""
     shape = workloads.Shape(f"overlap_m{M}", M, 4096, 4096, 128, 9701, 9702 + M)
     p = workloads.make(shape)
     d = DeviceProblem(p)
+    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE else None
     def chain(overlap):
         x = d.x.clone()
         outs = []
         for i in range(6):
             x = (x.float() * 0.5 + 0.25).to(torch.bfloat16)      # written by the preceding kernel
             y = any4.any4_matmul(x, d.packed, d.lut, d.scale, d.offset, shape.G,
-                                 overlap_prior=overlap)
+                                 overlap_prior=overlap, workspace=ws)
             outs.append(y.clone())                              # read by the following kernel
             x = torch.cat([y[:, :shape.K]], dim=1) if shape.N >= shape.K else x
             x = (x.float() / (x.float().abs().max() + 1)).to(torch.bfloat16)
@@ -147,7 +172,8 @@ def test_decode_overlap_prior_chain(M):
     for ya, yb in zip(a, b):
         assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
-    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, overlap_prior=True)
+    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, overlap_prior=True,
+                          workspace=ws)
     torch.cuda.synchronize()
     assert_matmul_close(host_bits(y1), y_ref, "overlap")
 
@@ -156,18 +182,20 @@ def test_decode_overlap_prior_chain(M):
                                           (3072, 300, 64, False), (8192, 2050, 128, False),
                                           (4096, 1500, 128, True), (2048, 9, 64, True)])
 def test_decode_m1_streamed_variants(K, N, G, shared):
-    """M = 1 shapes of the tensor-memory-streamed decode kernel: every group
-    size it takes, ragged rows, a last 1024-column slice cut short, the one
-    table mode; dev_status must stay clear."""
+    """M = 1 shapes of both tensor-memory-streamed decode kernels (the
+    pair-table kernel with its workspace, the shuffle kernel without): every
+    group size they take, ragged rows, a last slice cut short, the one table
+    mode; dev_status must stay clear."""
     shape = workloads.Shape(f"m1_{K}_{N}_{G}", 1, K, N, G, 9901 + K + N, 9951 + G)
     p = workloads.make(shape)
     d = DeviceProblem(p)
     lut = p.lut[11 % N].copy() if shared else p.lut
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    y = any4.any4_matmul(d.x, d.packed, dev_bf16(lut), d.scale, d.offset, shape.G,
-                         dev_status=status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, lut, p.scale, p.offset, shape.G,
                                per_tensor_lut=shared)
-    assert_matmul_close(host_bits(y), y_ref, shape.name)
+    for ws in (None, torch.empty(0, dtype=torch.uint8, device="cuda")):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        y = any4.any4_matmul(d.x, d.packed, dev_bf16(lut), d.scale, d.offset, shape.G,
+                             dev_status=status, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert_matmul_close(host_bits(y), y_ref, f"{shape.name} {ws is None}")

@@ -39,6 +39,10 @@ def test_static_scratch_size_matches_header():
     workloads.Shape("noalloc_ragged", 300, 1056, 520, 32, 9931, 9932),
     # 2 x 4 tiles of 32 stages over 64 blocks: every tile split across blocks
     workloads.Shape("noalloc_split", 512, 2048, 1024, 128, 9933, 9934),
+    # M >= 1024: the workspace entry point runs the two-pass route here (its
+    # workspace holds the dequantised weights), this entry point the one-pass
+    # kernel; they agree within the matmul tolerance, not bit for bit
+    workloads.Shape("noalloc_m1024", 1024, 1024, 1024, 128, 9935, 9936),
 ], ids=lambda s: s.name)
 def test_static_scratch_matches_workspace_entry(shape):
     p = workloads.make(shape)
