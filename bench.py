@@ -65,7 +65,7 @@ def kernel_source_hash() -> str:
     """Hash of the M = 1 pair-table decode kernel source (the only kernel of a step): a
     stored ncu traffic figure is only used while it was taken on this source."""
     h = hashlib.sha256()
-    for fn in ("decode_pair.cu", "common.cuh"):
+    for fn in ("decode_tma.cu", "common.cuh"):
         with open(os.path.join(ROOT, "learned_bit_lut_any4_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -74,7 +74,7 @@ def kernel_source_hash() -> str:
 def stored_traffic():
     """Per-launch DRAM bytes (read + write) of the decode kernel on this step,
     from the committed ncu summary, if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_pair_kernel_llama3_8b_layer_m1.md")
+    path = os.path.join(ROOT, "profiles", "decode_tma_kernel_llama3_8b_layer_m1.md")
     try:
         text = open(path).read()
     except OSError:
@@ -683,8 +683,9 @@ def nbit_dequant_detail(reps: int = 10):
     return out
 
 
-def profile_shape(name: str, calls: int):
-    """Run a few any4_matmul calls (auto path) on one workload shape."""
+def profile_shape(name: str, calls: int, op: str = "matmul"):
+    """Run a few calls of one operation (any4_matmul on the auto path, or
+    any4_dequant) on one workload shape: a small, fixed case for ncu."""
     import torch
     import learned_bit_lut_any4_b200 as any4
     shape = [s for s in workloads.all_shapes() if s.name == name]
@@ -695,10 +696,14 @@ def profile_shape(name: str, calls: int):
     packed = any4.any4_pack(torch.from_numpy(p.idx).cuda())
     lut, sc, of, x = (_dev_bf16(a) for a in (p.lut, p.scale, p.offset, p.x))
     y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
+    W = torch.empty((s.N, s.K), dtype=torch.bfloat16, device="cuda") if op == "dequant" else None
     for _ in range(calls):
-        any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
+        if op == "dequant":
+            any4.any4_dequant(packed, lut, sc, of, s.G, W=W)
+        else:
+            any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
     torch.cuda.synchronize()
-    print(f"profiled {name}: M={s.M} K={s.K} N={s.N} G={s.G}, {calls} calls", flush=True)
+    print(f"profiled {op} {name}: M={s.M} K={s.K} N={s.N} G={s.G}, {calls} calls", flush=True)
 
 
 def main():
@@ -720,6 +725,7 @@ def main():
                     help="no timing: run --profile-calls any4_matmul calls on one named "
                          "workload shape (a small, fixed case for ncu captures)")
     ap.add_argument("--profile-calls", type=int, default=3)
+    ap.add_argument("--profile-op", default="matmul", choices=["matmul", "dequant"])
     ap.add_argument("--quantize-detail", action="store_true",
                     help="no step: time any4_quantize on the Llama3-8B matrices (and the "
                          "oracle on a sample of rows) and print one JSON line")
@@ -728,7 +734,7 @@ def main():
                     help="leave the any4_quantize timing out of the JSON line")
     args = ap.parse_args()
     if args.profile_shape:
-        profile_shape(args.profile_shape, args.profile_calls)
+        profile_shape(args.profile_shape, args.profile_calls, args.profile_op)
         return
     if args.quantize_detail:
         print(json.dumps({"detail": "quantize",
@@ -768,7 +774,7 @@ def main():
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": stored_traffic(),
-                    "kernel": "decode_pair_kernel<1, 4> (the only kernel of the step)",
+                    "kernel": "decode_tma_kernel<8> (the only kernel of the step)",
                     "peak_source": peaks.get("source", "measured")}
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,

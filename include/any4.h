@@ -175,6 +175,27 @@ ANY4_API any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, in
                          int64_t N, int64_t K, int64_t G, any4_stream_t stream);
 
 /*
+ * any4_group_sums -- per-group sums of the activations:
+ *   xsum[m][g] = sum over the G columns k = g*G .. g*G+G-1 of x[m][k]
+ * The factor of the group offset when the product of paper §4.1 Eq. 8 is
+ * expanded with the group-affine weights of §2.5.2 (alpha * LUT[c] + beta):
+ *   sum_k x * (alpha * LUT[c] + beta) = alpha * sum_k x * LUT[c] + beta * xsum.
+ * For callers that apply the offsets themselves (a matmul on the bare table
+ * values, an offset correction, a calibration statistic); any4_matmul does not
+ * need it, it applies alpha and beta to every weight.
+ *   x      [M][K] bf16 (device, caller-owned, 16-byte aligned)
+ *   xsum   [M][K/G] fp32 (device, caller-owned output, 16-byte aligned)
+ *   M >= 1; K and G multiples of 32 with K % G == 0.
+ * fp32 sums in a fixed order (each 8-column chunk left to right, then the
+ * group's chunks left to right), so deterministic; every result is within
+ * gamma_{G-1} * sum |x| of the exact sum (gamma_n = n u / (1 - n u),
+ * u = 2^-24).  Returns ANY4_ERR_NULL, _SHAPE or _ALIGN without launching
+ * when a precondition fails; asynchronous on `stream` otherwise.
+ */
+ANY4_API any4_status any4_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K,
+                                     int64_t G, any4_stream_t stream);
+
+/*
  * any4_matmul -- y = x * dequant(W)^T (paper §4.1 Eq. 8, orientation §4.2),
  * dequantisation fused (W is never written to memory on the decode path).
  *   x               [M][K] bf16
@@ -231,7 +252,13 @@ typedef enum any4_flags {
    * tensor memory released, so the device and stream stay usable.  Kernels
    * with bounded waits only: the pair-table and weight-streaming decode
    * kernels and the prefill kernel (others ignore it). */
-  ANY4_FLAG_TEST_STALL = 4
+  ANY4_FLAG_TEST_STALL = 4,
+  /* Decode path, M = 1: run the pair-table kernel (the M = 2 default) instead
+   * of the weight-streaming kernel that M = 1 takes by default.  Needs the
+   * workspace any4_matmul_workspace_size returns for the shape; without it,
+   * or where the pair-table kernel does not take the shape, the flag is
+   * ignored. */
+  ANY4_FLAG_PAIR_TABLE = 8
 } any4_flags;
 
 /* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16)

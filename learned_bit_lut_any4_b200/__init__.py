@@ -25,6 +25,7 @@ from ._native import (  # noqa: F401
     any4_bits_per_weight,
     any4_dequant,
     any4_dequant_bits,
+    any4_group_sums,
     any4_matmul,
     any4_matmul_choose_path,
     any4_matmul_static_scratch,

@@ -31,6 +31,7 @@ ANY4_STATIC_SCRATCH_BYTES = 148 * 262144 + 1024
 ANY4_FLAG_OVERLAP_PRIOR = 1
 ANY4_FLAG_FP32_OUT = 2
 ANY4_FLAG_TEST_STALL = 4
+ANY4_FLAG_PAIR_TABLE = 8
 # Limits of any4_quantize (the row lives in one block's shared memory).
 ANY4_QUANTIZE_MAX_K = 16384
 ANY4_QUANTIZE_MAX_ITER = 100000
@@ -86,6 +87,8 @@ def library() -> ctypes.CDLL:
     lib.any4_matmul_choose_path.restype = i32
     lib.any4_status_string.argtypes = [i32]
     lib.any4_status_string.restype = ctypes.c_char_p
+    lib.any4_group_sums.argtypes = [vp, vp, i64, i64, i64, vp]
+    lib.any4_group_sums.restype = i32
     lib.any4_bits_per_weight.argtypes = [i64, i64]
     lib.any4_bits_per_weight.restype = ctypes.c_double
     lib.any4_version.argtypes = []
@@ -374,6 +377,25 @@ def any4_dequant(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
     return W
 
 
+def any4_group_sums(x: torch.Tensor, G: int, xsum: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 xsum[M, K/G]: the sum of x[m, k] over each group of G columns."""
+    _need(x, "x", _BF16)
+    if x.dim() != 2:
+        raise ValueError("x must be [M, K]")
+    dev = x.device
+    M, K = x.shape
+    if G < 1 or K % G:
+        raise ValueError("K must be a multiple of G")
+    if xsum is None:
+        xsum = torch.empty((M, K // G), dtype=torch.float32, device=dev)
+    _need(xsum, "xsum", (torch.float32,), dev)
+    _need_shape(xsum, "xsum", (M, K // G))
+    with _on_device(dev):
+        _check(library().any4_group_sums(_ptr(x), _ptr(xsum), M, K, G, _stream(dev)),
+               "any4_group_sums")
+    return xsum
+
+
 def any4_matmul_workspace_size(M: int, N: int, K: int, G: int, path: str = "auto") -> int:
     return int(library().any4_matmul_workspace_size_ex(M, N, K, G, PATHS[path]))
 
@@ -388,7 +410,7 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                 y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 path: str = "auto", dev_status: torch.Tensor | None = None,
                 overlap_prior: bool = False, fp32_out: bool = False,
-                test_stall: bool = False) -> torch.Tensor:
+                test_stall: bool = False, pair_table: bool = False) -> torch.Tensor:
     """bf16 y[M, N] = x[M, K] * dequant(W)^T, fp32 accumulation.
 
     workspace: a CUDA tensor of at least any4_matmul_workspace_size() bytes, or
@@ -398,7 +420,9 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
     work still running on the stream; the decode kernel may then overlap it).
     fp32_out: ANY4_FLAG_FP32_OUT, y is fp32 and holds the sums unrounded.
     test_stall: ANY4_FLAG_TEST_STALL, a test of the failure handling (one
-    block's stream stops, the call ends with ANY4_ERR_TIMEOUT in dev_status)."""
+    block's stream stops, the call ends with ANY4_ERR_TIMEOUT in dev_status).
+    pair_table: ANY4_FLAG_PAIR_TABLE, M = 1 on the pair-table kernel (needs
+    the workspace) instead of the weight-streaming kernel."""
     M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y,
                                              dev_status, fp32_out)
     dev = x.device
@@ -423,7 +447,8 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                                   _ptr(dev_status), p,
                                   (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
                                   | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
-                                  | (ANY4_FLAG_TEST_STALL if test_stall else 0),
+                                  | (ANY4_FLAG_TEST_STALL if test_stall else 0)
+                                  | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
                                   _stream(dev)), "any4_matmul")
     return y
 

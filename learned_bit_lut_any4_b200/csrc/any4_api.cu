@@ -235,6 +235,17 @@ any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut
                         (cudaStream_t)stream, dev);
 }
 
+any4_status any4_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K, int64_t G,
+                             any4_stream_t stream) {
+  if (!x || !xsum) return ANY4_ERR_NULL;
+  if (M < 1 || !shape_ok(M, K, G)) return ANY4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(xsum)) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_group_sums(x, xsum, M, K, G, (cudaStream_t)stream, dev);
+}
+
 any4_path any4_matmul_choose_path(int64_t M, int64_t N, int64_t K, int64_t G) {
   (void)N; (void)K; (void)G;
   return M <= kDecodeMaxM ? ANY4_PATH_DECODE : ANY4_PATH_PREFILL;
@@ -277,7 +288,8 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (workspace && !aligned16(workspace)) return ANY4_ERR_ALIGN;
   if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
   if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
-  if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL))
+  if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL |
+                         ANY4_FLAG_PAIR_TABLE))
     return ANY4_ERR_UNSUPPORTED;
   float* y32 = (flags & ANY4_FLAG_FP32_OUT) ? reinterpret_cast<float*>(y) : nullptr;
   const bool test_stall = (flags & ANY4_FLAG_TEST_STALL) != 0;
@@ -296,7 +308,8 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (path == ANY4_PATH_DECODE) {
     return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
                          workspace, workspace_bytes, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,
-                         dev_status, test_stall, (cudaStream_t)stream, dev);
+                         (flags & ANY4_FLAG_PAIR_TABLE) != 0, dev_status, test_stall,
+                         (cudaStream_t)stream, dev);
   }
   if (prefill_use_two_pass(M, N, K) &&
       workspace_bytes >= prefill_two_pass_workspace_size(M, N, K, G))

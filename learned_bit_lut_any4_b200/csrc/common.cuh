@@ -135,13 +135,15 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const uint16_t* scale, const uint16_t* offset, uint16_t* W,
                            int64_t N, int64_t K, int64_t G, cudaStream_t stream,
                            const DeviceInfo& dev);
+any4_status launch_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K, int64_t G,
+                              cudaStream_t stream, const DeviceInfo& dev);
 // The decode path (M <= 16).  y32, when not NULL, receives the fp32 sums
 // instead of y (the unrounded results).  A workspace of at least
 // decode_pair_workspace_size bytes selects the pair-table kernel for M <= 2.
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
                           uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
-                          void* workspace, size_t workspace_bytes, bool overlap,
+                          void* workspace, size_t workspace_bytes, bool overlap, bool pair_at_m1,
                           int32_t* dev_status, bool test_stall, cudaStream_t stream,
                           const DeviceInfo& dev);
 // Pair-table decode for M <= 2 (decode_pair.cu): workspace bytes it needs on

@@ -372,18 +372,23 @@ any4_status run(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
 any4_status launch_decode(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                           int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
                           uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K, int64_t G,
-                          void* workspace, size_t workspace_bytes, bool overlap,
+                          void* workspace, size_t workspace_bytes, bool overlap, bool pair_at_m1,
                           int32_t* dev_status, bool test_stall, cudaStream_t stream,
                           const DeviceInfo& dev) {
-  // M <= 2 with its workspace: pair-table lookups, stream-K over 64-row sets
-  // (decode_pair.cu)
+  // The kernel measured fastest for each M on B200 where several apply:
+  //   M = 1  the weight-streaming shuffle kernel (decode_tma.cu), unless the
+  //          caller asks for the pair-table kernel;
+  //   M = 2  the pair-table kernel (decode_pair.cu), stream-K over 64-row
+  //          sets, when the caller passes its workspace.
   const size_t pair_ws = decode_pair_workspace_size(M, N, K, G, dev);
-  if (pair_ws > 0 && workspace != nullptr && workspace_bytes >= pair_ws)
+  const bool pair_ok = pair_ws > 0 && workspace != nullptr && workspace_bytes >= pair_ws;
+  const bool tma_ok = decode_tma_supported(M, N, K, G);
+  if (pair_ok && (M == 2 || pair_at_m1 || !tma_ok))
     return launch_decode_pair(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
                               workspace, overlap, dev_status, test_stall, stream, dev);
   // M = 1 with a 1024-column slice holding whole 16-byte runs of scales:
-  // weights streamed by the tensor-memory-access engine (decode_tma.cu)
-  if (decode_tma_supported(M, N, K, G))
+  // weights streamed by the tensor-memory-access engine
+  if (tma_ok)
     return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G,
                              overlap, dev_status, test_stall, stream, dev);
   // M >= 2: the skinny kernel (one dequantisation of the weights for all rows

@@ -32,11 +32,12 @@
 //    with g == t), so C[g][t] and C[g+8][t] are that lane's two rows' partial
 //    sums; 256 weights per MMA, fp32 accumulation.  With M = 2 the second
 //    row of x sits in columns 4..7 (lanes with g == t + 4).
-//  * Weights stream through a per-warp ring of 3 stages filled by
+//  * Weights stream through a per-warp ring of 4 stages filled by
 //    cp.async.bulk.tensor (codes [64 rows][64 B] with the 64-byte swizzle, so
-//    each lane's 16-byte reads are conflict free; x [M][128]); scales and
-//    offsets arrive per window of 8 groups ([64 rows][16 B] each) in two
-//    window slots per warp and are kept in registers for the window.
+//    each lane's 16-byte reads are conflict free; x [M][128]).  The warps of
+//    a block split a set's chunks into contiguous ranges.  A lane loads its
+//    two rows' scales and offsets for the chunk itself (a few bytes, shared
+//    with its neighbouring chunks through L1), one chunk ahead of their use.
 //  * Work split (stream-K): the (row set, 128-column chunk) units are divided
 //    evenly over the blocks (one per SM).  A block whose range starts inside
 //    a row set publishes its 64 x M partial sums in the workspace and then
@@ -66,9 +67,8 @@ constexpr int kPWarps = 8;
 constexpr int kPThreads = kPWarps * 32;
 constexpr int kPRows = 64;                          // rows of a set: two per lane
 constexpr int kPChunk = 128;                        // columns per ring stage
-constexpr int kPStages = 3;
+constexpr int kPStages = 4;
 constexpr int kPCodeBytes = kPRows * kPChunk / 2;   // 4096
-constexpr int kPWinBytes = kPRows * 16;             // 8 groups of scales (or offsets)
 constexpr int kPLutBytes = kPRows * 32;             // the set's 64 tables
 constexpr uint32_t kPTableBytes = 65536;
 constexpr unsigned long long kPWaitNs = 2000000000ull;
@@ -81,14 +81,18 @@ struct PLayout {
   static constexpr int kStage = ((kPCodeBytes + MT * kPChunk * 2 + 511) / 512) * 512;
   static constexpr uint32_t kTxCodes = kPCodeBytes;
   static constexpr uint32_t kTxX = MT * kPChunk * 2;
-  static constexpr uint32_t kTxWin = 2 * kPWinBytes;
+};
+
+// Unit ranges of the blocks (block b: units ub[b] .. ub[b + 1] - 1), worked
+// out on the host so that the kernel needs no 64-bit division.
+constexpr int kPMaxGrid = 160;
+struct PSched {
+  int ub[kPMaxGrid + 1];
 };
 
 struct PMaps {
   CUtensorMap codes;   // u8 [N][K/2], box {64, 64}, 64-byte swizzle
   CUtensorMap x;       // bf16 [M][K], box {128, MT}
-  CUtensorMap scale;   // bf16 [N][K/G], box {8, 64}
-  CUtensorMap offset;  // bf16 [N][K/G], box {8, 64}
   CUtensorMap lut;     // bf16 [N][16], box {16, 64} (a table per row)
 };
 
@@ -162,58 +166,59 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// bf16 value q (0..7) of a window held as 4 bf16x2 words, in both halves
-__device__ __forceinline__ uint32_t win_dup(const uint32_t (&w)[4], int q) {
-  const uint32_t lo = (q & 2) ? w[1] : w[0];
-  const uint32_t hi = (q & 2) ? w[3] : w[2];
-  const uint32_t v = (q & 4) ? hi : lo;
-  return prmt(v, 0u, (q & 1) ? 0x3232u : 0x1010u);
+// bf16 scale or offset pairs (s, s) of the 32-column sub-blocks of a chunk:
+// one group for G = 128 (GS = 4), two for G = 64, four for G = 32.  The raw
+// 2, 4 or 8 bytes of a row's groups of the chunk sit in `raw` (2 words).
+template <int GS>
+__device__ __forceinline__ uint32_t group_dup(const uint2& raw, int sub) {
+  const int q = sub / GS;  // group of the sub-block within the chunk
+  const uint32_t w = (q & 2) ? raw.y : raw.x;
+  return prmt(w, 0u, (q & 1) ? 0x3232u : 0x1010u);
+}
+template <int GS>
+__device__ __forceinline__ uint2 load_groups(const uint16_t* p) {
+  if constexpr (GS == 4) return make_uint2((uint32_t)ldg_u16(p), 0u);
+  if constexpr (GS == 2) return make_uint2(__ldg(reinterpret_cast<const uint32_t*>(p)), 0u);
+  return __ldg(reinterpret_cast<const uint2*>(p));
 }
 
 // The block's units [u0, u1) of the flattened (row set, chunk) space and the
-// chunks of row set r that warp w handles.
+// chunks of row set r that warp w handles: an eighth of the block's chunks
+// of the set, contiguous (each warp streams long runs of its rows).
 struct PRange {
-  int64_t u0, u1;
+  int u0, u1;  // units of the block (fewer than 2^31: N K / 8192 <= 2^27)
   int KC;
-  __device__ void warp_chunks(int64_t r, int w, int& lo, int& hi) const {
-    const int64_t base = r * KC;
-    const int cl = (int)((u0 > base ? u0 : base) - base);
-    const int ch = (int)((u1 < base + KC ? u1 : base + KC) - base);
-    const int n = ch - cl;
+  __device__ void warp_chunks(int r, int w, int& lo, int& hi) const {
+    const int base = r * KC;
+    const int cl = (u0 > base ? u0 : base) - base;
+    const int n = (u1 < base + KC ? u1 : base + KC) - base - cl;
     lo = cl + (n * w) / kPWarps;
     hi = cl + (n * (w + 1)) / kPWarps;
   }
 };
 
-// The sequence of (row set, chunk) items of one warp, in consumption order,
-// with a flag for the items that start a new window of scales (the warp's
-// first chunk in a set, or a chunk in a later window than the one before).
+// The sequence of (row set, chunk) items of one warp, in consumption order.
 struct PIter {
   PRange rg;
-  int warp, wshift;
-  int64_t r, r_last;
-  int c, c_hi, prev_win;
-  __device__ void start(const PRange& range, int w, int window_shift) {
+  int warp;
+  int r, r_last;
+  int c, c_hi;
+  __device__ void start(const PRange& range, int w) {
     rg = range;
     warp = w;
-    wshift = window_shift;
     r = range.u0 / range.KC;
     r_last = (range.u1 - 1) / range.KC;
     range.warp_chunks(r, w, c, c_hi);
-    prev_win = -1;
     skip();
   }
   __device__ void skip() {
     while (r <= r_last && c >= c_hi) {
       ++r;
-      prev_win = -1;
       if (r <= r_last) rg.warp_chunks(r, warp, c, c_hi);
     }
   }
   __device__ bool valid() const { return r <= r_last; }
-  __device__ bool new_window() const { return (c >> wshift) != prev_win; }
   __device__ void next() {
-    prev_win = c >> wshift;
     ++c;
     skip();
   }
@@ -222,18 +227,26 @@ struct PIter {
 template <int MT, int GS>  // rows of x (1, 2); G / 32 (1, 2, 4)
 __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
     const __grid_constant__ PMaps maps, const uint16_t* __restrict__ lut_shared,
-    uint16_t* __restrict__ y, float* __restrict__ y32, int N, int K, int KC, int64_t units,
+    const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
+    uint16_t* __restrict__ y, float* __restrict__ y32, int N, int K, int KC,
+    const __grid_constant__ PSched sched,
     float* __restrict__ ws_part, unsigned long long* __restrict__ ws_flag, int dyn_bytes,
     int32_t* dev_status, int test_stall) {
   using L = PLayout<MT>;
-  // window = 8 groups = 8 G columns = (8 G / 128) chunks: chunk c is in window c >> wshift
-  constexpr int kWShift = GS == 1 ? 1 : (GS == 2 ? 2 : 3);
+  constexpr int kGPC = 4 / GS;  // groups per 128-column chunk
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // test_stall: warp 0 of block 0 stops its weight stream after one item, so
   // its next wait runs out (1 ms limit) and the kernel ends cleanly
   const unsigned long long wait_ns = test_stall ? kPTestWaitNs : kPWaitNs;
   const bool stalled = test_stall && blockIdx.x == 0 && warp == 0;
+  if (threadIdx.x == 0) {
+    // fetch the tensor-map descriptors now rather than at each first use
+    asm volatile("prefetch.tensormap [%0];" :: "l"(&maps.codes) : "memory");
+    asm volatile("prefetch.tensormap [%0];" :: "l"(&maps.x) : "memory");
+    if (lut_shared == nullptr)
+      asm volatile("prefetch.tensormap [%0];" :: "l"(&maps.lut) : "memory");
+  }
 
   // ---- shared-memory layout: the 64 KiB-aligned pair table, then everything
   // else first-fit in the space below and above it
@@ -250,14 +263,10 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
     fits = false;
     return 0u;
   };
-  uint32_t my_stage0 = 0, my_win0 = 0;
+  uint32_t my_stage0 = 0;
   for (int w = 0; w < kPWarps; ++w) {  // per warp: kPStages stages of L::kStage bytes
     const uint32_t a = alloc(kPStages * L::kStage, 512);
     if (w == warp) my_stage0 = a;
-  }
-  for (int w = 0; w < kPWarps; ++w) {  // per warp: 2 window slots of (scales, offsets)
-    const uint32_t a = alloc(2 * 2 * kPWinBytes, 128);
-    if (w == warp) my_win0 = a;
   }
   const uint32_t lutbuf = alloc(2 * kPLutBytes, 128);
   const uint32_t part = alloc(kPWarps * MT * kPRows * 4, 16);
@@ -269,6 +278,7 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
   }
   uint8_t* const gsm = smem - base;  // generic pointer of shared address a: gsm + a
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + flags);
+  volatile int* late_flag = reinterpret_cast<volatile int*>(gsm + flags + 4);
   float* const s_part = reinterpret_cast<float*>(gsm + part);
   const uint32_t my_bars = bars + 8u * (uint32_t)(warp * kPStages);
   const uint32_t lut_bars = bars + 8u * (uint32_t)(kPWarps * kPStages);
@@ -287,44 +297,28 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
 
   PRange rg;
   rg.KC = KC;
-  rg.u0 = units * (int64_t)blockIdx.x / gridDim.x;
-  rg.u1 = units * (int64_t)(blockIdx.x + 1) / gridDim.x;
-  const int64_t r_first = rg.u0 / KC, r_last = (rg.u1 - 1) / KC;
+  rg.u0 = sched.ub[blockIdx.x];
+  rg.u1 = sched.ub[blockIdx.x + 1];
+  const int r_first = rg.u0 / KC, r_last = (rg.u1 - 1) / KC;
   const int nsets = (int)(r_last - r_first + 1);
 
   // ---- producer state (lane 0 of each warp): items issued ahead of use
   PIter pit;
-  pit.start(rg, warp, kWShift);
-  int issued = 0, pw_loads = 0;
-  int win_item0 = -1, win_item1 = -1;  // item that last filled each window slot
+  pit.start(rg, warp);
+  int issued = 0;
   auto issue = [&](int consumed, bool with_x) {
     while (pit.valid() && issued < consumed + kPStages && !(stalled && issued >= 1)) {
-      const bool nw = pit.new_window();
-      const int wslot = pw_loads & 1;
-      if (nw && (wslot ? win_item1 : win_item0) >= consumed) break;  // still to be read
       const int st = issued % kPStages;
       const uint32_t dst = my_stage0 + (uint32_t)(st * L::kStage);
       const uint32_t bar = my_bars + 8u * st;
-      const uint32_t tx = L::kTxCodes + L::kTxX + (nw ? L::kTxWin : 0u);
+      const uint32_t tx = L::kTxCodes + L::kTxX;
       if (with_x) {
         mbar_arrive_expect(bar, tx);
       } else {
         mbar_expect(bar, tx);  // the arrival comes once x is issued too
       }
-      const int row = (int)(pit.r * kPRows);
-      tma_2d(dst, &maps.codes, pit.c * (kPChunk / 2), row, bar);
+      tma_2d(dst, &maps.codes, pit.c * (kPChunk / 2), (int)(pit.r * kPRows), bar);
       if (with_x) tma_2d(dst + kPCodeBytes, &maps.x, pit.c * kPChunk, 0, bar);
-      if (nw) {
-        const uint32_t wd = my_win0 + (uint32_t)(wslot * 2 * kPWinBytes);
-        const int gx = (pit.c >> kWShift) * 8;
-        tma_2d(wd, &maps.scale, gx, row, bar);
-        tma_2d(wd + kPWinBytes, &maps.offset, gx, row, bar);
-        if (wslot)
-          win_item1 = issued;
-        else
-          win_item0 = issued;
-        ++pw_loads;
-      }
       ++issued;
       pit.next();
     }
@@ -338,25 +332,46 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
            bar);
   };
 
-  // weights (codes, scales, tables) may stream before the preceding kernel
-  // finishes; x is read and y written only after griddepcontrol.wait
+  // weights (codes, tables) may stream before the preceding kernel finishes;
+  // x is read and y written only after griddepcontrol.wait
   int early = 0;
   if (lane == 0) {
-    issue(0, false);
-    early = issued;
     if (warp == 0) {
       issue_lut(0);
       issue_lut(1);
     }
+    issue(0, false);
+    early = issued;
   }
+  // the scales and offsets of a lane's two rows for one item: rows
+  // r * 64 + lane and r * 64 + 32 + lane, the chunk's groups (zeros past N)
+  const int groups = K / (32 * GS);
+  auto load_so = [&](int r, int c, uint2 (&so)[4]) {
+    const int ra = r * kPRows + lane, rb = ra + 32;
+    const int g0 = c * kGPC;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) so[i] = make_uint2(0u, 0u);
+    if (ra < N) {
+      so[0] = load_groups<GS>(scale + (int64_t)ra * groups + g0);
+      so[1] = load_groups<GS>(offset + (int64_t)ra * groups + g0);
+    }
+    if (rb < N) {
+      so[2] = load_groups<GS>(scale + (int64_t)rb * groups + g0);
+      so[3] = load_groups<GS>(offset + (int64_t)rb * groups + g0);
+    }
+  };
+  PIter cit;  // the consumer's copy of the item sequence (all lanes)
+  cit.start(rg, warp);
+  uint2 so_next[4];
+  if (cit.valid()) load_so(cit.r, cit.c, so_next);
+
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (lane == 0) {
-    for (int i = 0; i < early; ++i) {
+    PIter it;  // the early items again, for their chunk index
+    it.start(rg, warp);
+    for (int i = 0; i < early; ++i, it.next()) {
       const int st = i % kPStages;
-      PIter it;  // the i-th item again, for its chunk index
-      it.start(rg, warp, kWShift);
-      for (int j = 0; j < i; ++j) it.next();
       tma_2d(my_stage0 + (uint32_t)(st * L::kStage) + kPCodeBytes, &maps.x, it.c * kPChunk, 0,
              my_bars + 8u * st);
       mbar_arrive(my_bars + 8u * st);
@@ -369,14 +384,15 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
   const uint32_t xoff = (uint32_t)((g >> 2) * kPChunk * 2);
   const uint32_t lb0 = tab | (uint32_t)(lane << 2);
   const uint32_t lb1 = tab | 128u | (uint32_t)(lane << 2);
+  // 16-byte unit j of a lane's code row sits at unit j ^ swz (64-byte swizzle);
+  // both of its rows (lane, 32 + lane) share it
+  const uint32_t swz = (uint32_t)((lane >> 1) & 3);
 
   bool ok = true;
-  int item = 0, wloads = 0;
-  uint32_t ws_[4] = {0u, 0u, 0u, 0u}, wo_[4] = {0u, 0u, 0u, 0u};   // slot 0 window
-  uint32_t ws1[4] = {0u, 0u, 0u, 0u}, wo1[4] = {0u, 0u, 0u, 0u};   // slot 1 window
+  int item = 0;
 
   for (int s = 0; s < nsets; ++s) {
-    const int64_t r = r_first + s;
+    const int r = r_first + s;
     // ---- the pair tables of this set: warp w builds entries 32w .. 32w+31
     {
       uint32_t la[8], lb[8], lwa, lwb;
@@ -421,57 +437,40 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
     if (threadIdx.x == 0) issue_lut(s + 2);
 
     // ---- this warp's chunks of the set
-    int c_lo, c_hi;
-    rg.warp_chunks(r, warp, c_lo, c_hi);
     float acc[MT == 1 ? 4 : 2][4];
 #pragma unroll
     for (int q = 0; q < (MT == 1 ? 4 : 2); ++q)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
-    int prev_win = -1, cur_slot = 0;
-    for (int c = c_lo; c < c_hi; ++c, ++item) {
+    while (cit.valid() && cit.r == r) {
+      const int c = cit.c;
+      uint2 so[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) so[i] = so_next[i];
+      cit.next();  // the next item's scales and offsets, one item ahead
+      if (cit.valid()) load_so(cit.r, cit.c, so_next);
+      // after an abort the remaining items are skipped, not consumed: the
+      // drain at the end waits for the copies of those already issued
       if (*abort_flag != 0) ok = false;
-      if (!ok) break;
+      if (!ok) continue;
       const int st = item % kPStages;
       if (!mbar_wait(my_bars + 8u * st, (uint32_t)((item / kPStages) & 1), wait_ns)) {
         if (lane == 0) report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
         *abort_flag = 1;
         ok = false;
-        break;
+        continue;
       }
       const uint32_t sp = my_stage0 + (uint32_t)(st * L::kStage);
-      if ((c >> kWShift) != prev_win) {
-        prev_win = c >> kWShift;
-        cur_slot = wloads & 1;
-        ++wloads;
-        const uint32_t wd = my_win0 + (uint32_t)(cur_slot * 2 * kPWinBytes);
-        const uint4 s0 = lds128(wd + (uint32_t)(lane * 16));
-        const uint4 s1 = lds128(wd + (uint32_t)((32 + lane) * 16));
-        const uint4 o0 = lds128(wd + kPWinBytes + (uint32_t)(lane * 16));
-        const uint4 o1 = lds128(wd + kPWinBytes + (uint32_t)((32 + lane) * 16));
-        ws_[0] = s0.x; ws_[1] = s0.y; ws_[2] = s0.z; ws_[3] = s0.w;
-        ws1[0] = s1.x; ws1[1] = s1.y; ws1[2] = s1.z; ws1[3] = s1.w;
-        wo_[0] = o0.x; wo_[1] = o0.y; wo_[2] = o0.z; wo_[3] = o0.w;
-        wo1[0] = o1.x; wo1[1] = o1.y; wo1[2] = o1.z; wo1[3] = o1.w;
-      }
+      const uint32_t rowa = sp + (uint32_t)(lane * 64), rowb = rowa + 32u * 64u;
       const int nsub = min(4, (K - c * kPChunk) / 32);  // K % 32 == 0
-      uint32_t sa2 = 0, oa2 = 0, sb2 = 0, ob2 = 0;
-      int cur_q = -1;
 #pragma unroll 1
       for (int sub = 0; sub < nsub; ++sub) {
-        // group of these 32 columns within the window (8 groups)
-        const int q = ((c * 4 + sub) / GS) & 7;
-        if (q != cur_q) {
-          cur_q = q;
-          sa2 = win_dup(ws_, q); oa2 = win_dup(wo_, q);
-          sb2 = win_dup(ws1, q); ob2 = win_dup(wo1, q);
-        }
-        // codes of the lane's two rows, columns 32 sub .. 32 sub + 31 (16 bytes;
-        // 16-byte unit j of row r sits at unit j ^ ((r >> 1) & 3) of the row)
-        const uint32_t ja = (uint32_t)(sub ^ ((lane >> 1) & 3));
-        const uint32_t jb = (uint32_t)(sub ^ (((32 + lane) >> 1) & 3));
-        const uint4 qa = lds128(sp + (uint32_t)(lane * 64) + (ja << 4));
-        const uint4 qb = lds128(sp + (uint32_t)((32 + lane) * 64) + (jb << 4));
+        const uint32_t sa2 = group_dup<GS>(so[0], sub), oa2 = group_dup<GS>(so[1], sub);
+        const uint32_t sb2 = group_dup<GS>(so[2], sub), ob2 = group_dup<GS>(so[3], sub);
+        // codes of the lane's two rows, columns 32 sub .. 32 sub + 31
+        const uint32_t ju = ((uint32_t)sub ^ swz) << 4;
+        const uint4 qa = lds128(rowa + ju);
+        const uint4 qb = lds128(rowb + ju);
         const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
         const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
@@ -494,11 +493,12 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
           }
         }
       }
+      ++item;
       // stage consumed: let the tensor loads refill it
       __syncwarp();
       if (lane == 0) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(item + 1, true);
+        issue(item, true);
       }
     }
     // ---- partial sums of the 64 rows (x MT) over this warp's chunks
@@ -521,49 +521,50 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
       dst[32 + l0] = tot[2];
       dst[32 + l0 + 1] = tot[3];
     }
-    __syncthreads();
     // ---- the set's sums: fixed order over warps, then over blocks
-    const int64_t set_u0 = r * KC, set_u1 = set_u0 + KC;
+    const int set_u0 = r * KC, set_u1 = set_u0 + KC;
     const bool starts = rg.u0 <= set_u0;  // this block holds chunk 0 of the set
     const bool whole = starts && rg.u1 >= set_u1;
-    bool publish = false, consumed = false;
-    if (threadIdx.x < MT * kPRows && *abort_flag == 0) {
+    // blocks holding later parts of the set: blockIdx + 1 .. blockIdx + nlater
+    int nlater = 0;
+    if (starts && !whole)
+      while (blockIdx.x + 1 + nlater < gridDim.x && sched.ub[blockIdx.x + 1 + nlater] < set_u1)
+        ++nlater;
+    if (threadIdx.x == 0) *late_flag = 0;
+    __syncthreads();
+    if (threadIdx.x < nlater && *abort_flag == 0) {
+      // one thread per later block: wait (bounded) for its published partials
+      const unsigned long long* fp = ws_flag + blockIdx.x + 1 + threadIdx.x;
+      unsigned long long f;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(fp) : "memory");
+      if (f != kPPublished) {
+        const unsigned long long t0 = gtime();
+        for (uint32_t i = 1;; ++i) {
+          asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(fp) : "memory");
+          if (f == kPPublished) break;
+          if ((i & 15u) == 0u && gtime() - t0 > wait_ns) break;
+        }
+      }
+      if (f != kPPublished) {
+        report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
+        *late_flag = 1;
+      }
+    }
+    __syncthreads();
+    const bool good = *abort_flag == 0 && *late_flag == 0;
+    if (threadIdx.x < MT * kPRows && good) {
       const int m = threadIdx.x / kPRows, slot = threadIdx.x % kPRows;
       float v = 0.f;
       for (int w = 0; w < kPWarps; ++w) v += s_part[(size_t)(w * MT + m) * kPRows + slot];
-      const int64_t row = r * kPRows + slot;
+      const int row = r * kPRows + slot;
       if (!starts) {
         // a later part of the set: hand the partial sums to the set's first block
         __stcg(ws_part + (size_t)blockIdx.x * (MT * kPRows) + threadIdx.x, v);
-        publish = true;
       } else {
-        bool got = true;
-        if (!whole) {
-          // add the later blocks' parts in block order
-          for (int64_t b = blockIdx.x + 1; b < gridDim.x; ++b) {
-            if (units * b / gridDim.x >= set_u1) break;
-            const unsigned long long* fp = ws_flag + b;
-            unsigned long long f;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(fp) : "memory");
-            if (f != kPPublished) {
-              const unsigned long long t0 = gtime();
-              for (uint32_t i = 1;; ++i) {
-                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(fp)
-                             : "memory");
-                if (f == kPPublished) break;
-                if ((i & 63u) == 0u && gtime() - t0 > wait_ns) break;
-              }
-            }
-            if (f != kPPublished) {
-              report_status(dev_status, (int32_t)ANY4_ERR_TIMEOUT);
-              got = false;
-              break;
-            }
-            v += __ldcg(ws_part + (size_t)b * (MT * kPRows) + threadIdx.x);
-          }
-        }
-        if (got) consumed = true;
-        if (got && row < N) {
+        // add the later blocks' parts in block order (their flags were seen above)
+        for (int b = 1; b <= nlater; ++b)
+          v += __ldcg(ws_part + (size_t)(blockIdx.x + b) * (MT * kPRows) + threadIdx.x);
+        if (row < N) {
           if (y32 != nullptr)
             y32[(int64_t)m * N + row] = v;
           else
@@ -572,19 +573,17 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_pair_kernel(
       }
     }
     __syncthreads();  // partial sums read; table and s_part may be rewritten
-    if (publish && threadIdx.x == 0) {
-      __threadfence();
-      asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(ws_flag + blockIdx.x),
-                   "l"(kPPublished) : "memory");
-    }
-    if (consumed && threadIdx.x == 0 && !whole) {
-      // every reader of the later blocks' partials is past the barrier above:
-      // their flags go back to "not published" for the next launch
-      for (int64_t b = blockIdx.x + 1; b < gridDim.x; ++b) {
-        if (units * b / gridDim.x >= set_u1) break;
-        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(ws_flag + b), "l"(0ull)
-                     : "memory");
+    if (threadIdx.x == 0 && good) {
+      if (!starts) {
+        __threadfence();
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(ws_flag + blockIdx.x),
+                     "l"(kPPublished) : "memory");
       }
+    }
+    if (threadIdx.x < nlater && good) {
+      // the consumed flags go back to "not published" for the next launch
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;"
+                   :: "l"(ws_flag + blockIdx.x + 1 + threadIdx.x), "l"(0ull) : "memory");
     }
   }
   // before leaving, no tensor load of this warp may still be writing its ring
@@ -641,18 +640,14 @@ any4_status run_pair(const uint16_t* x, const uint8_t* packed, const uint16_t* l
   if (!map2d(enc, &maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2,
              (uint64_t)N, (uint64_t)K / 2, kPChunk / 2, kPRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !map2d(enc, &maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)K, (uint64_t)M,
-             (uint64_t)K * 2, kPChunk, MT, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map2d(enc, &maps.scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, scale, (uint64_t)(K / G),
-             (uint64_t)N, (uint64_t)(K / G) * 2, 8, kPRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map2d(enc, &maps.offset, CU_TENSOR_MAP_DATA_TYPE_UINT16, offset, (uint64_t)(K / G),
-             (uint64_t)N, (uint64_t)(K / G) * 2, 8, kPRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+             (uint64_t)K * 2, kPChunk, MT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ANY4_ERR_CUDA;
   if (lut_row_stride == 16) {
     if (!map2d(enc, &maps.lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, lut, 16, (uint64_t)N, 32, 16,
                kPRows, CU_TENSOR_MAP_SWIZZLE_NONE))
       return ANY4_ERR_CUDA;
   } else {
-    maps.lut = maps.scale;  // unused: one table for the matrix, read directly
+    maps.lut = maps.codes;  // unused: one table for the matrix, read directly
   }
   auto kern = decode_pair_kernel<MT, GS>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), kPDynBytes) != ANY4_OK)
@@ -660,7 +655,9 @@ any4_status run_pair(const uint16_t* x, const uint8_t* packed, const uint16_t* l
   const int KC = (int)((K + kPChunk - 1) / kPChunk);
   const int64_t sets = (N + kPRows - 1) / kPRows;
   const int64_t units = sets * KC;
-  const int grid = (int)std::min<int64_t>(units, dev.sm_count);
+  const int grid = (int)std::min<int64_t>({units, (int64_t)dev.sm_count, (int64_t)kPMaxGrid});
+  PSched sched;
+  for (int b = 0; b <= grid; ++b) sched.ub[b] = (int)(units * b / grid);
   float* ws_part = static_cast<float*>(workspace);
   auto* ws_flag = reinterpret_cast<unsigned long long*>(
       static_cast<uint8_t*>(workspace) + (size_t)dev.sm_count * MT * kPRows * sizeof(float));
@@ -675,8 +672,9 @@ any4_status run_pair(const uint16_t* x, const uint8_t* packed, const uint16_t* l
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const uint16_t* lut_shared = lut_row_stride == 0 ? lut : nullptr;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, lut_shared, y, y32, (int)N, (int)K,
-                                             KC, units, ws_part, ws_flag, kPDynBytes, dev_status,
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, lut_shared, scale, offset, y, y32,
+                                             (int)N, (int)K,
+                                             KC, sched, ws_part, ws_flag, kPDynBytes, dev_status,
                                              test_stall ? 1 : 0);
   return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
@@ -686,8 +684,12 @@ any4_status run_pair(const uint16_t* x, const uint8_t* packed, const uint16_t* l
 bool decode_pair_supported(int64_t M, int64_t N, int64_t K, int64_t G) {
   if (M < 1 || M > 2) return false;
   if (G != 32 && G != 64 && G != 128) return false;
-  if ((K / G) % 8 != 0) return false;  // 16-byte rows of scales for the tensor maps
-  if (N > INT32_MAX / 2 || K > INT32_MAX / 2) return false;
+  // whole 128-column chunks, so that a chunk holds 4 / (G / 32) whole groups
+  // and its scales are one aligned 2-, 4- or 8-byte load per row
+  if (K % kPChunk != 0) return false;
+  // unit, row and column indices in 32 bits
+  if (N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return false;
+  if (((N + kPRows - 1) / kPRows) * (K / kPChunk) > (int64_t(1) << 30)) return false;
   return true;
 }
 

@@ -113,19 +113,24 @@ __global__ void __launch_bounds__(kNbWarps * 32)
 dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut,
                     int64_t lut_row_stride, const uint16_t* __restrict__ scale,
                     const uint16_t* __restrict__ offset, uint16_t* __restrict__ W, int64_t N,
-                    int64_t K, int64_t G) {
+                    int K, int G, int g_shift) {
   __shared__ __align__(128) uint16_t s_out[kNbWarps][2][kNbSeg];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t segs_per_row = (K + kNbSeg - 1) / kNbSeg;
+  const int segs_per_row = (K + kNbSeg - 1) / kNbSeg;
   const int64_t nseg = N * segs_per_row;
-  const int64_t groups = K / G;
+  const int groups = K / G;
+  const int64_t first = (int64_t)blockIdx.x * kNbWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * kNbWarps;
+  // (row, segment) of the warp's segments without a division per step
+  int64_t n = first / segs_per_row;
+  int seg = (int)(first % segs_per_row);
+  const int64_t n_step = stride / segs_per_row;
+  const int s_step = (int)(stride % segs_per_row);
   int buf = 0;
-  for (int64_t sg = (int64_t)blockIdx.x * kNbWarps + warp; sg < nseg;
-       sg += (int64_t)gridDim.x * kNbWarps) {
-    const int64_t n = sg / segs_per_row;
-    const int64_t col0 = (sg - n * segs_per_row) * kNbSeg;
-    const int cols = (int)min((int64_t)kNbSeg, K - col0);  // a multiple of 32
-    const int64_t k0 = col0 + 32 * lane;
+  for (int64_t sg = first; sg < nseg; sg += stride) {
+    const int col0 = seg * kNbSeg;
+    const int cols = min(kNbSeg, K - col0);  // a multiple of 32
+    const int k0 = col0 + 32 * lane;
     const bool on = 32 * lane < cols;
     uint32_t t0, t1, t2 = 0, t3 = 0;
     if constexpr (BITS == 3) {
@@ -144,7 +149,7 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
 #pragma unroll
     for (int b = 0; b < BITS; ++b) v[b] = 0u;
     if (on) {
-      const int64_t g = k0 / G;
+      const uint32_t g = g_shift >= 0 ? ((uint32_t)k0 >> g_shift) : (uint32_t)k0 / (uint32_t)G;
       s = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
       o = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
       load_chunk<BITS>(packed + (n * K + k0) / 8 * BITS, v);
@@ -181,10 +186,22 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
     buf ^= 1;
+    n += n_step;
+    seg += s_step;
+    if (seg >= segs_per_row) {
+      seg -= segs_per_row;
+      ++n;
+    }
   }
   // every bulk copy of this warp has finished before the block's shared memory goes
   if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   __syncwarp();
+}
+
+int nb_pow2_shift(int64_t G) {
+  for (int s = 0; s < 31; ++s)
+    if ((int64_t(1) << s) == G) return s;
+  return -1;
 }
 
 int nb_grid(int64_t chunks, const DeviceInfo& dev) {
@@ -222,8 +239,9 @@ any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
   if (per_sm < 1) per_sm = 1;
   const int64_t want = (segs + kNbWarps - 1) / kNbWarps;
   const int64_t cap = (int64_t)dev.sm_count * per_sm;
+  if (K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   kern<<<(unsigned)std::max<int64_t>(1, std::min(want, cap)), kNbWarps * 32, 0, stream>>>(
-      packed, lut, lut_row_stride, scale, offset, W, N, K, G);
+      packed, lut, lut_row_stride, scale, offset, W, N, (int)K, (int)G, nb_pow2_shift(G));
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 

@@ -67,38 +67,78 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
   return r;
 }
 
+// The segments of one warp, in order: segment index sg = first + i * stride
+// walked as (row, segment within the row) without a division per step.
+struct SegWalk {
+  int64_t n;       // row
+  int seg;         // segment within the row
+  int64_t n_step;  // stride / segments per row
+  int s_step;      // stride % segments per row
+  int spr;         // segments per row
+  __device__ SegWalk(int64_t first, int64_t stride, int segs_per_row)
+      : n(first / segs_per_row), seg((int)(first % segs_per_row)),
+        n_step(stride / segs_per_row), s_step((int)(stride % segs_per_row)),
+        spr(segs_per_row) {}
+  __device__ void next() {
+    n += n_step;
+    seg += s_step;
+    if (seg >= spr) {
+      seg -= spr;
+      ++n;
+    }
+  }
+};
+
+// group of column k: a shift when G is a power of two (g_shift >= 0)
+__device__ __forceinline__ uint32_t group_of(uint32_t k, int g_shift, uint32_t G) {
+  return g_shift >= 0 ? (k >> g_shift) : k / G;
+}
+
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
     const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-    uint16_t* __restrict__ W, int64_t N, int64_t K, int64_t G) {
+    uint16_t* __restrict__ W, int64_t N, int K, int G, int g_shift) {
   __shared__ __align__(128) uint16_t s_out[kDqWarps][2][kDqSeg];
   __shared__ float s_lut[kDqWarps][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t segs_per_row = (K + kDqSeg - 1) / kDqSeg;
+  const int segs_per_row = (K + kDqSeg - 1) / kDqSeg;
   const int64_t nseg = N * segs_per_row;
-  const int64_t groups = K / G;
-  int64_t cur_row = -1;
-  int buf = 0;
-  for (int64_t sg = (int64_t)blockIdx.x * kDqWarps + warp; sg < nseg;
-       sg += (int64_t)gridDim.x * kDqWarps) {
-    const int64_t n = sg / segs_per_row;
-    const int64_t col0 = (sg - n * segs_per_row) * kDqSeg;
-    const int cols = (int)min((int64_t)kDqSeg, K - col0);  // a multiple of 32
+  const int groups = K / G;
+  const int64_t first = (int64_t)blockIdx.x * kDqWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * kDqWarps;
+  if (first >= nseg) return;
+  SegWalk wk(first, stride, segs_per_row);
+  // codes and the group's scale and offset of one segment, per lane
+  struct Seg {
     uint32_t w[4];
-    float sv[4], ov[4];
+    float s[4], o[4];
+  };
+  auto load = [&](int64_t n, int col0, Seg& d) {
+    const int cols = min(kDqSeg, K - col0);
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int c = 256 * v + 8 * lane;
-      w[v] = 0u;
-      sv[v] = ov[v] = 0.f;
+      d.w[v] = 0u;
+      d.s[v] = d.o[v] = 0.f;
       if (c < cols) {
-        const int64_t k = col0 + c;
-        w[v] = ldg_nc_u32(packed + (n * K + k) / 2);
-        const int64_t gi = n * groups + k / G;
-        sv[v] = bf16_lo_to_f32(ldg_u16(scale + gi));
-        ov[v] = bf16_lo_to_f32(ldg_u16(offset + gi));
+        const uint32_t k = (uint32_t)(col0 + c);
+        d.w[v] = ldg_nc_u32(packed + (n * K + k) / 2);
+        const int64_t gi = n * groups + group_of(k, g_shift, (uint32_t)G);
+        d.s[v] = bf16_lo_to_f32(ldg_u16(scale + gi));
+        d.o[v] = bf16_lo_to_f32(ldg_u16(offset + gi));
       }
     }
+  };
+  Seg cur, nxt;
+  load(wk.n, wk.seg * kDqSeg, cur);
+  int64_t cur_row = -1;
+  int buf = 0;
+  for (int64_t sg = first; sg < nseg; sg += stride) {
+    const int64_t n = wk.n;
+    const int col0 = wk.seg * kDqSeg;
+    const int cols = min(kDqSeg, K - col0);  // a multiple of 32
+    wk.next();
+    if (sg + stride < nseg) load(wk.n, wk.seg * kDqSeg, nxt);  // the next segment in flight
     if (n != cur_row) {  // this warp moves to a new row: its table as fp32
       __syncwarp();
       if (lane < 16) s_lut[warp][lane] = bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + lane));
@@ -118,9 +158,9 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
           // byte p of the word: codes of columns c + 2p (low nibble), c + 2p + 1
-          const uint32_t byte = (w[v] >> (8 * p)) & 0xffu;
-          const float lo = __fmaf_rn(t[byte & 15u], sv[v], ov[v]);
-          const float hi = __fmaf_rn(t[byte >> 4], sv[v], ov[v]);
+          const uint32_t byte = (cur.w[v] >> (8 * p)) & 0xffu;
+          const float lo = __fmaf_rn(t[byte & 15u], cur.s[v], cur.o[v]);
+          const float hi = __fmaf_rn(t[byte >> 4], cur.s[v], cur.o[v]);
           o[p] = pack_bf16x2_rn(lo, hi);
         }
         *reinterpret_cast<uint4*>(out + c) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -135,10 +175,17 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
     buf ^= 1;
+    cur = nxt;
   }
   // every bulk copy of this warp has finished before the block's shared memory goes
   if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   __syncwarp();
+}
+
+int pow2_shift(int64_t G) {
+  for (int s = 0; s < 31; ++s)
+    if ((int64_t(1) << s) == G) return s;
+  return -1;
 }
 
 int grid_for(int64_t work_items, int threads, const DeviceInfo& dev, int blocks_per_sm) {
@@ -164,8 +211,9 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
   const int64_t segs = N * ((K + kDqSeg - 1) / kDqSeg);
   int per_sm = cached_occupancy(reinterpret_cast<const void*>(dequant_kernel), kDqThreads, 0);
   if (per_sm < 1) per_sm = 1;
+  if (K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   dequant_kernel<<<grid_for(segs * 32, kDqThreads, dev, per_sm), kDqThreads, 0, stream>>>(
-      packed, lut, lut_row_stride, scale, offset, W, N, K, G);
+      packed, lut, lut_row_stride, scale, offset, W, N, (int)K, (int)G, pow2_shift(G));
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 

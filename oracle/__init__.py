@@ -12,6 +12,9 @@ Every function follows "any4: Learned 4-bit Numeric Representation for LLMs"
   dequant            §2.5.2 dequant(w_Q) = alpha*w_Q + beta with w_Q = LUT[code];
                      §2.5.1 group k covers columns k*G .. (k+1)*G-1
   matmul             §4.1 Eq. 8 and §4.2 (y = x W^T, x is M x K, W is N x K)
+  group_sums         per-group activation sums, the factor of the group offset
+                     when Eq. 8 is expanded with the group-affine weights of
+                     §2.5.2 (the pages do not name it; this is that reading)
   bits_per_weight    §2.4.1 storage accounting (4.3125 bits at G=128, K=4096)
   group_scale        §2.5.1 Eq. 1-2 (alpha = (max - min) / 15, beta = min)
   scaled_weights     §2.5.1 Eq. 1 (w_S = (w - beta) / alpha)
@@ -99,6 +102,8 @@ def _bind(lib):
     lib.oracle_dequant_bits.restype = None
     lib.oracle_bits_per_weight_n.argtypes = [i64, i64, ci]
     lib.oracle_bits_per_weight_n.restype = ctypes.c_double
+    lib.oracle_group_sums.argtypes = [u16p, f64p, i64, i64, i64]
+    lib.oracle_group_sums.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -261,6 +266,19 @@ def matmul_rows(x, packed, lut, scale, offset, G: int, rows, per_tensor_lut: boo
                                _ptr(y, ctypes.c_double), _ptr(wrow, ctypes.c_uint16),
                                M, N, K, G)
     return y
+
+
+def group_sums(x: np.ndarray, G: int) -> np.ndarray:
+    """xsum[m][g] = sum of x[m][k] over the G columns of group g, fp64 [M, K/G].
+
+    x is uint16 (bf16 bits) [M, K]; K must be a multiple of G."""
+    x = _c(x, np.uint16)
+    if x.ndim != 2 or G < 1 or x.shape[1] % G:
+        raise ValueError("x must be [M, K] with K a multiple of G")
+    M, K = x.shape
+    out = np.empty((M, K // G), dtype=np.float64)
+    _load().oracle_group_sums(_ptr(x, ctypes.c_uint16), _ptr(out, ctypes.c_double), M, K, G)
+    return out
 
 
 def any4_matmul(x, packed, lut, scale, offset, G: int, per_tensor_lut: bool = False):

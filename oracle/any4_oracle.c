@@ -461,3 +461,21 @@ void oracle_dequant_bits(const uint8_t* packed, const uint16_t* lut, int64_t lut
 double oracle_bits_per_weight_n(int64_t K, int64_t G, int bits) {
   return (double)bits + 32.0 / (double)G + (16.0 * (double)(1 << bits)) / (double)K;
 }
+
+/* Per-group sums of the activations: xsum[m][g] = sum over the columns k of
+ * group g (k = g*G .. g*G+G-1, §2.5.1) of x[m][k], in fp64, k ascending.
+ * This is the factor that multiplies the group offset beta when Eq. 8's
+ * product is taken with the group-affine weights alpha*LUT[c] + beta
+ * (§4.1 Eq. 8, §2.5.2):  sum_k x*(alpha*LUT + beta)
+ *   = alpha * sum_k x*LUT + beta * xsum.
+ * x: [M][K] bf16, xsum: [M][K/G] fp64. */
+void oracle_group_sums(const uint16_t* x, double* xsum, int64_t M, int64_t K, int64_t G) {
+  const int64_t groups = K / G;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t g = 0; g < groups; ++g) {
+      double acc = 0.0;
+      for (int64_t k = g * G; k < (g + 1) * G; ++k) acc += (double)oracle_bf16_to_f32(x[m * K + k]);
+      xsum[m * groups + g] = acc;
+    }
+  }
+}

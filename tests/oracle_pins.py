@@ -416,6 +416,62 @@ def pin_matmul_rows_equals_full():
     assert np.array_equal(part, full[:, rows])
 
 
+def pin_group_sums_brute_force_exact():
+    """Tiny shapes: every group sum against the exact rational sum of the
+    group's bf16 values (Fractions).  Exponents span [-20, 12): 32 binades
+    plus 8 significand bits plus 7 bits of carries for 128 terms fit in the
+    53 bits of fp64, so its sum is exact and the values must be identical
+    (an fp32 accumulator, 24 bits, is not)."""
+    rng = np.random.default_rng(17)
+    for (M, K, G) in [(1, 64, 32), (3, 256, 64), (2, 384, 128)]:
+        x = random_bf16(rng, (M, K), lo_exp=-20, hi_exp=12)
+        xs = oracle.group_sums(x, G)
+        xv = torch_bf16_to_f64(x)
+        assert xs.shape == (M, K // G)
+        for m in range(M):
+            for g in range(K // G):
+                exact = sum((Fraction(float(v)) for v in xv[m, g * G:(g + 1) * G]), Fraction(0))
+                assert Fraction(float(xs[m, g])) == exact, (M, K, G, m, g)
+
+
+def pin_group_sums_constant_and_one_hot():
+    """Constant rows sum to G * c; a single nonzero column lands in its own
+    group k // G and nowhere else (a shifted group boundary fails this)."""
+    M, K, G = 2, 512, 128
+    c = torch_bf16_bits(np.array([0.75], np.float32))[0]
+    xs = oracle.group_sums(np.full((M, K), c, dtype=np.uint16), G)
+    assert (xs == G * 0.75).all()
+    one = torch_bf16_bits(np.array([1.0], np.float32))[0]
+    for k in (0, 1, 127, 128, 129, 383, 384, 511):
+        x = np.zeros((M, K), dtype=np.uint16)
+        x[1, k] = one
+        xs = oracle.group_sums(x, G)
+        want = np.zeros((M, K // G))
+        want[1, k // G] = 1.0
+        assert np.array_equal(xs, want), k
+
+
+def pin_group_sums_expand_eq8_with_group_affine_weights():
+    """The reason the sums exist: with unrounded group-affine weights
+    W = LUT[c] * alpha + beta, x W^T equals
+    sum_g alpha_g * (sum_{k in g} x * LUT[c]) + beta_g * xsum_g (exact algebra;
+    both sides in fp64 with numpy, equal to within rounding)."""
+    rng = np.random.default_rng(18)
+    M, N, K, G = 3, 10, 256, 64
+    idx, lut, scale, offset, x = _small_problem(rng, M, N, K, G)
+    xv = torch_bf16_to_f64(x)
+    T = torch_bf16_to_f64(lut)
+    a = np.repeat(torch_bf16_to_f64(scale), G, axis=1)
+    b = np.repeat(torch_bf16_to_f64(offset), G, axis=1)
+    Wq = np.take_along_axis(T, idx.astype(np.int64), axis=1)        # LUT[n][c]
+    direct = xv @ (Wq * a + b).T
+    xs = oracle.group_sums(x, G)                                     # [M, K/G]
+    lut_part = np.einsum("mgk,ngk->mng", xv.reshape(M, K // G, G), Wq.reshape(N, K // G, G))
+    expanded = (np.einsum("mng,ng->mn", lut_part, torch_bf16_to_f64(scale))
+                + xs @ torch_bf16_to_f64(offset).T)
+    assert np.allclose(expanded, direct, rtol=1e-12, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # learning the table: §2.5.1 Eq. 1-2 scaling, §4.1 E-step (Eq. 18) and M-step
 # (Eq. 23), Appendix A.1 Alg. 1 (k-means per row, sample weight alpha * E|x|)

@@ -80,7 +80,7 @@ def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, sc
     (dict(M=17, path=1), any4.ANY4_ERR_UNSUPPORTED),
     (dict(path=7), any4.ANY4_ERR_UNSUPPORTED),
     (dict(flags=16), any4.ANY4_ERR_UNSUPPORTED),
-    (dict(flags=8), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(flags=32), any4.ANY4_ERR_UNSUPPORTED),
     (dict(ws=FAKE + 8, ws_bytes=1 << 20), any4.ANY4_ERR_ALIGN),
 ])
 def test_matmul_rejects_bad_arguments(kw, expect):
@@ -182,7 +182,7 @@ def test_workspace_sizes_by_path():
         assert any4.any4_matmul_workspace_size(M, N, K, G) == \
             ((sms * M * 64 * 4 + sms * 8 + 255) // 256) * 256
     assert any4.any4_matmul_workspace_size(1, N, K, 256) == 0       # G outside {32, 64, 128}
-    assert any4.any4_matmul_workspace_size(1, N, 1024 + 64, 64) == 0  # K/G not a multiple of 8
+    assert any4.any4_matmul_workspace_size(1, N, 1024 + 64, 64) == 0  # K not a multiple of 128
     for M in (3, 8, 16):
         assert any4.any4_matmul_workspace_size(M, N, K, G) == 0
     one = any4.any4_matmul_workspace_size(17, N, K, G)

@@ -11,8 +11,8 @@ correct fp32 sums of the bf16 weights pass with orders of magnitude to spare.
 The same calls' bf16 outputs report the literal statistic
 max |y - y_ref| / rms(y_ref[m, :]) per configuration in the test log.
 
-Routes: the pair-table decode kernel (M <= 2 with its workspace), the
-weight-streaming shuffle kernel (M = 1 without), the generic decode kernel
+Routes: the pair-table decode kernel (M = 2 with its workspace, M = 1 on
+request), the weight-streaming shuffle kernel (M = 1), the generic decode kernel
 (a group size the streaming kernels do not take), the skinny kernel
 (3 <= M <= 16), and the tensor-core prefill in one pass (below M = 1024, or
 with a one-pass workspace) and in two passes (M >= 1024).
@@ -40,12 +40,12 @@ def _check_fp32(y32: np.ndarray, y_ref: np.ndarray, what: str) -> float:
     return worst
 
 
-def _call(d, shape, workspace=None, path="auto"):
+def _call(d, shape, workspace=None, path="auto", pair_table=False):
     """bf16 and fp32 outputs of one call route."""
     outs = {}
     for fp32 in (False, True):
         y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path=path,
-                             workspace=workspace, fp32_out=fp32)
+                             workspace=workspace, fp32_out=fp32, pair_table=pair_table)
         torch.cuda.synchronize()
         outs[fp32] = y.cpu().numpy() if fp32 else host_bits(y)
     return outs[False], outs[True]
@@ -74,9 +74,9 @@ def test_fp32_m1_decode_kernels(shape):
     p = workloads.make(shape)
     d = DeviceProblem(p, check_pack=False)
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
-    y16, y32 = _call(d, shape)                       # pair-table kernel
+    y16, y32 = _call(d, shape, pair_table=True)      # pair-table kernel
     _report(shape.name, "pair table", y16, y32, y_ref)
-    y16, y32 = _call(d, shape, workspace=_empty())   # weight-streaming shuffle kernel
+    y16, y32 = _call(d, shape)                       # weight-streaming shuffle kernel
     _report(shape.name, "shuffle stream", y16, y32, y_ref)
 
 

@@ -23,16 +23,24 @@ DECODE_SHAPES = (workloads.TINY + workloads.LLAMA3_8B_DECODE
 
 
 NO_WORKSPACE = "no_workspace"
+PAIR = "pair_table"
+
+
+def _ws_args(workspace):
+    """workspace None: the binding allocates what the path asks for (M = 2
+    then runs the pair-table kernel, M = 1 the weight-streaming kernel);
+    NO_WORKSPACE: none is passed, so M = 2 runs the skinny kernel; PAIR: the
+    workspace plus ANY4_FLAG_PAIR_TABLE, the pair-table kernel at M = 1 too."""
+    if workspace == NO_WORKSPACE:
+        return dict(workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))
+    if workspace == PAIR:
+        return dict(workspace=None, pair_table=True)
+    return dict(workspace=workspace)
 
 
 def _run(d, shape, path="auto", workspace=None):
-    """workspace None: the binding allocates what the path asks for (the
-    pair-table kernel at M <= 2); NO_WORKSPACE: none is passed, so M <= 2
-    runs the decode kernels that need none."""
-    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE \
-        else workspace
     y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, path=path,
-                         workspace=ws)
+                         **_ws_args(workspace))
     torch.cuda.synchronize()
     return host_bits(y)
 
@@ -47,10 +55,11 @@ def test_decode_full_shapes(shape):
     st = assert_matmul_close(y, y_ref, shape.name)
     print(shape.name, st)
     if shape.M <= 2:
-        # the same shape on the kernels that need no workspace
-        y = _run(d, shape, workspace=NO_WORKSPACE)
-        st = assert_matmul_close(y, y_ref, shape.name + " without workspace")
-        print(shape.name, "without workspace", st)
+        # the same shape on the other kernel that takes it
+        other = PAIR if shape.M == 1 else NO_WORKSPACE
+        y = _run(d, shape, workspace=other)
+        st = assert_matmul_close(y, y_ref, f"{shape.name} {other}")
+        print(shape.name, other, st)
 
 
 @pytest.mark.parametrize("M", list(range(1, 17)))
@@ -61,7 +70,7 @@ def test_decode_every_m_ragged(M):
     p = workloads.make(shape)
     d = DeviceProblem(p)
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
-    for ws in (None, NO_WORKSPACE):
+    for ws in (None, NO_WORKSPACE, PAIR):
         y = _run(d, shape, path="decode", workspace=ws)
         assert_matmul_close(y, y_ref, f"{shape.name} {ws}")
 
@@ -80,23 +89,21 @@ def test_decode_edge_shapes(K, N, G):
         assert_matmul_close(y, y_ref, shape.name)
 
 
-@pytest.mark.parametrize("workspace", [None, NO_WORKSPACE])
+@pytest.mark.parametrize("workspace", [PAIR, None])
 def test_decode_one_hot_is_exact(workspace):
     """x = e_k returns column k of the dequantised weight, bit for bit: the
     fused group-affine form reduces to fmaf(LUT, scale, offset) rounded once.
-    Both M = 1 kernels (pair table with its workspace, weight streaming
-    without)."""
+    Both M = 1 kernels (pair table on request, weight streaming by default)."""
     shape = workloads.Shape("onehot", 1, 4096, 2000, 128, 9401, 9901)
     p = workloads.make(shape)
     d = DeviceProblem(p)
     W_ref = oracle.dequant(d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     one = torch_bf16_bits(np.array([1.0], np.float32))[0]
-    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE else None
     for k in (0, 1, 31, 32, 127, 128, 1023, 1024, 2047, 4095):
         x = np.zeros((1, shape.K), np.uint16)
         x[0, k] = one
         y = any4.any4_matmul(dev_bf16(x), d.packed, d.lut, d.scale, d.offset, shape.G,
-                             workspace=ws)
+                             **_ws_args(workspace))
         torch.cuda.synchronize()
         got = bits_to_f64(host_bits(y))[0]
         assert np.array_equal(got, bits_to_f64(W_ref[:, k])), k
@@ -143,25 +150,26 @@ def test_decode_writes_only_its_output(M):
     assert_matmul_close(host_bits(y), y_ref, "guard")
 
 
-@pytest.mark.parametrize("M,workspace", [(1, None), (2, None), (1, NO_WORKSPACE), (4, None),
-                                         (12, None)])
+@pytest.mark.parametrize("M,workspace", [(1, PAIR), (2, None), (1, None), (2, NO_WORKSPACE),
+                                         (4, None), (12, None)])
 def test_decode_overlap_prior_chain(M, workspace):
     """ANY4_FLAG_OVERLAP_PRIOR: x is produced by the kernel just before each
     call and y is consumed by the kernel just after; a chain of overlapped
     calls must match the same chain run without overlap, bit for bit, and the
-    oracle within tolerance (M <= 2: pair-table kernel, or weight streaming
-    without a workspace; M > 2: skinny)."""
+    oracle within tolerance (M = 1: weight streaming, or the pair-table
+    kernel on request; M = 2: pair table, or skinny without a workspace;
+    M > 2: skinny)."""
     shape = workloads.Shape(f"overlap_m{M}", M, 4096, 4096, 128, 9701, 9702 + M)
     p = workloads.make(shape)
     d = DeviceProblem(p)
-    ws = torch.empty(0, dtype=torch.uint8, device="cuda") if workspace == NO_WORKSPACE else None
+    wa = _ws_args(workspace)
     def chain(overlap):
         x = d.x.clone()
         outs = []
         for i in range(6):
             x = (x.float() * 0.5 + 0.25).to(torch.bfloat16)      # written by the preceding kernel
             y = any4.any4_matmul(x, d.packed, d.lut, d.scale, d.offset, shape.G,
-                                 overlap_prior=overlap, workspace=ws)
+                                 overlap_prior=overlap, **wa)
             outs.append(y.clone())                              # read by the following kernel
             x = torch.cat([y[:, :shape.K]], dim=1) if shape.N >= shape.K else x
             x = (x.float() / (x.float().abs().max() + 1)).to(torch.bfloat16)
@@ -173,7 +181,7 @@ def test_decode_overlap_prior_chain(M, workspace):
         assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, shape.G)
     y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, overlap_prior=True,
-                          workspace=ws)
+                          **wa)
     torch.cuda.synchronize()
     assert_matmul_close(host_bits(y1), y_ref, "overlap")
 
@@ -183,7 +191,7 @@ def test_decode_overlap_prior_chain(M, workspace):
                                           (4096, 1500, 128, True), (2048, 9, 64, True)])
 def test_decode_m1_streamed_variants(K, N, G, shared):
     """M = 1 shapes of both tensor-memory-streamed decode kernels (the
-    pair-table kernel with its workspace, the shuffle kernel without): every
+    pair-table kernel on request, the shuffle kernel by default): every
     group size they take, ragged rows, a last slice cut short, the one table
     mode; dev_status must stay clear."""
     shape = workloads.Shape(f"m1_{K}_{N}_{G}", 1, K, N, G, 9901 + K + N, 9951 + G)
@@ -192,10 +200,10 @@ def test_decode_m1_streamed_variants(K, N, G, shared):
     lut = p.lut[11 % N].copy() if shared else p.lut
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, lut, p.scale, p.offset, shape.G,
                                per_tensor_lut=shared)
-    for ws in (None, torch.empty(0, dtype=torch.uint8, device="cuda")):
+    for ws in (PAIR, None):
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         y = any4.any4_matmul(d.x, d.packed, dev_bf16(lut), d.scale, d.offset, shape.G,
-                             dev_status=status, workspace=ws)
+                             dev_status=status, **_ws_args(ws))
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        assert_matmul_close(host_bits(y), y_ref, f"{shape.name} {ws is None}")
+        assert_matmul_close(host_bits(y), y_ref, f"{shape.name} {ws}")

@@ -1,5 +1,5 @@
-"""The pair-table decode kernel (M <= 2, given its workspace) against the fp64
-oracle: the stream-K split of 64-row sets over the blocks, its cross-block
+"""The pair-table decode kernel (M = 2 given its workspace, M = 1 on request)
+against the fp64 oracle: the stream-K split of 64-row sets over the blocks, its cross-block
 exchange (partial sums published with a per-launch flag), repeated calls and
 CUDA-graph replays that reuse one workspace, and the shape edges of the
 kernel (ragged rows and chunks, every group size, one table for the matrix).
@@ -7,6 +7,8 @@ kernel (ragged rows and chunks, every group size, one table for the matrix).
 Tolerance as in the other matmul tests: |y - y_ref| <= 1e-2 * rms(y_ref[m, :])
 + ulp_bf16(y_ref) per element.
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -17,6 +19,9 @@ import learned_bit_lut_any4_b200 as any4
 from tests.gpu_helpers import DeviceProblem, assert_matmul_close, dev_bf16, host_bits
 
 pytestmark = pytest.mark.gpu
+
+# M = 1 runs the weight-streaming kernel unless the pair-table kernel is asked for
+_mm = functools.partial(any4.any4_matmul, pair_table=True)
 
 
 def _sms():
@@ -42,6 +47,9 @@ def _ws(M, N, K, G):
     (2, 768, 65, 32),        # six chunks, 65 rows
     (1, 256, 5, 32),         # two chunks, five rows (K/G = 8 makes K a multiple of 256)
     (2, 8192, 28672 // 8, 128),
+    (1, 1152, 300, 128),     # K / G = 9 groups per row (odd)
+    (2, 640, 77, 64),        # K / G = 10
+    (1, 384, 1000, 32),      # three chunks, twelve groups per row
 ])
 def test_pair_stream_k_shapes(M, K, N, G):
     shape = workloads.Shape(f"pair_{M}_{K}_{N}_{G}", M, K, N, G, 8801 + N, 8802 + K // 32)
@@ -49,7 +57,7 @@ def test_pair_stream_k_shapes(M, K, N, G):
     d = DeviceProblem(p)
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, G)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    y = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, G, workspace=_ws(M, N, K, G),
+    y = _mm(d.x, d.packed, d.lut, d.scale, d.offset, G, workspace=_ws(M, N, K, G),
                          dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -62,7 +70,7 @@ def test_pair_shared_table(M):
     p = workloads.make(shape)
     d = DeviceProblem(p)
     table = p.lut[7].copy()
-    y = any4.any4_matmul(d.x, d.packed, dev_bf16(table), d.scale, d.offset, shape.G,
+    y = _mm(d.x, d.packed, dev_bf16(table), d.scale, d.offset, shape.G,
                          workspace=_ws(M, shape.N, shape.K, shape.G))
     torch.cuda.synchronize()
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, table, p.scale, p.offset, shape.G,
@@ -84,9 +92,9 @@ def test_pair_repeated_calls_share_one_workspace():
     rng = np.random.default_rng(8915)
     for i in range(4):
         xa = workloads._to_bf16_bits(rng.normal(0, 1, (1, a.K)).astype(np.float32))
-        ya = any4.any4_matmul(dev_bf16(xa), da.packed, da.lut, da.scale, da.offset, a.G,
+        ya = _mm(dev_bf16(xa), da.packed, da.lut, da.scale, da.offset, a.G,
                               workspace=ws)
-        yb = any4.any4_matmul(db.x, db.packed, db.lut, db.scale, db.offset, b.G, workspace=ws)
+        yb = _mm(db.x, db.packed, db.lut, db.scale, db.offset, b.G, workspace=ws)
         torch.cuda.synchronize()
         assert_matmul_close(host_bits(ya), oracle.any4_matmul(xa, da.packed_ref, pa.lut,
                                                               pa.scale, pa.offset, a.G), f"a{i}")
@@ -106,11 +114,11 @@ def test_pair_graph_replays():
     y = torch.empty((1, shape.N), dtype=torch.bfloat16, device="cuda")
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
-        any4.any4_matmul(x, d.packed, d.lut, d.scale, d.offset, shape.G, y=y, workspace=ws)
+        _mm(x, d.packed, d.lut, d.scale, d.offset, shape.G, y=y, workspace=ws)
     s.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        any4.any4_matmul(x, d.packed, d.lut, d.scale, d.offset, shape.G, y=y, workspace=ws)
+        _mm(x, d.packed, d.lut, d.scale, d.offset, shape.G, y=y, workspace=ws)
     rng = np.random.default_rng(8923)
     for i in range(3):
         xb = workloads._to_bf16_bits(rng.normal(0, 1, (1, shape.K)).astype(np.float32))
@@ -127,7 +135,7 @@ def test_pair_is_deterministic():
     p = workloads.make(shape)
     d = DeviceProblem(p, check_pack=False)
     ws = _ws(2, shape.N, shape.K, shape.G)
-    y1 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, workspace=ws)
-    y2 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, workspace=ws)
+    y1 = _mm(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, workspace=ws)
+    y2 = _mm(d.x, d.packed, d.lut, d.scale, d.offset, shape.G, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))

@@ -41,7 +41,7 @@ def test_stalled_stream_times_out_cleanly(name, M, K, N, G, ws):
     y = buf[pad:pad + M * N].view(M, N).view(torch.bfloat16)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, G, y=y, workspace=workspace,
-                     dev_status=status, test_stall=True)
+                     dev_status=status, test_stall=True, pair_table=name == "pair_table")
     torch.cuda.synchronize()
     assert int(status.item()) == any4.ANY4_ERR_TIMEOUT
     assert (buf[:pad] == -3).all() and (buf[pad + M * N:] == -3).all()
@@ -51,7 +51,7 @@ def test_stalled_stream_times_out_cleanly(name, M, K, N, G, ws):
         workspace.zero_()
     status.zero_()
     y2 = any4.any4_matmul(d.x, d.packed, d.lut, d.scale, d.offset, G, workspace=workspace,
-                          dev_status=status)
+                          dev_status=status, pair_table=name == "pair_table")
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     y_ref = oracle.any4_matmul(p.x, d.packed_ref, p.lut, p.scale, p.offset, G)

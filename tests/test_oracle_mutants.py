@@ -77,6 +77,12 @@ MUTANTS = [
     ("bits_per_weight_n_sixteen_entries",
      "return (double)bits + 32.0 / (double)G + (16.0 * (double)(1 << bits)) / (double)K;",
      "return (double)bits + 32.0 / (double)G + (16.0 * 16.0) / (double)K;"),
+    ("group_sums_boundary_shifted", "for (int64_t k = g * G; k < (g + 1) * G; ++k) acc +=",
+     "for (int64_t k = g * G + (g > 0); k < (g + 1) * G + (g + 1 < groups); ++k) acc +="),
+    ("group_sums_row_zero", "acc += (double)oracle_bf16_to_f32(x[m * K + k]);\n      xsum",
+     "acc += (double)oracle_bf16_to_f32(x[k]);\n      xsum"),
+    ("group_sums_fp32_accumulate", "      double acc = 0.0;\n      for (int64_t k = g * G;",
+     "      float acc = 0.0f;\n      for (int64_t k = g * G;"),
     ("storage_bits_one_param", "4.0 + (2.0 * (double)group_param_bits) / (double)G",
      "4.0 + (1.0 * (double)group_param_bits) / (double)G"),
 ]
