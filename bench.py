@@ -335,6 +335,35 @@ def time_weight_set(shapes, stream, overlap, peaks):
     return out
 
 
+# The layer's seven matmuls as the four calls a decoder makes: the projections
+# that read the same activations run as one grouped call (q/k/v; gate/up).
+LAYER_CALLS = (("8b_q", "8b_k", "8b_v"), ("8b_o",), ("8b_gate", "8b_up"), ("8b_down",))
+
+
+def layer_plan(sets, grouped):
+    """Index lists into `sets`: one list per call of a layer step."""
+    names = [s.name for (s, *_r) in sets]
+    if not grouped:
+        return [[i] for i in range(len(sets))]
+    return [[names.index(n) for n in call] for call in LAYER_CALLS]
+
+
+def run_call(sets, idxs, c, copies, overlap, x=None, ys=None):
+    """One call of a layer step on weight copy c: any4_matmul for one matrix,
+    any4_matmul_grouped for matrices sharing x (the first matrix's x)."""
+    import learned_bit_lut_any4_b200 as any4
+    s0, reps0, x0, y0, _ = sets[idxs[0]]
+    x = x0 if x is None else x
+    if len(idxs) == 1:
+        w = reps0[c % copies]
+        any4.any4_matmul(x, w[0], w[1], w[2], w[3], s0.G, y=y0 if ys is None else ys[0],
+                         overlap_prior=overlap, workspace=ws_for(s0))
+    else:
+        any4.any4_matmul_grouped(x, [sets[i][1][c % copies] for i in idxs], s0.G,
+                                 ys=[sets[i][3] for i in idxs] if ys is None else ys,
+                                 overlap_prior=overlap, workspace=ws_for(s0))
+
+
 def gpu_arm(args, rank, world):
     import torch
     import learned_bit_lut_any4_b200 as any4
@@ -348,11 +377,11 @@ def gpu_arm(args, rank, world):
     overlap = not args.no_overlap
     stream = torch.cuda.Stream()
 
-    def step(c):
-        for (s, reps, x, y, _) in sets:
-            w = reps[c % copies]
-            any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y, overlap_prior=overlap,
-                             workspace=ws_for(s))
+    plan = layer_plan(sets, grouped=not args.ungrouped)
+
+    def step(c, plan=plan):
+        for idxs in plan:
+            run_call(sets, idxs, c, copies, overlap)
 
     # one graph = `copies` steps (each step on the next weight copy)
     with torch.cuda.stream(stream):
@@ -417,6 +446,18 @@ def gpu_arm(args, rank, world):
         detail[s.name] = {"us": round(us, 3), "GB/s": round(gbs, 1),
                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
         del g
+
+    # the layer both ways: the four calls of the step (q/k/v and gate/up
+    # grouped) and seven separate calls, same rotation, one graph each
+    layer_calls = {}
+    for key, grouped in (("grouped_4_calls", True), ("separate_7_calls", False)):
+        pl = layer_plan(sets, grouped)
+        us = _time_graph(stream, [(lambda c=c, pl=pl: step(c, pl)) for c in range(copies)],
+                         max(1, 200 // copies))
+        gbs = step_bytes / (us * 1e-6) / 1e9
+        layer_calls[key] = {"us_per_layer": round(us, 3), "GB/s": round(gbs, 1),
+                            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                            "launches_per_layer": len(pl)}
 
     # single-call latency of each M = 1 shape: one launch between an event
     # pair, after a write of twice the L2 size (cold caches); 3 discarded, 20 kept
@@ -492,7 +533,8 @@ def gpu_arm(args, rank, world):
     # end to end through the public API with host buffers: every step copies
     # the step's inputs (every call's x) from pinned host memory in one
     # transfer and reads the step's results (every call's y) back in one
-    xs = [np.ascontiguousarray(hx).view(np.int16).reshape(-1) for (_, _, _, _, hx) in sets]
+    lead = [idxs[0] for idxs in plan]  # the matrices whose x a call reads
+    xs = [np.ascontiguousarray(sets[i][4]).view(np.int16).reshape(-1) for i in lead]
     x_off = np.cumsum([0] + [a.size for a in xs])
     host_x = torch.from_numpy(np.concatenate(xs)).pin_memory()
     dev_x = torch.empty(host_x.numel(), dtype=torch.int16, device="cuda")
@@ -500,8 +542,8 @@ def gpu_arm(args, rank, world):
     y_off = np.cumsum([0] + y_sizes)
     host_y = torch.empty(int(y_off[-1]), dtype=torch.int16).pin_memory()
     dev_y = torch.empty(int(y_off[-1]), dtype=torch.int16, device="cuda")
-    x_views = [dev_x[x_off[i]:x_off[i + 1]].view(torch.bfloat16).view(s.M, s.K)
-               for i, (s, *_r) in enumerate(sets)]
+    x_views = [dev_x[x_off[j]:x_off[j + 1]].view(torch.bfloat16).view(sets[i][0].M, sets[i][0].K)
+               for j, i in enumerate(lead)]
     y_views = [dev_y[y_off[i]:y_off[i + 1]].view(torch.bfloat16).view(s.M, s.N)
                for i, (s, *_r) in enumerate(sets)]
     h2d = host_x.numel() * 2
@@ -510,10 +552,8 @@ def gpu_arm(args, rank, world):
 
     def e2e_step(c):
         dev_x.copy_(host_x, non_blocking=True)
-        for i, (s, reps, _x, _y, _) in enumerate(sets):
-            w = reps[c % copies]
-            any4.any4_matmul(x_views[i], w[0], w[1], w[2], w[3], s.G, y=y_views[i],
-                             workspace=ws_for(s))
+        for j, idxs in enumerate(plan):
+            run_call(sets, idxs, c, copies, False, x=x_views[j], ys=[y_views[i] for i in idxs])
         host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -535,13 +575,14 @@ def gpu_arm(args, rank, world):
 
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
-        "clocks": clocks, "detail": detail, "single": single, "prefill": prefill,
+        "clocks": clocks, "detail": detail, "layer_calls": layer_calls, "single": single,
+        "prefill": prefill,
         "batch": batch, "more_m1": more_m1, "fig3": fig3,
         "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "launches": len(sets) * steps_timed,
+        "launches": len(plan) * steps_timed,
     }
 
 
@@ -683,6 +724,51 @@ def nbit_dequant_detail(reps: int = 10):
     return out
 
 
+def nbit_matmul_detail():
+    """any4_matmul_bits at M = 1 (n = 2, 3, 4: the codes read directly by the
+    weight-streaming kernel) on the Llama3-8B gate and Llama3-70B gate
+    matrices, G = 128, on rotating weight copies larger than L2 replayed in a
+    CUDA graph: us per call, GB/s of the algorithmic bytes (codes, scales,
+    offsets, tables, x, y) and the fraction of the HBM peak."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    peaks = load_peaks()
+    G = 128
+    rng = np.random.default_rng(4700)
+    stream = torch.cuda.Stream()
+    out = {}
+    for name, K, N in (("8b_gate", 4096, 14336), ("70b_gate", 8192, 28672)):
+        res = {"K": K, "N": N, "G": G}
+        for bits in (2, 3, 4):
+            nq = 1 << bits
+            wbytes = N * K * bits // 8 + 4 * N * (K // G) + 2 * nq * N
+            copies = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
+            packed = torch.from_numpy(rng.integers(0, 256, size=(N, bits * K // 8),
+                                                   dtype=np.uint8)).cuda()
+            lut = _dev_bf16(workloads._to_bf16_bits(
+                np.sort(rng.normal(0, 0.5, (N, nq)), axis=1).astype(np.float32)))
+            scale = _dev_bf16(workloads._to_bf16_bits(
+                (np.abs(rng.normal(0, 0.01, (N, K // G))) + 1e-3).astype(np.float32)))
+            offset = _dev_bf16(workloads._to_bf16_bits(
+                rng.normal(0, 0.002, (N, K // G)).astype(np.float32)))
+            reps = [(packed, lut, scale, offset)] + [
+                (packed.clone(), lut.clone(), scale.clone(), offset.clone())
+                for _ in range(copies - 1)]
+            x = _dev_bf16(workloads._to_bf16_bits(rng.normal(0, 1, (1, K)).astype(np.float32)))
+            y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+            calls = [(lambda w=w: any4.any4_matmul_bits(x, w[0], w[1], w[2], w[3], G, bits, y=y,
+                                                        overlap_prior=True))
+                     for w in reps]
+            us = _time_graph(stream, calls, max(2, 200 // copies))
+            alg = wbytes + 2 * K + 2 * N
+            res[f"any{bits}"] = {"us": round(us, 3), "GB/s": round(alg / us / 1e3, 1),
+                                 "frac_hbm": round(alg / us / 1e3 / peaks["hbm_gbs"], 4)}
+            del reps, packed, lut, scale, offset, x, y
+            torch.cuda.synchronize()
+        out[name] = res
+    return out
+
+
 def profile_shape(name: str, calls: int, op: str = "matmul"):
     """Run a few calls of one operation (any4_matmul on the auto path, or
     any4_dequant) on one workload shape: a small, fixed case for ncu."""
@@ -712,6 +798,9 @@ def main():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=40)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ungrouped", action="store_true",
+                    help="run the layer step as seven separate any4_matmul calls instead of "
+                         "four (q/k/v and gate/up as grouped calls)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the decode kernels without programmatic dependent launch")
     ap.add_argument("--skip-prefill", action="store_true")
@@ -764,12 +853,16 @@ def main():
                          "matrices": table_learning_detail(args.quantize_iters, 4.0, reps=2)}
             except Exception as e:  # pragma: no cover - only on a GPU machine
                 table = {"error": f"{type(e).__name__}: {e}"}
-        nbit = None
+        nbit = nbit_mm = None
         if world == 1:
             try:  # a detail beside the step: its failure is reported, not fatal
                 nbit = nbit_dequant_detail()
             except Exception as e:  # pragma: no cover - only on a GPU machine
                 nbit = {"error": f"{type(e).__name__}: {e}"}
+            try:
+                nbit_mm = nbit_matmul_detail()
+            except Exception as e:  # pragma: no cover - only on a GPU machine
+                nbit_mm = {"error": f"{type(e).__name__}: {e}"}
         achieved = r["value"] / world  # per-GPU decode throughput over the whole step
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -786,7 +879,9 @@ def main():
                        "shapes": [[s.name, s.K, s.N] for s in workloads.LLAMA3_8B_DECODE],
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs larger than L2: {r['copies']} rotating weight copies",
-                       "overlap_prior": not args.no_overlap},
+                       "overlap_prior": not args.no_overlap,
+                       "calls": ("q/k/v grouped, o, gate/up grouped, down (4 launches)"
+                                 if not args.ungrouped else "7 separate calls")},
             "us_per_layer": round(r["ms_per_step"] * 1e3, 2),
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -798,8 +893,10 @@ def main():
             "fig3_square_m1": r["fig3"],
             "table_learning": table,
             "nbit_dequant": nbit,
+            "nbit_matmul_m1": nbit_mm,
             "single_call_m1": r["single"],
             "detail_batch": r["batch"],
+            "layer_m1_calls": r["layer_calls"],
             "detail_m1": r["detail"],
             "detail_m1_more": r["more_m1"],
             "prefill_m2048": r["prefill"],

@@ -157,6 +157,30 @@ ANY4_API any4_status any4_quantize_bits(const uint16_t* w, const float* ex_abs, 
                                         uint16_t* offset, int32_t* iters, any4_stream_t stream);
 
 /*
+ * any4_matmul_bits -- y = x * dequant(W)^T for n-bit codes (n = 2, 3 or 4;
+ * the any3 / any2 formats of paper §5, a table of 2^n values per row, §4.1
+ * Eq. 9), codes in the layout of any4_pack_bits, lut_row_stride 2^n or 0.
+ * n = 4 runs any4_matmul_ex (auto path).  For n = 2, 3:
+ *   M = 1, G of 32, 64 or 128, K/G a multiple of 8 and n K a multiple of 128:
+ *     the weight-streaming decode kernel reads the n-bit codes directly
+ *     (fused lookup, scale and offset; no workspace);
+ *   otherwise two passes as any4_matmul's large-M path: the n-bit dequant
+ *     into the workspace (bf16 W, bit-exact with any4_dequant_bits), then the
+ *     tensor-core GEMM.
+ * workspace: at least any4_matmul_bits_workspace_size bytes (0: none).
+ * flags: ANY4_FLAG_OVERLAP_PRIOR, _FP32_OUT, _TEST_STALL as for any4_matmul_ex.
+ * Tolerance and determinism as any4_matmul.
+ */
+ANY4_API any4_status any4_matmul_bits(const uint16_t* x, const uint8_t* packed,
+                                      const uint16_t* lut, int64_t lut_row_stride,
+                                      const uint16_t* scale, const uint16_t* offset, uint16_t* y,
+                                      int64_t M, int64_t N, int64_t K, int64_t G, int32_t bits,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, uint32_t flags, any4_stream_t stream);
+ANY4_API size_t any4_matmul_bits_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G,
+                                                int32_t bits);
+
+/*
  * any4_dequant -- materialise the bf16 weight (paper §2.5.2 dequant with the
  * per-row table of §2.4.1):
  *   W[n][k] = bf16_rne( fmaf( LUT[n][c], scale[n][k/G], offset[n][k/G] ) )
@@ -327,6 +351,49 @@ ANY4_API any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t
  * size this function returns for M < 1024), runs the one-pass kernel, which
  * dequantises the weights tile by tile. */
 ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+
+/*
+ * any4_matmul_grouped -- several weight matrices applied to the same x:
+ *   y_i = x * dequant(W_i)^T   for i = 0 .. count-1
+ * (the q, k and v projections of a transformer layer, or gate and up: the
+ * matmuls of paper §4.1 Eq. 8 that share their input).  Each result is
+ * exactly what any4_matmul_ex gives for that matrix alone (same bits).
+ * At M = 1, on the shapes the weight-streaming decode kernel takes (G of 32,
+ * 64 or 128 with K/G a multiple of 8), all matrices run in ONE launch whose
+ * blocks stream the matrices' rows one after the other, so small matrices no
+ * longer pay a launch and a pipeline ramp each; otherwise the matrices run
+ * as count calls of any4_matmul_ex, one after the other on `stream`, sharing
+ * the workspace.
+ *   x          [M][K] bf16
+ *   w          count descriptors (host memory, read during the call only):
+ *              packed [N_i][K/2], lut (lut_row_stride 16: [N_i][16]; 0: one
+ *              [16] table), scale and offset [N_i][K/G], y [M][N_i] bf16 (or
+ *              fp32 with ANY4_FLAG_FP32_OUT), N_i >= 1; device pointers,
+ *              16-byte aligned; no y may overlap another y or any input
+ *   count      1 .. ANY4_GROUP_MAX
+ *   workspace  at least the largest any4_matmul_workspace_size_ex(M, N_i, K,
+ *              G, path) of the group where the per-matrix calls need one
+ *   flags      as any4_matmul_ex (ANY4_FLAG_OVERLAP_PRIOR, _FP32_OUT,
+ *              _TEST_STALL; ANY4_FLAG_PAIR_TABLE makes M = 1 take the
+ *              per-matrix calls)
+ * Returns the first error of the validation (nothing launched), or of the
+ * per-matrix calls (the earlier ones launched).
+ */
+#define ANY4_GROUP_MAX 4
+typedef struct any4_weight {
+  const uint8_t* packed;
+  const uint16_t* lut;
+  int64_t lut_row_stride;
+  const uint16_t* scale;
+  const uint16_t* offset;
+  uint16_t* y;
+  int64_t N;
+} any4_weight;
+
+ANY4_API any4_status any4_matmul_grouped(const uint16_t* x, const any4_weight* w, int32_t count,
+                                         int64_t M, int64_t K, int64_t G, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_status,
+                                         any4_path path, uint32_t flags, any4_stream_t stream);
 
 /* Same for an explicit path. */
 ANY4_API size_t any4_matmul_workspace_size_ex(int64_t M, int64_t N, int64_t K, int64_t G,

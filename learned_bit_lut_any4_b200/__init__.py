@@ -17,6 +17,7 @@ from ._native import (  # noqa: F401
     ANY4_ERR_TIMEOUT,
     ANY4_ERR_UNSUPPORTED,
     ANY4_ERR_WORKSPACE,
+    ANY4_GROUP_MAX,
     ANY4_QUANTIZE_MAX_ITER,
     ANY4_QUANTIZE_MAX_K,
     ANY4_STATIC_SCRATCH_BYTES,
@@ -27,7 +28,10 @@ from ._native import (  # noqa: F401
     any4_dequant_bits,
     any4_group_sums,
     any4_matmul,
+    any4_matmul_bits,
+    any4_matmul_bits_workspace_size,
     any4_matmul_choose_path,
+    any4_matmul_grouped,
     any4_matmul_static_scratch,
     any4_matmul_workspace_size,
     any4_pack,

@@ -45,6 +45,16 @@ class Any4Error(RuntimeError):
         super().__init__(f"{where}: any4 status {status} ({any4_status_string(status)})")
 
 
+class Any4Weight(ctypes.Structure):
+    """any4_weight of include/any4.h: one matrix of any4_matmul_grouped."""
+    _fields_ = [("packed", ctypes.c_void_p), ("lut", ctypes.c_void_p),
+                ("lut_row_stride", ctypes.c_int64), ("scale", ctypes.c_void_p),
+                ("offset", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64)]
+
+
+ANY4_GROUP_MAX = 4
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -87,6 +97,14 @@ def library() -> ctypes.CDLL:
     lib.any4_matmul_choose_path.restype = i32
     lib.any4_status_string.argtypes = [i32]
     lib.any4_status_string.restype = ctypes.c_char_p
+    lib.any4_matmul_grouped.argtypes = [vp, ctypes.POINTER(Any4Weight), i32, i64, i64, i64, vp,
+                                        sz, vp, i32, ctypes.c_uint32, vp]
+    lib.any4_matmul_grouped.restype = i32
+    lib.any4_matmul_bits.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, i32, vp,
+                                     sz, vp, ctypes.c_uint32, vp]
+    lib.any4_matmul_bits.restype = i32
+    lib.any4_matmul_bits_workspace_size.argtypes = [i64, i64, i64, i64, i32]
+    lib.any4_matmul_bits_workspace_size.restype = sz
     lib.any4_group_sums.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.any4_group_sums.restype = i32
     lib.any4_bits_per_weight.argtypes = [i64, i64]
@@ -308,7 +326,8 @@ def _need_status(dev_status, dev):
     _need(dev_status, "dev_status", (torch.int32,), dev)
 
 
-def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_out=False):
+def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_out=False,
+                     bits=4):
     """Validate the operands of a matmul call on the host, before any launch:
     the C ABI sees bare pointers and cannot check that a buffer is large
     enough, so a short y, scale or offset is caught here.  Sizes are checked
@@ -321,14 +340,14 @@ def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_
         if t.dtype not in dts:
             raise TypeError(f"{nm} must have dtype in {dts}, got {t.dtype}")
     if x.dim() != 2 or packed.dim() != 2:
-        raise ValueError("x must be [M, K] and packed [N, K/2]")
+        raise ValueError(f"x must be [M, K] and packed [N, {bits} K / 8]")
     M, K = x.shape
     N, Kh = packed.shape
-    if 2 * Kh != K:
-        raise ValueError(f"x has K={K} but packed holds {2 * Kh} columns")
+    if Kh * 8 != K * bits:
+        raise ValueError(f"x has K={K} but packed holds {Kh * 8 // bits} {bits}-bit columns")
     if G <= 0 or K % G != 0:
         raise ValueError(f"G={G} must be positive and divide K={K}")
-    stride = _lut_stride(lut, N)
+    stride = _lut_stride(lut, N, 1 << bits)
     if scale.numel() != N * (K // G) or offset.numel() != N * (K // G):
         raise ValueError(f"scale and offset must hold N * K/G = {N * (K // G)} values")
     if y is not None:
@@ -346,12 +365,12 @@ def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_
     return M, N, K, stride, y
 
 
-def _lut_stride(lut: torch.Tensor, N: int) -> int:
-    if lut.dim() == 1 and lut.numel() == 16:
+def _lut_stride(lut: torch.Tensor, N: int, entries: int = 16) -> int:
+    if lut.dim() == 1 and lut.numel() == entries:
         return 0
-    if lut.dim() == 2 and tuple(lut.shape) == (N, 16):
-        return 16
-    raise ValueError(f"lut must be [N, 16] or [16], got {tuple(lut.shape)}")
+    if lut.dim() == 2 and tuple(lut.shape) == (N, entries):
+        return entries
+    raise ValueError(f"lut must be [N, {entries}] or [{entries}], got {tuple(lut.shape)}")
 
 
 def any4_dequant(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
@@ -451,6 +470,92 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                                   | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
                                   _stream(dev)), "any4_matmul")
     return y
+
+
+def any4_matmul_bits_workspace_size(M: int, N: int, K: int, G: int, bits: int) -> int:
+    return int(library().any4_matmul_bits_workspace_size(M, N, K, G, bits))
+
+
+def any4_matmul_bits(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
+                     scale: torch.Tensor, offset: torch.Tensor, G: int, bits: int,
+                     y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None, overlap_prior: bool = False,
+                     fp32_out: bool = False, test_stall: bool = False) -> torch.Tensor:
+    """y[M, N] = x * dequant(W)^T for n-bit codes (any4_pack_bits layout; lut
+    [N, 2^bits] or [2^bits]).  bits = 4 is any4_matmul."""
+    if bits not in (2, 3, 4):
+        raise ValueError("bits must be 2, 3 or 4")
+    M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status,
+                                          fp32_out, bits)
+    dev = x.device
+    lib = library()
+    need = int(lib.any4_matmul_bits_workspace_size(M, N, K, G, bits))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), dev)
+        ws_bytes = workspace.numel()
+        if ws_bytes == 0:
+            workspace = None
+    _need_status(dev_status, dev)
+    with _on_device(dev):
+        _check(lib.any4_matmul_bits(_ptr(x), _ptr(packed), _ptr(lut), stride, _ptr(scale),
+                                    _ptr(offset), _ptr(y), M, N, K, G, bits, _ptr(workspace),
+                                    ws_bytes, _ptr(dev_status),
+                                    (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
+                                    | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
+                                    | (ANY4_FLAG_TEST_STALL if test_stall else 0),
+                                    _stream(dev)), "any4_matmul_bits")
+    return y
+
+
+def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
+                        workspace: torch.Tensor | None = None, path: str = "auto",
+                        dev_status: torch.Tensor | None = None, overlap_prior: bool = False,
+                        fp32_out: bool = False, test_stall: bool = False,
+                        pair_table: bool = False):
+    """[y_i = x * dequant(W_i)^T for each (packed, lut, scale, offset) in
+    weights]: matrices that share x, in one launch at M = 1 (see
+    any4_matmul_grouped in include/any4.h).  Returns the list of y_i."""
+    weights = list(weights)
+    if not 1 <= len(weights) <= ANY4_GROUP_MAX:
+        raise ValueError(f"between 1 and {ANY4_GROUP_MAX} matrices")
+    if ys is not None and len(ys) != len(weights):
+        raise ValueError("one y per matrix")
+    descs = (Any4Weight * len(weights))()
+    outs = []
+    M = K = None
+    need_ws = 0
+    lib = library()
+    p = PATHS[path]
+    for i, (packed, lut, scale, offset) in enumerate(weights):
+        y = None if ys is None else ys[i]
+        M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status,
+                                              fp32_out)
+        outs.append(y)
+        descs[i] = Any4Weight(_ptr(packed), _ptr(lut), stride, _ptr(scale), _ptr(offset),
+                              _ptr(y), N)
+        need_ws = max(need_ws, int(lib.any4_matmul_workspace_size_ex(M, N, K, G, p)))
+    dev = x.device
+    if workspace is None and need_ws > 0:
+        workspace = torch.empty(need_ws, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), dev)
+        ws_bytes = workspace.numel()
+        if ws_bytes == 0:
+            workspace = None
+    _need_status(dev_status, dev)
+    with _on_device(dev):
+        _check(lib.any4_matmul_grouped(_ptr(x), descs, len(weights), M, K, G, _ptr(workspace),
+                                       ws_bytes, _ptr(dev_status), p,
+                                       (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
+                                       | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
+                                       | (ANY4_FLAG_TEST_STALL if test_stall else 0)
+                                       | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
+                                       _stream(dev)), "any4_matmul_grouped")
+    return outs
 
 
 def any4_matmul_static_scratch(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,

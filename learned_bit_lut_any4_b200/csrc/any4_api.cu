@@ -19,6 +19,15 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
                                     int64_t N, int64_t K, int64_t G, void* workspace,
                                     size_t workspace_bytes, int32_t* dev_status, bool test_stall,
                                     cudaStream_t stream, const DeviceInfo& dev);
+// The same with codes of 2 or 3 bits (the n-bit dequant as the first pass).
+any4_status launch_prefill_two_pass_bits(const uint16_t* x, const uint8_t* packed,
+                                         const uint16_t* lut, int64_t lut_row_stride,
+                                         const uint16_t* scale, const uint16_t* offset,
+                                         uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K,
+                                         int64_t G, int bits, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_status,
+                                         bool test_stall, cudaStream_t stream,
+                                         const DeviceInfo& dev);
 
 // Table learning (quantize.cu): one thread block per weight row; bits = 2, 3, 4.
 size_t quantize_smem_bytes(int64_t K, int64_t G);
@@ -30,10 +39,6 @@ any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64
 any4_status launch_pack_bits(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
                              int bits, int32_t* dev_status, cudaStream_t stream,
                              const DeviceInfo& dev);
-any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
-                                int64_t lut_row_stride, const uint16_t* scale,
-                                const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
-                                int64_t G, int bits, cudaStream_t stream, const DeviceInfo& dev);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -233,6 +238,100 @@ any4_status any4_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut
   if (st != ANY4_OK) return st;
   return launch_dequant(packed, lut, lut_row_stride, scale, offset, W, N, K, G,
                         (cudaStream_t)stream, dev);
+}
+
+any4_status any4_matmul_grouped(const uint16_t* x, const any4_weight* w, int32_t count,
+                                int64_t M, int64_t K, int64_t G, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, any4_path path,
+                                uint32_t flags, any4_stream_t stream) {
+  if (!x || !w) return ANY4_ERR_NULL;
+  if (count < 1 || count > ANY4_GROUP_MAX) return ANY4_ERR_SHAPE;
+  for (int i = 0; i < count; ++i) {
+    if (!w[i].packed || !w[i].lut || !w[i].scale || !w[i].offset || !w[i].y)
+      return ANY4_ERR_NULL;
+    if (M < 1 || !shape_ok(w[i].N, K, G) || !stride_ok(w[i].lut_row_stride))
+      return ANY4_ERR_SHAPE;
+    if (!aligned16(w[i].packed) || !aligned16(w[i].lut) || !aligned16(w[i].scale) ||
+        !aligned16(w[i].offset) || !aligned16(w[i].y))
+      return ANY4_ERR_ALIGN;
+  }
+  if (!aligned16(x)) return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL |
+                         ANY4_FLAG_PAIR_TABLE))
+    return ANY4_ERR_UNSUPPORTED;
+  const any4_path chosen = path == ANY4_PATH_AUTO ? any4_matmul_choose_path(M, 1, K, G) : path;
+  bool one_launch = chosen == ANY4_PATH_DECODE && !(flags & ANY4_FLAG_PAIR_TABLE);
+  for (int i = 0; i < count && one_launch; ++i)
+    one_launch = decode_tma_supported(M, w[i].N, K, G);
+  if (one_launch) {
+    DeviceInfo dev;
+    any4_status st = current_device(&dev);
+    if (st != ANY4_OK) return st;
+    const bool fp32 = (flags & ANY4_FLAG_FP32_OUT) != 0;
+    DecodeWeights dw[ANY4_GROUP_MAX];
+    for (int i = 0; i < count; ++i)
+      dw[i] = {w[i].packed, w[i].lut, w[i].lut_row_stride, w[i].scale, w[i].offset,
+               fp32 ? nullptr : w[i].y, fp32 ? reinterpret_cast<float*>(w[i].y) : nullptr,
+               w[i].N};
+    return launch_decode_tma_group(x, dw, count, K, G, 4, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,
+                                   dev_status, (flags & ANY4_FLAG_TEST_STALL) != 0,
+                                   (cudaStream_t)stream, dev);
+  }
+  for (int i = 0; i < count; ++i) {
+    const any4_status st =
+        any4_matmul_ex(x, w[i].packed, w[i].lut, w[i].lut_row_stride, w[i].scale, w[i].offset,
+                       w[i].y, M, w[i].N, K, G, workspace, workspace_bytes, dev_status, path,
+                       flags, stream);
+    if (st != ANY4_OK) return st;
+  }
+  return ANY4_OK;
+}
+
+size_t any4_matmul_bits_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G,
+                                       int32_t bits) {
+  if (bits == 4) return any4_matmul_workspace_size(M, N, K, G);
+  if (bits < 2 || bits > 3 || M < 1 || !shape_ok(N, K, G)) return 0;
+  if (decode_tma_supported(M, N, K, G, bits)) return 0;
+  return prefill_two_pass_workspace_size(M, N, K, G);
+}
+
+any4_status any4_matmul_bits(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
+                             int64_t lut_row_stride, const uint16_t* scale,
+                             const uint16_t* offset, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                             int64_t G, int32_t bits, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_status, uint32_t flags, any4_stream_t stream) {
+  if (bits == 4)
+    return any4_matmul_ex(x, packed, lut, lut_row_stride, scale, offset, y, M, N, K, G,
+                          workspace, workspace_bytes, dev_status, ANY4_PATH_AUTO, flags, stream);
+  if (!x || !packed || !lut || !scale || !offset || !y) return ANY4_ERR_NULL;
+  if (bits < 2 || bits > 3 || M < 1 || !shape_ok(N, K, G) ||
+      (lut_row_stride != 0 && lut_row_stride != (int64_t(1) << bits)))
+    return ANY4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(lut) || !aligned16(scale) ||
+      !aligned16(offset) || !aligned16(y))
+    return ANY4_ERR_ALIGN;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
+  if (workspace && !aligned16(workspace)) return ANY4_ERR_ALIGN;
+  if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL))
+    return ANY4_ERR_UNSUPPORTED;
+  const size_t need = any4_matmul_bits_workspace_size(M, N, K, G, bits);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return ANY4_ERR_WORKSPACE;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  const bool fp32 = (flags & ANY4_FLAG_FP32_OUT) != 0;
+  float* y32 = fp32 ? reinterpret_cast<float*>(y) : nullptr;
+  const bool test_stall = (flags & ANY4_FLAG_TEST_STALL) != 0;
+  if (need == 0) {
+    const DecodeWeights w = {packed, lut, lut_row_stride, scale, offset, fp32 ? nullptr : y, y32,
+                             N};
+    return launch_decode_tma_group(x, &w, 1, K, G, bits, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,
+                                   dev_status, test_stall, (cudaStream_t)stream, dev);
+  }
+  return launch_prefill_two_pass_bits(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N,
+                                      K, G, bits, workspace, workspace_bytes, dev_status,
+                                      test_stall, (cudaStream_t)stream, dev);
 }
 
 any4_status any4_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K, int64_t G,

@@ -157,13 +157,37 @@ any4_status launch_decode_pair(const uint16_t* x, const uint8_t* packed, const u
                                int64_t N, int64_t K, int64_t G, void* workspace, bool overlap,
                                int32_t* dev_status, bool test_stall, cudaStream_t stream,
                                const DeviceInfo& dev);
-bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G);
+// The weight-streaming decode kernel takes the shape (bits: code width 2..4).
+bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G, int bits = 4);
+// One weight matrix of a grouped decode launch (y32, when not NULL, receives
+// the fp32 sums instead of y).
+struct DecodeWeights {
+  const uint8_t* packed;
+  const uint16_t* lut;
+  int64_t lut_row_stride;
+  const uint16_t* scale;
+  const uint16_t* offset;
+  uint16_t* y;
+  float* y32;
+  int64_t N;
+};
+// M = 1 on the weight-streaming kernel for up to ANY4_GROUP_MAX matrices that
+// share x, K and G, in one launch.
+any4_status launch_decode_tma_group(const uint16_t* x, const DecodeWeights* w, int count,
+                                    int64_t K, int64_t G, int bits, bool overlap,
+                                    int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                                    const DeviceInfo& dev);
 any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                               int64_t lut_row_stride, const uint16_t* scale,
                               const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
                               int64_t K, int64_t G, bool overlap, int32_t* dev_status,
                               bool test_stall, cudaStream_t stream, const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
+// n-bit (2 or 3) dequant into a bf16 W (nbit.cu).
+any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,
+                                int64_t lut_row_stride, const uint16_t* scale,
+                                const uint16_t* offset, uint16_t* W, int64_t N, int64_t K,
+                                int64_t G, int bits, cudaStream_t stream, const DeviceInfo& dev);
 // Skinny matmul for 2 <= M <= 16 (standard tensor-core mapping, table
 // lookups by byte permute): skinny.cu.
 any4_status launch_skinny(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,

@@ -23,6 +23,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,16 +32,9 @@ namespace any4 {
 namespace {
 
 constexpr int kTmaMaxWarps = 8;
+constexpr int kTmaMaxGroup = ANY4_GROUP_MAX;
 constexpr int kTmaRows = 8;      // P: rows per stage
 constexpr int kTmaStages = 2;    // S: stages per warp (2 keeps two blocks per SM)
-// Row pairs of a stage (counted from the last) whose table lookups run as
-// byte permutes on the integer pipe instead of warp shuffles, so that the
-// two kinds of lookup proceed on different pipes.
-#ifndef ANY4_DECODE_PRMT_PAIRS
-#define ANY4_DECODE_PRMT_PAIRS 0
-#endif
-constexpr int kTmaPrmtPairs = ANY4_DECODE_PRMT_PAIRS;
-static_assert(kTmaPrmtPairs >= 0 && kTmaPrmtPairs <= kTmaRows / 2, "pairs on the permute path");
 
 constexpr unsigned long long kTmaWaitNs = 2000000000ull;
 constexpr unsigned long long kTmaTestWaitNs = 1000000ull;  // the test-stall mode's limit
@@ -87,6 +81,20 @@ struct TmaMaps {
   CUtensorMap lut;     // bf16 [N][16], box {16, P}
   CUtensorMap scale;   // bf16 [N][K/G], box {1024/G, P}
   CUtensorMap offset;  // bf16 [N][K/G], box {1024/G, P}
+};
+
+// Up to kTmaMaxGroup matrices that multiply the same x (the q, k, v or gate,
+// up projections of a layer) in one launch: their row blocks are numbered one
+// after the other, block b of the launch belongs to the first matrix i with
+// b < blk_end[i].  All share K and G.
+struct TmaGroup {
+  TmaMaps maps[kTmaMaxGroup];
+  uint16_t* y[kTmaMaxGroup];
+  float* y32[kTmaMaxGroup];
+  const uint16_t* lut_shared[kTmaMaxGroup];  // one table for the matrix, or NULL
+  int N[kTmaMaxGroup];
+  int64_t blk_end[kTmaMaxGroup];
+  int count;
 };
 
 // D += A * B, m16n8k16 bf16 -> fp32 (legacy warp-level tensor-core MMA).
@@ -141,22 +149,49 @@ __device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
   return v[0];
 }
 
-template <int GPS>  // groups per 1024-column slice (1024 / G)
+// The stage layout of one warp's ring: P rows of codes (BITS * 128 bytes a
+// row: 1024 codes), the rows' tables (2^BITS bf16 each), scales, offsets.
+template <int GPS, int BITS>
+struct TmaStage {
+  static constexpr int P = kTmaRows;
+  static constexpr int kEntries = 1 << BITS;
+  static constexpr int kCodeBytes = P * 128 * BITS;
+  static constexpr int kLutBytes = P * kEntries * 2;
+  static constexpr int kLutSlot = ((kLutBytes + 127) / 128) * 128;
+  static constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
+  static constexpr int kBytes = kCodeBytes + kLutSlot + 2 * kGrpBytes;
+  static constexpr uint32_t kTx = kCodeBytes + kLutBytes + 2 * P * GPS * 2;
+  static_assert(kBytes % 128 == 0, "stage alignment");
+};
+
+__device__ __forceinline__ void tma1d(uint32_t dst, const CUtensorMap* map, int c0, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2}], [%3];"
+      :: "r"(dst), "l"(map), "r"(c0), "r"(bar) : "memory");
+}
+
+// Code j (0..31) of a lane's 32 codes held in BITS words (a little-endian
+// bit stream), in the low bits of the result; the bits above it are the
+// following codes, which the table shuffle ignores.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_word(const uint32_t (&w)[BITS], int j) {
+  const int bit = BITS * j, wi = bit >> 5, off = bit & 31;
+  if (wi + 1 < BITS) return __funnelshift_r(w[wi], w[wi + 1], off);
+  return w[wi] >> off;
+}
+
+template <int GPS, int BITS>  // groups per 1024-column slice (1024 / G), code width
 __global__ void __maxnreg__(96) decode_tma_kernel(
-    const __grid_constant__ TmaMaps maps, const uint16_t* __restrict__ x,
-    const uint16_t* __restrict__ lut_shared, uint16_t* __restrict__ y, float* __restrict__ y32,
-    int N, int K, int nslices, int rows_per_block, int32_t* dev_status, int test_stall) {
+    const __grid_constant__ TmaGroup grp, const uint16_t* __restrict__ x, int K, int nslices,
+    int rows_per_block, int32_t* dev_status, int test_stall) {
   // test_stall: warp 0 of block 0 stops its weight stream after one stage,
   // so its next wait runs out (1 ms limit) and the kernel ends cleanly
   const unsigned long long wait_ns = test_stall ? kTmaTestWaitNs : kTmaWaitNs;
-  constexpr int P = kTmaRows;
+  using St = TmaStage<GPS, BITS>;
+  constexpr int P = St::P;
   constexpr int S = kTmaStages;
-  constexpr int kCodeBytes = P * 512;
-  constexpr int kLutBytes = P * 32;
-  constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
-  constexpr int kStageBytes = kCodeBytes + kLutBytes + 2 * kGrpBytes;
-  constexpr uint32_t kTx = kCodeBytes + kLutBytes + 2 * P * GPS * 2;
-  static_assert(kStageBytes % 128 == 0, "stage alignment");
+  constexpr int NE = St::kEntries;
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31;
@@ -164,15 +199,15 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
   const int nwarps = blockDim.x >> 5;
   const int RT = rows_per_block;
   const int RTP = ((RT + P - 1) / P) * P;
-  // layout: [rings: nwarps * S * kStageBytes][bars: nwarps * S * 8][partials]
+  // layout: [rings: nwarps * S * St::kBytes][bars: nwarps * S * 8][partials]
   const uint32_t base = (smem_addr(smem_raw) + 127u) & ~127u;
   uint8_t* gbase = smem_raw + (base - smem_addr(smem_raw));
-  const uint32_t ring = base + (uint32_t)(warp * S * kStageBytes);
-  const uint8_t* gring = gbase + warp * S * kStageBytes;
-  const uint32_t bars = base + (uint32_t)(nwarps * S * kStageBytes) + (uint32_t)(warp * S * 8);
+  const uint32_t ring = base + (uint32_t)(warp * S * St::kBytes);
+  const uint8_t* gring = gbase + warp * S * St::kBytes;
+  const uint32_t bars = base + (uint32_t)(nwarps * S * St::kBytes) + (uint32_t)(warp * S * 8);
   float* s_part =
-      reinterpret_cast<float*>(gbase + nwarps * S * kStageBytes + nwarps * S * 8 + 16);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + nwarps * S * kStageBytes +
+      reinterpret_cast<float*>(gbase + nwarps * S * St::kBytes + nwarps * S * 8 + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + nwarps * S * St::kBytes +
                                                           nwarps * S * 8);
   if (threadIdx.x == 0) *s_abort = 0;
 
@@ -182,7 +217,7 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
   }
   __syncthreads();  // barriers and the abort flag are initialised
 
-  const int64_t nblocks = ((int64_t)N + RT - 1) / RT;
+  const int64_t nblocks = grp.blk_end[grp.count - 1];
   uint32_t it_issue = 0, it_use = 0;  // ring positions (issue and consumption order)
   bool waited = false, ok = true;
   const int gsub = (lane * 32) / (1024 / GPS);  // this lane's group within the slice
@@ -191,7 +226,12 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
   // a warp whose wait gave up only stops computing (ok = false) and raises
   // the block-wide flag so that no result of the block is written.
   for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
-    const int row0 = (int)(blk * RT);
+    int mi = 0;  // the matrix of this row block
+    while (mi + 1 < grp.count && blk >= grp.blk_end[mi]) ++mi;
+    const TmaMaps& maps = grp.maps[mi];
+    const int N = grp.N[mi];
+    const uint16_t* lut_shared = grp.lut_shared[mi];
+    const int row0 = (int)((blk - (mi > 0 ? grp.blk_end[mi - 1] : 0)) * RT);
     const int nrows = (N - row0) < RT ? (N - row0) : RT;
     const int nstages = (nrows + P - 1) / P;
     bool first_slice = true;
@@ -205,15 +245,19 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
           return;
         }
         const int st = (int)(it_issue % S);
-        const uint32_t dst = ring + (uint32_t)(st * kStageBytes);
+        const uint32_t dst = ring + (uint32_t)(st * St::kBytes);
         const uint32_t bar = bars + 8u * st;
         const int r = row0 + stage_idx * P;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     :: "r"(bar), "r"(kTx) : "memory");
-        tma2d(dst, &maps.codes, s * 128, r, bar);
-        tma2d(dst + kCodeBytes, &maps.lut, 0, r, bar);
-        tma2d(dst + kCodeBytes + kLutBytes, &maps.scale, s * GPS, r, bar);
-        tma2d(dst + kCodeBytes + kLutBytes + kGrpBytes, &maps.offset, s * GPS, r, bar);
+                     :: "r"(bar), "r"(St::kTx) : "memory");
+        tma2d(dst, &maps.codes, s * 32 * BITS, r, bar);
+        if constexpr (BITS == 2)
+          tma1d(dst + St::kCodeBytes, &maps.lut, r * NE, bar);
+        else
+          tma2d(dst + St::kCodeBytes, &maps.lut, 0, r, bar);
+        tma2d(dst + St::kCodeBytes + St::kLutSlot, &maps.scale, s * GPS, r, bar);
+        tma2d(dst + St::kCodeBytes + St::kLutSlot + St::kGrpBytes, &maps.offset, s * GPS, r,
+              bar);
         ++it_issue;
       };
       for (int q = 0; q < S && q < nstages; ++q) issue(q);
@@ -235,11 +279,8 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
 #pragma unroll
         for (int i = 0; i < 16; ++i) xw[i] = 0u;
       }
-      const uint32_t lv_shared = lut_shared ? (uint32_t)ldg_u16(lut_shared + (lane & 15)) : 0u;
-      // byte planes of the one shared table (pairs on the permute path)
-      uint32_t tls[4] = {0u, 0u, 0u, 0u}, ths[4] = {0u, 0u, 0u, 0u};
-      if (kTmaPrmtPairs > 0 && lut_shared)
-        table_planes(ldg_nc_v4(lut_shared), ldg_nc_v4(lut_shared + 8), tls, ths);
+      const uint32_t lv_shared =
+          lut_shared ? (uint32_t)ldg_u16(lut_shared + (lane & (NE - 1))) : 0u;
 
       for (int si = 0; si < nstages; ++si) {
         const int st = (int)(it_use % S);
@@ -250,12 +291,12 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
           *s_abort = 1;
           break;
         }
-        const uint8_t* sp = gring + st * kStageBytes;
-        const uint4* codes = reinterpret_cast<const uint4*>(sp);
-        const uint16_t* lt = reinterpret_cast<const uint16_t*>(sp + kCodeBytes);
-        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes);
-        const uint16_t* of =
-            reinterpret_cast<const uint16_t*>(sp + kCodeBytes + kLutBytes + kGrpBytes);
+        const uint8_t* sp = gring + st * St::kBytes;
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sp);
+        const uint16_t* lt = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes);
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot);
+        const uint16_t* of = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot +
+                                                               St::kGrpBytes);
         // The stage's rows a pair at a time (rows 2pp, 2pp+1 share the tensor-core
         // steps), so that few registers stay live and many warps fit per SM;
         // each pair accumulates in two chains (even and odd steps) to halve the
@@ -274,56 +315,49 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         for (int pp = 0; pp < npairs; ++pp) {
           const int ja = 2 * pp, jb = 2 * pp + 1;
           const bool va = ja < rows_left, vb = jb < rows_left;
-          const uint4 qa = va ? codes[ja * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
-          const uint4 qb = vb ? codes[jb * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t la = lut_shared ? lv_shared : (uint32_t)lt[ja * 16 + (lane & 15)];
-          const uint32_t lb = lut_shared ? lv_shared : (uint32_t)lt[jb * 16 + (lane & 15)];
-          const uint32_t sa = dup2(sc[ja * GPS + gsub]), oa = dup2(of[ja * GPS + gsub]);
-          const uint32_t sb = dup2(sc[jb * GPS + gsub]), ob = dup2(of[jb * GPS + gsub]);
-          const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w};
-          const uint32_t wb4[4] = {qb.x, qb.y, qb.z, qb.w};
-          float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-          // word t = codes 8t .. 8t + 7 of the lane's 32, two mma steps of 4
-          // codes: A rows 0-7 = row ja, rows 8-15 = row jb, B = x at the same
-          // four columns; the diagonals C[q][q], C[q+8][q] are the two rows'
-          // partial sums
-          if (kTmaPrmtPairs > 0 && pp >= NP - kTmaPrmtPairs) {
-            // this pair's lookups as byte permutes on the integer pipe
-            uint32_t tla[4], tha[4], tlb[4], thb[4];
-            if (lut_shared) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) { tla[i] = tlb[i] = tls[i]; tha[i] = thb[i] = ths[i]; }
-            } else {
-              const uint4* ea = reinterpret_cast<const uint4*>(lt + ja * 16);
-              const uint4* eb = reinterpret_cast<const uint4*>(lt + jb * 16);
-              table_planes(ea[0], ea[1], tla, tha);
-              table_planes(eb[0], eb[1], tlb, thb);
-            }
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint32_t A[4], B[4];
-              lookup8(wa4[t], tla, tha, A);
-              lookup8(wb4[t], tlb, thb, B);
-#pragma unroll
-              for (int p = 0; p < 4; ++p) {
-                A[p] = hfma2_bf16(A[p], sa, oa);
-                B[p] = hfma2_bf16(B[p], sb, ob);
-              }
-              mma16816(c0, A[0], B[0], A[1], B[1], xw[4 * t], xw[4 * t + 1]);
-              mma16816(c1, A[2], B[2], A[3], B[3], xw[4 * t + 2], xw[4 * t + 3]);
-            }
+          // the lane's 32 codes of each row: BITS consecutive words
+          uint32_t wa[BITS], wb[BITS];
+          if constexpr (BITS == 4) {
+            const uint4 qa = va ? reinterpret_cast<const uint4*>(codes)[ja * 32 + lane]
+                                : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 qb = vb ? reinterpret_cast<const uint4*>(codes)[jb * 32 + lane]
+                                : make_uint4(0u, 0u, 0u, 0u);
+            wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
+            wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
+          } else if constexpr (BITS == 2) {
+            const uint2 qa = va ? reinterpret_cast<const uint2*>(codes)[ja * 32 + lane]
+                                : make_uint2(0u, 0u);
+            const uint2 qb = vb ? reinterpret_cast<const uint2*>(codes)[jb * 32 + lane]
+                                : make_uint2(0u, 0u);
+            wa[0] = qa.x; wa[1] = qa.y;
+            wb[0] = qb.x; wb[1] = qb.y;
           } else {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint32_t A[4], B[4];
-#pragma unroll
-              for (int p = 0; p < 4; ++p) {
-                A[p] = dq_pair(la, wa4[t] >> (8 * p), wa4[t] >> (8 * p + 4), sa, oa);
-                B[p] = dq_pair(lb, wb4[t] >> (8 * p), wb4[t] >> (8 * p + 4), sb, ob);
-              }
-              mma16816(c0, A[0], B[0], A[1], B[1], xw[4 * t], xw[4 * t + 1]);
-              mma16816(c1, A[2], B[2], A[3], B[3], xw[4 * t + 2], xw[4 * t + 3]);
+            for (int b = 0; b < BITS; ++b) {
+              wa[b] = va ? codes[(ja * 32 + lane) * BITS + b] : 0u;
+              wb[b] = vb ? codes[(jb * 32 + lane) * BITS + b] : 0u;
             }
+          }
+          const uint32_t la = lut_shared ? lv_shared : (uint32_t)lt[ja * NE + (lane & (NE - 1))];
+          const uint32_t lb = lut_shared ? lv_shared : (uint32_t)lt[jb * NE + (lane & (NE - 1))];
+          const uint32_t sa = dup2(sc[ja * GPS + gsub]), oa = dup2(of[ja * GPS + gsub]);
+          const uint32_t sb = dup2(sc[jb * GPS + gsub]), ob = dup2(of[jb * GPS + gsub]);
+          float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+          // codes 8t .. 8t + 7 of the lane's 32, two mma steps of 4 codes:
+          // A rows 0-7 = row ja, rows 8-15 = row jb, B = x at the same four
+          // columns; the diagonals C[q][q], C[q+8][q] are the two rows'
+          // partial sums
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            uint32_t A[4], B[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int j = 8 * t + 2 * p;
+              A[p] = dq_pair(la, code_word<BITS>(wa, j), code_word<BITS>(wa, j + 1), sa, oa);
+              B[p] = dq_pair(lb, code_word<BITS>(wb, j), code_word<BITS>(wb, j + 1), sb, ob);
+            }
+            mma16816(c0, A[0], B[0], A[1], B[1], xw[4 * t], xw[4 * t + 1]);
+            mma16816(c1, A[2], B[2], A[3], B[3], xw[4 * t + 2], xw[4 * t + 3]);
           }
           const float da = (qd & 1) ? c0[1] + c1[1] : c0[0] + c1[0];
           const float db = (qd & 1) ? c0[3] + c1[3] : c0[2] + c1[2];
@@ -357,10 +391,10 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
       for (int t = threadIdx.x; t < nrows; t += blockDim.x) {
         float tot = 0.f;
         for (int w = 0; w < nw_used; ++w) tot += s_part[(size_t)w * RTP + t];
-        if (y32 != nullptr)
-          y32[row0 + t] = tot;
+        if (grp.y32[mi] != nullptr)
+          grp.y32[mi][row0 + t] = tot;
         else
-          y[row0 + t] = f32_to_bf16_rn(tot);
+          grp.y[mi][row0 + t] = f32_to_bf16_rn(tot);
       }
     }
     __syncthreads();
@@ -411,55 +445,83 @@ bool encode2d(EncodeFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int GPS>
-any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
-                    int64_t lut_row_stride, const uint16_t* scale, const uint16_t* offset,
-                    uint16_t* y, float* y32, int64_t N, int64_t K, int64_t G, bool overlap,
-                    int32_t* dev_status, bool test_stall, cudaStream_t stream,
-                    const DeviceInfo& dev) {
+// 1-D map over n u16 values (the 2-bit tables: 8 bytes a row, below the
+// 16-byte row stride a 2-D map needs), box of box_n values
+bool encode1d(EncodeFn enc, CUtensorMap* m, const void* ptr, uint64_t n, uint32_t box_n) {
+  const cuuint64_t dims[1] = {n};
+  // a rank-1 map has no stride, but the encoder rejects a NULL stride array
+  const cuuint64_t unused_stride[1] = {((n * 2 + 15) / 16) * 16};
+  const cuuint32_t box[1] = {box_n};
+  const cuuint32_t es[1] = {1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 1, const_cast<void*>(ptr), dims, unused_stride, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_weights(EncodeFn enc, TmaMaps* maps, const DecodeWeights& w, int64_t K, int64_t G,
+                    int GPS, int bits) {
   constexpr int P = kTmaRows;
+  const uint64_t N = (uint64_t)w.N;
+  const uint32_t ne = 1u << bits;
+  // codes as u32 [N][K bits / 32]: 1024 codes of a row = 32 * bits words
+  if (!encode2d(enc, &maps->codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, w.packed,
+                (uint64_t)K * bits / 32, N, (uint64_t)K * bits / 8, 32 * bits, P) ||
+      !encode2d(enc, &maps->scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.scale, (uint64_t)(K / G), N,
+                (uint64_t)(K / G) * 2, GPS, P) ||
+      !encode2d(enc, &maps->offset, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.offset, (uint64_t)(K / G),
+                N, (uint64_t)(K / G) * 2, GPS, P))
+    return false;
+  // One table for the matrix (lut_row_stride 0) is read directly by the
+  // kernel; the per-stage tensor load of the table slot still runs (rows past
+  // the first come back as zeros) so that every stage carries the same bytes.
+  const uint64_t lut_rows = w.lut_row_stride != 0 ? N : 1;
+  if (bits == 2) return encode1d(enc, &maps->lut, w.lut, lut_rows * ne, P * ne);
+  return encode2d(enc, &maps->lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.lut, ne, lut_rows, ne * 2,
+                  ne, P);
+}
+
+template <int GPS, int BITS>
+any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_t K, int64_t G,
+                    bool overlap, int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                    const DeviceInfo& dev) {
+  using St = TmaStage<GPS, BITS>;
+  constexpr int P = St::P;
   constexpr int S = kTmaStages;
-  constexpr int kGrpBytes = ((P * GPS * 2 + 127) / 128) * 128;
-  constexpr int kStageBytes = P * 512 + P * 32 + 2 * kGrpBytes;
+  if (count < 1 || count > kTmaMaxGroup) return ANY4_ERR_UNSUPPORTED;
   EncodeFn enc = get_encode();
   if (!enc) return ANY4_ERR_UNSUPPORTED;
-  TmaMaps maps;
-  if (!encode2d(enc, &maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, (uint64_t)K / 8,
-                (uint64_t)N, (uint64_t)K / 2, 128, P) ||
-      !encode2d(enc, &maps.scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, scale, (uint64_t)(K / G),
-                (uint64_t)N, (uint64_t)(K / G) * 2, GPS, P) ||
-      !encode2d(enc, &maps.offset, CU_TENSOR_MAP_DATA_TYPE_UINT16, offset, (uint64_t)(K / G),
-                (uint64_t)N, (uint64_t)(K / G) * 2, GPS, P))
-    return ANY4_ERR_CUDA;
-  if (lut_row_stride == 16) {
-    if (!encode2d(enc, &maps.lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, lut, 16, (uint64_t)N, 32, 16,
-                  P))
-      return ANY4_ERR_CUDA;
-  } else {
-    // one table for the matrix: read directly by the kernel; the per-stage
-    // tensor load of the table slot still runs (rows past the first come
-    // back as zeros) so that every stage carries the same byte count
-    if (!encode2d(enc, &maps.lut, CU_TENSOR_MAP_DATA_TYPE_UINT16, lut, 16, 1, 32, 16, P))
-      return ANY4_ERR_CUDA;
+  TmaGroup grp;
+  memset(&grp, 0, sizeof(grp));
+  int64_t total_rows = 0;
+  for (int i = 0; i < count; ++i) {
+    if (!encode_weights(enc, &grp.maps[i], w[i], K, G, GPS, BITS)) return ANY4_ERR_CUDA;
+    grp.y[i] = w[i].y;
+    grp.y32[i] = w[i].y32;
+    grp.lut_shared[i] = w[i].lut_row_stride == 0 ? w[i].lut : nullptr;
+    grp.N[i] = (int)w[i].N;
+    total_rows += w[i].N;
   }
+  grp.count = count;
   const int nslices = (int)((K + 1023) / 1024);
   const int per_warp = (nslices + kTmaMaxWarps - 1) / kTmaMaxWarps;
   const int nwarps = (nslices + per_warp - 1) / per_warp;
   const int threads = nwarps * 32;
 
-  auto kern = decode_tma_kernel<GPS>;
-  const size_t ring_bytes = (size_t)nwarps * S * kStageBytes + (size_t)nwarps * S * 8 + 16 + 128;
+  auto kern = decode_tma_kernel<GPS, BITS>;
+  const size_t ring_bytes = (size_t)nwarps * S * St::kBytes + (size_t)nwarps * S * 8 + 16 + 128;
   const int kMaxRT = 512;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern),
                           std::min<size_t>(dev.smem_optin, 227 * 1024)) != ANY4_OK)
     return ANY4_ERR_CUDA;
-  // rows per block from the blocks that fit per SM, which depends (through the
-  // partial sums) on the rows per block: settle it in two passes
+  // rows per block (one value for every matrix of the group) from the blocks
+  // that fit per SM, which depends (through the partial sums) on the rows per
+  // block: settle it in two passes
   int per_sm = 2;
   int64_t rt = 0, rtp = 0;
   for (int pass = 0; pass < 2; ++pass) {
     const int64_t wave = (int64_t)dev.sm_count * per_sm;
-    rt = std::min<int64_t>((N + wave - 1) / wave, kMaxRT);
+    rt = std::min<int64_t>((total_rows + wave - 1) / wave, kMaxRT);
     rtp = ((rt + P - 1) / P) * P;
     const size_t smem_try = ring_bytes + (size_t)nwarps * rtp * sizeof(float);
     int occ = cached_occupancy(reinterpret_cast<const void*>(kern), threads, smem_try);
@@ -468,9 +530,17 @@ any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lu
     per_sm = occ;
   }
   const int64_t wave = (int64_t)dev.sm_count * per_sm;
-  rt = std::min<int64_t>((N + wave - 1) / wave, kMaxRT);
+  rt = std::min<int64_t>((total_rows + wave - 1) / wave, kMaxRT);
+  // 2-bit tables come by a 1-D tensor load at element 4 r of the table
+  // array: its byte offset 8 r must be a multiple of 16, so every stage's
+  // first row r (row0 + a multiple of P) must be even, hence rt even
+  if (BITS == 2 && (rt & 1)) ++rt;
   rtp = ((rt + P - 1) / P) * P;
-  const int64_t nblocks = (N + rt - 1) / rt;
+  int64_t nblocks = 0;
+  for (int i = 0; i < count; ++i) {
+    nblocks += (w[i].N + rt - 1) / rt;
+    grp.blk_end[i] = nblocks;
+  }
   const int grid = (int)std::min<int64_t>(nblocks, wave);
   const size_t smem = ring_bytes + (size_t)nwarps * rtp * sizeof(float);
 
@@ -484,20 +554,53 @@ any4_status run_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lu
   attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const uint16_t* lut_shared = lut_row_stride == 0 ? lut : nullptr;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, maps, x, lut_shared, y, y32, (int)N, (int)K,
-                                             nslices, (int)rt, dev_status, test_stall ? 1 : 0);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, grp, x, (int)K, nslices, (int)rt,
+                                             dev_status, test_stall ? 1 : 0);
   return err == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
+
+template <int BITS>
+any4_status run_tma_bits(const uint16_t* x, const DecodeWeights* w, int count, int64_t K,
+                         int64_t G, bool overlap, int32_t* dev_status, bool test_stall,
+                         cudaStream_t stream, const DeviceInfo& dev) {
+  switch (G) {
+    case 128:
+      return run_tma<8, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    case 64:
+      return run_tma<16, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    case 32:
+      return run_tma<32, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    default:
+      return ANY4_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace
 
-bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G) {
+bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G, int bits) {
   if (M != 1) return false;
+  if (bits < 2 || bits > 4) return false;
   if (G != 32 && G != 64 && G != 128) return false;
-  if ((K / G) % 8 != 0) return false;  // 16-byte row stride of scale/offset
+  if ((K / G) % 8 != 0) return false;           // 16-byte row stride of scale/offset
+  if ((K * bits) % 128 != 0) return false;      // 16-byte row stride of the codes
   if (N > INT32_MAX / 2 || K > INT32_MAX / 2) return false;
   return true;
+}
+
+any4_status launch_decode_tma_group(const uint16_t* x, const DecodeWeights* w, int count,
+                                    int64_t K, int64_t G, int bits, bool overlap,
+                                    int32_t* dev_status, bool test_stall, cudaStream_t stream,
+                                    const DeviceInfo& dev) {
+  switch (bits) {
+    case 4:
+      return run_tma_bits<4>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    case 3:
+      return run_tma_bits<3>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    case 2:
+      return run_tma_bits<2>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+    default:
+      return ANY4_ERR_UNSUPPORTED;
+  }
 }
 
 any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
@@ -505,19 +608,9 @@ any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const ui
                               const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
                               int64_t K, int64_t G, bool overlap, int32_t* dev_status,
                               bool test_stall, cudaStream_t stream, const DeviceInfo& dev) {
-  switch (G) {
-    case 128:
-      return run_tma<8>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
-                        dev_status, test_stall, stream, dev);
-    case 64:
-      return run_tma<16>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
-                         dev_status, test_stall, stream, dev);
-    case 32:
-      return run_tma<32>(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G, overlap,
-                         dev_status, test_stall, stream, dev);
-    default:
-      return ANY4_ERR_UNSUPPORTED;
-  }
+  const DecodeWeights w = {packed, lut, lut_row_stride, scale, offset, y, y32, N};
+  return launch_decode_tma_group(x, &w, 1, K, G, 4, overlap, dev_status, test_stall, stream,
+                                 dev);
 }
 
 }  // namespace any4

@@ -7,8 +7,8 @@
 // §2.5.2:  sum_k x (alpha LUT + beta) = alpha sum_k x LUT + beta xsum.
 //
 // HBM-bound (reads 2 M K bytes, writes 4 M K / G).  A warp owns a "unit": a
-// run of whole groups of one row, about 2048 columns (8 KiB of loads in
-// flight per warp: 8 x 16-byte loads per lane, 512 coalesced bytes per warp
+// run of whole groups of one row (at most 32, one per lane), up to 2048
+// columns (8 KiB of loads in flight per warp: 8 x 16-byte loads per lane, 512 coalesced bytes per warp
 // instruction).  Fixed summation order, so results are deterministic:
 //   1. each 16-byte chunk (8 columns) is summed left to right in fp32;
 //   2. a group's chunk partials are summed left to right in fp32 by one lane.
@@ -38,10 +38,10 @@ __device__ __forceinline__ float sum8_bf16(uint4 v) {
   return s;
 }
 
-// Groups per unit: as many whole groups as fit in one pass (at least one; a
-// group wider than a pass is walked in passes).
+// Groups per unit: as many whole groups as fit in one pass, at most one per
+// lane (at least one; a group wider than a pass is walked in passes).
 __host__ __device__ inline int64_t groups_per_unit(int64_t G) {
-  return G >= kGsPassCols ? 1 : kGsPassCols / G;
+  return G >= kGsPassCols ? 1 : (kGsPassCols / G < 32 ? kGsPassCols / G : 32);
 }
 
 __global__ void __launch_bounds__(kGsThreads) group_sums_kernel(

@@ -99,14 +99,21 @@ __device__ __forceinline__ float table_entry(uint32_t t0, uint32_t t1, uint32_t 
 
 // dequant: one warp per 1024-column segment of a row, lane l on the segment's
 // 32-code chunk l (its n words are the n * 4 bytes after lane l - 1's, so the
-// warp's code loads are contiguous).  The 64 output bytes of a lane go to a
+// warp's code loads are contiguous).  The loads of the warp's next segment
+// (codes, the chunk's scale and offset, the row's table) are issued before the
+// current one is converted.  The 64 output bytes of a lane go to a
 // shared-memory copy of the segment's bf16 row, 16 bytes at a time in a
 // lane-rotated order (lanes 2i and 2i + 1 start at the 16-byte unit i mod 4
 // of their 64 bytes), which keeps every phase of 8 lanes on 8 distinct bank
-// groups; one bulk copy then writes the 2 KiB segment while the warp moves on
-// (two staging buffers per warp).
+// groups; the warp then writes the segment with 16-byte streaming stores,
+// 512 consecutive bytes per instruction.
 constexpr int kNbWarps = 8;
 constexpr int kNbSeg = 1024;
+
+__device__ __forceinline__ void nb_stg_cs_v4(void* p, const uint4& v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};"
+               :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
 
 template <int BITS>
 __global__ void __launch_bounds__(kNbWarps * 32)
@@ -114,58 +121,80 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
                     int64_t lut_row_stride, const uint16_t* __restrict__ scale,
                     const uint16_t* __restrict__ offset, uint16_t* __restrict__ W, int64_t N,
                     int K, int G, int g_shift) {
-  __shared__ __align__(128) uint16_t s_out[kNbWarps][2][kNbSeg];
+  __shared__ __align__(128) uint16_t s_out[kNbWarps][kNbSeg];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int segs_per_row = (K + kNbSeg - 1) / kNbSeg;
   const int64_t nseg = N * segs_per_row;
   const int groups = K / G;
   const int64_t first = (int64_t)blockIdx.x * kNbWarps + warp;
   const int64_t stride = (int64_t)gridDim.x * kNbWarps;
+  if (first >= nseg) return;
   // (row, segment) of the warp's segments without a division per step
-  int64_t n = first / segs_per_row;
-  int seg = (int)(first % segs_per_row);
   const int64_t n_step = stride / segs_per_row;
   const int s_step = (int)(stride % segs_per_row);
-  int buf = 0;
+  auto advance = [&](int64_t& n, int& seg) {
+    n += n_step;
+    seg += s_step;
+    if (seg >= segs_per_row) {
+      seg -= segs_per_row;
+      ++n;
+    }
+  };
+  // one segment's inputs, per lane
+  struct Seg {
+    uint32_t v[BITS];
+    uint32_t t[BITS == 3 ? 4 : 2];  // the row's table as bf16 pairs
+    uint32_t so;                    // scale (low half) and offset (high half)
+  };
+  auto load = [&](int64_t n, int seg, Seg& d) {
+    const int col0 = seg * kNbSeg;
+    const int k0 = col0 + 32 * lane;
+    if constexpr (BITS == 3) {
+      const uint4 t = __ldg(reinterpret_cast<const uint4*>(lut + n * lut_row_stride));
+      d.t[0] = t.x; d.t[1] = t.y; d.t[2] = t.z; d.t[3] = t.w;
+    } else {
+      const uint2 t = __ldg(reinterpret_cast<const uint2*>(lut + n * lut_row_stride));
+      d.t[0] = t.x; d.t[1] = t.y;
+    }
+#pragma unroll
+    for (int b = 0; b < BITS; ++b) d.v[b] = 0u;
+    d.so = 0u;
+    if (32 * lane < min(kNbSeg, K - col0)) {
+      const uint32_t g = g_shift >= 0 ? ((uint32_t)k0 >> g_shift) : (uint32_t)k0 / (uint32_t)G;
+      d.so = (uint32_t)ldg_u16(scale + n * groups + g) |
+             ((uint32_t)ldg_u16(offset + n * groups + g) << 16);
+      load_chunk<BITS>(packed + (n * K + k0) / 8 * BITS, d.v);
+    }
+  };
+  int64_t n = first / segs_per_row, ln = n;
+  int seg = (int)(first % segs_per_row), lseg = seg;
+  Seg nxt;
+  load(ln, lseg, nxt);
+  advance(ln, lseg);
   for (int64_t sg = first; sg < nseg; sg += stride) {
     const int col0 = seg * kNbSeg;
     const int cols = min(kNbSeg, K - col0);  // a multiple of 32
-    const int k0 = col0 + 32 * lane;
     const bool on = 32 * lane < cols;
-    uint32_t t0, t1, t2 = 0, t3 = 0;
-    if constexpr (BITS == 3) {
-      const uint4 t = __ldg(reinterpret_cast<const uint4*>(lut + n * lut_row_stride));
-      t0 = t.x;
-      t1 = t.y;
-      t2 = t.z;
-      t3 = t.w;
-    } else {
-      const uint2 t = __ldg(reinterpret_cast<const uint2*>(lut + n * lut_row_stride));
-      t0 = t.x;
-      t1 = t.y;
+    const Seg cur = nxt;
+    if (sg + stride < nseg) {  // the next segment's loads go out before this one's math
+      load(ln, lseg, nxt);
+      advance(ln, lseg);
     }
-    float s = 0.f, o = 0.f;
-    uint32_t v[BITS];
-#pragma unroll
-    for (int b = 0; b < BITS; ++b) v[b] = 0u;
-    if (on) {
-      const uint32_t g = g_shift >= 0 ? ((uint32_t)k0 >> g_shift) : (uint32_t)k0 / (uint32_t)G;
-      s = bf16_lo_to_f32(ldg_u16(scale + n * groups + g));
-      o = bf16_lo_to_f32(ldg_u16(offset + n * groups + g));
-      load_chunk<BITS>(packed + (n * K + k0) / 8 * BITS, v);
-    }
+    const uint32_t t0 = cur.t[0], t1 = cur.t[1];
+    const uint32_t t2 = BITS == 3 ? cur.t[BITS == 3 ? 2 : 0] : 0u;
+    const uint32_t t3 = BITS == 3 ? cur.t[BITS == 3 ? 3 : 1] : 0u;
+    const float s = bf16_lo_to_f32(cur.so), o = bf16_hi_to_f32(cur.so);
     uint32_t out[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
-      const float lo = __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(v, 2 * p)), s, o);
+      const float lo =
+          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(cur.v, 2 * p)), s, o);
       const float hi =
-          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(v, 2 * p + 1)), s, o);
+          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(cur.v, 2 * p + 1)), s, o);
       out[p] = pack_bf16x2_rn(lo, hi);
     }
-    // the bulk copy that last read this buffer (two segments ago) must be done
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-    __syncwarp();
-    uint16_t* seg_out = s_out[warp][buf];
+    uint16_t* seg_out = s_out[warp];
+    __syncwarp();  // the previous segment's row has been read back
     if (on) {
 #pragma unroll
       for (int step = 0; step < 4; ++step) {
@@ -177,25 +206,16 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
         *reinterpret_cast<uint4*>(seg_out + 32 * lane + 8 * q) = val;
       }
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (lane == 0) {
-      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                   :: "l"(W + n * K + col0), "r"((uint32_t)__cvta_generic_to_shared(seg_out)),
-                      "r"((uint32_t)cols * 2u) : "memory");
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    // 16-byte unit u = 32 q + lane of the segment's row: 512 contiguous bytes per q
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = 8 * (32 * q + lane);
+      if (c < cols)
+        nb_stg_cs_v4(W + n * K + col0 + c, *reinterpret_cast<const uint4*>(seg_out + c));
     }
-    buf ^= 1;
-    n += n_step;
-    seg += s_step;
-    if (seg >= segs_per_row) {
-      seg -= segs_per_row;
-      ++n;
-    }
+    advance(n, seg);
   }
-  // every bulk copy of this warp has finished before the block's shared memory goes
-  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-  __syncwarp();
 }
 
 int nb_pow2_shift(int64_t G) {

@@ -49,14 +49,17 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ i
 // (paper §2.5.2 dequant(w_Q) = alpha*w_Q + beta with w_Q = LUT[c], §2.4.1)
 // ---------------------------------------------------------------------------
 
-// One warp per 1024-column segment of a row.  Lane l converts the 8 codes at
-// columns 256 v + 8 l .. + 7 of the segment (v = 0..3), so each of the warp's
-// 4-byte code loads covers 128 consecutive bytes and each 16-byte result lands
-// next to its neighbour lane's in a shared-memory copy of the segment's bf16
-// row; one bulk copy (cp.async.bulk) then writes the whole segment, 2 KiB in
-// one piece, while the warp goes on with its next segment (two staging
-// buffers per warp).  The row's table sits in shared memory as fp32 (16
-// entries, 16 banks: conflict free).
+// One warp per 1024-column segment of a row, segments walked grid-stride.
+// Lane l converts the 8 codes at columns 256 v + 8 l .. + 7 (v = 0..3): each
+// of the warp's 4-byte code loads covers 128 consecutive bytes and each of
+// its 16-byte streaming stores 512 consecutive bytes of W.  The loads of the
+// warp's next segment are issued before the current one is converted (one
+// segment ahead, in registers).  The kernel moves 4 bytes of W out per byte
+// of codes in, and on B200 that mix of reads and writes streams at about
+// 5 TB/s with no arithmetic at all; a deeper prefetch (in registers, or
+// through a shared-memory ring fed by bulk copies) and bulk-copy stores were
+// both measured slower: they cost resident warps.  The row's table sits in
+// shared memory as fp32 (16 entries, 16 banks: conflict free).
 constexpr int kDqWarps = 8;
 constexpr int kDqThreads = kDqWarps * 32;
 constexpr int kDqSeg = 1024;
@@ -67,38 +70,22 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
   return r;
 }
 
-// The segments of one warp, in order: segment index sg = first + i * stride
-// walked as (row, segment within the row) without a division per step.
-struct SegWalk {
-  int64_t n;       // row
-  int seg;         // segment within the row
-  int64_t n_step;  // stride / segments per row
-  int s_step;      // stride % segments per row
-  int spr;         // segments per row
-  __device__ SegWalk(int64_t first, int64_t stride, int segs_per_row)
-      : n(first / segs_per_row), seg((int)(first % segs_per_row)),
-        n_step(stride / segs_per_row), s_step((int)(stride % segs_per_row)),
-        spr(segs_per_row) {}
-  __device__ void next() {
-    n += n_step;
-    seg += s_step;
-    if (seg >= spr) {
-      seg -= spr;
-      ++n;
-    }
-  }
-};
+__device__ __forceinline__ void stg_cs_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};"
+               :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
 
 // group of column k: a shift when G is a power of two (g_shift >= 0)
 __device__ __forceinline__ uint32_t group_of(uint32_t k, int g_shift, uint32_t G) {
   return g_shift >= 0 ? (k >> g_shift) : k / G;
 }
 
+// kFull: K is a multiple of the segment width, so no lane needs a bounds test
+template <bool kFull>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
     const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
     uint16_t* __restrict__ W, int64_t N, int K, int G, int g_shift) {
-  __shared__ __align__(128) uint16_t s_out[kDqWarps][2][kDqSeg];
   __shared__ float s_lut[kDqWarps][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int segs_per_row = (K + kDqSeg - 1) / kDqSeg;
@@ -107,79 +94,62 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
   const int64_t first = (int64_t)blockIdx.x * kDqWarps + warp;
   const int64_t stride = (int64_t)gridDim.x * kDqWarps;
   if (first >= nseg) return;
-  SegWalk wk(first, stride, segs_per_row);
-  // codes and the group's scale and offset of one segment, per lane
+  // codes and the groups' scale (low half) and offset (high half) of one
+  // segment, per lane
   struct Seg {
     uint32_t w[4];
-    float s[4], o[4];
+    uint32_t so[4];
   };
-  auto load = [&](int64_t n, int col0, Seg& d) {
-    const int cols = min(kDqSeg, K - col0);
+  auto load = [&](int64_t sg, Seg& d) {
+    const int64_t n = sg / segs_per_row;
+    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int c = 256 * v + 8 * lane;
-      d.w[v] = 0u;
-      d.s[v] = d.o[v] = 0.f;
-      if (c < cols) {
+      if (kFull || c < K - col0) {
         const uint32_t k = (uint32_t)(col0 + c);
         d.w[v] = ldg_nc_u32(packed + (n * K + k) / 2);
         const int64_t gi = n * groups + group_of(k, g_shift, (uint32_t)G);
-        d.s[v] = bf16_lo_to_f32(ldg_u16(scale + gi));
-        d.o[v] = bf16_lo_to_f32(ldg_u16(offset + gi));
+        d.so[v] = (uint32_t)ldg_u16(scale + gi) | ((uint32_t)ldg_u16(offset + gi) << 16);
+      } else {
+        d.w[v] = 0u;
+        d.so[v] = 0u;
       }
     }
   };
-  Seg cur, nxt;
-  load(wk.n, wk.seg * kDqSeg, cur);
+  Seg nxt;
+  load(first, nxt);
   int64_t cur_row = -1;
-  int buf = 0;
   for (int64_t sg = first; sg < nseg; sg += stride) {
-    const int64_t n = wk.n;
-    const int col0 = wk.seg * kDqSeg;
-    const int cols = min(kDqSeg, K - col0);  // a multiple of 32
-    wk.next();
-    if (sg + stride < nseg) load(wk.n, wk.seg * kDqSeg, nxt);  // the next segment in flight
+    const int64_t n = sg / segs_per_row;
+    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
     if (n != cur_row) {  // this warp moves to a new row: its table as fp32
       __syncwarp();
       if (lane < 16) s_lut[warp][lane] = bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + lane));
       __syncwarp();
       cur_row = n;
     }
-    // the bulk copy that last read this buffer (two segments ago) must be done
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-    __syncwarp();
+    const Seg cur = nxt;
+    if (sg + stride < nseg) load(sg + stride, nxt);  // out before this segment's math
     const float* t = s_lut[warp];
-    uint16_t* out = s_out[warp][buf];
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int c = 256 * v + 8 * lane;
-      if (c < cols) {
+      if (kFull || c < K - col0) {
+        const float sv = bf16_lo_to_f32(cur.so[v]), ov = bf16_hi_to_f32(cur.so[v]);
         uint32_t o[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
           // byte p of the word: codes of columns c + 2p (low nibble), c + 2p + 1
           const uint32_t byte = (cur.w[v] >> (8 * p)) & 0xffu;
-          const float lo = __fmaf_rn(t[byte & 15u], cur.s[v], cur.o[v]);
-          const float hi = __fmaf_rn(t[byte >> 4], cur.s[v], cur.o[v]);
+          const float lo = __fmaf_rn(t[byte & 15u], sv, ov);
+          const float hi = __fmaf_rn(t[byte >> 4], sv, ov);
           o[p] = pack_bf16x2_rn(lo, hi);
         }
-        *reinterpret_cast<uint4*>(out + c) = make_uint4(o[0], o[1], o[2], o[3]);
+        stg_cs_v4(W + n * K + col0 + c, o[0], o[1], o[2], o[3]);
       }
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncwarp();
-    if (lane == 0) {
-      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                   :: "l"(W + n * K + col0), "r"((uint32_t)__cvta_generic_to_shared(out)),
-                      "r"((uint32_t)cols * 2u) : "memory");
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
-    buf ^= 1;
-    cur = nxt;
   }
-  // every bulk copy of this warp has finished before the block's shared memory goes
-  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-  __syncwarp();
 }
 
 int pow2_shift(int64_t G) {
@@ -208,11 +178,12 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const uint16_t* scale, const uint16_t* offset, uint16_t* W,
                            int64_t N, int64_t K, int64_t G, cudaStream_t stream,
                            const DeviceInfo& dev) {
-  const int64_t segs = N * ((K + kDqSeg - 1) / kDqSeg);
-  int per_sm = cached_occupancy(reinterpret_cast<const void*>(dequant_kernel), kDqThreads, 0);
-  if (per_sm < 1) per_sm = 1;
   if (K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
-  dequant_kernel<<<grid_for(segs * 32, kDqThreads, dev, per_sm), kDqThreads, 0, stream>>>(
+  const int64_t segs = N * ((K + kDqSeg - 1) / kDqSeg);
+  auto kern = K % kDqSeg == 0 ? dequant_kernel<true> : dequant_kernel<false>;
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(kern), kDqThreads, 0);
+  if (per_sm < 1) per_sm = 1;
+  kern<<<grid_for(segs * 32, kDqThreads, dev, per_sm), kDqThreads, 0, stream>>>(
       packed, lut, lut_row_stride, scale, offset, W, N, (int)K, (int)G, pow2_shift(G));
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }

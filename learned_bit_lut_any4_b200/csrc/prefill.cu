@@ -778,4 +778,25 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
                                    K, G, workspace, fused, dev_status, test_stall, stream, dev);
 }
 
+// The same two passes for codes of 2 or 3 bits: the n-bit dequant kernel
+// fills the workspace with bf16 weights, then the same tensor-core pass.
+any4_status launch_prefill_two_pass_bits(const uint16_t* x, const uint8_t* packed,
+                                         const uint16_t* lut, int64_t lut_row_stride,
+                                         const uint16_t* scale, const uint16_t* offset,
+                                         uint16_t* y, float* y32, int64_t M, int64_t N, int64_t K,
+                                         int64_t G, int bits, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_status,
+                                         bool test_stall, cudaStream_t stream,
+                                         const DeviceInfo& dev) {
+  if (workspace == nullptr || workspace_bytes < prefill_two_pass_workspace_size(M, N, K, G))
+    return ANY4_ERR_WORKSPACE;
+  const size_t fused = prefill_workspace_size(M, N, K, G);
+  uint16_t* w = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + fused);
+  any4_status st = launch_dequant_bits(packed, lut, lut_row_stride, scale, offset, w, N, K, G,
+                                       bits, stream, dev);
+  if (st != ANY4_OK) return st;
+  return launch_prefill_impl<true>(x, packed, lut, lut_row_stride, scale, offset, w, y, y32, M, N,
+                                   K, G, workspace, fused, dev_status, test_stall, stream, dev);
+}
+
 }  // namespace any4

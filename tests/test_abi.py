@@ -288,3 +288,91 @@ def test_static_scratch_holds_a_148_sm_grid_and_no_more():
         _prefill_one_pass_bytes(slots)
     assert _prefill_one_pass_bytes(148) <= any4.ANY4_STATIC_SCRATCH_BYTES
     assert _prefill_one_pass_bytes(149) > any4.ANY4_STATIC_SCRATCH_BYTES
+
+
+def _grouped(items, M=1, K=128, G=32, x=FAKE, status=None, flags=0):
+    arr = (_native.Any4Weight * max(1, len(items)))()
+    for i, it in enumerate(items):
+        arr[i] = _native.Any4Weight(**it)
+    return _native.library().any4_matmul_grouped(x, arr, len(items), M, K, G, None, 0, status, 0,
+                                                 flags, None)
+
+
+def _item(**kw):
+    d = dict(packed=FAKE, lut=FAKE, lut_row_stride=16, scale=FAKE, offset=FAKE, y=FAKE, N=64)
+    d.update(kw)
+    return d
+
+
+def test_grouped_descriptor_layout_matches_header():
+    # seven 8-byte fields, no padding: pointers, an int64 stride, pointers, int64 N
+    assert ctypes.sizeof(_native.Any4Weight) == 56
+    assert _native.Any4Weight.N.offset == 48
+    text = open(os.path.join(HEADER_DIR, "any4.h")).read()
+    assert f"#define ANY4_GROUP_MAX {any4.ANY4_GROUP_MAX}" in text
+
+
+@pytest.mark.parametrize("items,kw,expect", [
+    ([], {}, any4.ANY4_ERR_SHAPE),                                   # count 0
+    ([_item()] * 5, {}, any4.ANY4_ERR_SHAPE),                        # above ANY4_GROUP_MAX
+    ([_item(), _item(y=None)], {}, any4.ANY4_ERR_NULL),
+    ([_item(), _item(N=0)], {}, any4.ANY4_ERR_SHAPE),
+    ([_item(lut_row_stride=8)], {}, any4.ANY4_ERR_SHAPE),
+    ([_item()], dict(K=100), any4.ANY4_ERR_SHAPE),
+    ([_item(), _item(scale=FAKE + 2)], {}, any4.ANY4_ERR_ALIGN),
+    ([_item()], dict(x=FAKE + 8), any4.ANY4_ERR_ALIGN),
+    ([_item()], dict(x=None), any4.ANY4_ERR_NULL),
+    ([_item()], dict(M=0), any4.ANY4_ERR_SHAPE),
+    ([_item()], dict(flags=64), any4.ANY4_ERR_UNSUPPORTED),
+    ([_item()], dict(status=FAKE + 2), any4.ANY4_ERR_ALIGN),
+])
+def test_grouped_rejects_bad_arguments(items, kw, expect):
+    assert _grouped(items, **kw) == expect
+
+
+def test_grouped_binding_checks_before_launch():
+    import torch
+    x = torch.zeros((1, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        any4.any4_matmul_grouped(x, [], 32)
+    with pytest.raises((TypeError, ValueError)):
+        any4.any4_matmul_grouped(x, [(torch.zeros((64, 64), dtype=torch.uint8),
+                                      torch.zeros((64, 16), dtype=torch.bfloat16),
+                                      torch.zeros((64, 4), dtype=torch.bfloat16),
+                                      torch.zeros((64, 4), dtype=torch.bfloat16))], 32)
+
+
+def _mbits(M=1, N=64, K=128, G=32, bits=3, x=FAKE, packed=FAKE, lut=FAKE, stride=8, scale=FAKE,
+           offset=FAKE, y=FAKE, ws=None, ws_bytes=0, status=None, flags=0):
+    return _native.library().any4_matmul_bits(x, packed, lut, stride, scale, offset, y, M, N, K,
+                                              G, bits, ws, ws_bytes, status, flags, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(bits=1), any4.ANY4_ERR_SHAPE),
+    (dict(bits=5), any4.ANY4_ERR_SHAPE),
+    (dict(stride=16), any4.ANY4_ERR_SHAPE),          # 3 bits: 8 entries a row or 0
+    (dict(bits=2, stride=8), any4.ANY4_ERR_SHAPE),   # 2 bits: 4 entries a row or 0
+    (dict(K=100), any4.ANY4_ERR_SHAPE),
+    (dict(M=0), any4.ANY4_ERR_SHAPE),
+    (dict(x=None), any4.ANY4_ERR_NULL),
+    (dict(y=FAKE + 4), any4.ANY4_ERR_ALIGN),
+    (dict(flags=8), any4.ANY4_ERR_UNSUPPORTED),      # the pair-table flag is any4-only
+    (dict(M=2), any4.ANY4_ERR_WORKSPACE),            # two passes need the workspace
+    (dict(M=1, K=1056, G=32), any4.ANY4_ERR_WORKSPACE),
+])
+def test_matmul_bits_rejects_bad_arguments(kw, expect):
+    assert _mbits(**kw) == expect
+
+
+def test_matmul_bits_workspace_sizes():
+    ws = any4.any4_matmul_bits_workspace_size
+    # M = 1 on the weight-streaming kernel's shapes: none
+    assert ws(1, 4096, 4096, 128, 3) == 0 and ws(1, 4096, 4096, 64, 2) == 0
+    # otherwise the two-pass workspace, the same as any4's large-M path
+    two = any4.any4_matmul_workspace_size(2048, 4096, 4096, 128)
+    assert ws(2, 4096, 4096, 128, 3) == two and ws(2048, 4096, 4096, 128, 2) == two
+    assert ws(1, 4096, 1056, 32, 3) == any4.any4_matmul_workspace_size(2048, 4096, 1056, 32)
+    assert ws(1, 4096, 4096, 256, 3) > 0
+    assert ws(1, 4096, 4096, 128, 4) == any4.any4_matmul_workspace_size(1, 4096, 4096, 128)
+    assert ws(1, 4096, 4096, 128, 5) == 0 and ws(0, 4096, 4096, 128, 3) == 0
