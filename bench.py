@@ -62,7 +62,7 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the M = 1 pair-table decode kernel source (the only kernel of a step): a
+    """Hash of the M = 1 weight-streaming decode kernel source (the only kernel of a step): a
     stored ncu traffic figure is only used while it was taken on this source."""
     h = hashlib.sha256()
     for fn in ("decode_tma.cu", "common.cuh"):

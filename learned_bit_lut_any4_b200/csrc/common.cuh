@@ -131,10 +131,12 @@ any4_status current_device(DeviceInfo* info);
 
 any4_status launch_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
                         int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev);
+// streaming: W written with evict-first stores (any4_dequant); false keeps
+// what fits of W in L2 for a kernel that reads it next (the two-pass prefill).
 any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
                            const uint16_t* scale, const uint16_t* offset, uint16_t* W,
                            int64_t N, int64_t K, int64_t G, cudaStream_t stream,
-                           const DeviceInfo& dev);
+                           const DeviceInfo& dev, bool streaming = true);
 any4_status launch_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K, int64_t G,
                               cudaStream_t stream, const DeviceInfo& dev);
 // The decode path (M <= 16).  y32, when not NULL, receives the fp32 sums

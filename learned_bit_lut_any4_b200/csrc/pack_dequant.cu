@@ -80,8 +80,10 @@ __device__ __forceinline__ uint32_t group_of(uint32_t k, int g_shift, uint32_t G
   return g_shift >= 0 ? (k >> g_shift) : k / G;
 }
 
-// kFull: K is a multiple of the segment width, so no lane needs a bounds test
-template <bool kFull>
+// kFull: K is a multiple of the segment width, so no lane needs a bounds test;
+// kStream: streaming stores (W is not read again soon) or plain write-back
+// stores (the two-pass prefill reads W right after: what stays in L2 helps)
+template <bool kFull, bool kStream>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
     const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut, int64_t lut_row_stride,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
@@ -146,7 +148,10 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
           const float hi = __fmaf_rn(t[byte >> 4], sv, ov);
           o[p] = pack_bf16x2_rn(lo, hi);
         }
-        stg_cs_v4(W + n * K + col0 + c, o[0], o[1], o[2], o[3]);
+        if (kStream)
+          stg_cs_v4(W + n * K + col0 + c, o[0], o[1], o[2], o[3]);
+        else
+          *reinterpret_cast<uint4*>(W + n * K + col0 + c) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -177,10 +182,11 @@ any4_status launch_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t 
 any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t lut_row_stride,
                            const uint16_t* scale, const uint16_t* offset, uint16_t* W,
                            int64_t N, int64_t K, int64_t G, cudaStream_t stream,
-                           const DeviceInfo& dev) {
+                           const DeviceInfo& dev, bool streaming) {
   if (K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   const int64_t segs = N * ((K + kDqSeg - 1) / kDqSeg);
-  auto kern = K % kDqSeg == 0 ? dequant_kernel<true> : dequant_kernel<false>;
+  auto kern = K % kDqSeg == 0 ? (streaming ? dequant_kernel<true, true> : dequant_kernel<true, false>)
+                              : (streaming ? dequant_kernel<false, true> : dequant_kernel<false, false>);
   int per_sm = cached_occupancy(reinterpret_cast<const void*>(kern), kDqThreads, 0);
   if (per_sm < 1) per_sm = 1;
   kern<<<grid_for(segs * 32, kDqThreads, dev, per_sm), kDqThreads, 0, stream>>>(

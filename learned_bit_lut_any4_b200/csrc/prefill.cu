@@ -199,6 +199,26 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
 
+// Phase alignment of the stream-K schedule (two-pass mode): block b starts at
+// unit U b / grid, mostly inside a tile, so without care the blocks sweep K at
+// offsets spread over the whole of it and every x and W panel is wanted at
+// many different times (the down shape re-read x about 9 times from DRAM).
+// Each tile's stages are therefore taken in a rotated order, starting at
+// stage rot(tile), chosen so that the block that finishes the tile reads
+// stage t of K at step t of its own range; the other blocks then run at most
+// one block range (mod the tile's stages) ahead, so at any moment all blocks
+// read a narrow band of K and each x and W panel is fetched from DRAM about
+// once.  Only the TMA coordinates change: the MMA consumes stages in issue
+// order, and a tile's partial sums still meet in block order.
+__device__ __forceinline__ int kb_rotation(int tile, int nkb, int64_t U, int64_t grid) {
+  const int64_t v = (int64_t)(tile + 1) * nkb;              // one past the tile's last unit
+  const int64_t b = (v * grid + U - 1) / U - 1;             // the block holding unit v - 1
+  const int64_t ub = U * b / grid;                          // where that block starts
+  int64_t r = ((int64_t)tile * nkb - ub) % nkb;
+  if (r < 0) r += nkb;
+  return (int)r;
+}
+
 // Walks a block's range [u, ue) of (tile, stage) units as segments: the
 // stages kb0 .. kb1-1 of one tile.
 struct SegIter {
@@ -307,7 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       int tile, kb0, kb1;
       while (seg.next(tile, kb0, kb1)) {
         const int mt = tile % n_mtiles;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int rot = kWTma ? kb_rotation(tile, nkb, U, gridDim.x) : 0;
+        for (int kbl = kb0; kbl < kb1; ++kbl, ++it) {
+          const int kb = kbl + rot < nkb ? kbl + rot : kbl + rot - nkb;
           const int s = (int)(it % kStages);
           const uint32_t ph = (it / kStages) & 1u;
           if (test_stall && blockIdx.x == 0 && it >= 1) goto done;  // the stream stops here
@@ -771,8 +793,10 @@ any4_status launch_prefill_two_pass(const uint16_t* x, const uint8_t* packed, co
     return ANY4_ERR_WORKSPACE;
   const size_t fused = prefill_workspace_size(M, N, K, G);
   uint16_t* w = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + fused);
+  // plain write-back stores: the GEMM pass reads W next, and what of it
+  // stays in L2 is not read from DRAM again
   any4_status st = launch_dequant(packed, lut, lut_row_stride, scale, offset, w, N, K, G, stream,
-                                  dev);
+                                  dev, /*streaming=*/false);
   if (st != ANY4_OK) return st;
   return launch_prefill_impl<true>(x, packed, lut, lut_row_stride, scale, offset, w, y, y32, M, N,
                                    K, G, workspace, fused, dev_status, test_stall, stream, dev);

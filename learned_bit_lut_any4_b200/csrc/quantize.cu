@@ -26,7 +26,8 @@
 //   - M-step: sample weight u_j = alpha_{g(j)} * E|x_j| (exact in fp64);
 //     numerator sum(u_j * w_S_j) and denominator sum(u_j) over ascending j,
 //     one lane of warp 0 per cluster and per sum, so the rounding order is the
-//     sequential one; a cluster whose weights sum to 0 keeps its entry;
+//     sequential one (the lane adds only its cluster's columns, found 32 at a
+//     time by warp ballots); a cluster whose weights sum to 0 keeps its entry;
 //   - stop after max_iter M-steps, or when an E-step changes no code;
 //   - LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
 //     LUT, packed as one little-endian bit stream per row (code k in bits
@@ -185,20 +186,36 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   int it = 0;
   while (it < max_iter) {
     if (warp == 0) {
-      // Eq. 23: lane q sums u_j * w_S_j, lane NQ + q sums u_j, over the
+      // Eq. 23: lane q sums u_j * w_S_j and lane NQ + q sums u_j over the
       // columns of cluster q in ascending order (lanes from 2 NQ up repeat
-      // that work and write nothing).
+      // that work and write nothing).  The columns go 32 at a time (one
+      // group, G % 32 == 0): lane t forms column j0 + t's two terms, a ballot
+      // per cluster gives each summing lane the bitmask of its cluster's
+      // columns in the chunk, and the lane adds those terms in ascending bit
+      // order, fetched by shuffle: the sequential order, in max_q popc steps
+      // per chunk instead of 32.
       const int q = lane & (NQ - 1);
       const bool den = (lane & NQ) != 0;
       double acc = 0.0;
-      for (int g = 0; g < NG; ++g) {
-        const double a = (double)alpha_s[g];
-        const int j1 = (g + 1) * G;
-#pragma unroll 4
-        for (int j = g * G; j < j1; ++j) {
-          const double u = __dmul_rn(a, (double)ex_s[j]);
-          const double t = den ? u : __dmul_rn(u, xs[j]);
-          if (code[j] == q) acc = __dadd_rn(acc, t);
+      for (int j0 = 0; j0 < K; j0 += 32) {
+        const int j = j0 + lane;
+        const double u = __dmul_rn((double)alpha_s[j0 / G], (double)ex_s[j]);
+        const double un = __dmul_rn(u, xs[j]);
+        const int cj = code[j];
+        uint32_t mask = 0;
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) {
+          const uint32_t m = __ballot_sync(kFullMask, cj == qq);
+          if (q == qq) mask = m;
+        }
+        while (__any_sync(kFullMask, mask != 0)) {
+          const int src = mask ? __ffs(mask) - 1 : lane;
+          const double vn = __shfl_sync(kFullMask, un, src);
+          const double vd = __shfl_sync(kFullMask, u, src);
+          if (mask) {
+            acc = __dadd_rn(acc, den ? vd : vn);
+            mask &= mask - 1;
+          }
         }
       }
       const double d = __shfl_down_sync(kFullMask, acc, NQ);
