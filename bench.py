@@ -770,10 +770,24 @@ def nbit_matmul_detail():
 
 
 def profile_shape(name: str, calls: int, op: str = "matmul"):
-    """Run a few calls of one operation (any4_matmul on the auto path, or
-    any4_dequant) on one workload shape: a small, fixed case for ncu."""
+    """Run a few calls of one operation (any4_matmul on the auto path,
+    any4_dequant, or any4_quantize on the first 148 rows of a quantiser
+    matrix, max_iter 20) on one workload shape: a small, fixed case for ncu."""
     import torch
     import learned_bit_lut_any4_b200 as any4
+    if op == "quantize":
+        qs = [q for q in workloads.QUANTIZE_LLAMA3_8B if q.name == name]
+        if not qs:
+            raise SystemExit(f"unknown quantiser matrix {name}")
+        q = qs[0]
+        w = _dev_bf16(workloads.draw_dense_weight(q)[:148])
+        ex = torch.from_numpy(workloads.draw_abs_act_mean(q)).cuda()
+        for _ in range(calls):
+            any4.any4_quantize(w, ex, q.G, max_iter=20)
+        torch.cuda.synchronize()
+        print(f"profiled quantize {name}: 148 of {q.N} rows, K={q.K} G={q.G}, {calls} calls",
+              flush=True)
+        return
     shape = [s for s in workloads.all_shapes() if s.name == name]
     if not shape:
         raise SystemExit(f"unknown shape {name}; known: {[s.name for s in workloads.all_shapes()]}")
@@ -790,6 +804,35 @@ def profile_shape(name: str, calls: int, op: str = "matmul"):
             any4.any4_matmul(x, packed, lut, sc, of, s.G, y=y)
     torch.cuda.synchronize()
     print(f"profiled {op} {name}: M={s.M} K={s.K} N={s.N} G={s.G}, {calls} calls", flush=True)
+
+
+def target_summary(r, nbit, table, peaks):
+    """The headline fractions in one small dict (fractions of the HBM peak
+    for the memory-bound paths, of the bf16 burst peak for prefill)."""
+    def get(d, *ks):
+        for k in ks:
+            if not isinstance(d, dict) or k not in d:
+                return None
+            d = d[k]
+        return d
+    t = {"peak_hbm_gbs": peaks["hbm_gbs"], "peak_bf16_tflops": peaks["bf16_tflops"],
+         "m1_8b_layer_grouped": get(r, "layer_calls", "grouped_4_calls", "frac_hbm"),
+         "m1_8b_layer_7_calls": get(r, "layer_calls", "separate_7_calls", "frac_hbm"),
+         "m1_70b_gate": get(r, "more_m1", "70b_gate_m1", "frac_hbm"),
+         "m1_70b_down": get(r, "more_m1", "70b_down_m1", "frac_hbm"),
+         "m2": get(r, "batch", "sweep_m2", "frac_hbm"),
+         "m4": get(r, "batch", "sweep_m4", "frac_hbm"),
+         "m8": get(r, "batch", "sweep_m8", "frac_hbm"),
+         "m16": get(r, "batch", "sweep_m16", "frac_hbm"),
+         "m8_70b_gate": get(r, "batch", "70b_gate_m8", "frac_hbm"),
+         "dequant_8b_gate": get(nbit, "any4", "frac_hbm"),
+         "prefill_gate_burst": get(r, "prefill", "prefill_gate", "frac_bf16_burst"),
+         "prefill_down_burst": get(r, "prefill", "prefill_down", "frac_bf16_burst")}
+    if isinstance(table, dict) and isinstance(table.get("matrices"), list):
+        for m in table["matrices"]:
+            if m.get("shape") == "8b_down":
+                t["quantize_8b_down_ms"] = m.get("gpu_ms")
+    return t
 
 
 def main():
@@ -814,7 +857,7 @@ def main():
                     help="no timing: run --profile-calls any4_matmul calls on one named "
                          "workload shape (a small, fixed case for ncu captures)")
     ap.add_argument("--profile-calls", type=int, default=3)
-    ap.add_argument("--profile-op", default="matmul", choices=["matmul", "dequant"])
+    ap.add_argument("--profile-op", default="matmul", choices=["matmul", "dequant", "quantize"])
     ap.add_argument("--quantize-detail", action="store_true",
                     help="no step: time any4_quantize on the Llama3-8B matrices (and the "
                          "oracle on a sample of rows) and print one JSON line")
@@ -900,6 +943,9 @@ def main():
             "detail_m1": r["detail"],
             "detail_m1_more": r["more_m1"],
             "prefill_m2048": r["prefill"],
+            # one compact summary of every target figure, last, where the
+            # kept tail of the line always holds it
+            "targets": target_summary(r, nbit, table, peaks),
         }
         print(json.dumps(line), flush=True)
     finally:

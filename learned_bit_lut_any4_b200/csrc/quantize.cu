@@ -25,9 +25,10 @@
 //   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q;
 //   - M-step: sample weight u_j = alpha_{g(j)} * E|x_j| (exact in fp64);
 //     numerator sum(u_j * w_S_j) and denominator sum(u_j) over ascending j,
-//     one lane of warp 0 per cluster and per sum, so the rounding order is the
-//     sequential one (the lane adds only its cluster's columns, found 32 at a
-//     time by warp ballots); a cluster whose weights sum to 0 keeps its entry;
+//     one lane per cluster and per sum (the clusters spread over the warps),
+//     so the rounding order is the sequential one (the lane adds only its
+//     cluster's columns, found 32 at a time by warp ballots); a cluster whose
+//     weights sum to 0 keeps its entry;
 //   - stop after max_iter M-steps, or when an E-step changes no code;
 //   - LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
 //     LUT, packed as one little-endian bit stream per row (code k in bits
@@ -39,13 +40,16 @@
 namespace any4 {
 namespace {
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantWarps = kQuantThreads / 32;
+// Threads per block (one block per row): 256, or 512 when the row's shared
+// memory leaves room for one block per SM only (long rows), so that the one
+// resident block has more warps to hide the M-step's add chains.
+constexpr int kQuantThreadsMax = 512;
+constexpr int kQuantWarpsMax = kQuantThreadsMax / 32;
 
 // Shared-memory layout of one row (K columns, NG = K / G groups, P = the
 // power of two >= K the sort runs over).
 struct QuantSmem {
-  size_t xs, ex, alpha, beta, cent, table, code, total;
+  size_t xs, ex, alpha, beta, cent, table, stage, code, total;
 };
 
 __host__ __device__ inline int64_t pow2_at_least(int64_t K) {
@@ -60,7 +64,8 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G) {
   s.xs = 0;                                            // double [P]
   s.cent = s.xs + 8 * (size_t)pow2_at_least(K);        // double [16]
   s.table = s.cent + 8 * 16;                           // double [16]
-  s.ex = s.table + 8 * 16;                             // float [K]
+  s.stage = s.table + 8 * 16;                          // double2 [warps][32] (M-step)
+  s.ex = s.stage + 16 * 32 * kQuantWarpsMax;           // float [K]
   s.alpha = s.ex + 4 * (size_t)K;                      // float [NG]
   s.beta = s.alpha + 4 * (size_t)NG;                   // float [NG]
   s.code = s.beta + 4 * (size_t)NG;                    // uint8 [K]
@@ -79,7 +84,7 @@ __device__ __forceinline__ double scaled_weight(float w, float alpha, float beta
 
 // E-step over the row: nearest of the NQ entries of c (ties to the lowest
 // index).  Returns (uniformly across the block) whether any code changed.
-template <int NQ>
+template <int NQ, int kQuantThreads>
 __device__ __forceinline__ bool estep(const double* xs, int K, const double* c, uint8_t* code) {
   double cr[NQ];
 #pragma unroll
@@ -104,12 +109,13 @@ __device__ __forceinline__ bool estep(const double* xs, int K, const double* c, 
 }
 
 // NQ = 2^n table entries (4, 8 or 16); the packed row has n K / 8 bytes.
-template <int NQ>
+template <int NQ, int kQuantThreads>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, int K, int G,
                 int max_iter, uint8_t* __restrict__ packed, uint16_t* __restrict__ lut,
                 uint16_t* __restrict__ scale, uint16_t* __restrict__ offset,
                 int32_t* __restrict__ iters) {
+  constexpr int kQuantWarps = kQuantThreads / 32;
   extern __shared__ __align__(16) unsigned char smem[];
   const QuantSmem L = quant_smem_layout(K, G);
   double* xs = reinterpret_cast<double*>(smem + L.xs);
@@ -119,6 +125,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   float* alpha_s = reinterpret_cast<float*>(smem + L.alpha);
   float* beta_s = reinterpret_cast<float*>(smem + L.beta);
   uint8_t* code = smem + L.code;
+  double2* stage = reinterpret_cast<double2*>(smem + L.stage);
 
   const int64_t n = blockIdx.x;
   const int NG = K / G;
@@ -182,48 +189,63 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
     xs[j] = scaled_weight(bf16_canon(wrow[j]), alpha_s[j / G], beta_s[j / G]);
   __syncthreads();
 
-  estep<NQ>(xs, K, cent, code);
+  estep<NQ, kQuantThreads>(xs, K, cent, code);
   int it = 0;
   while (it < max_iter) {
-    if (warp == 0) {
-      // Eq. 23: lane q sums u_j * w_S_j and lane NQ + q sums u_j over the
-      // columns of cluster q in ascending order (lanes from 2 NQ up repeat
-      // that work and write nothing).  The columns go 32 at a time (one
-      // group, G % 32 == 0): lane t forms column j0 + t's two terms, a ballot
-      // per cluster gives each summing lane the bitmask of its cluster's
-      // columns in the chunk, and the lane adds those terms in ascending bit
-      // order, fetched by shuffle: the sequential order, in max_q popc steps
-      // per chunk instead of 32.
-      const int q = lane & (NQ - 1);
-      const bool den = (lane & NQ) != 0;
-      double acc = 0.0;
-      for (int j0 = 0; j0 < K; j0 += 32) {
-        const int j = j0 + lane;
-        const double u = __dmul_rn((double)alpha_s[j0 / G], (double)ex_s[j]);
-        const double un = __dmul_rn(u, xs[j]);
-        const int cj = code[j];
-        uint32_t mask = 0;
+    {
+      // Eq. 23, every warp at once: warp w owns clusters q0 .. q0 + QPW - 1;
+      // lane i < QPW sums u_j * w_S_j and lane 16 + i sums u_j over the
+      // columns of cluster q0 + i in ascending order.  The columns go 32 at a
+      // time (one group, G % 32 == 0): lane t puts column j0 + t's two terms
+      // in the warp's staging row, a ballot per cluster gives each summing
+      // lane the bitmask of its cluster's columns in the chunk, and the lane
+      // adds those terms in ascending bit order: the sequential order, in
+      // max popc steps per chunk instead of 32.
+      constexpr int QPW = NQ >= kQuantWarps ? NQ / kQuantWarps : 1;  // clusters per warp
+      const int q0 = warp * QPW;
+      const int qi = lane & 15;
+      const bool owner = qi < QPW;
+      const int q = q0 + (owner ? qi : 0);
+      const bool den = lane >= 16;
+      double2* st = stage + warp * 32;
+      if (q0 < NQ) {  // warp-uniform
+        double acc = 0.0;
+        for (int j0 = 0; j0 < K; j0 += 32) {
+          const int j = j0 + lane;
+          const double u = __dmul_rn((double)alpha_s[j0 / G], (double)ex_s[j]);
+          st[lane] = make_double2(__dmul_rn(u, xs[j]), u);
+          const int cj = code[j];
+          uint32_t mask = 0;
 #pragma unroll
-        for (int qq = 0; qq < NQ; ++qq) {
-          const uint32_t m = __ballot_sync(kFullMask, cj == qq);
-          if (q == qq) mask = m;
-        }
-        while (__any_sync(kFullMask, mask != 0)) {
-          const int src = mask ? __ffs(mask) - 1 : lane;
-          const double vn = __shfl_sync(kFullMask, un, src);
-          const double vd = __shfl_sync(kFullMask, u, src);
-          if (mask) {
-            acc = __dadd_rn(acc, den ? vd : vn);
-            mask &= mask - 1;
+          for (int i = 0; i < QPW; ++i) {
+            const uint32_t m = __ballot_sync(kFullMask, cj == q0 + i);
+            if (owner && qi == i) mask = m;
           }
+          __syncwarp();
+          // up to four terms per round: their loads go out together, then
+          // the adds follow in ascending column order
+          const double* sv = reinterpret_cast<const double*>(st) + (den ? 1 : 0);
+          while (mask) {
+            // the term of the lowest set bit, or 0 past the last (exact: x + 0
+            // is x for every x the sums hold, none of them -0)
+            auto take = [&]() -> double {
+              if (!mask) return 0.0;
+              const double v = sv[2 * (__ffs(mask) - 1)];
+              mask &= mask - 1;
+              return v;
+            };
+            const double v0 = take(), v1 = take(), v2 = take(), v3 = take();
+            acc = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc, v0), v1), v2), v3);
+          }
+          __syncwarp();
         }
+        const double d = __shfl_down_sync(kFullMask, acc, 16);
+        if (owner && !den && d > 0.0) cent[q] = __ddiv_rn(acc, d);
       }
-      const double d = __shfl_down_sync(kFullMask, acc, NQ);
-      if (lane < NQ && d > 0.0) cent[q] = __ddiv_rn(acc, d);
     }
     __syncthreads();
     ++it;
-    if (!estep<NQ>(xs, K, cent, code)) break;
+    if (!estep<NQ, kQuantThreads>(xs, K, cent, code)) break;
   }
 
   if (tid < NQ) {
@@ -233,7 +255,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   }
   if (tid == 0 && iters) iters[n] = it;
   __syncthreads();
-  estep<NQ>(xs, K, table, code);
+  estep<NQ, kQuantThreads>(xs, K, table, code);
 
   // Pack 32 codes (BITS words) per thread step; K % 32 == 0.
   constexpr int BITS = NQ == 16 ? 4 : (NQ == 8 ? 3 : 2);
@@ -265,10 +287,18 @@ any4_status launch_quantize_nq(const uint16_t* w, const float* ex, int64_t N, in
                                int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
                                uint16_t* scale, uint16_t* offset, int32_t* iters, size_t smem,
                                cudaStream_t stream) {
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(quantize_kernel<NQ>), smem) != ANY4_OK)
-    return ANY4_ERR_CUDA;
-  quantize_kernel<NQ><<<(unsigned)N, kQuantThreads, smem, stream>>>(
-      w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
+  // long rows: one block fits per SM, give it 512 threads; else 256 threads
+  // and several blocks (rows) per SM
+  const bool wide = 2 * (smem + 1024) > (size_t)228 * 1024;
+  const void* kern = wide ? reinterpret_cast<const void*>(quantize_kernel<NQ, 512>)
+                          : reinterpret_cast<const void*>(quantize_kernel<NQ, 256>);
+  if (ensure_dynamic_smem(kern, smem) != ANY4_OK) return ANY4_ERR_CUDA;
+  if (wide)
+    quantize_kernel<NQ, 512><<<(unsigned)N, 512, smem, stream>>>(
+        w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
+  else
+    quantize_kernel<NQ, 256><<<(unsigned)N, 256, smem, stream>>>(
+        w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
