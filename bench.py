@@ -682,21 +682,22 @@ def table_learning_detail(max_iter: int, cpu_seconds: float, reps: int = 3):
     return out
 
 
-def nbit_dequant_detail(reps: int = 10):
+def nbit_dequant_detail():
     """Time any4_dequant_bits for n = 2, 3, 4 on the Llama3-8B gate matrix
-    (4096 -> 14336, G = 128), L2 flushed before each call: HBM GB/s of the
-    algorithmic bytes (codes, scales, offsets and tables read, bf16 W written)."""
+    (4096 -> 14336, G = 128) on rotating weight copies larger than L2, replayed
+    in a CUDA graph (events on its stream): HBM GB/s of the algorithmic bytes
+    (codes, scales, offsets and tables read, bf16 W written)."""
     import torch
     import learned_bit_lut_any4_b200 as any4
     peaks = load_peaks()
     N, K, G = 14336, 4096, 128
     rng = np.random.default_rng(4600)
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
-    W = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.Stream()
     out = {"N": N, "K": K, "G": G}
     for bits in (2, 3, 4):
         nq = 1 << bits
+        alg = N * K * bits // 8 + 4 * N * (K // G) + 2 * nq * N + 2 * N * K
+        copies = max(2, int(np.ceil(3 * L2_BYTES / alg)))
         packed = torch.from_numpy(rng.integers(0, 256, size=(N, bits * K // 8),
                                                dtype=np.uint8)).cuda()
         lut = _dev_bf16(workloads._to_bf16_bits(rng.normal(0, 0.5, (N, nq)).astype(np.float32)))
@@ -704,23 +705,16 @@ def nbit_dequant_detail(reps: int = 10):
             (np.abs(rng.normal(0, 0.01, (N, K // G))) + 1e-3).astype(np.float32)))
         offset = _dev_bf16(workloads._to_bf16_bits(
             rng.normal(0, 0.002, (N, K // G)).astype(np.float32)))
-        any4.any4_dequant_bits(packed, lut, scale, offset, G, bits, W=W)
-        times = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            any4.any4_dequant_bits(packed, lut, scale, offset, G, bits, W=W)
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b) * 1e3)
-        us = float(np.median(times))
-        alg = N * K * bits // 8 + 4 * N * (K // G) + 2 * nq * N + 2 * N * K
+        reps = [(packed, lut, scale, offset)] + [
+            (packed.clone(), lut.clone(), scale.clone(), offset.clone()) for _ in range(copies - 1)]
+        Ws = [torch.empty((N, K), dtype=torch.bfloat16, device="cuda") for _ in range(copies)]
+        calls = [(lambda w=w, W=W: any4.any4_dequant_bits(w[0], w[1], w[2], w[3], G, bits, W=W))
+                 for w, W in zip(reps, Ws)]
+        us = _time_graph(stream, calls, max(2, 100 // copies))
         out[f"any{bits}"] = {"us": round(us, 2), "GB/s": round(alg / us / 1e3, 1),
                              "frac_hbm": round(alg / us / 1e3 / peaks["hbm_gbs"], 4)}
-        del packed, lut, scale, offset
-    del flush, W
-    torch.cuda.synchronize()
+        del reps, Ws, packed, lut, scale, offset
+        torch.cuda.synchronize()
     return out
 
 

@@ -298,9 +298,9 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         const uint16_t* of = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot +
                                                                St::kGrpBytes);
         // The stage's rows a pair at a time (rows 2pp, 2pp+1 share the tensor-core
-        // steps), so that few registers stay live and many warps fit per SM;
-        // each pair accumulates in two chains (even and odd steps) to halve the
-        // dependent-MMA latency.
+        // steps), two pairs interleaved per loop step (more independent work per
+        // warp within the same 96 registers); each pair accumulates in two
+        // chains (even and odd steps) to halve the dependent-MMA latency.
         constexpr int NP = P / 2;
         float part[P];
 #pragma unroll
@@ -311,7 +311,7 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         // a block may be partly past its rows)
         const int rows_left = nrows - si * P;
         const int npairs = rows_left >= P ? NP : (rows_left + 1) / 2;
-#pragma unroll 1
+#pragma unroll(BITS == 3 ? 1 : 2)  // 3-bit codes: the funnel shifts leave no room
         for (int pp = 0; pp < npairs; ++pp) {
           const int ja = 2 * pp, jb = 2 * pp + 1;
           const bool va = ja < rows_left, vb = jb < rows_left;

@@ -42,9 +42,9 @@ namespace {
 
 // Threads per block (one block per row): 256, or 512 when the row's shared
 // memory leaves room for one block per SM only (long rows), so that the one
-// resident block has more warps to hide the M-step's add chains.
+// resident block has more warps to hide the M-step's add chains; the staging
+// row is sized for the larger count.
 constexpr int kQuantThreadsMax = 512;
-constexpr int kQuantWarpsMax = kQuantThreadsMax / 32;
 
 // Shared-memory layout of one row (K columns, NG = K / G groups, P = the
 // power of two >= K the sort runs over).
@@ -64,8 +64,8 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G) {
   s.xs = 0;                                            // double [P]
   s.cent = s.xs + 8 * (size_t)pow2_at_least(K);        // double [16]
   s.table = s.cent + 8 * 16;                           // double [16]
-  s.stage = s.table + 8 * 16;                          // double2 [warps][32] (M-step)
-  s.ex = s.stage + 16 * 32 * kQuantWarpsMax;           // float [K]
+  s.stage = s.table + 8 * 16;                          // double2 [threads] (M-step)
+  s.ex = s.stage + 16 * (size_t)kQuantThreadsMax;      // float [K]
   s.alpha = s.ex + 4 * (size_t)K;                      // float [NG]
   s.beta = s.alpha + 4 * (size_t)NG;                   // float [NG]
   s.code = s.beta + 4 * (size_t)NG;                    // uint8 [K]
@@ -193,55 +193,54 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   int it = 0;
   while (it < max_iter) {
     {
-      // Eq. 23, every warp at once: warp w owns clusters q0 .. q0 + QPW - 1;
-      // lane i < QPW sums u_j * w_S_j and lane 16 + i sums u_j over the
-      // columns of cluster q0 + i in ascending order.  The columns go 32 at a
-      // time (one group, G % 32 == 0): lane t puts column j0 + t's two terms
-      // in the warp's staging row, a ballot per cluster gives each summing
-      // lane the bitmask of its cluster's columns in the chunk, and the lane
-      // adds those terms in ascending bit order: the sequential order, in
-      // max popc steps per chunk instead of 32.
+      // Eq. 23, every warp at once: warp w owns clusters q0 .. q0 + QPW - 1,
+      // its lane i < QPW sums u_j * w_S_j (num) and u_j (den) of cluster
+      // q0 + i over ascending j.  The columns go one block-wide batch at a
+      // time: each thread stages one column's two terms in shared memory;
+      // then, 32 columns at a time (one group, G % 32 == 0), a warp ballot per
+      // cluster gives each summing lane the bitmask of its cluster's columns,
+      // and the lane adds those terms in ascending bit order, four loads per
+      // round: the sequential order, each term formed once for the block.
       constexpr int QPW = NQ >= kQuantWarps ? NQ / kQuantWarps : 1;  // clusters per warp
       const int q0 = warp * QPW;
-      const int qi = lane & 15;
-      const bool owner = qi < QPW;
-      const int q = q0 + (owner ? qi : 0);
-      const bool den = lane >= 16;
-      double2* st = stage + warp * 32;
-      if (q0 < NQ) {  // warp-uniform
-        double acc = 0.0;
-        for (int j0 = 0; j0 < K; j0 += 32) {
-          const int j = j0 + lane;
-          const double u = __dmul_rn((double)alpha_s[j0 / G], (double)ex_s[j]);
-          st[lane] = make_double2(__dmul_rn(u, xs[j]), u);
-          const int cj = code[j];
-          uint32_t mask = 0;
-#pragma unroll
-          for (int i = 0; i < QPW; ++i) {
-            const uint32_t m = __ballot_sync(kFullMask, cj == q0 + i);
-            if (owner && qi == i) mask = m;
-          }
-          __syncwarp();
-          // up to four terms per round: their loads go out together, then
-          // the adds follow in ascending column order
-          const double* sv = reinterpret_cast<const double*>(st) + (den ? 1 : 0);
-          while (mask) {
-            // the term of the lowest set bit, or 0 past the last (exact: x + 0
-            // is x for every x the sums hold, none of them -0)
-            auto take = [&]() -> double {
-              if (!mask) return 0.0;
-              const double v = sv[2 * (__ffs(mask) - 1)];
-              mask &= mask - 1;
-              return v;
-            };
-            const double v0 = take(), v1 = take(), v2 = take(), v3 = take();
-            acc = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc, v0), v1), v2), v3);
-          }
-          __syncwarp();
+      const bool owner = lane < QPW && q0 < NQ;
+      double acc_n = 0.0, acc_d = 0.0;
+      for (int b0 = 0; b0 < K; b0 += kQuantThreads) {
+        const int jb = b0 + tid;
+        if (jb < K) {
+          const double u = __dmul_rn((double)alpha_s[jb / G], (double)ex_s[jb]);
+          stage[tid] = make_double2(__dmul_rn(u, xs[jb]), u);
         }
-        const double d = __shfl_down_sync(kFullMask, acc, 16);
-        if (owner && !den && d > 0.0) cent[q] = __ddiv_rn(acc, d);
+        __syncthreads();
+        if (q0 < NQ) {  // warp-uniform
+          const int ncols = min(kQuantThreads, K - b0);  // a multiple of 32
+          for (int c0 = 0; c0 < ncols; c0 += 32) {
+            const int cj = code[b0 + c0 + lane];
+            uint32_t mask = 0;
+#pragma unroll
+            for (int i = 0; i < QPW; ++i) {
+              const uint32_t m = __ballot_sync(kFullMask, cj == q0 + i);
+              if (lane == i) mask = m;
+            }
+            const double2* sv = stage + c0;
+            while (mask) {
+              // the terms of the lowest set bit, or 0 past the last (exact:
+              // x + 0 is x for every x these sums hold, none of them -0)
+              auto take = [&]() -> double2 {
+                if (!mask) return make_double2(0.0, 0.0);
+                const double2 v = sv[__ffs(mask) - 1];
+                mask &= mask - 1;
+                return v;
+              };
+              const double2 v0 = take(), v1 = take(), v2 = take(), v3 = take();
+              acc_n = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_n, v0.x), v1.x), v2.x), v3.x);
+              acc_d = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_d, v0.y), v1.y), v2.y), v3.y);
+            }
+          }
+        }
+        __syncthreads();  // the batch's terms have been read
       }
+      if (owner && acc_d > 0.0) cent[q0 + lane] = __ddiv_rn(acc_n, acc_d);
     }
     __syncthreads();
     ++it;
