@@ -81,22 +81,6 @@ pack_bits_kernel(const uint8_t* __restrict__ idx, uint8_t* __restrict__ packed, 
   }
 }
 
-// Table entry `code` of a row table held as bf16 pairs in registers: t0..t3
-// hold entries (0,1) (2,3) (4,5) (6,7); with 4 entries only t0, t1 are used.
-template <int BITS>
-__device__ __forceinline__ float table_entry(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
-                                             uint32_t code) {
-  const uint32_t e = code & 3u;
-  const uint32_t sel = (2u * e) | ((2u * e + 1u) << 4);   // bytes 2e, 2e+1 of the pair
-  uint32_t v;
-  if constexpr (BITS == 3) {
-    v = (code & 4u) ? __byte_perm(t2, t3, sel) : __byte_perm(t0, t1, sel);
-  } else {
-    v = __byte_perm(t0, t1, sel);
-  }
-  return __uint_as_float(v << 16);
-}
-
 // dequant: one warp per 1024-column segment of a row, lane l on the segment's
 // 32-code chunk l (its n words are the n * 4 bytes after lane l - 1's, so the
 // warp's code loads are contiguous).  The loads of the warp's next segment
@@ -122,6 +106,7 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
                     const uint16_t* __restrict__ offset, uint16_t* __restrict__ W, int64_t N,
                     int K, int G, int g_shift) {
   __shared__ __align__(128) uint16_t s_out[kNbWarps][kNbSeg];
+  __shared__ float s_lut[kNbWarps][8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int segs_per_row = (K + kNbSeg - 1) / kNbSeg;
   const int64_t nseg = N * segs_per_row;
@@ -141,21 +126,16 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
     }
   };
   // one segment's inputs, per lane
+  constexpr int NQ = 1 << BITS;
   struct Seg {
     uint32_t v[BITS];
-    uint32_t t[BITS == 3 ? 4 : 2];  // the row's table as bf16 pairs
-    uint32_t so;                    // scale (low half) and offset (high half)
+    uint32_t lv;  // lanes 0 .. NQ-1: entry `lane` of the row's table (bf16 bits)
+    uint32_t so;  // scale (low half) and offset (high half)
   };
   auto load = [&](int64_t n, int seg, Seg& d) {
     const int col0 = seg * kNbSeg;
     const int k0 = col0 + 32 * lane;
-    if constexpr (BITS == 3) {
-      const uint4 t = __ldg(reinterpret_cast<const uint4*>(lut + n * lut_row_stride));
-      d.t[0] = t.x; d.t[1] = t.y; d.t[2] = t.z; d.t[3] = t.w;
-    } else {
-      const uint2 t = __ldg(reinterpret_cast<const uint2*>(lut + n * lut_row_stride));
-      d.t[0] = t.x; d.t[1] = t.y;
-    }
+    d.lv = lane < NQ ? (uint32_t)ldg_u16(lut + n * lut_row_stride + lane) : 0u;
 #pragma unroll
     for (int b = 0; b < BITS; ++b) d.v[b] = 0u;
     d.so = 0u;
@@ -171,6 +151,7 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
   Seg nxt;
   load(ln, lseg, nxt);
   advance(ln, lseg);
+  int64_t cur_row = -1;
   for (int64_t sg = first; sg < nseg; sg += stride) {
     const int col0 = seg * kNbSeg;
     const int cols = min(kNbSeg, K - col0);  // a multiple of 32
@@ -180,21 +161,22 @@ dequant_bits_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restri
       load(ln, lseg, nxt);
       advance(ln, lseg);
     }
-    const uint32_t t0 = cur.t[0], t1 = cur.t[1];
-    const uint32_t t2 = BITS == 3 ? cur.t[BITS == 3 ? 2 : 0] : 0u;
-    const uint32_t t3 = BITS == 3 ? cur.t[BITS == 3 ? 3 : 1] : 0u;
+    uint16_t* seg_out = s_out[warp];
+    float* tab = s_lut[warp];
+    __syncwarp();  // the previous segment's row and table have been read
+    if (n != cur_row) {  // a new row: its table as fp32 in shared memory
+      if (lane < NQ) tab[lane] = bf16_lo_to_f32(cur.lv);
+      __syncwarp();
+      cur_row = n;
+    }
     const float s = bf16_lo_to_f32(cur.so), o = bf16_hi_to_f32(cur.so);
     uint32_t out[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
-      const float lo =
-          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(cur.v, 2 * p)), s, o);
-      const float hi =
-          __fmaf_rn(table_entry<BITS>(t0, t1, t2, t3, code_of<BITS>(cur.v, 2 * p + 1)), s, o);
+      const float lo = __fmaf_rn(tab[code_of<BITS>(cur.v, 2 * p)], s, o);
+      const float hi = __fmaf_rn(tab[code_of<BITS>(cur.v, 2 * p + 1)], s, o);
       out[p] = pack_bf16x2_rn(lo, hi);
     }
-    uint16_t* seg_out = s_out[warp];
-    __syncwarp();  // the previous segment's row has been read back
     if (on) {
 #pragma unroll
       for (int step = 0; step < 4; ++step) {
