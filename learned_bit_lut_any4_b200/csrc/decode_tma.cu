@@ -298,9 +298,12 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         const uint16_t* of = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot +
                                                                St::kGrpBytes);
         // The stage's rows a pair at a time (rows 2pp, 2pp+1 share the tensor-core
-        // steps), two pairs interleaved per loop step (more independent work per
-        // warp within the same 96 registers); each pair accumulates in two
-        // chains (even and odd steps) to halve the dependent-MMA latency.
+        // steps), the pair loop unrolled so that the pairs' work interleaves and
+        // the per-pair slots of part[] are fixed registers; each pair
+        // accumulates in two chains (even and odd steps) to halve the
+        // dependent-MMA latency.  A stage's rows past the matrix come back as
+        // zeros from the tensor loads, and rows past the block's last are
+        // computed and dropped, so the code loads need no row test.
         constexpr int NP = P / 2;
         float part[P];
 #pragma unroll
@@ -311,31 +314,27 @@ __global__ void __maxnreg__(96) decode_tma_kernel(
         // a block may be partly past its rows)
         const int rows_left = nrows - si * P;
         const int npairs = rows_left >= P ? NP : (rows_left + 1) / 2;
-#pragma unroll(BITS == 3 ? 1 : 2)  // 3-bit codes: the funnel shifts leave no room
-        for (int pp = 0; pp < npairs; ++pp) {
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp) {
+          if (pp >= npairs) break;
           const int ja = 2 * pp, jb = 2 * pp + 1;
-          const bool va = ja < rows_left, vb = jb < rows_left;
           // the lane's 32 codes of each row: BITS consecutive words
           uint32_t wa[BITS], wb[BITS];
           if constexpr (BITS == 4) {
-            const uint4 qa = va ? reinterpret_cast<const uint4*>(codes)[ja * 32 + lane]
-                                : make_uint4(0u, 0u, 0u, 0u);
-            const uint4 qb = vb ? reinterpret_cast<const uint4*>(codes)[jb * 32 + lane]
-                                : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 qa = reinterpret_cast<const uint4*>(codes)[ja * 32 + lane];
+            const uint4 qb = reinterpret_cast<const uint4*>(codes)[jb * 32 + lane];
             wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
             wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
           } else if constexpr (BITS == 2) {
-            const uint2 qa = va ? reinterpret_cast<const uint2*>(codes)[ja * 32 + lane]
-                                : make_uint2(0u, 0u);
-            const uint2 qb = vb ? reinterpret_cast<const uint2*>(codes)[jb * 32 + lane]
-                                : make_uint2(0u, 0u);
+            const uint2 qa = reinterpret_cast<const uint2*>(codes)[ja * 32 + lane];
+            const uint2 qb = reinterpret_cast<const uint2*>(codes)[jb * 32 + lane];
             wa[0] = qa.x; wa[1] = qa.y;
             wb[0] = qb.x; wb[1] = qb.y;
           } else {
 #pragma unroll
             for (int b = 0; b < BITS; ++b) {
-              wa[b] = va ? codes[(ja * 32 + lane) * BITS + b] : 0u;
-              wb[b] = vb ? codes[(jb * 32 + lane) * BITS + b] : 0u;
+              wa[b] = codes[(ja * 32 + lane) * BITS + b];
+              wb[b] = codes[(jb * 32 + lane) * BITS + b];
             }
           }
           const uint32_t la = lut_shared ? lv_shared : (uint32_t)lt[ja * NE + (lane & (NE - 1))];
