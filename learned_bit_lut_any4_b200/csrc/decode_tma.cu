@@ -530,6 +530,10 @@ any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_
   }
   const int64_t wave = (int64_t)dev.sm_count * per_sm;
   rt = std::min<int64_t>((total_rows + wave - 1) / wave, kMaxRT);
+  // at least 4 rows a block: below that a block's fixed costs (barriers, its
+  // x loads, the partial-sum pass) outweigh its rows (1024-row matrices ran
+  // 25 % faster with 4 rows a block than with the 2 that one wave gives)
+  rt = std::max<int64_t>(rt, 4);
   // 2-bit tables come by a 1-D tensor load at element 4 r of the table
   // array: its byte offset 8 r must be a multiple of 16, so every stage's
   // first row r (row0 + a multiple of P) must be even, hence rt even
