@@ -81,6 +81,7 @@ __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int 
 
 struct TmaMaps {
   CUtensorMap codes;   // u32 [N][K/8], box {128, P}
+  CUtensorMap codes_head;  // the same, box {128, head_rows}
   CUtensorMap lut;     // bf16 [N][16], box {16, P}
   CUtensorMap scale;   // bf16 [N][K/G], box {1024/G, P}
   CUtensorMap offset;  // bf16 [N][K/G], box {1024/G, P}
@@ -98,6 +99,7 @@ struct TmaGroup {
   int N[kTmaMaxGroup];
   int64_t blk_end[kTmaMaxGroup];
   int count;
+  int head_rows;  // rows of a slice's first stage (folded-table kernel), 1..P
 };
 
 // D += A * B, m16n8k16 bf16 -> fp32 (legacy warp-level tensor-core MMA).
@@ -468,7 +470,12 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   const int RT = rows_per_block;
-  const int RTP = ((RT + P - 1) / P) * P;
+  // A slice's stages: head_rows rows (the block's rows modulo P, or P),
+  // then P rows each, so that a block's one short stage comes first and
+  // every later stage is full.
+  const int H = grp.head_rows;
+  const int RTP = RT <= H ? H : H + ((RT - H + P - 1) / P) * P;
+  auto stage_row = [H](int si) { return si == 0 ? 0 : H + (si - 1) * P; };
   const uint32_t base = (smem_addr(smem_raw) + 127u) & ~127u;
   uint8_t* gbase = smem_raw + (base - smem_addr(smem_raw));
   const uint32_t ring = base + (uint32_t)(warp * S * St::kBytes);
@@ -505,7 +512,7 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
     const uint16_t* lut_shared = grp.lut_shared[mi];
     const int row0 = (int)((blk - (mi > 0 ? grp.blk_end[mi - 1] : 0)) * RT);
     const int nrows = (N - row0) < RT ? (N - row0) : RT;
-    const int nstages = (nrows + P - 1) / P;
+    const int nstages = nrows <= H ? 1 : 1 + (nrows - H + P - 1) / P;
     bool first_slice = true;
     for (int s = warp; s < nslices && ok; s += nwarps) {
       auto issue = [&](int stage_idx) {
@@ -517,10 +524,11 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
         const int st = (int)(it_issue % S);
         const uint32_t dst = ring + (uint32_t)(st * St::kBytes);
         const uint32_t bar = bars + 8u * st;
-        const int r = row0 + stage_idx * P;
+        const int r = row0 + stage_row(stage_idx);
+        const uint32_t tx = stage_idx == 0 ? St::kTx - (uint32_t)((P - H) * kRowWords * 4) : St::kTx;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     :: "r"(bar), "r"(St::kTx) : "memory");
-        tma2d(dst, &maps.codes, s * kRowWords, r, bar);
+                     :: "r"(bar), "r"(tx) : "memory");
+        tma2d(dst, stage_idx == 0 ? &maps.codes_head : &maps.codes, s * kRowWords, r, bar);
         tma2d(dst + St::kCodeBytes, &maps.lut, 0, r, bar);
         tma2d(dst + St::kCodeBytes + St::kLutSlot, &maps.scale, s * GPS, r, bar);
         tma2d(dst + St::kCodeBytes + St::kLutSlot + St::kGrpBytes, &maps.offset, s * GPS, r,
@@ -590,7 +598,7 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
           return (a0.x + a0.y) + (a1.x + a1.y);
         };
         float part[P];
-        const int rows_left = nrows - si * P;
+        const int rows_left = si == 0 ? (nrows < H ? nrows : H) : nrows - stage_row(si);
         if (rows_left >= P) {
 #pragma unroll
           for (int j = 0; j < P; ++j) part[j] = row(j);
@@ -605,9 +613,9 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
           issue(si + S);
         }
         const float tot = reduce8(part, lane);
-        if ((lane & 3) == 0) {
-          const int idx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-          float* dst = s_part + (size_t)warp * RTP + si * P + idx;
+        const int idx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+        if ((lane & 3) == 0 && idx < (si == 0 ? H : P)) {
+          float* dst = s_part + (size_t)warp * RTP + stage_row(si) + idx;
           *dst = first_slice ? tot : *dst + tot;
         }
       }
@@ -687,13 +695,15 @@ bool encode1d(EncodeFn enc, CUtensorMap* m, const void* ptr, uint64_t n, uint32_
 }
 
 bool encode_weights(EncodeFn enc, TmaMaps* maps, const DecodeWeights& w, int64_t K, int64_t G,
-                    int GPS, int bits) {
+                    int GPS, int bits, int head_rows) {
   constexpr int P = kTmaRows;
   const uint64_t N = (uint64_t)w.N;
   const uint32_t ne = 1u << bits;
   // codes as u32 [N][K bits / 32]: 1024 codes of a row = 32 * bits words
   if (!encode2d(enc, &maps->codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, w.packed,
                 (uint64_t)K * bits / 32, N, (uint64_t)K * bits / 8, 32 * bits, P) ||
+      !encode2d(enc, &maps->codes_head, CU_TENSOR_MAP_DATA_TYPE_UINT32, w.packed,
+                (uint64_t)K * bits / 32, N, (uint64_t)K * bits / 8, 32 * bits, head_rows) ||
       !encode2d(enc, &maps->scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.scale, (uint64_t)(K / G), N,
                 (uint64_t)(K / G) * 2, GPS, P) ||
       !encode2d(enc, &maps->offset, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.offset, (uint64_t)(K / G),
@@ -721,15 +731,7 @@ any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_
   TmaGroup grp;
   memset(&grp, 0, sizeof(grp));
   int64_t total_rows = 0;
-  for (int i = 0; i < count; ++i) {
-    if (!encode_weights(enc, &grp.maps[i], w[i], K, G, GPS, BITS)) return ANY4_ERR_CUDA;
-    grp.y[i] = w[i].y;
-    grp.y32[i] = w[i].y32;
-    grp.lut_shared[i] = w[i].lut_row_stride == 0 ? w[i].lut : nullptr;
-    grp.N[i] = (int)w[i].N;
-    total_rows += w[i].N;
-  }
-  grp.count = count;
+  for (int i = 0; i < count; ++i) total_rows += w[i].N;
   const int nslices = (int)((K + 1023) / 1024);
   const int per_warp = (nslices + kTmaMaxWarps - 1) / kTmaMaxWarps;
   const int nwarps = (nslices + per_warp - 1) / per_warp;
@@ -770,6 +772,18 @@ any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_
   // first row r (row0 + a multiple of P) must be even, hence rt even
   if (BITS == 2 && (rt & 1)) ++rt;
   rtp = ((rt + P - 1) / P) * P;
+  // the folded-table kernel's first stage per slice: rt mod P rows (or P)
+  const int head_rows = kFold && rt % P != 0 ? (int)(rt % P) : P;
+  for (int i = 0; i < count; ++i) {
+    if (!encode_weights(enc, &grp.maps[i], w[i], K, G, GPS, BITS, head_rows))
+      return ANY4_ERR_CUDA;
+    grp.y[i] = w[i].y;
+    grp.y32[i] = w[i].y32;
+    grp.lut_shared[i] = w[i].lut_row_stride == 0 ? w[i].lut : nullptr;
+    grp.N[i] = (int)w[i].N;
+  }
+  grp.count = count;
+  grp.head_rows = head_rows;
   int64_t nblocks = 0;
   for (int i = 0; i < count; ++i) {
     nblocks += (w[i].N + rt - 1) / rt;
