@@ -74,7 +74,7 @@ def kernel_source_hash() -> str:
 def stored_traffic():
     """Per-launch DRAM bytes (read + write) of the decode kernel on this step,
     from the committed ncu summary, if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_tma_kernel_llama3_8b_layer_m1.md")
+    path = os.path.join(ROOT, "profiles", "decode_tma_ffma_kernel_llama3_8b_layer_m1.md")
     try:
         text = open(path).read()
     except OSError:
@@ -904,7 +904,7 @@ def main():
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": stored_traffic(),
-                    "kernel": "decode_tma_kernel<8> (the only kernel of the step)",
+                    "kernel": "decode_tma_ffma_kernel (the only kernel of the step)",
                     "peak_source": peaks.get("source", "measured")}
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
