@@ -26,6 +26,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cstring>
 #include <mutex>
 
@@ -569,14 +570,20 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot);
         const uint16_t* of = reinterpret_cast<const uint16_t*>(sp + St::kCodeBytes + St::kLutSlot +
                                                                St::kGrpBytes);
-        // one row of the stage: the lane's sum over its 32 columns
-        auto row = [&](int j) -> float {
+        // one row of the stage: the lane's sum over its 32 columns (shared:
+        // the matrix has one table, held in lv_shared; the choice is made
+        // once per stage, outside the unrolled rows)
+        auto row = [&](int j, auto shared) -> float {
           uint32_t w[4];
           w[0] = codes[j * kRowWords + wofs0];
           w[1] = codes[j * kRowWords + wofs1];
           w[2] = codes[j * kRowWords + wofs0 + 32];
           w[3] = codes[j * kRowWords + wofs1 + 32];
-          const uint32_t l2 = lut_shared ? lv_shared : dup2(lt[j * NE + e]);
+          uint32_t l2;
+          if constexpr (decltype(shared)::value)
+            l2 = lv_shared;
+          else
+            l2 = dup2(lt[j * NE + e]);
           const uint2 s4 = *reinterpret_cast<const uint2*>(sc + j * GPS + 4 * h);
           const uint2 o4 = *reinterpret_cast<const uint2*>(of + j * GPS + 4 * h);
           const uint32_t t01 = hfma2_bits(l2, s4.x, o4.x), t23 = hfma2_bits(l2, s4.y, o4.y);
@@ -599,13 +606,19 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
         };
         float part[P];
         const int rows_left = si == 0 ? (nrows < H ? nrows : H) : nrows - stage_row(si);
-        if (rows_left >= P) {
+        auto rows = [&](auto shared) {
+          if (rows_left >= P) {
 #pragma unroll
-          for (int j = 0; j < P; ++j) part[j] = row(j);
-        } else {
+            for (int j = 0; j < P; ++j) part[j] = row(j, shared);
+          } else {
 #pragma unroll
-          for (int j = 0; j < P; ++j) part[j] = j < rows_left ? row(j) : 0.f;
-        }
+            for (int j = 0; j < P; ++j) part[j] = j < rows_left ? row(j, shared) : 0.f;
+          }
+        };
+        if (lut_shared)
+          rows(std::true_type{});
+        else
+          rows(std::false_type{});
         ++it_use;
         __syncwarp();
         if (si + S < nstages) {
