@@ -49,7 +49,7 @@ constexpr int kQuantThreadsMax = 512;
 // Shared-memory layout of one row (K columns, NG = K / G groups, P = the
 // power of two >= K the sort runs over).
 struct QuantSmem {
-  size_t xs, ex, alpha, beta, cent, table, stage, code, total;
+  size_t xs, ex, alpha, beta, cent, table, stage, cnt, off, code, total;
 };
 
 __host__ __device__ inline int64_t pow2_at_least(int64_t K) {
@@ -65,7 +65,9 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G) {
   s.cent = s.xs + 8 * (size_t)pow2_at_least(K);        // double [16]
   s.table = s.cent + 8 * 16;                           // double [16]
   s.stage = s.table + 8 * 16;                          // double2 [threads] (M-step)
-  s.ex = s.stage + 16 * (size_t)kQuantThreadsMax;      // float [K]
+  s.cnt = s.stage + 16 * (size_t)kQuantThreadsMax;     // int [warps][16] (M-step)
+  s.off = s.cnt + 4 * 16 * (size_t)(kQuantThreadsMax / 32);  // int [warps][16]
+  s.ex = s.off + 4 * 16 * (size_t)(kQuantThreadsMax / 32);   // float [K]
   s.alpha = s.ex + 4 * (size_t)K;                      // float [NG]
   s.beta = s.alpha + 4 * (size_t)NG;                   // float [NG]
   s.code = s.beta + 4 * (size_t)NG;                    // uint8 [K]
@@ -126,6 +128,8 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   float* beta_s = reinterpret_cast<float*>(smem + L.beta);
   uint8_t* code = smem + L.code;
   double2* stage = reinterpret_cast<double2*>(smem + L.stage);
+  int* cnt = reinterpret_cast<int*>(smem + L.cnt);
+  int* off = reinterpret_cast<int*>(smem + L.off);
 
   const int64_t n = blockIdx.x;
   const int NG = K / G;
@@ -136,6 +140,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
     ex_s[j] = ex[j];
     code[j] = 0;
   }
+  for (int i = tid; i < kQuantWarps * 16; i += kQuantThreads) cnt[i] = 0;
 
   // Eq. 1-2: one warp per group; min and max are exact, so their order is free.
   for (int g = warp; g < NG; g += kQuantWarps) {
@@ -193,54 +198,78 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   int it = 0;
   while (it < max_iter) {
     {
-      // Eq. 23, every warp at once: warp w owns clusters q0 .. q0 + QPW - 1,
-      // its lane i < QPW sums u_j * w_S_j (num) and u_j (den) of cluster
-      // q0 + i over ascending j.  The columns go one block-wide batch at a
-      // time: each thread stages one column's two terms in shared memory;
-      // then, 32 columns at a time (one group, G % 32 == 0), a warp ballot per
-      // cluster gives each summing lane the bitmask of its cluster's columns,
-      // and the lane adds those terms in ascending bit order, four loads per
-      // round: the sequential order, each term formed once for the block.
-      constexpr int QPW = NQ >= kQuantWarps ? NQ / kQuantWarps : 1;  // clusters per warp
-      const int q0 = warp * QPW;
-      const bool owner = lane < QPW && q0 < NQ;
+      // Eq. 23.  Cluster q's numerator sum(u_j * w_S_j) and denominator
+      // sum(u_j) over ascending j, added by lane q of warp 0.  The columns go
+      // one block-wide batch at a time (thread t: column b0 + t):
+      //  1. each thread forms its column's two terms; within its warp (32
+      //     consecutive columns) __match_any_sync gives the lanes of the same
+      //     cluster, hence the thread's rank among them, and the first of
+      //     them stores the warp's count for that cluster;
+      //  2. lane q of warp 0 turns the counts into offsets (warps in order),
+      //     the clusters' list bases by a scan over the lanes, and clears the
+      //     counts for the next batch;
+      //  3. each thread stores its terms at base[q] + offset[warp][q] + rank:
+      //     the batch sorted by cluster, ascending column within a cluster;
+      //  4. lane q of warp 0 adds its list front to back, the loads issued
+      //     ahead of the adds, while the other warps start the next batch.
+      // The adds are the sequential ones, in the same order.
       double acc_n = 0.0, acc_d = 0.0;
+      int lbeg = 0, lend = 0;  // lane q < NQ of warp 0: its list in `stage`
       for (int b0 = 0; b0 < K; b0 += kQuantThreads) {
         const int jb = b0 + tid;
-        if (jb < K) {
+        const bool in = jb < K;  // whole warps: K % 32 == 0
+        int q = 0, rank = 0;
+        double2 term = make_double2(0.0, 0.0);
+        if (in) {
+          q = code[jb];
           const double u = __dmul_rn((double)alpha_s[jb / G], (double)ex_s[jb]);
-          stage[tid] = make_double2(__dmul_rn(u, xs[jb]), u);
+          term = make_double2(__dmul_rn(u, xs[jb]), u);
+          const uint32_t m = __match_any_sync(kFullMask, q);
+          rank = __popc(m & ((1u << lane) - 1u));
+          if (rank == 0) cnt[warp * 16 + q] = __popc(m);
         }
-        __syncthreads();
-        if (q0 < NQ) {  // warp-uniform
-          const int ncols = min(kQuantThreads, K - b0);  // a multiple of 32
-          for (int c0 = 0; c0 < ncols; c0 += 32) {
-            const int cj = code[b0 + c0 + lane];
-            uint32_t mask = 0;
-#pragma unroll
-            for (int i = 0; i < QPW; ++i) {
-              const uint32_t m = __ballot_sync(kFullMask, cj == q0 + i);
-              if (lane == i) mask = m;
-            }
-            const double2* sv = stage + c0;
-            while (mask) {
-              // the terms of the lowest set bit, or 0 past the last (exact:
-              // x + 0 is x for every x these sums hold, none of them -0)
-              auto take = [&]() -> double2 {
-                if (!mask) return make_double2(0.0, 0.0);
-                const double2 v = sv[__ffs(mask) - 1];
-                mask &= mask - 1;
-                return v;
-              };
-              const double2 v0 = take(), v1 = take(), v2 = take(), v3 = take();
-              acc_n = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_n, v0.x), v1.x), v2.x), v3.x);
-              acc_d = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_d, v0.y), v1.y), v2.y), v3.y);
+        __syncthreads();  // counts stored; the previous batch's adds are done
+        if (warp == 0) {
+          int run = 0;
+          if (lane < NQ) {
+            for (int w = 0; w < kQuantWarps; ++w) {
+              const int v = cnt[w * 16 + lane];
+              off[w * 16 + lane] = run;
+              cnt[w * 16 + lane] = 0;
+              run += v;
             }
           }
+          int base = run;  // inclusive scan over the cluster lanes
+#pragma unroll
+          for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, base, d);
+            if (lane >= d) base += y;
+          }
+          base -= run;
+          if (lane < NQ) {
+            for (int w = 0; w < kQuantWarps; ++w) off[w * 16 + lane] += base;
+          }
+          lbeg = base;
+          lend = base + run;
         }
-        __syncthreads();  // the batch's terms have been read
+        __syncthreads();  // offsets ready
+        if (in) stage[off[warp * 16 + q] + rank] = term;
+        __syncthreads();  // the batch is sorted by cluster
+        if (warp == 0 && lane < NQ) {
+          int i = lbeg;
+          for (; i + 4 <= lend; i += 4) {
+            const double2 v0 = stage[i], v1 = stage[i + 1], v2 = stage[i + 2], v3 = stage[i + 3];
+            acc_n = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_n, v0.x), v1.x), v2.x), v3.x);
+            acc_d = __dadd_rn(__dadd_rn(__dadd_rn(__dadd_rn(acc_d, v0.y), v1.y), v2.y), v3.y);
+          }
+          for (; i < lend; ++i) {
+            const double2 v = stage[i];
+            acc_n = __dadd_rn(acc_n, v.x);
+            acc_d = __dadd_rn(acc_d, v.y);
+          }
+        }
       }
-      if (owner && acc_d > 0.0) cent[q0 + lane] = __ddiv_rn(acc_n, acc_d);
+      if (warp == 0 && lane < NQ && acc_d > 0.0) cent[lane] = __ddiv_rn(acc_n, acc_d);
     }
     __syncthreads();
     ++it;
