@@ -47,7 +47,8 @@ namespace {
 constexpr int kQuantThreadsMax = 512;
 
 // Shared-memory layout of one row (K columns, NG = K / G groups, P = the
-// power of two >= K the sort runs over).
+// power of two >= K the sort runs over; cpt M-step columns per thread and
+// batch, 2 where the row leaves room, else 1).
 struct QuantSmem {
   size_t xs, ex, alpha, beta, cent, table, stage, cnt, off, code, total;
 };
@@ -58,16 +59,17 @@ __host__ __device__ inline int64_t pow2_at_least(int64_t K) {
   return p;
 }
 
-__host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G) {
+__host__ __device__ inline QuantSmem quant_smem_layout(int64_t K, int64_t G, int cpt) {
   QuantSmem s;
   const int64_t NG = K / G;
   s.xs = 0;                                            // double [P]
   s.cent = s.xs + 8 * (size_t)pow2_at_least(K);        // double [16]
   s.table = s.cent + 8 * 16;                           // double [16]
-  s.stage = s.table + 8 * 16;                          // double2 [threads] (M-step)
-  s.cnt = s.stage + 16 * (size_t)kQuantThreadsMax;     // int [warps][16] (M-step)
-  s.off = s.cnt + 4 * 16 * (size_t)(kQuantThreadsMax / 32);  // int [warps][16]
-  s.ex = s.off + 4 * 16 * (size_t)(kQuantThreadsMax / 32);   // float [K]
+  const size_t chunks = (size_t)cpt * (kQuantThreadsMax / 32);  // 32 columns each
+  s.stage = s.table + 8 * 16;                          // double2 [32 chunks] (M-step)
+  s.cnt = s.stage + 16 * 32 * chunks;                  // int [chunks][16] (M-step)
+  s.off = s.cnt + 4 * 16 * chunks;                     // int [chunks][16]
+  s.ex = s.off + 4 * 16 * chunks;                      // float [K]
   s.alpha = s.ex + 4 * (size_t)K;                      // float [NG]
   s.beta = s.alpha + 4 * (size_t)NG;                   // float [NG]
   s.code = s.beta + 4 * (size_t)NG;                    // uint8 [K]
@@ -111,7 +113,7 @@ __device__ __forceinline__ bool estep(const double* xs, int K, const double* c, 
 }
 
 // NQ = 2^n table entries (4, 8 or 16); the packed row has n K / 8 bytes.
-template <int NQ, int kQuantThreads>
+template <int NQ, int kQuantThreads, int kCPT>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, int K, int G,
                 int max_iter, uint8_t* __restrict__ packed, uint16_t* __restrict__ lut,
@@ -119,7 +121,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
                 int32_t* __restrict__ iters) {
   constexpr int kQuantWarps = kQuantThreads / 32;
   extern __shared__ __align__(16) unsigned char smem[];
-  const QuantSmem L = quant_smem_layout(K, G);
+  const QuantSmem L = quant_smem_layout(K, G, kCPT);
   double* xs = reinterpret_cast<double*>(smem + L.xs);
   double* cent = reinterpret_cast<double*>(smem + L.cent);
   double* table = reinterpret_cast<double*>(smem + L.table);
@@ -140,7 +142,7 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
     ex_s[j] = ex[j];
     code[j] = 0;
   }
-  for (int i = tid; i < kQuantWarps * 16; i += kQuantThreads) cnt[i] = 0;
+  for (int i = tid; i < kCPT * kQuantWarps * 16; i += kQuantThreads) cnt[i] = 0;
 
   // Eq. 1-2: one warp per group; min and max are exact, so their order is free.
   for (int g = warp; g < NG; g += kQuantWarps) {
@@ -200,7 +202,8 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
     {
       // Eq. 23.  Cluster q's numerator sum(u_j * w_S_j) and denominator
       // sum(u_j) over ascending j, added by lane q of warp 0.  The columns go
-      // one block-wide batch at a time (thread t: column b0 + t):
+      // one block-wide batch at a time (thread t: columns b0 + r T + t,
+      // r < kCPT, T threads; chunk r W + w is warp w's r-th set of 32):
       //  1. each thread forms its column's two terms; within its warp (32
       //     consecutive columns) __match_any_sync gives the lanes of the same
       //     cluster, hence the thread's rank among them, and the first of
@@ -215,31 +218,35 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
       // The adds are the sequential ones, in the same order.
       double acc_n = 0.0, acc_d = 0.0;
       int lbeg = 0, lend = 0;  // lane q < NQ of warp 0: its list in `stage`
-      for (int b0 = 0; b0 < K; b0 += kQuantThreads) {
-        const int jb = b0 + tid;
-        const bool in = jb < K;  // whole warps: K % 32 == 0
-        int q = 0, rank = 0;
-        double2 term = make_double2(0.0, 0.0);
-        if (in) {
-          q = code[jb];
-          const double u = __dmul_rn((double)alpha_s[jb / G], (double)ex_s[jb]);
-          term = make_double2(__dmul_rn(u, xs[jb]), u);
-          const uint32_t m = __match_any_sync(kFullMask, q);
-          rank = __popc(m & ((1u << lane) - 1u));
-          if (rank == 0) cnt[warp * 16 + q] = __popc(m);
+      constexpr int kBatch = kCPT * kQuantThreads;
+      for (int b0 = 0; b0 < K; b0 += kBatch) {
+        int q[kCPT], rank[kCPT];
+        double2 term[kCPT];
+#pragma unroll
+        for (int r = 0; r < kCPT; ++r) {
+          const int jb = b0 + r * kQuantThreads + tid;  // chunk r * warps + warp
+          q[r] = 0; rank[r] = 0; term[r] = make_double2(0.0, 0.0);
+          if (jb < K) {  // whole warps: K % 32 == 0
+            q[r] = code[jb];
+            const double u = __dmul_rn((double)alpha_s[jb / G], (double)ex_s[jb]);
+            term[r] = make_double2(__dmul_rn(u, xs[jb]), u);
+            const uint32_t m = __match_any_sync(kFullMask, q[r]);
+            rank[r] = __popc(m & ((1u << lane) - 1u));
+            if (rank[r] == 0) cnt[(r * kQuantWarps + warp) * 16 + q[r]] = __popc(m);
+          }
         }
-        __syncthreads();  // counts stored; the previous batch's adds are done
+        __syncthreads();
         if (warp == 0) {
           int run = 0;
           if (lane < NQ) {
-            for (int w = 0; w < kQuantWarps; ++w) {
-              const int v = cnt[w * 16 + lane];
-              off[w * 16 + lane] = run;
-              cnt[w * 16 + lane] = 0;
+            for (int c = 0; c < kCPT * kQuantWarps; ++c) {
+              const int v = cnt[c * 16 + lane];
+              off[c * 16 + lane] = run;
+              cnt[c * 16 + lane] = 0;
               run += v;
             }
           }
-          int base = run;  // inclusive scan over the cluster lanes
+          int base = run;
 #pragma unroll
           for (int d = 1; d < 32; d <<= 1) {
             const int y = __shfl_up_sync(kFullMask, base, d);
@@ -247,14 +254,18 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
           }
           base -= run;
           if (lane < NQ) {
-            for (int w = 0; w < kQuantWarps; ++w) off[w * 16 + lane] += base;
+            for (int c = 0; c < kCPT * kQuantWarps; ++c) off[c * 16 + lane] += base;
           }
           lbeg = base;
           lend = base + run;
         }
-        __syncthreads();  // offsets ready
-        if (in) stage[off[warp * 16 + q] + rank] = term;
-        __syncthreads();  // the batch is sorted by cluster
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < kCPT; ++r) {
+          const int jb = b0 + r * kQuantThreads + tid;
+          if (jb < K) stage[off[(r * kQuantWarps + warp) * 16 + q[r]] + rank[r]] = term[r];
+        }
+        __syncthreads();
         if (warp == 0 && lane < NQ) {
           int i = lbeg;
           for (; i + 4 <= lend; i += 4) {
@@ -310,29 +321,46 @@ quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ ex, in
   }
 }
 
-template <int NQ>
-any4_status launch_quantize_nq(const uint16_t* w, const float* ex, int64_t N, int64_t K,
-                               int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
-                               uint16_t* scale, uint16_t* offset, int32_t* iters, size_t smem,
-                               cudaStream_t stream) {
+template <int NQ, int kCPT>
+any4_status launch_quantize_cpt(const uint16_t* w, const float* ex, int64_t N, int64_t K,
+                                int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                                uint16_t* scale, uint16_t* offset, int32_t* iters, size_t smem,
+                                cudaStream_t stream) {
   // long rows: one block fits per SM, give it 512 threads; else 256 threads
   // and several blocks (rows) per SM
   const bool wide = 2 * (smem + 1024) > (size_t)228 * 1024;
-  const void* kern = wide ? reinterpret_cast<const void*>(quantize_kernel<NQ, 512>)
-                          : reinterpret_cast<const void*>(quantize_kernel<NQ, 256>);
+  const void* kern = wide ? reinterpret_cast<const void*>(quantize_kernel<NQ, 512, kCPT>)
+                          : reinterpret_cast<const void*>(quantize_kernel<NQ, 256, kCPT>);
   if (ensure_dynamic_smem(kern, smem) != ANY4_OK) return ANY4_ERR_CUDA;
   if (wide)
-    quantize_kernel<NQ, 512><<<(unsigned)N, 512, smem, stream>>>(
+    quantize_kernel<NQ, 512, kCPT><<<(unsigned)N, 512, smem, stream>>>(
         w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
   else
-    quantize_kernel<NQ, 256><<<(unsigned)N, 256, smem, stream>>>(
+    quantize_kernel<NQ, 256, kCPT><<<(unsigned)N, 256, smem, stream>>>(
         w, ex, (int)K, (int)G, (int)max_iter, packed, lut, scale, offset, iters);
   return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
 }
 
+// two M-step columns per thread and batch (half the batches and block
+// barriers) where the row's shared memory leaves room, else one (and one for
+// 2-bit codes, whose two-column form does not fit the 512-thread register
+// budget without spills)
+template <int NQ>
+any4_status launch_quantize_nq(const uint16_t* w, const float* ex, int64_t N, int64_t K,
+                               int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
+                               uint16_t* scale, uint16_t* offset, int32_t* iters,
+                               cudaStream_t stream, const DeviceInfo& dev) {
+  const size_t smem2 = quant_smem_layout(K, G, 2).total;
+  if (NQ >= 8 && smem2 <= dev.smem_optin)
+    return launch_quantize_cpt<NQ, NQ >= 8 ? 2 : 1>(w, ex, N, K, G, max_iter, packed, lut, scale, offset,
+                                      iters, smem2, stream);
+  return launch_quantize_cpt<NQ, 1>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
+                                    quant_smem_layout(K, G, 1).total, stream);
+}
+
 }  // namespace
 
-size_t quantize_smem_bytes(int64_t K, int64_t G) { return quant_smem_layout(K, G).total; }
+size_t quantize_smem_bytes(int64_t K, int64_t G) { return quant_smem_layout(K, G, 1).total; }
 
 any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64_t K, int64_t G,
                             int bits, int32_t max_iter, uint8_t* packed, uint16_t* lut,
@@ -343,13 +371,13 @@ any4_status launch_quantize(const uint16_t* w, const float* ex, int64_t N, int64
   switch (bits) {
     case 4:
       return launch_quantize_nq<16>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
-                                    smem, stream);
+                                    stream, dev);
     case 3:
       return launch_quantize_nq<8>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
-                                   smem, stream);
+                                   stream, dev);
     case 2:
       return launch_quantize_nq<4>(w, ex, N, K, G, max_iter, packed, lut, scale, offset, iters,
-                                   smem, stream);
+                                   stream, dev);
     default:
       return ANY4_ERR_SHAPE;
   }
