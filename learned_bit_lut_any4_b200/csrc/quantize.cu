@@ -25,9 +25,9 @@
 //   - E-step: nearest by |w_S - c_q| in fp64, ties to the lowest q;
 //   - M-step: sample weight u_j = alpha_{g(j)} * E|x_j| (exact in fp64);
 //     numerator sum(u_j * w_S_j) and denominator sum(u_j) over ascending j,
-//     one lane per cluster and per sum (the clusters spread over the warps),
-//     so the rounding order is the sequential one (the lane adds only its
-//     cluster's columns, found 32 at a time by warp ballots); a cluster whose
+//     one lane per cluster adding both sums, so the rounding order is the
+//     sequential one (the block first sorts each batch of columns' terms by
+//     cluster, keeping the column order within a cluster); a cluster whose
 //     weights sum to 0 keeps its entry;
 //   - stop after max_iter M-steps, or when an E-step changes no code;
 //   - LUT_q = bf16(fp32(c_q)); the codes are a final E-step against the stored
