@@ -157,6 +157,89 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
   }
 }
 
+// G a multiple of 128 and K a multiple of 1024: the table folded with the
+// group's scale and offset.  A warp still owns 1024-column segments and writes
+// them with the same 512-byte warp stores, but step p (0..3) of a lane in half
+// h covers columns 256 p + 128 h + 8 (lane & 15) .. + 7, so a half-warp spans
+// 128 columns of one group at a time.  Source lane e of half h then holds, for
+// its half's groups of steps 2i and 2i + 1, the bf16 pair
+//   (bf16(fmaf(LUT[e], s, o)) of step 2i, the same of step 2i + 1),
+// the weight of the definition for code e, and a lookup is one shuffle inside
+// the half-warp (segment mask 16) with the shifted code word, a byte permute
+// pairing two weights in the half of the step.  Per weight that is a shift, a
+// shuffle and half a permute instead of a table load, an fp32 FMA and half a
+// conversion: the arithmetic no longer competes with the memory stream.
+template <bool kStream>
+__global__ void __launch_bounds__(kDqThreads) dequant_fold_kernel(
+    const uint8_t* __restrict__ packed, const uint16_t* __restrict__ lut, int64_t lut_row_stride,
+    const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
+    uint16_t* __restrict__ W, int64_t N, int K, int G, int g_shift) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = lane >> 4, e = lane & 15;
+  const int segs_per_row = K / kDqSeg;
+  const int64_t nseg = N * segs_per_row;
+  const int groups = K / G;
+  const int64_t first = (int64_t)blockIdx.x * kDqWarps + warp;
+  const int64_t stride = (int64_t)gridDim.x * kDqWarps;
+  if (first >= nseg) return;
+  // codes, and the scale (low half) and offset (high half) of the lane's
+  // group at each step, of one segment
+  struct Seg {
+    uint32_t w[4];
+    uint32_t so[4];
+  };
+  auto load = [&](int64_t sg, Seg& d) {
+    const int64_t n = sg / segs_per_row;
+    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t k = (uint32_t)(col0 + 256 * p + 128 * h + 8 * e);
+      d.w[p] = ldg_nc_u32(packed + (n * K + k) / 2);
+      const int64_t gi = n * groups + group_of(k, g_shift, (uint32_t)G);
+      d.so[p] = (uint32_t)ldg_u16(scale + gi) | ((uint32_t)ldg_u16(offset + gi) << 16);
+    }
+  };
+  Seg nxt;
+  load(first, nxt);
+  int64_t cur_row = -1;
+  float lv = 0.f;  // LUT[row][e]
+  for (int64_t sg = first; sg < nseg; sg += stride) {
+    const int64_t n = sg / segs_per_row;
+    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+    if (n != cur_row) {
+      lv = bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + e));
+      cur_row = n;
+    }
+    const Seg cur = nxt;
+    if (sg + stride < nseg) load(sg + stride, nxt);  // out before this segment's math
+    uint32_t tab[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+      tab[i] = pack_bf16x2_rn(
+          __fmaf_rn(lv, bf16_lo_to_f32(cur.so[2 * i]), bf16_hi_to_f32(cur.so[2 * i])),
+          __fmaf_rn(lv, bf16_lo_to_f32(cur.so[2 * i + 1]), bf16_hi_to_f32(cur.so[2 * i + 1])));
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t sel = (p & 1) ? 0x7632u : 0x5410u;
+      uint32_t o[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        uint32_t a, b;
+        asm("shfl.sync.idx.b32 %0, %1, %2, 0x101f, 0xffffffff;"
+            : "=r"(a) : "r"(tab[p >> 1]), "r"(cur.w[p] >> (8 * m)));
+        asm("shfl.sync.idx.b32 %0, %1, %2, 0x101f, 0xffffffff;"
+            : "=r"(b) : "r"(tab[p >> 1]), "r"(cur.w[p] >> (8 * m + 4)));
+        o[m] = __byte_perm(a, b, sel);
+      }
+      uint16_t* dst = W + n * K + col0 + 256 * p + 128 * h + 8 * e;
+      if (kStream)
+        stg_cs_v4(dst, o[0], o[1], o[2], o[3]);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 int pow2_shift(int64_t G) {
   for (int s = 0; s < 31; ++s)
     if ((int64_t(1) << s) == G) return s;
@@ -185,8 +268,12 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const DeviceInfo& dev, bool streaming) {
   if (K > INT32_MAX / 2) return ANY4_ERR_SHAPE;
   const int64_t segs = N * ((K + kDqSeg - 1) / kDqSeg);
-  auto kern = K % kDqSeg == 0 ? (streaming ? dequant_kernel<true, true> : dequant_kernel<true, false>)
-                              : (streaming ? dequant_kernel<false, true> : dequant_kernel<false, false>);
+  // the folded-table kernel where a half-warp step stays inside one group
+  const bool fold = K % kDqSeg == 0 && G % 128 == 0;
+  auto kern = fold ? (streaming ? dequant_fold_kernel<true> : dequant_fold_kernel<false>)
+            : K % kDqSeg == 0
+                ? (streaming ? dequant_kernel<true, true> : dequant_kernel<true, false>)
+                : (streaming ? dequant_kernel<false, true> : dequant_kernel<false, false>);
   int per_sm = cached_occupancy(reinterpret_cast<const void*>(kern), kDqThreads, 0);
   if (per_sm < 1) per_sm = 1;
   kern<<<grid_for(segs * 32, kDqThreads, dev, per_sm), kDqThreads, 0, stream>>>(
