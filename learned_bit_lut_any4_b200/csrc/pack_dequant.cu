@@ -102,9 +102,8 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
     uint32_t w[4];
     uint32_t so[4];
   };
-  auto load = [&](int64_t sg, Seg& d) {
-    const int64_t n = sg / segs_per_row;
-    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+  auto load = [&](int64_t n, int si, Seg& d) {
+    const int col0 = si * kDqSeg;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int c = 256 * v + 8 * lane;
@@ -119,12 +118,24 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
       }
     }
   };
+  // the next segment's (row, segment of the row), advanced by the grid
+  // stride without a division per segment
+  const int64_t step_rows = stride / segs_per_row;
+  const int step_segs = (int)(stride - step_rows * segs_per_row);
+  int64_t n_nxt = first / segs_per_row;
+  int si_nxt = (int)(first - n_nxt * segs_per_row);
   Seg nxt;
-  load(first, nxt);
+  load(n_nxt, si_nxt, nxt);
   int64_t cur_row = -1;
   for (int64_t sg = first; sg < nseg; sg += stride) {
-    const int64_t n = sg / segs_per_row;
-    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+    const int64_t n = n_nxt;
+    const int col0 = si_nxt * kDqSeg;
+    n_nxt += step_rows;
+    si_nxt += step_segs;
+    if (si_nxt >= segs_per_row) {
+      si_nxt -= segs_per_row;
+      ++n_nxt;
+    }
     if (n != cur_row) {  // this warp moves to a new row: its table as fp32
       __syncwarp();
       if (lane < 16) s_lut[warp][lane] = bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + lane));
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(
       cur_row = n;
     }
     const Seg cur = nxt;
-    if (sg + stride < nseg) load(sg + stride, nxt);  // out before this segment's math
+    if (sg + stride < nseg) load(n_nxt, si_nxt, nxt);  // out before this segment's math
     const float* t = s_lut[warp];
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
@@ -188,9 +199,8 @@ __global__ void __launch_bounds__(kDqThreads) dequant_fold_kernel(
     uint32_t w[4];
     uint32_t so[4];
   };
-  auto load = [&](int64_t sg, Seg& d) {
-    const int64_t n = sg / segs_per_row;
-    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+  auto load = [&](int64_t n, int si, Seg& d) {
+    const int col0 = si * kDqSeg;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const uint32_t k = (uint32_t)(col0 + 256 * p + 128 * h + 8 * e);
@@ -199,19 +209,31 @@ __global__ void __launch_bounds__(kDqThreads) dequant_fold_kernel(
       d.so[p] = (uint32_t)ldg_u16(scale + gi) | ((uint32_t)ldg_u16(offset + gi) << 16);
     }
   };
+  // the next segment's (row, segment of the row), advanced by the grid
+  // stride without a division per segment
+  const int64_t step_rows = stride / segs_per_row;
+  const int step_segs = (int)(stride - step_rows * segs_per_row);
+  int64_t n_nxt = first / segs_per_row;
+  int si_nxt = (int)(first - n_nxt * segs_per_row);
   Seg nxt;
-  load(first, nxt);
+  load(n_nxt, si_nxt, nxt);
   int64_t cur_row = -1;
   float lv = 0.f;  // LUT[row][e]
   for (int64_t sg = first; sg < nseg; sg += stride) {
-    const int64_t n = sg / segs_per_row;
-    const int col0 = (int)(sg - n * segs_per_row) * kDqSeg;
+    const int64_t n = n_nxt;
+    const int col0 = si_nxt * kDqSeg;
+    n_nxt += step_rows;
+    si_nxt += step_segs;
+    if (si_nxt >= segs_per_row) {
+      si_nxt -= segs_per_row;
+      ++n_nxt;
+    }
     if (n != cur_row) {
       lv = bf16_lo_to_f32(ldg_u16(lut + n * lut_row_stride + e));
       cur_row = n;
     }
     const Seg cur = nxt;
-    if (sg + stride < nseg) load(sg + stride, nxt);  // out before this segment's math
+    if (sg + stride < nseg) load(n_nxt, si_nxt, nxt);  // out before this segment's math
     uint32_t tab[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
