@@ -23,6 +23,7 @@ from ._native import (  # noqa: F401
     ANY4_STATIC_SCRATCH_BYTES,
     PATHS,
     Any4Error,
+    Any4Prepared,
     any4_bits_per_weight,
     any4_dequant,
     any4_dequant_bits,
@@ -36,6 +37,7 @@ from ._native import (  # noqa: F401
     any4_matmul_workspace_size,
     any4_pack,
     any4_pack_bits,
+    any4_prepare,
     any4_quantize,
     any4_quantize_bits,
     any4_status_string,

@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 
 import torch
 
@@ -155,8 +156,19 @@ def _check(status: int, where: str):
         raise Any4Error(status, where)
 
 
+_RAW_STREAM = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def _stream_index(index: int) -> int:
+    """The current stream's handle on device `index` (torch's raw-handle
+    accessor where it has one: no Stream object per call)."""
+    if _RAW_STREAM is not None:
+        return _RAW_STREAM(index)
+    return torch.cuda.current_stream(index).cuda_stream
 
 
 def _ptr(t) -> int | None:
@@ -326,6 +338,32 @@ def _need_status(dev_status, dev):
     _need(dev_status, "dev_status", (torch.int32,), dev)
 
 
+def _weight_operands(packed, lut, scale, offset, G, K=None, bits=4):
+    """Check one matrix's packed codes, table, scales and offsets (types and
+    sizes; devices and layout by the caller).  Returns (N, K, lut_row_stride)."""
+    for t, nm, dts in ((packed, "packed", (torch.uint8,)), (lut, "lut", _BF16),
+                       (scale, "scale", _BF16), (offset, "offset", _BF16)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{nm} must be a torch.Tensor")
+        if t.dtype not in dts:
+            raise TypeError(f"{nm} must have dtype in {dts}, got {t.dtype}")
+    if packed.dim() != 2:
+        raise ValueError(f"packed must be [N, {bits} K / 8]")
+    N, Kh = packed.shape
+    if K is None:
+        if (Kh * 8) % bits != 0:
+            raise ValueError(f"packed rows of {Kh} bytes do not hold whole {bits}-bit codes")
+        K = Kh * 8 // bits
+    elif Kh * 8 != K * bits:
+        raise ValueError(f"x has K={K} but packed holds {Kh * 8 // bits} {bits}-bit columns")
+    if G <= 0 or K % G != 0:
+        raise ValueError(f"G={G} must be positive and divide K={K}")
+    stride = _lut_stride(lut, N, 1 << bits)
+    if scale.numel() != N * (K // G) or offset.numel() != N * (K // G):
+        raise ValueError(f"scale and offset must hold N * K/G = {N * (K // G)} values")
+    return N, K, stride
+
+
 def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_out=False,
                      bits=4):
     """Validate the operands of a matmul call on the host, before any launch:
@@ -333,23 +371,14 @@ def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_
     enough, so a short y, scale or offset is caught here.  Sizes are checked
     before devices, so the checks hold for any tensor.  Returns
     (M, N, K, lut_row_stride, y), allocating y when it is None."""
-    for t, nm, dts in ((x, "x", _BF16), (packed, "packed", (torch.uint8,)), (lut, "lut", _BF16),
-                       (scale, "scale", _BF16), (offset, "offset", _BF16)):
-        if not isinstance(t, torch.Tensor):
-            raise TypeError(f"{nm} must be a torch.Tensor")
-        if t.dtype not in dts:
-            raise TypeError(f"{nm} must have dtype in {dts}, got {t.dtype}")
-    if x.dim() != 2 or packed.dim() != 2:
-        raise ValueError(f"x must be [M, K] and packed [N, {bits} K / 8]")
+    if not isinstance(x, torch.Tensor):
+        raise TypeError("x must be a torch.Tensor")
+    if x.dtype not in _BF16:
+        raise TypeError(f"x must have dtype in {_BF16}, got {x.dtype}")
+    if x.dim() != 2:
+        raise ValueError("x must be [M, K]")
     M, K = x.shape
-    N, Kh = packed.shape
-    if Kh * 8 != K * bits:
-        raise ValueError(f"x has K={K} but packed holds {Kh * 8 // bits} {bits}-bit columns")
-    if G <= 0 or K % G != 0:
-        raise ValueError(f"G={G} must be positive and divide K={K}")
-    stride = _lut_stride(lut, N, 1 << bits)
-    if scale.numel() != N * (K // G) or offset.numel() != N * (K // G):
-        raise ValueError(f"scale and offset must hold N * K/G = {N * (K // G)} values")
+    N, K, stride = _weight_operands(packed, lut, scale, offset, G, K, bits)
     if y is not None:
         _need_shape(y, "y", (M, N))
     if isinstance(dev_status, torch.Tensor) and dev_status.numel() < 1:
@@ -363,6 +392,97 @@ def _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status=None, fp32_
         y = torch.empty((M, N), dtype=torch.float32 if fp32_out else torch.bfloat16, device=dev)
     _need(y, "y", (torch.float32,) if fp32_out else _BF16, dev)
     return M, N, K, stride, y
+
+
+class Any4Prepared:
+    """One any4 matrix checked once, for repeated matmul calls (a decode loop).
+
+    any4_prepare checks the packed codes, table, scales and offsets (dtypes,
+    sizes, device, contiguity) and keeps them; any4_matmul and
+    any4_matmul_grouped take it in place of those four tensors and then check
+    only x, y and the workspace, which keeps the host cost of a call small.
+    The tensors must stay as they are (not resized, not moved) while it is in
+    use."""
+    __slots__ = ("packed", "lut", "scale", "offset", "G", "N", "K", "lut_row_stride",
+                 "device", "_ptrs", "__weakref__")
+
+    def __init__(self, packed, lut, scale, offset, G):
+        N, K, stride = _weight_operands(packed, lut, scale, offset, G)
+        dev = packed.device
+        _need(packed, "packed", (torch.uint8,))
+        for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
+            _need(t, nm, _BF16, dev)
+        self.packed, self.lut, self.scale, self.offset = packed, lut, scale, offset
+        self.G, self.N, self.K, self.lut_row_stride = int(G), int(N), int(K), stride
+        self.device = dev
+        self._ptrs = (packed.data_ptr(), lut.data_ptr(), scale.data_ptr(), offset.data_ptr())
+
+    def __repr__(self):
+        return f"Any4Prepared(N={self.N}, K={self.K}, G={self.G}, device={self.device})"
+
+
+def any4_prepare(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
+                 offset: torch.Tensor, G: int) -> Any4Prepared:
+    """Check an any4 matrix once for repeated calls (see Any4Prepared)."""
+    return Any4Prepared(packed, lut, scale, offset, G)
+
+
+# Per thread: the ctypes descriptor array of each group of prepared weights
+# used in a call (only the y pointers change from call to call), and the
+# workspace each needs per M.
+_PREPARED_GROUPS = threading.local()
+_PREPARED_GROUPS_MAX = 4096
+
+
+def _prepared_group(weights):
+    cache = getattr(_PREPARED_GROUPS, "d", None)
+    if cache is None:
+        cache = _PREPARED_GROUPS.d = {}
+    key = tuple(weights)
+    g = cache.get(key)
+    if g is None:
+        w0 = weights[0]
+        for w in weights:
+            if not isinstance(w, Any4Prepared):
+                raise TypeError("mix of prepared and plain weights in one call")
+            if w.device != w0.device or w.K != w0.K or w.G != w0.G:
+                raise ValueError("prepared weights of one call must share device, K and G")
+        descs = (Any4Weight * len(weights))()
+        for i, w in enumerate(weights):
+            pk, lt, sc, of = w._ptrs
+            descs[i] = Any4Weight(pk, lt, w.lut_row_stride, sc, of, 0, w.N)
+        if len(cache) >= _PREPARED_GROUPS_MAX:
+            cache.clear()
+        di = w0.device.index if w0.device.index is not None else -1
+        g = cache[key] = [descs, w0.K, w0.G, w0.device, di, {}]
+    return g
+
+
+def _prepared_x(x, K, dev_index):
+    """Check x of a call on prepared weights (K columns, on device dev_index);
+    returns M."""
+    if not isinstance(x, torch.Tensor) or x.dtype not in _BF16:
+        raise TypeError("x must be a bf16 torch.Tensor")
+    if x.get_device() != dev_index:
+        raise ValueError(f"x must be on cuda:{dev_index}, the device of the weights")
+    shape = x.shape
+    if len(shape) != 2 or shape[1] != K:
+        raise ValueError(f"x must be [M, {K}], got {tuple(shape)}")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    return shape[0]
+
+
+def _prepared_y(y, M, N, dev_index, fp32_out):
+    dts = (torch.float32,) if fp32_out else _BF16
+    if not isinstance(y, torch.Tensor) or y.dtype not in dts:
+        raise TypeError(f"y must be a torch.Tensor with dtype in {dts}")
+    if y.get_device() != dev_index:
+        raise ValueError(f"y must be on cuda:{dev_index}, the device of the weights")
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"y must have shape {(M, N)}, got {tuple(y.shape)}")
+    if not y.is_contiguous():
+        raise ValueError("y must be contiguous")
 
 
 def _lut_stride(lut: torch.Tensor, N: int, entries: int = 16) -> int:
@@ -517,7 +637,9 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
                         pair_table: bool = False):
     """[y_i = x * dequant(W_i)^T for each (packed, lut, scale, offset) in
     weights]: matrices that share x, in one launch at M = 1 (see
-    any4_matmul_grouped in include/any4.h).  Returns the list of y_i."""
+    any4_matmul_grouped in include/any4.h).  Returns the list of y_i.  The
+    entries may instead all be Any4Prepared (any4_prepare): then only x, the
+    y's and the workspace are checked per call."""
     weights = list(weights)
     if not 1 <= len(weights) <= ANY4_GROUP_MAX:
         raise ValueError(f"between 1 and {ANY4_GROUP_MAX} matrices")
@@ -529,10 +651,53 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
     need_ws = 0
     lib = library()
     p = PATHS[path]
-    for i, (packed, lut, scale, offset) in enumerate(weights):
+    if isinstance(weights[0], Any4Prepared):
+        # prepared weights: only x, the y's and the workspace are checked here
+        descs, K, Gp, dev, di, ws_need = _prepared_group(weights)
+        if G != Gp:
+            raise ValueError(f"G={G} but the weights were prepared with G={Gp}")
+        M = _prepared_x(x, K, di)
+        for i, w in enumerate(weights):
+            if ys is None:
+                y = torch.empty((M, w.N), dtype=torch.float32 if fp32_out else torch.bfloat16,
+                                device=dev)
+            else:
+                y = ys[i]
+                _prepared_y(y, M, w.N, di, fp32_out)
+            outs.append(y)
+            descs[i].y = y.data_ptr()
+        need_ws = ws_need.get((M, p))
+        if need_ws is None:
+            need_ws = ws_need[(M, p)] = max(
+                int(lib.any4_matmul_workspace_size_ex(M, w.N, K, G, p)) for w in weights)
+        if workspace is None and need_ws > 0:
+            workspace = torch.empty(need_ws, dtype=torch.uint8, device=dev)
+        ws_bytes = 0
+        if workspace is not None:
+            if (not isinstance(workspace, torch.Tensor) or workspace.dtype != torch.uint8
+                    or workspace.get_device() != di or not workspace.is_contiguous()):
+                raise ValueError(f"workspace must be a contiguous uint8 tensor on cuda:{di}")
+            ws_bytes = workspace.numel()
+            if ws_bytes == 0:
+                workspace = None
+        _need_status(dev_status, dev)
+        st = _stream_index(di)
+        with _on_device(dev):
+            _check(lib.any4_matmul_grouped(x.data_ptr(), descs, len(weights), M, K, G,
+                                           _ptr(workspace), ws_bytes, _ptr(dev_status), p,
+                                           (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
+                                           | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
+                                           | (ANY4_FLAG_TEST_STALL if test_stall else 0)
+                                           | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
+                                           st), "any4_matmul_grouped")
+        return outs
+    for i, wt in enumerate(weights):
+        if isinstance(wt, Any4Prepared):
+            raise TypeError("mix of prepared and plain weights in one call")
+        packed, lut, scale, offset = wt
         y = None if ys is None else ys[i]
-        M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y, dev_status,
-                                              fp32_out)
+        M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y,
+                                              dev_status, fp32_out)
         outs.append(y)
         descs[i] = Any4Weight(_ptr(packed), _ptr(lut), stride, _ptr(scale), _ptr(offset),
                               _ptr(y), N)

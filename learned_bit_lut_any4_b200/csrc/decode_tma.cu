@@ -29,6 +29,7 @@
 #include <type_traits>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 
@@ -680,31 +681,87 @@ EncodeFn get_encode() {
   return fn;
 }
 
+// Encoded maps, kept on the host: a decode loop calls the same matrices over
+// and over, and a map depends only on the arguments in MapKey (address,
+// sizes, box, element type; not the device), so each distinct map is encoded
+// once.  Keys are zero-filled before use, so padding compares equal.
+struct MapKey {
+  const void* ptr;
+  uint64_t dims[2];
+  uint64_t stride;
+  uint32_t box[2];
+  int32_t dtype;
+  int32_t rank;
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    const unsigned char* b = reinterpret_cast<const unsigned char*>(&k);
+    uint64_t h = 1469598103934665603ull;  // FNV-1a
+    for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ b[i]) * 1099511628211ull;
+    return (size_t)h;
+  }
+};
+struct MapKeyEq {
+  bool operator()(const MapKey& a, const MapKey& b) const {
+    return memcmp(&a, &b, sizeof(MapKey)) == 0;
+  }
+};
+constexpr size_t kMapCacheMax = 8192;  // cleared when full
+
+bool cached_encode(EncodeFn enc, CUtensorMap* m, const MapKey& key) {
+  static std::mutex mu;
+  static auto* cache = new std::unordered_map<MapKey, CUtensorMap, MapKeyHash, MapKeyEq>();
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache->find(key);
+    if (it != cache->end()) {
+      *m = it->second;
+      return true;
+    }
+  }
+  const cuuint64_t dims[2] = {key.dims[0], key.dims[1]};
+  // a rank-1 map has no stride, but the encoder rejects a NULL stride array
+  const cuuint64_t strides[1] = {key.stride};
+  const cuuint32_t box[2] = {key.box[0], key.box[1]};
+  const cuuint32_t es[2] = {1, 1};
+  if (enc(m, (CUtensorMapDataType)key.dtype, (cuuint32_t)key.rank, const_cast<void*>(key.ptr),
+          dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache->size() >= kMapCacheMax) cache->clear();
+  cache->emplace(key, *m);
+  return true;
+}
+
 bool encode2d(EncodeFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* ptr,
               uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_inner,
               uint32_t box_rows) {
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t es[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  MapKey k;
+  memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = inner;
+  k.dims[1] = rows;
+  k.stride = row_bytes;
+  k.box[0] = box_inner;
+  k.box[1] = box_rows;
+  k.dtype = (int32_t)dt;
+  k.rank = 2;
+  return cached_encode(enc, m, k);
 }
 
 // 1-D map over n u16 values (the 2-bit tables: 8 bytes a row, below the
 // 16-byte row stride a 2-D map needs), box of box_n values
 bool encode1d(EncodeFn enc, CUtensorMap* m, const void* ptr, uint64_t n, uint32_t box_n) {
-  const cuuint64_t dims[1] = {n};
-  // a rank-1 map has no stride, but the encoder rejects a NULL stride array
-  const cuuint64_t unused_stride[1] = {((n * 2 + 15) / 16) * 16};
-  const cuuint32_t box[1] = {box_n};
-  const cuuint32_t es[1] = {1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 1, const_cast<void*>(ptr), dims, unused_stride, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  MapKey k;
+  memset(&k, 0, sizeof(k));
+  k.ptr = ptr;
+  k.dims[0] = n;
+  k.stride = ((n * 2 + 15) / 16) * 16;
+  k.box[0] = box_n;
+  k.dtype = (int32_t)CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  k.rank = 1;
+  return cached_encode(enc, m, k);
 }
 
 bool encode_weights(EncodeFn enc, TmaMaps* maps, const DecodeWeights& w, int64_t K, int64_t G,

@@ -376,3 +376,26 @@ def test_matmul_bits_workspace_sizes():
     assert ws(1, 4096, 4096, 256, 3) > 0
     assert ws(1, 4096, 4096, 128, 4) == any4.any4_matmul_workspace_size(1, 4096, 4096, 128)
     assert ws(1, 4096, 4096, 128, 5) == 0 and ws(0, 4096, 4096, 128, 3) == 0
+
+
+def test_prepare_checks_the_weights_once():
+    """any4_prepare checks a matrix's sizes, dtypes and device up front (sizes
+    first, so host tensors show them); a host matrix is refused."""
+    import torch
+    N, K, G = 16, 256, 64
+    packed = torch.zeros((N, K // 2), dtype=torch.uint8)
+    lut = torch.zeros((N, 16), dtype=torch.bfloat16)
+    so = torch.zeros((N, K // G), dtype=torch.bfloat16)
+    short = torch.zeros((N, K // G - 1), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="scale and offset"):
+        any4.any4_prepare(packed, lut, short, so, G)
+    with pytest.raises(ValueError, match="divide K"):
+        any4.any4_prepare(packed, lut, so, so, 96)
+    with pytest.raises(ValueError, match="lut must be"):
+        any4.any4_prepare(packed, lut[:8], so, so, G)
+    with pytest.raises(TypeError):
+        any4.any4_prepare(packed.to(torch.int32), lut, so, so, G)
+    with pytest.raises(TypeError):
+        any4.any4_prepare(packed, lut.float(), so, so, G)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        any4.any4_prepare(packed, lut, so, so, G)

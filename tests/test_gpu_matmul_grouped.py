@@ -115,3 +115,43 @@ def test_grouped_stall_times_out_cleanly():
     for (s, p, d, _), y in zip(probs, out):
         y_ref = oracle.any4_matmul(x, d.packed_ref, p.lut, p.scale, p.offset, 128)
         assert_matmul_close(host_bits(y), y_ref, s.name + " after the stall")
+
+
+@pytest.mark.parametrize("M,K,G,Ns,seed", [
+    (1, 4096, 128, (4096, 1024, 1024), 12101),   # q/k/v, the folded-table kernel
+    (1, 2048, 64, (333, 1024), 12102),           # G = 64 and a ragged N: the per-weight kernel
+    (4, 1024, 128, (512,), 12103),               # M > 1: one matrix per launch
+])
+def test_prepared_weights_equal_plain_call(M, K, G, Ns, seed):
+    """Weights checked once (any4_prepare) give the same bits as the plain call."""
+    x, probs = _problems(M, K, G, Ns, seed)
+    xd = dev_bf16(x)
+    weights = [(d.packed, dev_bf16(lut), d.scale, d.offset) for (_, _, d, lut) in probs]
+    prepared = [any4.any4_prepare(*w, G) for w in weights]
+    plain = any4.any4_matmul_grouped(xd, weights, G)
+    fast = any4.any4_matmul_grouped(xd, prepared, G)
+    ys = [torch.empty_like(y) for y in plain]
+    fast2 = any4.any4_matmul_grouped(xd, prepared, G, ys=ys)
+    torch.cuda.synchronize()
+    assert all(a is b for a, b in zip(fast2, ys))
+    for a, b, c in zip(plain, fast, fast2):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+
+
+def test_prepared_weights_check_x_and_y():
+    x, probs = _problems(1, 1024, 128, (256,), 12104)
+    _, _, d, lut = probs[0]
+    w = any4.any4_prepare(d.packed, dev_bf16(lut), d.scale, d.offset, 128)
+    xd = dev_bf16(x)
+    with pytest.raises(ValueError):
+        any4.any4_matmul_grouped(xd[:, :512].contiguous(), [w], 128)       # wrong K
+    with pytest.raises(ValueError):
+        any4.any4_matmul_grouped(xd, [w], 64)                              # another G
+    with pytest.raises(ValueError):
+        any4.any4_matmul_grouped(xd, [w], 128,
+                                 ys=[torch.empty((1, 255), dtype=torch.bfloat16, device="cuda")])
+    with pytest.raises(TypeError):
+        any4.any4_matmul_grouped(xd.float(), [w], 128)
+    with pytest.raises(TypeError):
+        any4.any4_matmul_grouped(xd, [w, (d.packed, dev_bf16(lut), d.scale, d.offset)], 128)
