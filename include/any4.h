@@ -282,7 +282,15 @@ typedef enum any4_flags {
    * workspace any4_matmul_workspace_size returns for the shape; without it,
    * or where the pair-table kernel does not take the shape, the flag is
    * ignored. */
-  ANY4_FLAG_PAIR_TABLE = 8
+  ANY4_FLAG_PAIR_TABLE = 8,
+  /* packed holds the codes in the decode layout that any4_repack writes, not
+   * any4_pack's.  Taken only where the M = 1 weight-streaming kernel with
+   * folded tables runs: M = 1, G = 128, K a multiple of 1024, path auto or
+   * decode, without ANY4_FLAG_PAIR_TABLE (any4_matmul_ex and
+   * any4_matmul_grouped); any other call with this flag returns
+   * ANY4_ERR_UNSUPPORTED.  Results are the same bits as the call on
+   * any4_pack's layout. */
+  ANY4_FLAG_DECODE_LAYOUT = 16
 } any4_flags;
 
 /* any4_matmul with an explicit kernel family (ANY4_PATH_DECODE needs M <= 16)
@@ -353,6 +361,27 @@ ANY4_API any4_status any4_matmul_static_scratch(const uint16_t* x, const uint8_t
 ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 
 /*
+ * any4_repack -- the packed codes rearranged for the M = 1 decode kernel
+ * (ANY4_FLAG_DECODE_LAYOUT).  The idea is the paper's (§4.2: its kernel reads
+ * weights pre-permuted into the order its threads consume them); the order
+ * here is this library's own.  Each row's codes go in 1024-column slices of
+ * 128 32-bit words (word w of a slice: codes of columns 8w .. 8w + 7, the
+ * even column in the low nibble, as any4_pack); within a slice, the 16-byte
+ * chunk l (l = 0..31, bytes 16 l .. 16 l + 15) holds, as its words t = 0..3,
+ * the input words 16 (4 h + (t XOR h)) + e with h = l / 16, e = l mod 16:
+ * the four words lane l of the kernel reads, one per step, so a lane loads
+ * them with one 16-byte load.  A permutation of whole 32-bit words within
+ * each slice; the tables, scales and offsets are unchanged.
+ *   packed    [N][K/2] uint8, any4_pack's layout                    (input)
+ *   repacked  [N][K/2] uint8, the decode layout; must not overlap packed
+ *   K         a multiple of 1024; N >= 1
+ * Both pointers 16-byte aligned device memory.  Errors: ANY4_ERR_NULL,
+ * ANY4_ERR_SHAPE, ANY4_ERR_ALIGN, ANY4_ERR_CUDA (launch).
+ */
+ANY4_API any4_status any4_repack(const uint8_t* packed, uint8_t* repacked, int64_t N, int64_t K,
+                                 any4_stream_t stream);
+
+/*
  * any4_matmul_grouped -- several weight matrices applied to the same x:
  *   y_i = x * dequant(W_i)^T   for i = 0 .. count-1
  * (the q, k and v projections of a transformer layer, or gate and up: the
@@ -375,7 +404,8 @@ ANY4_API size_t any4_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int6
  *              G, path) of the group where the per-matrix calls need one
  *   flags      as any4_matmul_ex (ANY4_FLAG_OVERLAP_PRIOR, _FP32_OUT,
  *              _TEST_STALL; ANY4_FLAG_PAIR_TABLE makes M = 1 take the
- *              per-matrix calls)
+ *              per-matrix calls; ANY4_FLAG_DECODE_LAYOUT: every packed is
+ *              in any4_repack's layout, M = 1 and G = 128 only)
  * Returns the first error of the validation (nothing launched), or of the
  * per-matrix calls (the earlier ones launched).
  */

@@ -38,6 +38,7 @@ from ._native import (  # noqa: F401
     any4_pack,
     any4_pack_bits,
     any4_prepare,
+    any4_repack,
     any4_quantize,
     any4_quantize_bits,
     any4_status_string,

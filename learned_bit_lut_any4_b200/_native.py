@@ -33,6 +33,7 @@ ANY4_FLAG_OVERLAP_PRIOR = 1
 ANY4_FLAG_FP32_OUT = 2
 ANY4_FLAG_TEST_STALL = 4
 ANY4_FLAG_PAIR_TABLE = 8
+ANY4_FLAG_DECODE_LAYOUT = 16
 # Limits of any4_quantize (the row lives in one block's shared memory).
 ANY4_QUANTIZE_MAX_K = 16384
 ANY4_QUANTIZE_MAX_ITER = 100000
@@ -72,6 +73,8 @@ def library() -> ctypes.CDLL:
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     lib.any4_pack.argtypes = [vp, vp, i64, i64, vp, vp]
     lib.any4_pack.restype = i32
+    lib.any4_repack.argtypes = [vp, vp, i64, i64, vp]
+    lib.any4_repack.restype = i32
     lib.any4_quantize.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
     lib.any4_quantize.restype = i32
     lib.any4_quantize_bits.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -211,6 +214,27 @@ def any4_pack(idx: torch.Tensor, packed: torch.Tensor | None = None,
         _check(library().any4_pack(_ptr(idx), _ptr(packed), N, K, _ptr(dev_status),
                                    _stream(idx.device)), "any4_pack")
     return packed
+
+
+def any4_repack(packed: torch.Tensor, repacked: torch.Tensor | None = None) -> torch.Tensor:
+    """uint8 packed [N, K/2] (any4_pack's layout) -> the same codes in the M = 1
+    decode kernel's layout (see any4_repack in include/any4.h); K a multiple of
+    1024.  Use the result with decode_layout=True (M = 1, G = 128 only)."""
+    if not isinstance(packed, torch.Tensor) or packed.dim() != 2:
+        raise ValueError("packed must be a [N, K/2] tensor")
+    N, Kh = packed.shape
+    if (2 * Kh) % 1024 != 0 or Kh == 0:
+        raise ValueError(f"K = {2 * Kh} must be a positive multiple of 1024")
+    if repacked is not None:
+        _need_shape(repacked, "repacked", (N, Kh))
+    _need(packed, "packed", (torch.uint8,))
+    if repacked is None:
+        repacked = torch.empty_like(packed)
+    _need(repacked, "repacked", (torch.uint8,), packed.device)
+    with torch.cuda.device(packed.device):
+        _check(library().any4_repack(_ptr(packed), _ptr(repacked), N, 2 * Kh,
+                                     _stream(packed.device)), "any4_repack")
+    return repacked
 
 
 def any4_quantize(w: torch.Tensor, ex_abs: torch.Tensor, G: int, max_iter: int = 100,
@@ -404,10 +428,12 @@ class Any4Prepared:
     The tensors must stay as they are (not resized, not moved) while it is in
     use."""
     __slots__ = ("packed", "lut", "scale", "offset", "G", "N", "K", "lut_row_stride",
-                 "device", "_ptrs", "__weakref__")
+                 "device", "decode_layout", "_ptrs", "__weakref__")
 
-    def __init__(self, packed, lut, scale, offset, G):
+    def __init__(self, packed, lut, scale, offset, G, decode_layout=False):
         N, K, stride = _weight_operands(packed, lut, scale, offset, G)
+        if decode_layout and (G != 128 or K % 1024 != 0):
+            raise ValueError("the decode layout needs G = 128 and K a multiple of 1024")
         dev = packed.device
         _need(packed, "packed", (torch.uint8,))
         for t, nm in ((lut, "lut"), (scale, "scale"), (offset, "offset")):
@@ -415,6 +441,7 @@ class Any4Prepared:
         self.packed, self.lut, self.scale, self.offset = packed, lut, scale, offset
         self.G, self.N, self.K, self.lut_row_stride = int(G), int(N), int(K), stride
         self.device = dev
+        self.decode_layout = bool(decode_layout)
         self._ptrs = (packed.data_ptr(), lut.data_ptr(), scale.data_ptr(), offset.data_ptr())
 
     def __repr__(self):
@@ -422,9 +449,10 @@ class Any4Prepared:
 
 
 def any4_prepare(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
-                 offset: torch.Tensor, G: int) -> Any4Prepared:
-    """Check an any4 matrix once for repeated calls (see Any4Prepared)."""
-    return Any4Prepared(packed, lut, scale, offset, G)
+                 offset: torch.Tensor, G: int, decode_layout: bool = False) -> Any4Prepared:
+    """Check an any4 matrix once for repeated calls (see Any4Prepared);
+    decode_layout: packed comes from any4_repack."""
+    return Any4Prepared(packed, lut, scale, offset, G, decode_layout)
 
 
 # Per thread: the ctypes descriptor array of each group of prepared weights
@@ -445,8 +473,10 @@ def _prepared_group(weights):
         for w in weights:
             if not isinstance(w, Any4Prepared):
                 raise TypeError("mix of prepared and plain weights in one call")
-            if w.device != w0.device or w.K != w0.K or w.G != w0.G:
-                raise ValueError("prepared weights of one call must share device, K and G")
+            if (w.device != w0.device or w.K != w0.K or w.G != w0.G
+                    or w.decode_layout != w0.decode_layout):
+                raise ValueError("prepared weights of one call must share device, K, G and "
+                                 "code layout")
         descs = (Any4Weight * len(weights))()
         for i, w in enumerate(weights):
             pk, lt, sc, of = w._ptrs
@@ -454,7 +484,7 @@ def _prepared_group(weights):
         if len(cache) >= _PREPARED_GROUPS_MAX:
             cache.clear()
         di = w0.device.index if w0.device.index is not None else -1
-        g = cache[key] = [descs, w0.K, w0.G, w0.device, di, {}]
+        g = cache[key] = [descs, w0.K, w0.G, w0.device, di, {}, w0.decode_layout]
     return g
 
 
@@ -549,7 +579,8 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                 y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 path: str = "auto", dev_status: torch.Tensor | None = None,
                 overlap_prior: bool = False, fp32_out: bool = False,
-                test_stall: bool = False, pair_table: bool = False) -> torch.Tensor:
+                test_stall: bool = False, pair_table: bool = False,
+                decode_layout: bool = False) -> torch.Tensor:
     """bf16 y[M, N] = x[M, K] * dequant(W)^T, fp32 accumulation.
 
     workspace: a CUDA tensor of at least any4_matmul_workspace_size() bytes, or
@@ -561,7 +592,9 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
     test_stall: ANY4_FLAG_TEST_STALL, a test of the failure handling (one
     block's stream stops, the call ends with ANY4_ERR_TIMEOUT in dev_status).
     pair_table: ANY4_FLAG_PAIR_TABLE, M = 1 on the pair-table kernel (needs
-    the workspace) instead of the weight-streaming kernel."""
+    the workspace) instead of the weight-streaming kernel.
+    decode_layout: ANY4_FLAG_DECODE_LAYOUT, packed comes from any4_repack
+    (M = 1, G = 128 only)."""
     M, N, K, stride, y = _matmul_operands(x, packed, lut, scale, offset, G, y,
                                              dev_status, fp32_out)
     dev = x.device
@@ -587,7 +620,8 @@ def any4_matmul(x: torch.Tensor, packed: torch.Tensor, lut: torch.Tensor,
                                   (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
                                   | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
                                   | (ANY4_FLAG_TEST_STALL if test_stall else 0)
-                                  | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
+                                  | (ANY4_FLAG_PAIR_TABLE if pair_table else 0)
+                                  | (ANY4_FLAG_DECODE_LAYOUT if decode_layout else 0),
                                   _stream(dev)), "any4_matmul")
     return y
 
@@ -634,12 +668,14 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
                         workspace: torch.Tensor | None = None, path: str = "auto",
                         dev_status: torch.Tensor | None = None, overlap_prior: bool = False,
                         fp32_out: bool = False, test_stall: bool = False,
-                        pair_table: bool = False):
+                        pair_table: bool = False, decode_layout: bool = False):
     """[y_i = x * dequant(W_i)^T for each (packed, lut, scale, offset) in
     weights]: matrices that share x, in one launch at M = 1 (see
     any4_matmul_grouped in include/any4.h).  Returns the list of y_i.  The
     entries may instead all be Any4Prepared (any4_prepare): then only x, the
-    y's and the workspace are checked per call."""
+    y's and the workspace are checked per call, and their decode_layout
+    (any4_repack'd codes) applies.  decode_layout: the plain entries' packed
+    come from any4_repack (M = 1, G = 128 only)."""
     weights = list(weights)
     if not 1 <= len(weights) <= ANY4_GROUP_MAX:
         raise ValueError(f"between 1 and {ANY4_GROUP_MAX} matrices")
@@ -653,7 +689,7 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
     p = PATHS[path]
     if isinstance(weights[0], Any4Prepared):
         # prepared weights: only x, the y's and the workspace are checked here
-        descs, K, Gp, dev, di, ws_need = _prepared_group(weights)
+        descs, K, Gp, dev, di, ws_need, dl = _prepared_group(weights)
         if G != Gp:
             raise ValueError(f"G={G} but the weights were prepared with G={Gp}")
         M = _prepared_x(x, K, di)
@@ -688,7 +724,8 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
                                            (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
                                            | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
                                            | (ANY4_FLAG_TEST_STALL if test_stall else 0)
-                                           | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
+                                           | (ANY4_FLAG_PAIR_TABLE if pair_table else 0)
+                                           | (ANY4_FLAG_DECODE_LAYOUT if dl else 0),
                                            st), "any4_matmul_grouped")
         return outs
     for i, wt in enumerate(weights):
@@ -718,7 +755,8 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
                                        (ANY4_FLAG_OVERLAP_PRIOR if overlap_prior else 0)
                                        | (ANY4_FLAG_FP32_OUT if fp32_out else 0)
                                        | (ANY4_FLAG_TEST_STALL if test_stall else 0)
-                                       | (ANY4_FLAG_PAIR_TABLE if pair_table else 0),
+                                       | (ANY4_FLAG_PAIR_TABLE if pair_table else 0)
+                                       | (ANY4_FLAG_DECODE_LAYOUT if decode_layout else 0),
                                        _stream(dev)), "any4_matmul_grouped")
     return outs
 

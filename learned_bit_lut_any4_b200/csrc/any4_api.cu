@@ -163,6 +163,20 @@ any4_status any4_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
   return launch_pack(idx, packed, N, K, dev_status, (cudaStream_t)stream, dev);
 }
 
+any4_status any4_repack(const uint8_t* packed, uint8_t* repacked, int64_t N, int64_t K,
+                        any4_stream_t stream) {
+  if (!packed || !repacked) return ANY4_ERR_NULL;
+  if (N < 1 || K < 1024 || K % 1024 != 0 || N > (int64_t(1) << 40) / K) return ANY4_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(repacked)) return ANY4_ERR_ALIGN;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(packed), b0 = reinterpret_cast<uintptr_t>(repacked);
+  const uintptr_t bytes = (uintptr_t)(N * (K / 2));
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return ANY4_ERR_SHAPE;  // the buffers overlap
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_repack(packed, repacked, N, K, (cudaStream_t)stream, dev);
+}
+
 any4_status any4_quantize(const uint16_t* w, const float* ex_abs, int64_t N, int64_t K,
                           int64_t G, int32_t max_iter, uint8_t* packed, uint16_t* lut,
                           uint16_t* scale, uint16_t* offset, int32_t* iters,
@@ -258,9 +272,15 @@ any4_status any4_matmul_grouped(const uint16_t* x, const any4_weight* w, int32_t
   if (!aligned16(x)) return ANY4_ERR_ALIGN;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return ANY4_ERR_ALIGN;
   if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL |
-                         ANY4_FLAG_PAIR_TABLE))
+                         ANY4_FLAG_PAIR_TABLE | ANY4_FLAG_DECODE_LAYOUT))
     return ANY4_ERR_UNSUPPORTED;
   const any4_path chosen = path == ANY4_PATH_AUTO ? any4_matmul_choose_path(M, 1, K, G) : path;
+  const bool decode_layout = (flags & ANY4_FLAG_DECODE_LAYOUT) != 0;
+  if (decode_layout) {
+    if (chosen != ANY4_PATH_DECODE || (flags & ANY4_FLAG_PAIR_TABLE)) return ANY4_ERR_UNSUPPORTED;
+    for (int i = 0; i < count; ++i)
+      if (!decode_layout_supported(M, w[i].N, K, G)) return ANY4_ERR_UNSUPPORTED;
+  }
   bool one_launch = chosen == ANY4_PATH_DECODE && !(flags & ANY4_FLAG_PAIR_TABLE);
   for (int i = 0; i < count && one_launch; ++i)
     one_launch = decode_tma_supported(M, w[i].N, K, G);
@@ -276,7 +296,7 @@ any4_status any4_matmul_grouped(const uint16_t* x, const any4_weight* w, int32_t
                w[i].N};
     return launch_decode_tma_group(x, dw, count, K, G, 4, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,
                                    dev_status, (flags & ANY4_FLAG_TEST_STALL) != 0,
-                                   (cudaStream_t)stream, dev);
+                                   (cudaStream_t)stream, dev, decode_layout);
   }
   for (int i = 0; i < count; ++i) {
     const any4_status st =
@@ -388,7 +408,11 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   if (path == ANY4_PATH_AUTO) path = any4_matmul_choose_path(M, N, K, G);
   if (path != ANY4_PATH_DECODE && path != ANY4_PATH_PREFILL) return ANY4_ERR_UNSUPPORTED;
   if (flags & ~(uint32_t)(ANY4_FLAG_OVERLAP_PRIOR | ANY4_FLAG_FP32_OUT | ANY4_FLAG_TEST_STALL |
-                         ANY4_FLAG_PAIR_TABLE))
+                         ANY4_FLAG_PAIR_TABLE | ANY4_FLAG_DECODE_LAYOUT))
+    return ANY4_ERR_UNSUPPORTED;
+  const bool decode_layout = (flags & ANY4_FLAG_DECODE_LAYOUT) != 0;
+  if (decode_layout && (path != ANY4_PATH_DECODE || (flags & ANY4_FLAG_PAIR_TABLE) ||
+                        !decode_layout_supported(M, N, K, G)))
     return ANY4_ERR_UNSUPPORTED;
   float* y32 = (flags & ANY4_FLAG_FP32_OUT) ? reinterpret_cast<float*>(y) : nullptr;
   const bool test_stall = (flags & ANY4_FLAG_TEST_STALL) != 0;
@@ -404,6 +428,10 @@ any4_status any4_matmul_ex(const uint16_t* x, const uint8_t* packed, const uint1
   DeviceInfo dev;
   any4_status st = current_device(&dev);
   if (st != ANY4_OK) return st;
+  if (decode_layout)  // only the folded-table M = 1 kernel reads this layout
+    return launch_decode_tma(x, packed, lut, lut_row_stride, scale, offset, y, y32, N, K, G,
+                             (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0, dev_status, test_stall,
+                             (cudaStream_t)stream, dev, true);
   if (path == ANY4_PATH_DECODE) {
     return launch_decode(x, packed, lut, lut_row_stride, scale, offset, y, y32, M, N, K, G,
                          workspace, workspace_bytes, (flags & ANY4_FLAG_OVERLAP_PRIOR) != 0,

@@ -174,16 +174,24 @@ struct DecodeWeights {
   int64_t N;
 };
 // M = 1 on the weight-streaming kernel for up to ANY4_GROUP_MAX matrices that
-// share x, K and G, in one launch.
+// share x, K and G, in one launch (decode_layout: the codes are in
+// any4_repack's layout; only where decode_layout_supported).
 any4_status launch_decode_tma_group(const uint16_t* x, const DecodeWeights* w, int count,
                                     int64_t K, int64_t G, int bits, bool overlap,
                                     int32_t* dev_status, bool test_stall, cudaStream_t stream,
-                                    const DeviceInfo& dev);
+                                    const DeviceInfo& dev, bool decode_layout = false);
 any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const uint16_t* lut,
                               int64_t lut_row_stride, const uint16_t* scale,
                               const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
                               int64_t K, int64_t G, bool overlap, int32_t* dev_status,
-                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev);
+                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev,
+                              bool decode_layout = false);
+// The folded-table M = 1 kernel takes the shape, so codes in any4_repack's
+// layout can be used (M = 1, G = 128, K a multiple of 1024).
+bool decode_layout_supported(int64_t M, int64_t N, int64_t K, int64_t G);
+// any4_repack: packed codes into the decode layout (pack_dequant.cu).
+any4_status launch_repack(const uint8_t* packed, uint8_t* repacked, int64_t N, int64_t K,
+                          cudaStream_t stream, const DeviceInfo& dev);
 size_t prefill_workspace_size(int64_t M, int64_t N, int64_t K, int64_t G);
 // n-bit (2 or 3) dequant into a bf16 W (nbit.cu).
 any4_status launch_dequant_bits(const uint8_t* packed, const uint16_t* lut,

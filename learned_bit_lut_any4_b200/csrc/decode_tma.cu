@@ -453,10 +453,10 @@ __device__ __forceinline__ float fold_fetch(uint32_t tab, uint32_t code) {
   return __uint_as_float(v);
 }
 
-#ifndef ANY4_FFMA_REGS
-#define ANY4_FFMA_REGS 128
-#endif
-__global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
+// kDecodeLayout: the codes are in any4_repack's layout, where the four words
+// a lane reads in a row's 1024-column slice sit together (one 16-byte load)
+template <bool kDecodeLayout>
+__global__ void __maxnreg__(128) decode_tma_ffma_kernel(
     const __grid_constant__ TmaGroup grp, const uint16_t* __restrict__ x, int K, int nslices,
     int rows_per_block, int32_t* dev_status, int test_stall) {
   constexpr int GPS = 8, BITS = 4;
@@ -576,10 +576,15 @@ __global__ void __maxnreg__(ANY4_FFMA_REGS) decode_tma_ffma_kernel(
         // once per stage, outside the unrolled rows)
         auto row = [&](int j, auto shared) -> float {
           uint32_t w[4];
-          w[0] = codes[j * kRowWords + wofs0];
-          w[1] = codes[j * kRowWords + wofs1];
-          w[2] = codes[j * kRowWords + wofs0 + 32];
-          w[3] = codes[j * kRowWords + wofs1 + 32];
+          if constexpr (kDecodeLayout) {
+            const uint4 q4 = reinterpret_cast<const uint4*>(codes + j * kRowWords)[lane];
+            w[0] = q4.x; w[1] = q4.y; w[2] = q4.z; w[3] = q4.w;
+          } else {
+            w[0] = codes[j * kRowWords + wofs0];
+            w[1] = codes[j * kRowWords + wofs1];
+            w[2] = codes[j * kRowWords + wofs0 + 32];
+            w[3] = codes[j * kRowWords + wofs1 + 32];
+          }
           uint32_t l2;
           if constexpr (decltype(shared)::value)
             l2 = lv_shared;
@@ -790,8 +795,8 @@ bool encode_weights(EncodeFn enc, TmaMaps* maps, const DecodeWeights& w, int64_t
 
 template <int GPS, int BITS>
 any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_t K, int64_t G,
-                    bool overlap, int32_t* dev_status, bool test_stall, cudaStream_t stream,
-                    const DeviceInfo& dev) {
+                    bool overlap, int32_t* dev_status, bool test_stall, bool decode_layout,
+                    cudaStream_t stream, const DeviceInfo& dev) {
   using St = TmaStage<GPS, BITS>;
   constexpr int P = St::P;
   constexpr int S = kTmaStages;
@@ -810,7 +815,9 @@ any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_
   // G = 128 with 4-bit codes: the folded-table kernel; every other shape:
   // the per-weight multiply-add kernel
   constexpr bool kFold = GPS == 8 && BITS == 4;
-  auto kern = kFold ? decode_tma_ffma_kernel : decode_tma_kernel<GPS, BITS>;
+  if (decode_layout && (!kFold || K % 1024 != 0)) return ANY4_ERR_UNSUPPORTED;
+  auto kern = kFold ? (decode_layout ? decode_tma_ffma_kernel<true> : decode_tma_ffma_kernel<false>)
+                    : decode_tma_kernel<GPS, BITS>;
   const size_t ring_bytes = (size_t)nwarps * S * St::kBytes + (size_t)nwarps * S * 8 + 16 + 128;
   const int kMaxRT = 512;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern),
@@ -880,14 +887,17 @@ any4_status run_tma(const uint16_t* x, const DecodeWeights* w, int count, int64_
 template <int BITS>
 any4_status run_tma_bits(const uint16_t* x, const DecodeWeights* w, int count, int64_t K,
                          int64_t G, bool overlap, int32_t* dev_status, bool test_stall,
-                         cudaStream_t stream, const DeviceInfo& dev) {
+                         bool decode_layout, cudaStream_t stream, const DeviceInfo& dev) {
   switch (G) {
     case 128:
-      return run_tma<8, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma<8, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, decode_layout,
+                              stream, dev);
     case 64:
-      return run_tma<16, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma<16, BITS>(x, w, count, K, G, overlap, dev_status, test_stall,
+                               decode_layout, stream, dev);
     case 32:
-      return run_tma<32, BITS>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma<32, BITS>(x, w, count, K, G, overlap, dev_status, test_stall,
+                               decode_layout, stream, dev);
     default:
       return ANY4_ERR_UNSUPPORTED;
   }
@@ -908,14 +918,17 @@ bool decode_tma_supported(int64_t M, int64_t N, int64_t K, int64_t G, int bits) 
 any4_status launch_decode_tma_group(const uint16_t* x, const DecodeWeights* w, int count,
                                     int64_t K, int64_t G, int bits, bool overlap,
                                     int32_t* dev_status, bool test_stall, cudaStream_t stream,
-                                    const DeviceInfo& dev) {
+                                    const DeviceInfo& dev, bool decode_layout) {
   switch (bits) {
     case 4:
-      return run_tma_bits<4>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma_bits<4>(x, w, count, K, G, overlap, dev_status, test_stall, decode_layout,
+                             stream, dev);
     case 3:
-      return run_tma_bits<3>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma_bits<3>(x, w, count, K, G, overlap, dev_status, test_stall, decode_layout,
+                             stream, dev);
     case 2:
-      return run_tma_bits<2>(x, w, count, K, G, overlap, dev_status, test_stall, stream, dev);
+      return run_tma_bits<2>(x, w, count, K, G, overlap, dev_status, test_stall, decode_layout,
+                             stream, dev);
     default:
       return ANY4_ERR_UNSUPPORTED;
   }
@@ -925,10 +938,15 @@ any4_status launch_decode_tma(const uint16_t* x, const uint8_t* packed, const ui
                               int64_t lut_row_stride, const uint16_t* scale,
                               const uint16_t* offset, uint16_t* y, float* y32, int64_t N,
                               int64_t K, int64_t G, bool overlap, int32_t* dev_status,
-                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev) {
+                              bool test_stall, cudaStream_t stream, const DeviceInfo& dev,
+                              bool decode_layout) {
   const DecodeWeights w = {packed, lut, lut_row_stride, scale, offset, y, y32, N};
   return launch_decode_tma_group(x, &w, 1, K, G, 4, overlap, dev_status, test_stall, stream,
-                                 dev);
+                                 dev, decode_layout);
+}
+
+bool decode_layout_supported(int64_t M, int64_t N, int64_t K, int64_t G) {
+  return M == 1 && G == 128 && K % 1024 == 0 && decode_tma_supported(M, N, K, G);
 }
 
 }  // namespace any4

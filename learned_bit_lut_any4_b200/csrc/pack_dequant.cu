@@ -274,7 +274,36 @@ int grid_for(int64_t work_items, int threads, const DeviceInfo& dev, int blocks_
   return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+// any4_repack: one thread per 16-byte chunk of the decode layout (chunk l of
+// a row's 1024-column slice: the slice's words 16 (4h + (t ^ h)) + e for
+// t = 0..3, h = l / 16, e = l mod 16).  The four gathered words of a warp's
+// threads come from the same 512-byte slice (one cache line set), the store
+// is one coalesced 16-byte write per thread.
+__global__ void __launch_bounds__(256) repack_kernel(const uint32_t* __restrict__ in,
+                                                      uint4* __restrict__ out, int64_t chunks) {
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int l = (int)(c & 31);
+    const int h = l >> 4, e = l & 15;
+    const uint32_t* slice = in + (c >> 5) * 128;
+    uint4 v;
+    v.x = __ldg(slice + 16 * (4 * h + (0 ^ h)) + e);
+    v.y = __ldg(slice + 16 * (4 * h + (1 ^ h)) + e);
+    v.z = __ldg(slice + 16 * (4 * h + (2 ^ h)) + e);
+    v.w = __ldg(slice + 16 * (4 * h + (3 ^ h)) + e);
+    out[c] = v;
+  }
+}
+
 }  // namespace
+
+any4_status launch_repack(const uint8_t* packed, uint8_t* repacked, int64_t N, int64_t K,
+                          cudaStream_t stream, const DeviceInfo& dev) {
+  const int64_t chunks = N * (K / 1024) * 32;  // a slice is 1024 codes = 32 chunks of 16 bytes
+  repack_kernel<<<grid_for(chunks, 256, dev, 8), 256, 0, stream>>>(
+      reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<uint4*>(repacked), chunks);
+  return cudaGetLastError() == cudaSuccess ? ANY4_OK : ANY4_ERR_CUDA;
+}
 
 any4_status launch_pack(const uint8_t* idx, uint8_t* packed, int64_t N, int64_t K,
                         int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {

@@ -12,6 +12,8 @@ Every function follows "any4: Learned 4-bit Numeric Representation for LLMs"
   dequant            §2.5.2 dequant(w_Q) = alpha*w_Q + beta with w_Q = LUT[code];
                      §2.5.1 group k covers columns k*G .. (k+1)*G-1
   matmul             §4.1 Eq. 8 and §4.2 (y = x W^T, x is M x K, W is N x K)
+  repack_decode_layout  §4.2's pre-permuted weight order, for the library's
+                     M = 1 kernel: which 8 columns a thread reads at a step
   group_sums         per-group activation sums, the factor of the group offset
                      when Eq. 8 is expanded with the group-affine weights of
                      §2.5.2 (the pages do not name it; this is that reading)
@@ -66,6 +68,8 @@ def _bind(lib):
     lib.oracle_pack.restype = i64
     lib.oracle_unpack.argtypes = [u8p, u8p, i64, i64]
     lib.oracle_unpack.restype = None
+    lib.oracle_repack_decode_layout.argtypes = [u8p, u8p, i64, i64]
+    lib.oracle_repack_decode_layout.restype = ctypes.c_int
     lib.oracle_bits_per_weight.argtypes = [i64, i64, i64, i64]
     lib.oracle_bits_per_weight.restype = ctypes.c_double
     lib.oracle_dequant_one.argtypes = [ctypes.c_uint16] * 3
@@ -187,6 +191,19 @@ def unpack(packed: np.ndarray) -> np.ndarray:
     idx = np.empty((N, 2 * Kh), dtype=np.uint8)
     _load().oracle_unpack(_ptr(packed, ctypes.c_uint8), _ptr(idx, ctypes.c_uint8), N, 2 * Kh)
     return idx
+
+
+def repack_decode_layout(packed: np.ndarray) -> np.ndarray:
+    """packed uint8 [N, K/2] (pack's layout) -> the same codes in the order the
+    library's M = 1 decode kernel reads them (any4_repack); K a multiple of
+    1024.  The statement is oracle_repack_decode_layout in any4_oracle.c."""
+    packed = _c(packed, np.uint8)
+    N, Kh = packed.shape
+    out = np.empty_like(packed)
+    if _load().oracle_repack_decode_layout(_ptr(packed, ctypes.c_uint8),
+                                           _ptr(out, ctypes.c_uint8), N, 2 * Kh) != 0:
+        raise ValueError("K must be a positive multiple of 1024")
+    return out
 
 
 def bits_per_weight(K: int, G: int, lut_bits: int = 16, group_param_bits: int = 16) -> float:

@@ -113,6 +113,31 @@ void oracle_unpack(const uint8_t* packed, uint8_t* idx, int64_t N, int64_t K) {
       idx[n * K + k] = (uint8_t)code_at(packed, K, n, k);
 }
 
+/* The packed codes in the order the library's M = 1 decode kernel reads them
+ * (§4.2: the paper's kernel reads weights pre-permuted into the order its
+ * threads consume them).  In each row's 1024-column slice, thread l (0..31)
+ * of a warp covers at step t (0..3) the 8 columns 128 q + 8 (l mod 16) .. + 7
+ * of the slice, q = 4 h + (t XOR h) with h = l div 16; the layout stores the
+ * 4 bytes holding those 8 codes, for l in order and, within l, t in order.
+ * Returns 0, or -1 when K is not a positive multiple of 1024. */
+int oracle_repack_decode_layout(const uint8_t* packed, uint8_t* out, int64_t N, int64_t K) {
+  if (K <= 0 || K % 1024 != 0) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* src = packed + n * (K / 2);
+    uint8_t* dst = out + n * (K / 2);
+    for (int64_t s = 0; s < K / 1024; ++s)
+      for (int l = 0; l < 32; ++l) {
+        int h = l / 16, e = l % 16;
+        for (int t = 0; t < 4; ++t) {
+          int64_t col = 1024 * s + 128 * (4 * h + (t ^ h)) + 8 * e;
+          int64_t at = 512 * s + 16 * l + 4 * t;
+          for (int b = 0; b < 4; ++b) dst[at + b] = src[col / 2 + b];
+        }
+      }
+  }
+  return 0;
+}
+
 /* Bits stored per weight: the 4-bit code, plus a 16-bit scale and a 16-bit
  * zero point per group of G, plus a 16-entry table of lut_bits-wide values
  * per row of K weights (§2.4.1 works this out as 4 + 0.25 + 0.0625 = 4.3125

@@ -841,4 +841,43 @@ def pin_quantize_bits_error_falls_with_more_bits():
     assert errs[0] > 2 * errs[1] > 4 * errs[2], errs
 
 
+# --------------------------------------------------------------------------
+# the M = 1 decode layout (any4_repack): positions worked by hand, invariants
+# --------------------------------------------------------------------------
+
+def _word_index_rows(K: int) -> np.ndarray:
+    """One row whose 32-bit word w holds the value w in each of its bytes
+    (w < 256), so a byte of the repacked row names the word it came from."""
+    words = np.arange(K // 8, dtype=np.uint32)
+    assert words.max() < 256
+    return np.repeat(words.astype(np.uint8), 4).reshape(1, K // 2)
+
+
+def pin_repack_decode_layout_worked_positions():
+    for row in read_golden("repack_decode_layout.txt"):
+        K, lane, w0, w1, w2, w3, sl = (int(v) for v in row.split())
+        got = oracle.repack_decode_layout(_word_index_rows(K))[0]
+        for t, want in enumerate((w0, w1, w2, w3)):
+            at = 512 * sl + 16 * lane + 4 * t
+            assert np.all(got[at:at + 4] == want), (K, lane, t, got[at:at + 4], want)
+
+
+def pin_repack_decode_layout_is_a_word_permutation():
+    # whole 32-bit words move, inside their own 1024-column slice, row by row
+    rng = np.random.default_rng(11)
+    packed = rng.integers(0, 256, size=(3, 14336 // 2), dtype=np.uint8)
+    out = oracle.repack_decode_layout(packed)
+    for n in range(3):
+        a = packed[n].view(np.uint32).reshape(-1, 128)
+        b = out[n].view(np.uint32).reshape(-1, 128)
+        for sl in range(a.shape[0]):
+            assert np.array_equal(np.sort(a[sl]), np.sort(b[sl])), (n, sl)
+        assert np.array_equal(out[n], oracle.repack_decode_layout(packed[n:n + 1])[0])
+    try:
+        oracle.repack_decode_layout(np.zeros((1, 768), dtype=np.uint8))
+    except ValueError:
+        return
+    raise AssertionError("K = 1536 was accepted")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

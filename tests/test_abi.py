@@ -79,12 +79,35 @@ def _matmul(M=1, N=64, K=128, G=32, x=FAKE, packed=FAKE, lut=FAKE, stride=16, sc
     (dict(status=FAKE + 2), any4.ANY4_ERR_ALIGN),
     (dict(M=17, path=1), any4.ANY4_ERR_UNSUPPORTED),
     (dict(path=7), any4.ANY4_ERR_UNSUPPORTED),
-    (dict(flags=16), any4.ANY4_ERR_UNSUPPORTED),
     (dict(flags=32), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(flags=64), any4.ANY4_ERR_UNSUPPORTED),
+    # the decode layout: only M = 1, G = 128, K a multiple of 1024, decode path
+    (dict(flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(M=2, K=4096, G=128, flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(K=4096, G=64, flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(K=3072 - 1024 + 512, G=128, flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(K=4096, G=128, path=2, flags=16), any4.ANY4_ERR_UNSUPPORTED),
+    (dict(K=4096, G=128, flags=16 | 8), any4.ANY4_ERR_UNSUPPORTED),
     (dict(ws=FAKE + 8, ws_bytes=1 << 20), any4.ANY4_ERR_ALIGN),
 ])
 def test_matmul_rejects_bad_arguments(kw, expect):
     assert _matmul(**kw) == expect
+
+
+def test_repack_rejects_bad_arguments():
+    lib = _native.library()
+    N, K = 4, 2048
+    assert lib.any4_repack(None, FAKE, N, K, None) == any4.ANY4_ERR_NULL
+    assert lib.any4_repack(FAKE, None, N, K, None) == any4.ANY4_ERR_NULL
+    assert lib.any4_repack(FAKE, FAKE + (1 << 20), N, 1536, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_repack(FAKE, FAKE + (1 << 20), 0, K, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_repack(FAKE + 4, FAKE + (1 << 20), N, K, None) == any4.ANY4_ERR_ALIGN
+    # in place, or overlapping, is refused (the layout is a gather)
+    assert lib.any4_repack(FAKE, FAKE, N, K, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_repack(FAKE, FAKE + 1024, N, K, None) == any4.ANY4_ERR_SHAPE
+    import torch
+    with pytest.raises(ValueError, match="multiple of 1024"):
+        any4.any4_repack(torch.zeros((4, 768), dtype=torch.uint8))
 
 
 def test_pack_and_dequant_reject_bad_arguments():

@@ -85,6 +85,11 @@ MUTANTS = [
      "      float acc = 0.0f;\n      for (int64_t k = g * G;"),
     ("storage_bits_one_param", "4.0 + (2.0 * (double)group_param_bits) / (double)G",
      "4.0 + (1.0 * (double)group_param_bits) / (double)G"),
+    ("repack_without_xor", "int64_t col = 1024 * s + 128 * (4 * h + (t ^ h)) + 8 * e;",
+     "int64_t col = 1024 * s + 128 * (4 * h + t) + 8 * e;"),
+    ("repack_halves_interleaved", "int h = l / 16, e = l % 16;", "int h = l % 2, e = l / 2;"),
+    ("repack_steps_reversed", "int64_t at = 512 * s + 16 * l + 4 * t;",
+     "int64_t at = 512 * s + 16 * l + 4 * (3 - t);"),
 ]
 
 
