@@ -304,24 +304,28 @@ def fig3_square_sweep(stream, overlap):
     return out
 
 
-def time_weight_set(shapes, stream, overlap, peaks):
+def time_weight_set(shapes, stream, overlap, peaks, decode_layout=False):
     """Time any4_matmul on one weight set (the shapes share a weight seed and
     differ in M and x) on rotating weight copies larger than L2, replayed in
     a CUDA graph; per shape µs per call, GB/s of its algorithmic bytes and the
-    fraction of the HBM peak (+ TFLOPS for M > 16)."""
+    fraction of the HBM peak (+ TFLOPS for M > 16).  decode_layout: the codes
+    repacked by any4_repack (set-up, untimed) and read with that flag."""
     import torch
     import learned_bit_lut_any4_b200 as any4
     s0 = shapes[0]
     wbytes = s0.N * s0.K // 2 + 4 * s0.N * (s0.K // s0.G) + 32 * s0.N
     bc = max(2, int(np.ceil(3 * L2_BYTES / wbytes)))
     (_, reps, _, _, _), = prepare_layer([s0], bc)
+    if decode_layout:
+        reps = [(any4.any4_repack(w[0]), w[1], w[2], w[3]) for w in reps]
     out = {}
     for s in shapes:
         x = _dev_bf16(workloads.draw_x(s))
         y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device="cuda")
         ws = ws_for(s)
         calls = [(lambda w=w: any4.any4_matmul(x, w[0], w[1], w[2], w[3], s.G, y=y,
-                                               overlap_prior=overlap, workspace=ws))
+                                               overlap_prior=overlap, workspace=ws,
+                                               decode_layout=decode_layout))
                  for w in reps]
         us = _time_graph(stream, calls, max(2, 200 // bc))
         gbs = s.alg_bytes() / (us * 1e-6) / 1e9
@@ -516,7 +520,7 @@ def gpu_arm(args, rank, world):
     # the other M = 1 targets (tiny, the G = 64 variant, the 70B-shaped
     # matrices) and the batch sweep (M = 2 .. 32, 70B at M = 8): each weight set
     # once on rotating copies larger than L2, timed at every M it is used with
-    more_m1, batch = {}, {}
+    more_m1, batch, decode_layout = {}, {}, {}
     if not args.skip_batch:
         groups = [workloads.TINY, [s for s in workloads.SKINNY_SWEEP if s.G == 64]]
         groups.append([s for s in workloads.SKINNY_SWEEP if s.G == 128])
@@ -526,6 +530,13 @@ def gpu_arm(args, rank, world):
             res = time_weight_set(grp, stream, overlap, peaks)
             for s in grp:
                 (more_m1 if s.M == 1 and s.name != "sweep_m1" else batch)[s.name] = res[s.name]
+        torch.cuda.synchronize()
+        # the same M = 1 shapes on codes in the decode layout (any4_repack)
+        for s in ([s for s in workloads.LLAMA3_8B_DECODE if s.name in ("8b_gate", "8b_down")]
+                  + [s for s in workloads.LLAMA3_70B_DECODE
+                     if s.name in ("70b_gate_m1", "70b_down_m1")]):
+            decode_layout[s.name] = time_weight_set([s], stream, overlap, peaks,
+                                                    decode_layout=True)[s.name]
         torch.cuda.synchronize()
 
     fig3 = fig3_square_sweep(stream, overlap) if not args.skip_fig3 else {}
@@ -586,7 +597,7 @@ def gpu_arm(args, rank, world):
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
         "clocks": clocks, "detail": detail, "layer_calls": layer_calls, "single": single,
         "prefill": prefill,
-        "batch": batch, "more_m1": more_m1, "fig3": fig3,
+        "batch": batch, "more_m1": more_m1, "decode_layout": decode_layout, "fig3": fig3,
         "peaks": peaks,
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -945,6 +956,7 @@ def main():
             "layer_m1_calls": r["layer_calls"],
             "detail_m1": r["detail"],
             "detail_m1_more": r["more_m1"],
+            "m1_decode_layout": r["decode_layout"],
             "prefill_m2048": r["prefill"],
             # one compact summary of every target figure, last, where the
             # kept tail of the line always holds it
