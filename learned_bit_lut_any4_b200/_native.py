@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 import threading
+import weakref
 
 import torch
 
@@ -457,7 +458,9 @@ def any4_prepare(packed: torch.Tensor, lut: torch.Tensor, scale: torch.Tensor,
 
 # Per thread: the ctypes descriptor array of each group of prepared weights
 # used in a call (only the y pointers change from call to call), and the
-# workspace each needs per M.
+# workspace each needs per M.  Entries are keyed by the objects' ids and hold
+# only weak references to them, so the cache keeps no weights alive; an entry
+# whose objects are gone (an id reused by a new object) is rebuilt.
 _PREPARED_GROUPS = threading.local()
 _PREPARED_GROUPS_MAX = 4096
 
@@ -466,25 +469,27 @@ def _prepared_group(weights):
     cache = getattr(_PREPARED_GROUPS, "d", None)
     if cache is None:
         cache = _PREPARED_GROUPS.d = {}
-    key = tuple(weights)
+    key = tuple(id(w) for w in weights)
     g = cache.get(key)
-    if g is None:
-        w0 = weights[0]
-        for w in weights:
-            if not isinstance(w, Any4Prepared):
-                raise TypeError("mix of prepared and plain weights in one call")
-            if (w.device != w0.device or w.K != w0.K or w.G != w0.G
-                    or w.decode_layout != w0.decode_layout):
-                raise ValueError("prepared weights of one call must share device, K, G and "
-                                 "code layout")
-        descs = (Any4Weight * len(weights))()
-        for i, w in enumerate(weights):
-            pk, lt, sc, of = w._ptrs
-            descs[i] = Any4Weight(pk, lt, w.lut_row_stride, sc, of, 0, w.N)
-        if len(cache) >= _PREPARED_GROUPS_MAX:
-            cache.clear()
-        di = w0.device.index if w0.device.index is not None else -1
-        g = cache[key] = [descs, w0.K, w0.G, w0.device, di, {}, w0.decode_layout]
+    if g is not None and all(r() is w for r, w in zip(g[7], weights)):
+        return g
+    w0 = weights[0]
+    for w in weights:
+        if not isinstance(w, Any4Prepared):
+            raise TypeError("mix of prepared and plain weights in one call")
+        if (w.device != w0.device or w.K != w0.K or w.G != w0.G
+                or w.decode_layout != w0.decode_layout):
+            raise ValueError("prepared weights of one call must share device, K, G and "
+                             "code layout")
+    descs = (Any4Weight * len(weights))()
+    for i, w in enumerate(weights):
+        pk, lt, sc, of = w._ptrs
+        descs[i] = Any4Weight(pk, lt, w.lut_row_stride, sc, of, 0, w.N)
+    if len(cache) >= _PREPARED_GROUPS_MAX:
+        cache.clear()
+    di = w0.device.index if w0.device.index is not None else -1
+    g = cache[key] = [descs, w0.K, w0.G, w0.device, di, {}, w0.decode_layout,
+                      tuple(weakref.ref(w) for w in weights)]
     return g
 
 
@@ -689,7 +694,7 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
     p = PATHS[path]
     if isinstance(weights[0], Any4Prepared):
         # prepared weights: only x, the y's and the workspace are checked here
-        descs, K, Gp, dev, di, ws_need, dl = _prepared_group(weights)
+        descs, K, Gp, dev, di, ws_need, dl, _refs = _prepared_group(weights)
         if G != Gp:
             raise ValueError(f"G={G} but the weights were prepared with G={Gp}")
         M = _prepared_x(x, K, di)

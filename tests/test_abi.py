@@ -422,3 +422,25 @@ def test_prepare_checks_the_weights_once():
         any4.any4_prepare(packed, lut.float(), so, so, G)
     with pytest.raises(ValueError, match="CUDA tensor"):
         any4.any4_prepare(packed, lut, so, so, G)
+
+
+def test_prepared_group_cache_keeps_no_weights_alive():
+    """The binding caches each group of prepared weights' descriptor array,
+    but must not keep the weights (and their device tensors) alive."""
+    import gc
+    import weakref
+    import torch
+    ws = []
+    for n in (8, 16):
+        w = object.__new__(_native.Any4Prepared)   # host stand-ins: no CUDA needed
+        w.packed = torch.zeros((n, 512), dtype=torch.uint8)
+        w.lut = w.scale = w.offset = None
+        w.G, w.N, w.K, w.lut_row_stride = 128, n, 1024, 16
+        w.device, w.decode_layout, w._ptrs = w.packed.device, False, (0, 0, 0, 0)
+        ws.append(w)
+    g = _native._prepared_group(ws)
+    assert g is _native._prepared_group(ws)          # a hit the second time
+    refs = [weakref.ref(w) for w in ws]
+    del ws, g
+    gc.collect()
+    assert all(r() is None for r in refs)
