@@ -441,6 +441,6 @@ def test_prepared_group_cache_keeps_no_weights_alive():
     g = _native._prepared_group(ws)
     assert g is _native._prepared_group(ws)          # a hit the second time
     refs = [weakref.ref(w) for w in ws]
-    del ws, g
+    del ws, g, w  # (w: the loop variable still names the last one)
     gc.collect()
     assert all(r() is None for r in refs)
