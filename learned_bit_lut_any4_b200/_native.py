@@ -469,10 +469,14 @@ def _prepared_group(weights):
     cache = getattr(_PREPARED_GROUPS, "d", None)
     if cache is None:
         cache = _PREPARED_GROUPS.d = {}
-    key = tuple(id(w) for w in weights)
+    key = tuple(map(id, weights))
     g = cache.get(key)
-    if g is not None and all(r() is w for r, w in zip(g[7], weights)):
-        return g
+    if g is not None:
+        for r, w in zip(g[7], weights):
+            if r() is not w:
+                break
+        else:
+            return g
     w0 = weights[0]
     for w in weights:
         if not isinstance(w, Any4Prepared):
