@@ -593,6 +593,30 @@ def gpu_arm(args, rank, world):
     e2e_ms = allreduce_max(a.elapsed_time(b), world)
     e2e_gbs = allreduce_sum(step_bytes * e2e_steps, world) / (e2e_ms * 1e-3) / 1e9
 
+    # the same step as a serving loop replays it: the host copies and the four
+    # calls captured once (one step per weight copy) in a CUDA graph, so the
+    # host issues one launch per `copies` steps instead of six operations a step
+    e2e_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(e2e_graph, stream=stream):
+        for c in range(copies):
+            e2e_step(c)
+    g_reps = max(1, e2e_steps // copies)
+    with torch.cuda.stream(stream):
+        e2e_graph.replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(g_reps):
+            e2e_graph.replay()
+        b.record(stream)
+    b.synchronize()
+    barrier(world)
+    eg_ms = allreduce_max(a.elapsed_time(b), world)
+    eg_gbs = allreduce_sum(step_bytes * g_reps * copies, world) / (eg_ms * 1e-3) / 1e9
+    del e2e_graph
+
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
         "clocks": clocks, "detail": detail, "layer_calls": layer_calls, "single": single,
@@ -602,6 +626,11 @@ def gpu_arm(args, rank, world):
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "e2e_graph": {"value": round(eg_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h,
+                      "us_per_step": round(eg_ms * 1e3 / (g_reps * copies), 2),
+                      "how": "the e2e step (pinned H2D of x, four calls, D2H of y) "
+                             "captured in a CUDA graph and replayed"},
         "launches": len(plan) * steps_timed,
     }
 
@@ -943,6 +972,7 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
+            "e2e_graph": r["e2e_graph"],
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
             # bulky details first; the target numbers (per-shape M = 1 and the
