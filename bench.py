@@ -235,6 +235,32 @@ def prepare_layer(shapes, copies):
     return sets
 
 
+def read_stream_rate(stream, nbytes=2 << 30, reps=10):
+    """HBM read bandwidth (GB/s, median and best of `reps` launches) of
+    any4_read_probe over a buffer of nbytes (16x the L2), CUDA events on
+    `stream`: the read-only ceiling of the decode matmuls, which read about 250
+    bytes for each byte they write."""
+    import torch
+    import learned_bit_lut_any4_b200 as any4
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty(1, dtype=torch.int32, device="cuda")
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            any4.any4_read_probe(buf, out)
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            any4.any4_read_probe(buf, out)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b) * 1e-3)
+    del buf
+    rates = sorted(nbytes / t / 1e9 for t in times)
+    return {"gbs_median": round(float(np.median(rates)), 1), "gbs_best": round(rates[-1], 1),
+            "bytes": nbytes, "launches": reps, "kernel": "read_probe_kernel (any4_read_probe)"}
+
+
 def _time_graph(stream, calls, n_rep):
     """µs per call of `calls` (a list of no-argument callables) captured once in
     a CUDA graph and replayed n_rep times on `stream` (events on that stream)."""
@@ -616,6 +642,7 @@ def gpu_arm(args, rank, world):
     eg_ms = allreduce_max(a.elapsed_time(b), world)
     eg_gbs = allreduce_sum(step_bytes * g_reps * copies, world) / (eg_ms * 1e-3) / 1e9
     del e2e_graph
+    read_stream = read_stream_rate(stream)
 
     return {
         "value": value_gbs, "ms_per_step": ms_per_step, "steps_timed": steps_timed,
@@ -626,6 +653,7 @@ def gpu_arm(args, rank, world):
         "copies": copies, "step_bytes": step_bytes,
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "read_stream": read_stream,
         "e2e_graph": {"value": round(eg_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h,
                       "us_per_step": round(eg_ms * 1e3 / (g_reps * copies), 2),
@@ -970,6 +998,8 @@ def main():
                                  if not args.ungrouped else "7 separate calls")},
             "us_per_layer": round(r["ms_per_step"] * 1e3, 2),
             "roofline": roofline,
+            "hbm_read_stream": dict(r["read_stream"], layer_frac=round(
+                r["value"] / r["read_stream"]["gbs_median"], 4)),
             "cpu_baseline": cpu,
             "e2e": r["e2e"],
             "e2e_graph": r["e2e_graph"],

@@ -220,6 +220,24 @@ ANY4_API any4_status any4_group_sums(const uint16_t* x, float* xsum, int64_t M, 
                                      int64_t G, any4_stream_t stream);
 
 /*
+ * any4_read_probe -- a read-only stream over a device buffer, the measurement
+ * of the read bandwidth that bounds the decode matmuls (they read the packed
+ * codes, tables, scales and offsets once and write only y, so their roofline
+ * is HBM delivering reads alone, not a copy's mix of reads and writes):
+ *   *out = XOR of the 32-bit words buf[0 .. bytes / 4)
+ *   buf    device, caller-owned, 16-byte aligned (may be NULL when bytes == 0)
+ *   bytes  >= 0, a multiple of 16
+ *   out    one uint32 in device memory, caller-owned, 4-byte aligned; zeroed
+ *          on `stream` before the kernel runs (0 for an empty buffer)
+ * Every byte is read once, with 16-byte loads that skip L1, by a grid of
+ * 8 blocks of 256 threads per SM.  The result does not depend on the order of
+ * the reads.  Returns ANY4_ERR_NULL, _SHAPE or _ALIGN without launching when a
+ * precondition fails; asynchronous on `stream` otherwise.
+ */
+ANY4_API any4_status any4_read_probe(const void* buf, int64_t bytes, uint32_t* out,
+                                     any4_stream_t stream);
+
+/*
  * any4_matmul -- y = x * dequant(W)^T (paper §4.1 Eq. 8, orientation §4.2),
  * dequantisation fused (W is never written to memory on the decode path).
  *   x               [M][K] bf16

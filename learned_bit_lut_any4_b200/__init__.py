@@ -28,6 +28,7 @@ from ._native import (  # noqa: F401
     any4_dequant,
     any4_dequant_bits,
     any4_group_sums,
+    any4_read_probe,
     any4_matmul,
     any4_matmul_bits,
     any4_matmul_bits_workspace_size,

@@ -112,6 +112,8 @@ def library() -> ctypes.CDLL:
     lib.any4_matmul_bits_workspace_size.restype = sz
     lib.any4_group_sums.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.any4_group_sums.restype = i32
+    lib.any4_read_probe.argtypes = [vp, i64, vp, vp]
+    lib.any4_read_probe.restype = i32
     lib.any4_bits_per_weight.argtypes = [i64, i64]
     lib.any4_bits_per_weight.restype = ctypes.c_double
     lib.any4_version.argtypes = []
@@ -572,6 +574,30 @@ def any4_group_sums(x: torch.Tensor, G: int, xsum: torch.Tensor | None = None) -
         _check(library().any4_group_sums(_ptr(x), _ptr(xsum), M, K, G, _stream(dev)),
                "any4_group_sums")
     return xsum
+
+
+def any4_read_probe(buf: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """A read-only stream over buf (a contiguous CUDA tensor of a multiple of
+    16 bytes): returns a one-element int32 tensor holding the XOR of its 32-bit
+    words.  Timed, it measures the HBM read bandwidth that bounds the decode
+    matmuls."""
+    if not isinstance(buf, torch.Tensor) or not buf.is_cuda:
+        raise ValueError("buf must be a CUDA tensor")
+    if not buf.is_contiguous():
+        raise ValueError("buf must be contiguous")
+    dev = buf.device
+    nbytes = buf.numel() * buf.element_size()
+    if nbytes % 16:
+        raise ValueError(f"buf holds {nbytes} bytes, not a multiple of 16")
+    if out is None:
+        out = torch.empty(1, dtype=torch.int32, device=dev)
+    _need(out, "out", (torch.int32,), dev)
+    if out.numel() < 1:
+        raise ValueError("out must hold one int32")
+    with _on_device(dev):
+        _check(library().any4_read_probe(_ptr(buf) if nbytes else None, nbytes, _ptr(out),
+                                         _stream(dev)), "any4_read_probe")
+    return out
 
 
 def any4_matmul_workspace_size(M: int, N: int, K: int, G: int, path: str = "auto") -> int:

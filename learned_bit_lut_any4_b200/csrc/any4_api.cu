@@ -365,6 +365,17 @@ any4_status any4_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K
   return launch_group_sums(x, xsum, M, K, G, (cudaStream_t)stream, dev);
 }
 
+any4_status any4_read_probe(const void* buf, int64_t bytes, uint32_t* out,
+                            any4_stream_t stream) {
+  if (!out || (!buf && bytes > 0)) return ANY4_ERR_NULL;
+  if (bytes < 0 || bytes % 16 != 0) return ANY4_ERR_SHAPE;
+  if ((buf && !aligned16(buf)) || reinterpret_cast<uintptr_t>(out) % 4 != 0) return ANY4_ERR_ALIGN;
+  DeviceInfo dev;
+  any4_status st = current_device(&dev);
+  if (st != ANY4_OK) return st;
+  return launch_read_probe(buf, bytes, out, (cudaStream_t)stream, dev);
+}
+
 any4_path any4_matmul_choose_path(int64_t M, int64_t N, int64_t K, int64_t G) {
   (void)N; (void)K; (void)G;
   return M <= kDecodeMaxM ? ANY4_PATH_DECODE : ANY4_PATH_PREFILL;

@@ -139,6 +139,10 @@ any4_status launch_dequant(const uint8_t* packed, const uint16_t* lut, int64_t l
                            const DeviceInfo& dev, bool streaming = true);
 any4_status launch_group_sums(const uint16_t* x, float* xsum, int64_t M, int64_t K, int64_t G,
                               cudaStream_t stream, const DeviceInfo& dev);
+// out = XOR of the 32-bit words of buf[0 .. bytes) (bytes a multiple of 16);
+// zeroes *out first, on the stream.
+any4_status launch_read_probe(const void* buf, int64_t bytes, uint32_t* out, cudaStream_t stream,
+                              const DeviceInfo& dev);
 // The decode path (M <= 16).  y32, when not NULL, receives the fp32 sums
 // instead of y (the unrounded results).  A workspace of at least
 // decode_pair_workspace_size bytes selects the pair-table kernel for M <= 2.

@@ -110,6 +110,19 @@ def test_repack_rejects_bad_arguments():
         any4.any4_repack(torch.zeros((4, 768), dtype=torch.uint8))
 
 
+def test_read_probe_rejects_bad_arguments():
+    lib = _native.library()
+    assert lib.any4_read_probe(FAKE, 64, None, None) == any4.ANY4_ERR_NULL
+    assert lib.any4_read_probe(None, 64, FAKE, None) == any4.ANY4_ERR_NULL
+    assert lib.any4_read_probe(FAKE, 40, FAKE + 64, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_read_probe(FAKE, -16, FAKE + 64, None) == any4.ANY4_ERR_SHAPE
+    assert lib.any4_read_probe(FAKE + 8, 64, FAKE + 4096, None) == any4.ANY4_ERR_ALIGN
+    assert lib.any4_read_probe(FAKE, 64, FAKE + 4098, None) == any4.ANY4_ERR_ALIGN
+    import torch
+    with pytest.raises(ValueError, match="CUDA"):
+        any4.any4_read_probe(torch.zeros(16, dtype=torch.uint8))
+
+
 def test_pack_and_dequant_reject_bad_arguments():
     lib = _native.library()
     assert lib.any4_pack(None, FAKE, 4, 64, None, None) == any4.ANY4_ERR_NULL
