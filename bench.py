@@ -695,6 +695,31 @@ def oracle_layer_rate(max_seconds: float):
                       f"(dequant + fp64 matmul), {dt:.1f} s"}
 
 
+def oracle_single_thread():
+    """The oracle on one host thread for the Tiny and 8B gate M = 1 configs:
+    seconds of its dequant alone and of its whole matmul (dequant, then the
+    fp64 product), one call each."""
+    import oracle
+    prev = oracle.num_threads()
+    oracle.set_num_threads(1)
+    out = {}
+    try:
+        for s in [workloads.TINY[0]] + [s for s in workloads.LLAMA3_8B_DECODE
+                                        if s.name == "8b_gate"]:
+            p = workloads.make(s)
+            packed = oracle.pack(p.idx)
+            t0 = time.perf_counter()
+            oracle.dequant(packed, p.lut, p.scale, p.offset, s.G)
+            t1 = time.perf_counter()
+            oracle.any4_matmul(p.x, packed, p.lut, p.scale, p.offset, s.G)
+            t2 = time.perf_counter()
+            out[s.name] = {"dequant_s": round(t1 - t0, 4), "matmul_s": round(t2 - t1, 4),
+                           "GB/s": round(s.alg_bytes() / (t2 - t1) / 1e9, 4)}
+    finally:
+        oracle.set_num_threads(prev)
+    return {"cores": 1, "configs": out}
+
+
 def reference_arm(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -960,6 +985,8 @@ def main():
             return
         peaks = r["peaks"]
         cpu = oracle_layer_rate(max_seconds=args.cpu_seconds) if world == 1 else None
+        if cpu is not None:
+            cpu["single_thread"] = oracle_single_thread()
         table = None
         if world == 1 and not args.skip_table_learning:
             try:  # a detail beside the step: its failure is reported, not fatal
