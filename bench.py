@@ -140,7 +140,8 @@ def allreduce_sum(v, world):
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "clocks.mem")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -165,7 +166,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sms, maxs, reasons = [], [], set()
+        sms, maxs, mems, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
@@ -179,6 +180,11 @@ class ClockSampler:
             for nm, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
+            if len(parts) > 9:
+                try:
+                    mems.append(float(parts[9]))
+                except ValueError:
+                    pass
         try:
             os.remove(self.path)
         except OSError:
@@ -186,7 +192,8 @@ class ClockSampler:
         if not sms:
             return None
         return {"sm_mhz": float(np.median(sms)), "sm_max_mhz": float(max(maxs)),
-                "reasons": sorted(reasons), "samples": len(sms)}
+                "reasons": sorted(reasons), "samples": len(sms),
+                "mem_mhz": float(np.median(mems)) if mems else None}
 
 
 # ---------------------------------------------------------------------------
