@@ -479,9 +479,20 @@ def gpu_arm(args, rank, world):
             b.record(stream)
         b.synchronize()
         us = a.elapsed_time(b) * 1e3 / (n_rep * copies)
+        # 10 replays timed one by one: best and median µs per call
+        per = []
+        with torch.cuda.stream(stream):
+            for _ in range(10):
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                b.synchronize()
+                per.append(a.elapsed_time(b) * 1e3 / copies)
         gbs = s.alg_bytes() / (us * 1e-6) / 1e9
         detail[s.name] = {"us": round(us, 3), "GB/s": round(gbs, 1),
-                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                          "us_best_of_10": round(min(per), 3),
+                          "us_median_of_10": round(float(np.median(per)), 3)}
         del g
 
     # the layer both ways: the four calls of the step (q/k/v and gate/up
