@@ -716,7 +716,6 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
         raise ValueError(f"between 1 and {ANY4_GROUP_MAX} matrices")
     if ys is not None and len(ys) != len(weights):
         raise ValueError("one y per matrix")
-    descs = (Any4Weight * len(weights))()
     outs = []
     M = K = None
     need_ws = 0
@@ -763,6 +762,7 @@ def any4_matmul_grouped(x: torch.Tensor, weights, G: int, ys=None,
                                            | (ANY4_FLAG_DECODE_LAYOUT if dl else 0),
                                            st), "any4_matmul_grouped")
         return outs
+    descs = (Any4Weight * len(weights))()
     for i, wt in enumerate(weights):
         if isinstance(wt, Any4Prepared):
             raise TypeError("mix of prepared and plain weights in one call")
