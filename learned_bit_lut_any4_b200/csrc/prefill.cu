@@ -119,7 +119,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-// mbar_wait by every lane of a warp, with one verdict for the whole warp (so
+// mbar_wait by every lane of a warp, with one outcome for the whole warp (so
 // that no lane is left alone in a later warp-synchronous instruction).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, int32_t* dev_status,
