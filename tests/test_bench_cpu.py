@@ -29,3 +29,38 @@ def test_target_summary_tolerates_missing_details():
     t = bench.target_summary({}, {"error": "x"}, None, {"hbm_gbs": 1.0, "bf16_tflops": 1.0})
     assert t["m1_8b_layer_grouped"] is None and t["dequant_8b_gate"] is None
     assert "quantize_8b_down_ms" not in t
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        pass
+
+
+def test_clock_sampler_reads_sm_and_memory_clocks(tmp_path):
+    import os
+    c = bench.ClockSampler(0)
+    c.path = str(tmp_path / "clocks.csv")
+    with open(c.path, "w") as f:
+        f.write("0, 1965, 1965, 512.0, 0x0, Not Active, Not Active, Not Active, Not Active, 3996\n")
+        f.write("0, 1800, 1965, 990.5, 0x4, Not Active, Not Active, Not Active, Active, 3996\n")
+        f.write("0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active, 3996\n")
+        f.write("garbage line\n")
+    c.proc = _FakeProc()
+    c.fh = open(os.devnull, "w")
+    got = c.stop()
+    assert got == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3, "mem_mhz": 3996.0}
+    assert not os.path.exists(c.path)
+
+
+def test_oracle_single_thread_restores_the_thread_count():
+    import oracle
+    before = oracle.num_threads()
+    got = bench.oracle_single_thread()
+    assert oracle.num_threads() == before
+    assert got["cores"] == 1 and set(got["configs"]) == {"tiny", "8b_gate"}
+    for v in got["configs"].values():
+        assert v["dequant_s"] > 0 and v["matmul_s"] > 0 and v["GB/s"] > 0
